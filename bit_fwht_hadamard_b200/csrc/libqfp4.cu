@@ -1,0 +1,7 @@
+// libqfp4.cu -- single translation unit of the library (so the device-side
+// error word and the inline helpers need no relocatable device code).
+#include "runtime.cu"
+#include "quantize1d.cu"
+#include "dequant_fp32scale.cu"
+#include "pending.cu"
+#include "api.cu"

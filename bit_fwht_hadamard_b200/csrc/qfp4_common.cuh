@@ -1,0 +1,290 @@
+// qfp4_common.cuh -- shared device/host helpers of libqfp4 (sm_100a only).
+//
+// Holds: the status plumbing, PTX wrappers for mbarriers and TMA, the
+// tensor-map encoder (reached through the driver entry point, so the
+// library does not link libcuda), and the device numerics of the method:
+// Philox4x32-10, the E2M1 / E4M3 conversions, the truncation-free E8M0
+// exponent and the Walsh-Hadamard butterflies.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/qfp4.h"
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ != 1000)
+#error "libqfp4 is built for sm_100a only"
+#endif
+
+namespace qfp4 {
+
+template <class T>
+__host__ __device__ __forceinline__ T imin(T a, T b) { return a < b ? a : b; }
+template <class T>
+__host__ __device__ __forceinline__ T imax(T a, T b) { return a < b ? b : a; }
+
+// ------------------------------------------------------------------ errors
+// Device-side sticky error word (bounded waits that gave up, bounds checks).
+enum : int { DEV_ERR_NONE = 0, DEV_ERR_TIMEOUT = 1, DEV_ERR_BOUNDS = 2 };
+static __device__ int g_dev_error = 0;   // one copy: the library is a single translation unit
+
+// A spin on an mbarrier gives up after this many polls (seconds of wall
+// time), records DEV_ERR_TIMEOUT and lets the kernel return.
+constexpr uint32_t kSpinLimit = 1u << 28;
+
+__device__ __forceinline__ void record_error(int code) { atomicCAS(&g_dev_error, 0, code); }
+
+// ------------------------------------------------------------------ PTX: mbarrier
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fence_mbar_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Bounded wait: true when the phase completed, false (error recorded) when
+// kWaitLimitNs of wall time (or kSpinLimit polls) ran out.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 0; i < kSpinLimit; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 255u) == 255u && global_ns() - t0 > kWaitLimitNs) break;
+    }
+    record_error(DEV_ERR_TIMEOUT);
+    return false;
+}
+
+// ------------------------------------------------------------------ PTX: TMA
+__device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(void *smem_dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1,
+                                            int c2)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map)
+{
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ------------------------------------------------------------------ numerics
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11): multipliers 0xD2511F53
+// and 0xCD9E8D57, Weyl increments 0x9E3779B9 / 0xBB67AE85, ten rounds.
+// Counter (c0, c1, 0, 0); key (k0, k1).
+__device__ __forceinline__ uint4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t k0, uint32_t k1)
+{
+    uint32_t c2 = 0u, c3 = 0u;
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        const uint32_t hi0 = __umulhi(0xD2511F53u, c0), lo0 = 0xD2511F53u * c0;
+        const uint32_t hi1 = __umulhi(0xCD9E8D57u, c2), lo1 = 0xCD9E8D57u * c2;
+        const uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+        c0 = n0;
+        c1 = lo1;
+        c2 = n2;
+        c3 = lo0;
+        k0 += 0x9E3779B9u;
+        k1 += 0xBB67AE85u;
+    }
+    return make_uint4(c0, c1, c2, c3);
+}
+
+// The four random words of elements 4q .. 4q+3 (counter q = e / 4).
+__device__ __forceinline__ uint4 sr_words4(uint64_t seed, uint64_t q)
+{
+    return philox4x32_10(static_cast<uint32_t>(q), static_cast<uint32_t>(q >> 32), static_cast<uint32_t>(seed),
+                         static_cast<uint32_t>(seed >> 32));
+}
+
+// Two bf16 packed in a 32-bit word -> binary32 (exact widening).
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// E2M1 round-to-nearest-even with saturation to +-6, eight values packed
+// into one 32-bit word (element t in nibble t).  Uses the sm_100 hardware
+// conversion; the code's sign bit is then forced to the sign of the input
+// so that values rounding to zero keep their sign (the oracle's rule).
+__device__ __forceinline__ uint32_t e2m1x8_rne(const float *v)
+{
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out)
+        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+    uint32_t s = 0;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) s |= (__float_as_uint(v[t]) >> 31) << (4 * t + 3);
+    return out | s;
+}
+
+// E2M1 stochastic rounding of one value (|v| <= 6 or saturating):
+// lo <= |v| < hi adjacent grid values, up iff u < (|v| - lo) / (hi - lo)
+// with u = (w >> 8) * 2^-24.  Returns the 4-bit code.
+__device__ __forceinline__ uint32_t e2m1_sr(float v, uint32_t w)
+{
+    const uint32_t sign = (__float_as_uint(v) >> 28) & 8u;
+    const float a = fabsf(v);
+    float lo, sp, inv_sp;              // lower grid value, spacing, 1/spacing
+    if (a >= 1.0f) {
+        const uint32_t spb = (__float_as_uint(a) & 0x7F800000u) - 0x00800000u;   // 2^(exp-1)
+        lo = __uint_as_float(__float_as_uint(a) & 0x7FC00000u);                 // 1 mantissa bit
+        sp = __uint_as_float(spb);
+        inv_sp = __uint_as_float((254u << 23) - spb);
+    } else {
+        lo = a >= 0.5f ? 0.5f : 0.0f;
+        sp = 0.5f;
+        inv_sp = 2.0f;
+    }
+    const float p = __fmul_rn(__fsub_rn(a, lo), inv_sp);   // exact: power-of-two spacing
+    const float u = __fmul_rn(static_cast<float>(w >> 8), 5.9604644775390625e-08f);  // 2^-24
+    float r = (u < p) ? __fadd_rn(lo, sp) : lo;
+    r = fminf(r, 6.0f);
+    uint32_t code;
+    asm("{\n\t.reg .b8 b;\n\tcvt.rn.satfinite.e2m1x2.f32 b, %1, %1;\n\tcvt.u32.u8 %0, b;\n\t}" : "=r"(code) : "f"(r));
+    return (code & 7u) | sign;
+}
+
+// E4M3 (OCP) round-to-nearest-even, saturating to +-448: returns the byte.
+__device__ __forceinline__ uint32_t e4m3_rne(float v)
+{
+    uint16_t out;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %1;" : "=h"(out) : "f"(v));
+    return out & 0xFFu;
+}
+
+// Two values -> two E4M3 bytes (a in the low byte).
+__device__ __forceinline__ uint32_t e4m3x2_rne(float a, float b)
+{
+    uint16_t out;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(b), "f"(a));
+    return out;
+}
+
+// E4M3 byte -> binary32 (exact), from the bit fields.
+__device__ __forceinline__ float e4m3_value(uint32_t b)
+{
+    const uint32_t E = (b >> 3) & 15u, m = b & 7u;
+    // E == 0: m * 2^-9 (2^-9 has binary32 exponent field 118); E > 0: (1 + m/8) 2^(E-7)
+    const float mag = (E == 0) ? static_cast<float>(m) * __uint_as_float(118u << 23)
+                               : __uint_as_float(((E + 120u) << 23) | (m << 20));
+    return (b & 0x80u) ? -mag : mag;
+}
+
+// Least k in [-127, 127] with top * 2^k >= amax, top = top_m * 2^top_e with
+// top_m in [1, 2) given by its 23-bit fraction (6 = 1.5 * 2^2: 0x400000, 2;
+// 448 = 1.75 * 2^8: 0x600000, 8).  amax = m * 2^e: k = e - top_e when
+// m <= top_m, else e - top_e + 1.  amax == 0 gives -127.
+__device__ __forceinline__ int scale_exp(float amax, uint32_t top_frac, int top_e)
+{
+    const uint32_t u = __float_as_uint(amax) & 0x7FFFFFFFu;
+    if (u == 0) return -127;
+    int e;
+    uint32_t f;
+    const uint32_t E = u >> 23;
+    if (E == 0) {                                  // subnormal: normalise
+        const int lead = 31 - __clz(u);
+        e = lead - 149;
+        f = (u << (23 - lead)) & 0x7FFFFFu;
+    } else {
+        e = static_cast<int>(E) - 127;
+        f = u & 0x7FFFFFu;
+    }
+    const int k = (f <= top_frac) ? e - top_e : e - top_e + 1;
+    return max(-127, min(127, k));
+}
+
+// 2^k as binary32 for k in [-127, 127] (2^-127 is the subnormal 0x00400000).
+__device__ __forceinline__ float exp2i(int k)
+{
+    return k >= -126 ? __uint_as_float(static_cast<uint32_t>(k + 127) << 23) : __uint_as_float(0x00400000u);
+}
+
+// binary32 constant nearest 1/sqrt(128) = 2^-3.5.
+__device__ __forceinline__ float inv_sqrt128() { return __uint_as_float(0x3DB504F3u); }
+
+}  // namespace qfp4
+
+// ------------------------------------------------------------------ host side
+namespace qfp4 {
+
+int encode_tensor_map(CUtensorMap *map, CUtensorMapDataType dtype, int rank, void *gaddr, const uint64_t *dims,
+                      const uint64_t *strides_bytes /* rank-1 entries */, const uint32_t *box,
+                      CUtensorMapSwizzle swizzle);
+
+int num_sms();
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace qfp4
+
+#define QFP4_LAUNCH_CHECK()                                                                        \
+    do {                                                                                           \
+        if (cudaPeekAtLastError() != cudaSuccess) {                                                \
+            (void)cudaGetLastError();                                                              \
+            return QFP4_ERR_CUDA;                                                                  \
+        }                                                                                          \
+    } while (0)

@@ -1,0 +1,523 @@
+// quantize1d.cu -- 1D FP4 microscaling quantize (MXFP4 / NVFP4), optional
+// 128-point Walsh-Hadamard rotation, RNE or Philox stochastic rounding,
+// optional four-over-six; plus the NVFP4 tensor-amax pass.
+//
+// Method ([QN] Hadamard rotation + QuTLASS online quantization; [LB] §FP4,
+// §2, §3, §7; [46] Methodology): per 128 block along K an optional
+// normalised FWHT, per group of g a scale (E8M0 truncation-free for MXFP4,
+// E4M3 under the tensor scale for NVFP4), v = x / S, round onto E2M1.
+//
+// Layout: the input is a flat stream of n = M*K elements (groups never cross
+// rows because K % g == 0, and rotation blocks never cross rows because
+// K % 128 == 0).  A thread owns one 64-element unit (a 128-byte bf16 row of
+// the tile); the two threads of a 128-element rotation block exchange one
+// butterfly stage with a warp shuffle, every other stage runs in registers.
+// bf16 tiles of 512 units (64 KiB) are brought into shared memory by TMA
+// with 128-byte swizzle (so the per-thread 16-byte reads are bank-conflict
+// free) through a 3-stage mbarrier pipeline; the grid is persistent.
+#include "qfp4_common.cuh"
+#include "quantize1d.cuh"
+
+namespace qfp4 {
+
+constexpr int QT_THREADS = 512;                 // one 64-element unit per thread
+constexpr int QT_TILE_ROWS = QT_THREADS;        // 64-element rows per tile
+constexpr int QT_BOX_ROWS = 256;                // TMA box height (hardware limit 256)
+constexpr int QT_STAGES = 3;
+constexpr int QT_STAGE_BYTES = QT_TILE_ROWS * 128;
+constexpr int QT_SMEM_BYTES = QT_STAGES * QT_STAGE_BYTES + 1024;
+
+// E2M1 code -> binary32 value (exact), from the bit fields.
+__device__ __forceinline__ float e2m1_value(uint32_t c)
+{
+    const uint32_t E = (c >> 1) & 3u, m = c & 1u;
+    const float mag = (E == 0) ? (m ? 0.5f : 0.0f) : __uint_as_float(((E + 126u) << 23) | (m << 22));
+    return (c & 8u) ? -mag : mag;
+}
+
+// Walsh-Hadamard transform of a 128 block held as 64 values in each of two
+// lanes (lane^1 partner; the even lane holds elements 0..63).  Stages
+// h = 1..32 are local, h = 64 crosses the pair, then the 1/sqrt(128) scale.
+__device__ __forceinline__ void fwht128_pair(float (&v)[64], bool upper)
+{
+#pragma unroll
+    for (int h = 1; h < 64; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+            if ((i & h) == 0) {
+                const float a = v[i], b = v[i + h];
+                v[i] = __fadd_rn(a, b);
+                v[i + h] = __fsub_rn(a, b);
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+        const float o = __shfl_xor_sync(0xFFFFFFFFu, v[i], 1);
+        v[i] = upper ? __fsub_rn(o, v[i]) : __fadd_rn(v[i], o);
+    }
+    const float c = inv_sqrt128();
+#pragma unroll
+    for (int i = 0; i < 64; ++i) v[i] = __fmul_rn(v[i], c);
+}
+
+// Result of one unit: 64 nibbles (8 words) and up to 4 scale bytes.
+struct UnitOut {
+    uint32_t codes[8];
+    uint32_t scales;        // byte g = scale of group g within the unit
+};
+
+// Quantize 16 values under effective scale S (RNE): codes (2 words), and
+// when `sse` is given the binary32 squared error summed as a fixed tree.
+__device__ __forceinline__ void nv_block_rne(const float *x, float S, uint32_t *w2, float *sse)
+{
+    float q[16];
+    if (S == 0.0f) {
+        w2[0] = w2[1] = 0u;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) q[i] = 0.0f;
+    } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) q[i] = __fdiv_rn(x[i], S);
+        w2[0] = e2m1x8_rne(q);
+        w2[1] = e2m1x8_rne(q + 8);
+    }
+    if (sse) {
+        float e[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const uint32_t code = (w2[i >> 3] >> (4 * (i & 7))) & 15u;
+            const float deq = __fmul_rn(e2m1_value(code), S);
+            const float d = __fsub_rn(deq, x[i]);
+            e[i] = __fmul_rn(d, d);
+        }
+#pragma unroll
+        for (int h = 8; h >= 1; h >>= 1)
+#pragma unroll
+            for (int i = 0; i < h; ++i) e[i] = __fadd_rn(e[i], e[i + h]);
+        *sse = e[0];
+    }
+}
+
+// Stochastic rounding of 16 (NVFP4) or 32 (MXFP4) values v (already divided
+// by the scale) whose first element has logical index e (e % 4 == 0).
+template <int G>
+__device__ __forceinline__ void sr_group(const float *v, uint64_t e, uint64_t seed, uint32_t *words)
+{
+#pragma unroll
+    for (int w = 0; w < G / 8; ++w) words[w] = 0u;
+#pragma unroll
+    for (int q = 0; q < G / 4; ++q) {
+        const uint4 r = sr_words4(seed, (e >> 2) + q);
+        const uint32_t c0 = e2m1_sr(v[4 * q + 0], r.x), c1 = e2m1_sr(v[4 * q + 1], r.y);
+        const uint32_t c2 = e2m1_sr(v[4 * q + 2], r.z), c3 = e2m1_sr(v[4 * q + 3], r.w);
+        words[q >> 1] |= (c0 | (c1 << 4) | (c2 << 8) | (c3 << 12)) << (16 * (q & 1));
+    }
+}
+
+template <int FMT, bool SR, bool FOUR6>
+__device__ __forceinline__ void quant_unit(const float (&v)[64], uint64_t e0, float s_t, uint64_t seed, UnitOut &o)
+{
+    o.scales = 0u;
+    if (FMT == QFP4_MXFP4) {
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+            float amax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[32 * g + i]));
+            uint32_t *w = o.codes + 4 * g;
+            if (amax == 0.0f) {                      // all-zero group: byte 0, +0 codes
+                w[0] = w[1] = w[2] = w[3] = 0u;
+                continue;
+            }
+            const int k = scale_exp(amax, 0x400000u, 2);
+            o.scales |= static_cast<uint32_t>(k + 127) << (8 * g);
+            const float mul = exp2i(-k);             // x * 2^-k == x / 2^k exactly
+            float q[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) q[i] = __fmul_rn(v[32 * g + i], mul);
+            if (SR) {
+                sr_group<32>(q, e0 + 32 * g, seed, w);
+            } else {
+#pragma unroll
+                for (int t = 0; t < 4; ++t) w[t] = e2m1x8_rne(q + 8 * t);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const float *x = v + 16 * b;
+            float amax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
+            uint32_t *w = o.codes + 2 * b;
+            uint32_t enc = 0u;
+            float S = 0.0f;
+            if (s_t != 0.0f) {
+                enc = e4m3_rne(__fdiv_rn(__fdiv_rn(amax, 6.0f), s_t));
+                S = __fmul_rn(e4m3_value(enc), s_t);
+            }
+            if (FOUR6) {
+                uint32_t w6[2], w4[2];
+                float sse6, sse4;
+                uint32_t enc4 = 0u;
+                float S4 = 0.0f;
+                if (s_t != 0.0f) {
+                    enc4 = e4m3_rne(__fdiv_rn(__fdiv_rn(amax, 4.0f), s_t));
+                    S4 = __fmul_rn(e4m3_value(enc4), s_t);
+                }
+                nv_block_rne(x, S, w6, &sse6);
+                nv_block_rne(x, S4, w4, &sse4);
+                const bool pick4 = sse4 < sse6;
+                w[0] = pick4 ? w4[0] : w6[0];
+                w[1] = pick4 ? w4[1] : w6[1];
+                enc = pick4 ? enc4 : enc;
+            } else if (SR) {
+                if (S == 0.0f) {
+                    w[0] = w[1] = 0u;
+                } else {
+                    float q[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) q[i] = __fdiv_rn(x[i], S);
+                    sr_group<16>(q, e0 + 16 * b, seed, w);
+                }
+            } else {
+                nv_block_rne(x, S, w, nullptr);
+            }
+            o.scales |= enc << (8 * b);
+        }
+    }
+}
+
+__device__ __forceinline__ float block_max(float m, float *red)
+{
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __syncthreads();
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+    if (warp == 0) {
+        m = lane < static_cast<int>(blockDim.x >> 5) ? red[lane] : 0.0f;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+        if (lane == 0) red[0] = m;
+    }
+    __syncthreads();
+    return red[0];
+}
+
+// s_t = amax_t / (6 * 448), amax_t the max of the partial maxima.
+__device__ __forceinline__ float tensor_scale(const QuantParams &p, float *red)
+{
+    float m = 0.0f;
+    for (int i = threadIdx.x; i < p.n_partials; i += blockDim.x) m = fmaxf(m, p.partials[i]);
+    m = block_max(m, red);
+    return __fdiv_rn(m, 2688.0f);
+}
+
+template <int G>
+__device__ __forceinline__ void store_unit(const UnitOut &o, const QuantParams &p, uint64_t e0, int64_t n_valid)
+{
+    // n_valid: elements of this unit inside the launch range (a multiple of G)
+    uint8_t *cdst = p.codes + (e0 >> 1);
+    uint8_t *sdst = p.scales + e0 / G;
+    if (n_valid >= 64) {
+        uint4 *c4 = reinterpret_cast<uint4 *>(cdst);
+        c4[0] = make_uint4(o.codes[0], o.codes[1], o.codes[2], o.codes[3]);
+        c4[1] = make_uint4(o.codes[4], o.codes[5], o.codes[6], o.codes[7]);
+        if (G == 32) *reinterpret_cast<uint16_t *>(sdst) = static_cast<uint16_t>(o.scales);
+        else *reinterpret_cast<uint32_t *>(sdst) = o.scales;
+    } else {
+#pragma unroll
+        for (int gi = 0; gi < 64 / G; ++gi) {
+            if (gi * G < n_valid) {
+#pragma unroll
+                for (int w = 0; w < G / 8; ++w)
+                    reinterpret_cast<uint32_t *>(cdst)[gi * (G / 8) + w] = o.codes[gi * (G / 8) + w];
+                sdst[gi] = static_cast<uint8_t>(o.scales >> (8 * gi));
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------- TMA kernel
+template <int MODE, int FMT, bool ROT, bool SR, bool FOUR6>
+__global__ void __launch_bounds__(QT_THREADS, 1) k_quant1d_tma(const __grid_constant__ CUtensorMap tm, QuantParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ __align__(8) uint64_t full[QT_STAGES];
+    __shared__ float red[32];
+
+    const int tid = threadIdx.x;
+    const int64_t rows = p.n / 64;
+    const int64_t ntiles = (rows + QT_TILE_ROWS - 1) / QT_TILE_ROWS;
+    constexpr int G = FMT == QFP4_MXFP4 ? 32 : 16;
+
+    float s_t = 0.0f;
+    if (MODE == MODE_QUANT && FMT == QFP4_NVFP4) {
+        s_t = tensor_scale(p, red);
+        if (p.write_tscale && blockIdx.x == 0 && tid == 0) *p.tscale_out = s_t;
+    }
+    if (tid == 0) {
+        for (int s = 0; s < QT_STAGES; ++s) mbar_init(&full[s], 1);
+        fence_mbar_init();
+        prefetch_tensormap(&tm);
+    }
+    __syncthreads();
+
+    auto issue = [&](int64_t t, int s) {
+        uint8_t *dst = smem + s * QT_STAGE_BYTES;
+        mbar_arrive_expect_tx(&full[s], QT_STAGE_BYTES);
+        const int r0 = static_cast<int>(t * QT_TILE_ROWS);
+        tma_load_2d(dst, &tm, &full[s], 0, r0);
+        tma_load_2d(dst + QT_BOX_ROWS * 128, &tm, &full[s], 0, r0 + QT_BOX_ROWS);
+    };
+    if (tid == 0)
+        for (int s = 0; s < QT_STAGES; ++s) {
+            const int64_t t = blockIdx.x + static_cast<int64_t>(s) * gridDim.x;
+            if (t < ntiles) issue(t, s);
+        }
+
+    float tmax = 0.0f;
+    int it = 0;
+    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
+        const int s = it % QT_STAGES;
+        const uint32_t ph = (it / QT_STAGES) & 1u;
+        const bool ok = mbar_wait(&full[s], ph);
+        if (__syncthreads_or(!ok)) return;
+
+        const uint8_t *st = smem + s * QT_STAGE_BYTES + tid * 128;
+        float v[64];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const uint4 w = *reinterpret_cast<const uint4 *>(st + ((c ^ (tid & 7)) << 4));
+            v[8 * c + 0] = bf16lo(w.x);
+            v[8 * c + 1] = bf16hi(w.x);
+            v[8 * c + 2] = bf16lo(w.y);
+            v[8 * c + 3] = bf16hi(w.y);
+            v[8 * c + 4] = bf16lo(w.z);
+            v[8 * c + 5] = bf16hi(w.z);
+            v[8 * c + 6] = bf16lo(w.w);
+            v[8 * c + 7] = bf16hi(w.w);
+        }
+        __syncthreads();
+        if (tid == 0) {
+            const int64_t tn = t + static_cast<int64_t>(QT_STAGES) * gridDim.x;
+            if (tn < ntiles) issue(tn, s);
+        }
+
+        const int64_t row = t * QT_TILE_ROWS + tid;
+        const bool valid = row < rows;
+        if (ROT) fwht128_pair(v, (tid & 1) != 0);
+        if (MODE == MODE_AMAX) {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) tmax = fmaxf(tmax, fabsf(v[i]));
+        } else if (valid) {
+            const uint64_t e0 = p.e_base + static_cast<uint64_t>(row) * 64u;
+            UnitOut o;
+            quant_unit<FMT, SR, FOUR6>(v, e0, s_t, p.seed, o);
+            store_unit<G>(o, p, e0, 64);
+        }
+    }
+    if (MODE == MODE_AMAX) {
+        tmax = block_max(tmax, red);
+        if (tid == 0) p.partials_out[blockIdx.x] = tmax;
+    }
+}
+
+// ---------------------------------------------------------------- direct kernel
+// Loads straight from global memory (bf16 or binary32), one unit per thread;
+// serves binary32 inputs and the ragged tail (n % 64) of bf16 inputs.
+template <int MODE, int FMT, bool ROT, bool SR, bool FOUR6, typename T>
+__global__ void __launch_bounds__(128) k_quant1d_direct(const T *__restrict__ x, QuantParams p)
+{
+    __shared__ float red[32];
+    constexpr int G = FMT == QFP4_MXFP4 ? 32 : 16;
+    float s_t = 0.0f;
+    if (MODE == MODE_QUANT && FMT == QFP4_NVFP4) {
+        s_t = tensor_scale(p, red);
+        if (p.write_tscale && blockIdx.x == 0 && threadIdx.x == 0) *p.tscale_out = s_t;
+    }
+    const int64_t units = (p.n + 63) / 64;
+    float tmax = 0.0f;
+    for (int64_t u0 = static_cast<int64_t>(blockIdx.x) * blockDim.x; u0 < units;
+         u0 += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t u = u0 + threadIdx.x;
+        const int64_t off = u * 64;
+        const int64_t n_valid = u < units ? imin<int64_t>(64, p.n - off) : 0;
+        float v[64];
+#pragma unroll
+        for (int i = 0; i < 64; ++i) v[i] = 0.0f;
+        if (n_valid > 0) {
+            if (sizeof(T) == 4) {
+                const float4 *src = reinterpret_cast<const float4 *>(x + off);
+#pragma unroll
+                for (int c = 0; c < 16; ++c)
+                    if (4 * c < n_valid) {
+                        const float4 f = src[c];
+                        v[4 * c] = f.x;
+                        v[4 * c + 1] = f.y;
+                        v[4 * c + 2] = f.z;
+                        v[4 * c + 3] = f.w;
+                    }
+            } else {
+                const uint4 *src = reinterpret_cast<const uint4 *>(x + off);
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    if (8 * c < n_valid) {
+                        const uint4 w = src[c];
+                        v[8 * c] = bf16lo(w.x);
+                        v[8 * c + 1] = bf16hi(w.x);
+                        v[8 * c + 2] = bf16lo(w.y);
+                        v[8 * c + 3] = bf16hi(w.y);
+                        v[8 * c + 4] = bf16lo(w.z);
+                        v[8 * c + 5] = bf16hi(w.z);
+                        v[8 * c + 6] = bf16lo(w.w);
+                        v[8 * c + 7] = bf16hi(w.w);
+                    }
+            }
+        }
+        if (ROT) fwht128_pair(v, (threadIdx.x & 1) != 0);   // n % 128 == 0: pairs are whole
+        if (MODE == MODE_AMAX) {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) tmax = fmaxf(tmax, fabsf(v[i]));
+        } else if (n_valid > 0) {
+            const uint64_t e0 = p.e_base + static_cast<uint64_t>(off);
+            UnitOut o;
+            quant_unit<FMT, SR, FOUR6>(v, e0, s_t, p.seed, o);
+            store_unit<G>(o, p, e0, n_valid);
+        }
+    }
+    if (MODE == MODE_AMAX) {
+        tmax = block_max(tmax, red);
+        if (threadIdx.x == 0) p.partials_out[blockIdx.x] = tmax;
+    }
+}
+
+// ---------------------------------------------------------------- host launchers
+static int smem_configured[2][2][2][2][2] = {};
+
+template <int MODE, int FMT, bool ROT, bool SR, bool FOUR6>
+static int launch_tma(const CUtensorMap &tm, const QuantParams &p, int grid, cudaStream_t stream)
+{
+    auto kern = k_quant1d_tma<MODE, FMT, ROT, SR, FOUR6>;
+    int &done = smem_configured[MODE][FMT][ROT][SR][FOUR6];
+    if (!done) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, QT_SMEM_BYTES) != cudaSuccess)
+            return QFP4_ERR_CUDA;
+        done = 1;
+    }
+    kern<<<grid, QT_THREADS, QT_SMEM_BYTES, stream>>>(tm, p);
+    QFP4_LAUNCH_CHECK();
+    return QFP4_OK;
+}
+
+template <int MODE, int FMT, bool ROT, bool SR, bool FOUR6, typename T>
+static int launch_direct(const T *x, const QuantParams &p, int grid, cudaStream_t stream)
+{
+    k_quant1d_direct<MODE, FMT, ROT, SR, FOUR6, T><<<grid, 128, 0, stream>>>(x, p);
+    QFP4_LAUNCH_CHECK();
+    return QFP4_OK;
+}
+
+// One pass (amax or quantize) over x[0, n): the bf16 64-aligned body through
+// the TMA kernel, the rest through the direct kernel.  Partial maxima are
+// written to partials_out[0 ..) (amax pass); returns the number written.
+template <int MODE, int FMT, bool ROT, bool SR, bool FOUR6>
+static int run_pass(const void *x, qfp4_dtype xdt, int64_t n, QuantParams p, cudaStream_t stream, int *n_parts)
+{
+    const int nsm = num_sms();
+    int parts = 0;
+    int64_t body = 0;
+    const bool was_write = p.write_tscale;
+    if (xdt == QFP4_BF16) {
+        body = (n / 64) * 64;
+        if (body > 0) {
+            CUtensorMap tm;
+            const uint64_t dims[2] = {64, static_cast<uint64_t>(body / 64)};
+            const uint64_t strides[1] = {128};
+            const uint32_t box[2] = {64, QT_BOX_ROWS};
+            int st = encode_tensor_map(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x), dims, strides,
+                                       box, CU_TENSOR_MAP_SWIZZLE_128B);
+            if (st != QFP4_OK) return st;
+            const int64_t ntiles = (body / 64 + QT_TILE_ROWS - 1) / QT_TILE_ROWS;
+            const int grid = static_cast<int>(imin<int64_t>(ntiles, nsm));
+            QuantParams q = p;
+            q.n = body;
+            q.partials_out = p.partials_out;
+            st = launch_tma<MODE, FMT, ROT, SR, FOUR6>(tm, q, grid, stream);
+            if (st != QFP4_OK) return st;
+            parts += grid;
+            p.write_tscale = false;
+        }
+    }
+    const int64_t rest = n - body;
+    if (rest > 0) {
+        QuantParams q = p;
+        q.n = rest;
+        q.e_base = p.e_base + body;
+        q.write_tscale = body > 0 ? false : was_write;
+        q.partials_out = p.partials_out ? p.partials_out + parts : nullptr;
+        const int64_t units = (rest + 63) / 64;
+        const int grid = static_cast<int>(imin<int64_t>((units + 127) / 128, 4 * nsm));
+        int st;
+        if (xdt == QFP4_BF16)
+            st = launch_direct<MODE, FMT, ROT, SR, FOUR6>(static_cast<const uint16_t *>(x) + body, q, grid, stream);
+        else
+            st = launch_direct<MODE, FMT, ROT, SR, FOUR6>(static_cast<const float *>(x), q, grid, stream);
+        if (st != QFP4_OK) return st;
+        parts += grid;
+    }
+    if (n_parts) *n_parts = parts;
+    return QFP4_OK;
+}
+
+template <int FMT, bool ROT, bool SR, bool FOUR6>
+static int quantize1d_t(const void *x, qfp4_dtype xdt, int64_t n, uint64_t seed, uint8_t *codes, uint8_t *scales,
+                        float *tscale, float *partials, int *n_parts_out, cudaStream_t stream)
+{
+    QuantParams p{};
+    p.n = n;
+    p.e_base = 0;
+    p.codes = codes;
+    p.scales = scales;
+    p.seed = seed;
+    p.tscale_out = tscale;
+    p.write_tscale = true;
+    int n_parts = 0;
+    if (FMT == QFP4_NVFP4) {
+        p.partials_out = partials;
+        int st = run_pass<MODE_AMAX, FMT, ROT, false, false>(x, xdt, n, p, stream, &n_parts);
+        if (st != QFP4_OK) return st;
+        p.partials_out = nullptr;
+        p.partials = partials;
+        p.n_partials = n_parts;
+    }
+    if (n_parts_out) *n_parts_out = n_parts;
+    return run_pass<MODE_QUANT, FMT, ROT, SR, FOUR6>(x, xdt, n, p, stream, nullptr);
+}
+
+int quantize1d(const void *x, qfp4_dtype xdt, int64_t n, qfp4_fmt fmt, qfp4_round rounding, int rotate, int four6,
+               uint64_t seed, uint8_t *codes, uint8_t *scales, float *tscale, float *partials, int *n_parts_out,
+               cudaStream_t stream)
+{
+    const bool sr = rounding == QFP4_SR;
+    if (fmt == QFP4_MXFP4) {
+        if (rotate) return sr ? quantize1d_t<QFP4_MXFP4, true, true, false>(x, xdt, n, seed, codes, scales, tscale, partials, n_parts_out, stream)
+                              : quantize1d_t<QFP4_MXFP4, true, false, false>(x, xdt, n, seed, codes, scales, tscale, partials, n_parts_out, stream);
+        return sr ? quantize1d_t<QFP4_MXFP4, false, true, false>(x, xdt, n, seed, codes, scales, tscale, partials, n_parts_out, stream)
+                  : quantize1d_t<QFP4_MXFP4, false, false, false>(x, xdt, n, seed, codes, scales, tscale, partials, n_parts_out, stream);
+    }
+    if (four6) {
+        if (rotate) return quantize1d_t<QFP4_NVFP4, true, false, true>(x, xdt, n, seed, codes, scales, tscale, partials, n_parts_out, stream);
+        return quantize1d_t<QFP4_NVFP4, false, false, true>(x, xdt, n, seed, codes, scales, tscale, partials, n_parts_out, stream);
+    }
+    if (rotate) return sr ? quantize1d_t<QFP4_NVFP4, true, true, false>(x, xdt, n, seed, codes, scales, tscale, partials, n_parts_out, stream)
+                          : quantize1d_t<QFP4_NVFP4, true, false, false>(x, xdt, n, seed, codes, scales, tscale, partials, n_parts_out, stream);
+    return sr ? quantize1d_t<QFP4_NVFP4, false, true, false>(x, xdt, n, seed, codes, scales, tscale, partials, n_parts_out, stream)
+              : quantize1d_t<QFP4_NVFP4, false, false, false>(x, xdt, n, seed, codes, scales, tscale, partials, n_parts_out, stream);
+}
+
+}  // namespace qfp4

@@ -1,0 +1,29 @@
+// quantize1d.cuh -- interface between the 1D quantize kernels and the C ABI.
+#pragma once
+#include "qfp4_common.cuh"
+
+namespace qfp4 {
+
+enum { MODE_AMAX = 0, MODE_QUANT = 1 };
+
+// Upper bound on the number of partial tensor maxima a pass writes.
+constexpr int kMaxPartials = 1024;
+
+struct QuantParams {
+    int64_t n;                 // elements of this launch
+    uint64_t e_base;           // logical index of its first element
+    uint8_t *codes;            // whole-tensor outputs (indexed by logical element)
+    uint8_t *scales;
+    uint64_t seed;
+    const float *partials;     // NVFP4 quantize: partial maxima of the amax pass
+    int n_partials;
+    float *partials_out;       // amax pass: where this launch writes its partials
+    float *tscale_out;         // NVFP4: s_t output
+    bool write_tscale;         // this launch's block 0 writes *tscale_out
+};
+
+int quantize1d(const void *x, qfp4_dtype xdt, int64_t n, qfp4_fmt fmt, qfp4_round rounding, int rotate, int four6,
+               uint64_t seed, uint8_t *codes, uint8_t *scales, float *tscale, float *partials, int *n_parts_out,
+               cudaStream_t stream);
+
+}  // namespace qfp4

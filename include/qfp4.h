@@ -1,0 +1,215 @@
+/*
+ * qfp4.h -- C ABI of libqfp4: FP4 microscaling quantization of training
+ * tensors and the block-scaled FP4 matmul that consumes them, on NVIDIA
+ * B200 (sm_100a).
+ *
+ * Sources (the method; citations name the page and its section):
+ *   [QN] "Quartet -- Native 4-bit training that actually trains" (GPU-MODE
+ *        lecture 069 notes): Hadamard rotation y = xW = (xH)(H^T W); QuTLASS
+ *        fused rotation, online quantization, stochastic-rounding kernel,
+ *        MXFP4/NVFP4 GEMM with FP32 accumulate, FP4 forward / FP8 backward.
+ *   [LB] "low-bit quantization" blog (caveduck, series #4): §FP4 (E2M1 grid
+ *        +-{0,.5,1,1.5,2,3,4,6}, S = |W|max/6), §2 (group scales, MXFP4 = FP4
+ *        elements + one shared scale per 32), §3 (E8M0 2^k scale, effective
+ *        bits 4.25), §7 (Hadamard rotation, +-1/sqrt(n), O(n log n)).
+ *   [TI] "Stable FP4 Training via Transposition-Invariant Block
+ *        Quantization" (abstract): 2D blocks shared by X and X^T,
+ *        truncation-free scaling, stochastic rounding, MXFP8 for Q/K.
+ *   [46] "Four Over Six: More Accurate NVFP4 Quantization with Adaptive
+ *        Block Scaling" (summary, Methodology 1-3): per block, the better of
+ *        two candidate scales.
+ *
+ * General conventions
+ *   - Every pointer argument is DEVICE memory owned by the caller, unless a
+ *     parameter says otherwise.  The library allocates no device memory.
+ *   - Calls are asynchronous on `stream` (0 = legacy default stream).  The
+ *     returned status covers argument validation and kernel launch; it is
+ *     decided before anything is launched, so an error return leaves every
+ *     output untouched.
+ *   - Matrices are row-major.  X is M x K; element (i, j) has the logical
+ *     index e = i*K + j.
+ *   - FP4 (E2M1) codes: two per byte, element 2t in bits 0-3 and element
+ *     2t+1 in bits 4-7; bit 3 of a code is the sign.  A row of K elements
+ *     takes K/2 bytes.
+ *   - Scale bytes: one per group, row-major M x (K/g).  MXFP4 (g = 32): an
+ *     E8M0 byte, the scale is 2^(byte-127).  NVFP4 (g = 16): an OCP E4M3
+ *     byte, the scale is e4m3(byte) * s_t with s_t the per-tensor scale.
+ *   - All buffers need 16-byte aligned base pointers.
+ */
+#ifndef QFP4_H
+#define QFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *qfp4_stream_t;   /* == cudaStream_t */
+
+typedef enum { QFP4_MXFP4 = 0, QFP4_NVFP4 = 1 } qfp4_fmt;
+typedef enum { QFP4_RNE = 0, QFP4_SR = 1 } qfp4_round;
+typedef enum { QFP4_BF16 = 0, QFP4_F32 = 1 } qfp4_dtype;
+typedef enum {
+    QFP4_GRAN_TENSOR = 0, QFP4_GRAN_ROW = 1, QFP4_GRAN_GROUP16 = 2, QFP4_GRAN_GROUP32 = 3
+} qfp4_gran;
+
+enum {
+    QFP4_OK = 0,
+    QFP4_ERR_ARG = -1,          /* NULL where a buffer is required, bad enum, short workspace */
+    QFP4_ERR_SHAPE = -2,        /* dimensions violate the call's divisibility rules           */
+    QFP4_ERR_UNSUPPORTED = -3,  /* option combination not defined by the method              */
+    QFP4_ERR_ALIGN = -4,        /* a pointer is not 16-byte aligned                           */
+    QFP4_ERR_CUDA = -5,         /* a CUDA launch or driver call failed                        */
+    QFP4_ERR_TIMEOUT = -6       /* a bounded device-side wait gave up (see qfp4_last_device_error) */
+};
+
+/* ------------------------------------------------------------------------
+ * qfp4_quantize -- quantize X to FP4 with per-group scales.
+ *
+ * Per row block ([QN] Hadamard rotation and QuTLASS online quantization;
+ * [LB] §FP4, §2, §3, §7; [TI]; [46]):
+ *   (1) rotate != 0: each contiguous 128-element block along K is replaced
+ *       by its normalised Walsh-Hadamard transform (Sylvester order, stages
+ *       h = 1..64 of (a+b, a-b) in binary32, then one multiply by the
+ *       binary32 value of 1/sqrt(128)).  Needs K % 128 == 0.
+ *   (2) scales.  MXFP4: groups of 32 along K; the E8M0 exponent k is the
+ *       least integer with 6 * 2^k >= amax (truncation-free; k clamped to
+ *       [-127, 127]; an all-zero group gets byte 0 and +0 codes).  NVFP4:
+ *       s_t = amax_t / (6*448) in binary32 over the whole (rotated) tensor;
+ *       per 16-block enc = E4M3_RNE_satfinite((amax_b / 6) / s_t) and the
+ *       effective scale S = e4m3(enc) * s_t (binary32).
+ *   (3) four6 != 0 (NVFP4, RNE, 1D only): a second candidate scale from
+ *       amax_b / 4; each block keeps the candidate whose binary32 squared
+ *       error sum(deq - x)^2 (summed as pairs i,i+8; +4; +2; +1) is lower,
+ *       ties keeping amax/6.
+ *   (4) v = x / S in binary32, then round to E2M1: rounding = QFP4_RNE,
+ *       nearest grid value with ties to the even mantissa and saturation to
+ *       +-6; rounding = QFP4_SR, stochastic: with lo <= |v| < hi adjacent
+ *       grid values, up iff u < (|v|-lo)/(hi-lo), u = (w >> 8) * 2^-24 where
+ *       w is word (e mod 4) of Philox4x32-10 keyed (seed low 32, seed high
+ *       32) at counter (e/4 low 32, e/4 high 32, 0, 0).  The code's sign
+ *       bit is the sign of v.
+ *   (5) block2d != 0 (NVFP4 only, no rotation, no four6): 16x16 tiles share
+ *       one scale (amax over the tile), so X and X^T use the same scales.
+ *       scales[i][j/16] and scalesT[j][i/16] both hold tile (i/16, j/16);
+ *       codesT (K x M/2) is exactly the transpose of codes.  Needs M % 16
+ *       == 0 and K % 16 == 0.
+ *   In 1D mode a non-NULL codesT/scalesT asks for an independent
+ *   quantization of every column (groups of g along M; K x M/2 codes,
+ *   K x M/g scales), the baseline [TI] contrasts with 2D blocks; needs
+ *   M % g == 0 and rotate == 0.
+ *
+ * Arguments
+ *   x            M x K input, bf16 (xdt = QFP4_BF16) or binary32 (QFP4_F32).
+ *   codes        out, M*K/2 bytes.       scales   out, M*(K/g) bytes.
+ *   codesT       out or NULL, K*M/2.     scalesT  out or NULL, K*(M/g).
+ *   tscale       NVFP4: out, one float, the decode tensor scale s_t.
+ *                MXFP4: ignored (may be NULL).
+ *   workspace    NVFP4: device scratch of at least
+ *                qfp4_quantize_workspace_bytes() bytes (holds the partial
+ *                tensor maxima; contents on entry do not matter).  MXFP4:
+ *                may be NULL.
+ * Errors: QFP4_ERR_SHAPE for K % g != 0, K % 128 != 0 with rotate, M or K
+ *   not a multiple of 16 with block2d, M % g != 0 with a 1D codesT;
+ *   QFP4_ERR_UNSUPPORTED for four6 with MXFP4, SR or block2d, block2d with
+ *   MXFP4 or rotate, rotate with a 1D codesT.
+ * ---------------------------------------------------------------------- */
+size_t qfp4_quantize_workspace_bytes(int64_t M, int64_t K, qfp4_fmt fmt, int rotate, int block2d);
+
+int qfp4_quantize(const void *x, qfp4_dtype xdt, int64_t M, int64_t K,
+                  qfp4_fmt fmt, qfp4_round rounding, int rotate, int block2d, int four6,
+                  uint64_t seed,
+                  uint8_t *codes, uint8_t *scales,
+                  uint8_t *codesT, uint8_t *scalesT,
+                  float *tscale,
+                  void *workspace, size_t workspace_bytes,
+                  qfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * qfp4_quantize_mxfp8 -- MXFP8 variant ([TI]: MXFP8 for the sensitive Q/K
+ * projections; [QN]: FP8 backward): E4M3 elements in groups of 32 along K
+ * under an E8M0 scale with k the least integer such that 448 * 2^k >= amax.
+ * Elements: E4M3 round-to-nearest-even saturating to +-448, or the
+ * stochastic rule of qfp4_quantize on the E4M3 grid (same Philox words).
+ * codes M*K bytes, scales M*(K/32); codesT/scalesT (K*M and K*(M/32), or
+ * NULL) hold the column-wise quantization (groups of 32 along M).
+ * Needs K % 32 == 0 (and M % 32 == 0 with codesT).
+ * ---------------------------------------------------------------------- */
+int qfp4_quantize_mxfp8(const void *x, qfp4_dtype xdt, int64_t M, int64_t K,
+                        qfp4_round rounding, uint64_t seed,
+                        uint8_t *codes, uint8_t *scales,
+                        uint8_t *codesT, uint8_t *scalesT,
+                        qfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * qfp4_quantize_fp32scale -- the per-tensor / per-row / per-group FP32
+ * scale modes of [LB] §1-§2: S = amax / 6 in binary32 over the tensor, each
+ * row, or each group of 16 or 32 along K; v = x / S rounded to the nearest
+ * E2M1 value (ties to even, saturating); S == 0 gives +0 codes.
+ * scales: 1, M, M*K/16 or M*K/32 binary32 values.  Needs K % 2 == 0 and
+ * K % g == 0 for the group modes.  workspace: qfp4_quantize_workspace_bytes
+ * (M, K, QFP4_NVFP4, 0, 0) bytes for QFP4_GRAN_TENSOR, else may be NULL.
+ * ---------------------------------------------------------------------- */
+int qfp4_quantize_fp32scale(const void *x, qfp4_dtype xdt, int64_t M, int64_t K,
+                            qfp4_gran gran, uint8_t *codes, float *scales,
+                            void *workspace, size_t workspace_bytes,
+                            qfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * qfp4_dequantize -- out[i][j] = value(code) * scale (* s_t for NVFP4),
+ * formed exactly and rounded once to out_dt (nearest even).  tscale:
+ * NVFP4 device pointer to s_t, MXFP4 ignored.  Needs K % g == 0.
+ * ---------------------------------------------------------------------- */
+int qfp4_dequantize(const uint8_t *codes, const uint8_t *scales, const float *tscale,
+                    int64_t M, int64_t K, qfp4_fmt fmt, qfp4_dtype out_dt, void *out,
+                    qfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * qfp4_gemm_blockscaled -- Y = deq(A) * deq(B)^T ([QN] §QuTLASS: MXFP4 /
+ * NVFP4 operands, FP32 accumulation; [LB] §FP4: Blackwell FP4 tensor
+ * cores).  A is M x K and B is N x K, both K-major (codes + scales exactly
+ * as qfp4_quantize writes them); for NVFP4 the tensor scales multiply the
+ * accumulated sum: Y = acc * s_tA * s_tB (A_tscale, B_tscale device
+ * pointers; ignored for MXFP4).  out: M x N row-major, binary32 or bf16.
+ * Runs on 5th-generation tensor cores (tcgen05 block-scaled MMA, fp32
+ * accumulators in tensor memory).  Needs K % 256 == 0 (K may be padded
+ * with zero codes and zero scales), M >= 1, N >= 1 and N % 4 == 0.
+ * ---------------------------------------------------------------------- */
+int qfp4_gemm_blockscaled(const uint8_t *A_codes, const uint8_t *A_scales, const float *A_tscale,
+                          const uint8_t *B_codes, const uint8_t *B_scales, const float *B_tscale,
+                          int64_t M, int64_t N, int64_t K, qfp4_fmt fmt,
+                          qfp4_dtype out_dt, void *out, qfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * qfp4_gemm_fused_rq -- the same GEMM with A given in bf16: A is rotated
+ * (rotate != 0, along K in 128 blocks) and quantized (fmt, RNE, four6 as in
+ * qfp4_quantize) inside the call, then multiplied by the pre-quantized B
+ * ([QN] §QuTLASS: fused rotation and online quantization in the prologue;
+ * B is expected to be rotated the same way offline, so that
+ * (xH)(WH)^T = xW^T).  workspace: qfp4_gemm_fused_rq_workspace_bytes bytes
+ * of device scratch (quantized A and the partial maxima).
+ * ---------------------------------------------------------------------- */
+size_t qfp4_gemm_fused_rq_workspace_bytes(int64_t M, int64_t K, qfp4_fmt fmt);
+
+int qfp4_gemm_fused_rq(const void *A_bf16, int64_t M, int64_t K, int rotate, int four6, qfp4_fmt fmt,
+                       const uint8_t *B_codes, const uint8_t *B_scales, const float *B_tscale, int64_t N,
+                       void *workspace, size_t workspace_bytes,
+                       qfp4_dtype out_dt, void *out, qfp4_stream_t stream);
+
+/* Human-readable text of a status code (static storage). */
+const char *qfp4_status_string(int status);
+
+/* Sticky device-side error word of the current device: 0 when clean, else
+ * the code a bounded wait or a bounds check recorded (cleared by the read).
+ * Synchronizes the current device. */
+int qfp4_last_device_error(void);
+
+/* Library version, as MAJOR*10000 + MINOR*100 + PATCH. */
+int qfp4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QFP4_H */

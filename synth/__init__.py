@@ -83,6 +83,7 @@ def uniform(n: int, seed: int, stream: int = 0) -> np.ndarray:
 
 def permutation_prefix(n: int, k: int, seed: int, stream: int = 0) -> np.ndarray:
     """first k entries of a seeded Fisher-Yates shuffle of range(n)."""
+    k = min(k, n)
     a = np.arange(n, dtype=np.int64)
     w = _words(_key(seed, stream), 0, k)
     for t in range(k):
