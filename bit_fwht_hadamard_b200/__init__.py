@@ -27,7 +27,8 @@ OK, ERR_ARG, ERR_SHAPE, ERR_UNSUPPORTED, ERR_ALIGN, ERR_CUDA, ERR_TIMEOUT = 0, -
 
 EXPORTS = [
     "qfp4_quantize_workspace_bytes", "qfp4_quantize", "qfp4_quantize_mxfp8", "qfp4_quantize_fp32scale",
-    "qfp4_dequantize", "qfp4_gemm_blockscaled", "qfp4_gemm_fused_rq_workspace_bytes", "qfp4_gemm_fused_rq",
+    "qfp4_dequantize", "qfp4_gemm_workspace_bytes", "qfp4_gemm_blockscaled", "qfp4_gemm_fused_rq_workspace_bytes",
+    "qfp4_gemm_fused_rq",
     "qfp4_status_string", "qfp4_last_device_error", "qfp4_version",
 ]
 
@@ -60,10 +61,13 @@ def lib():
         L.qfp4_quantize_fp32scale.argtypes = [P, c_int, c_int64, c_int64, c_int, P, P, P, c_size_t, P]
         L.qfp4_dequantize.restype = c_int
         L.qfp4_dequantize.argtypes = [P, P, P, c_int64, c_int64, c_int, c_int, P, P]
+        L.qfp4_gemm_workspace_bytes.restype = c_size_t
+        L.qfp4_gemm_workspace_bytes.argtypes = [c_int64, c_int64, c_int64, c_int]
         L.qfp4_gemm_blockscaled.restype = c_int
-        L.qfp4_gemm_blockscaled.argtypes = [P, P, P, P, P, P, c_int64, c_int64, c_int64, c_int, c_int, P, P]
+        L.qfp4_gemm_blockscaled.argtypes = [P, P, P, P, P, P, c_int64, c_int64, c_int64, c_int, c_int, P, P,
+                                            c_size_t, P]
         L.qfp4_gemm_fused_rq_workspace_bytes.restype = c_size_t
-        L.qfp4_gemm_fused_rq_workspace_bytes.argtypes = [c_int64, c_int64, c_int]
+        L.qfp4_gemm_fused_rq_workspace_bytes.argtypes = [c_int64, c_int64, c_int64, c_int]
         L.qfp4_gemm_fused_rq.restype = c_int
         L.qfp4_gemm_fused_rq.argtypes = [P, c_int64, c_int64, c_int, c_int, c_int, P, P, P, c_int64, P, c_size_t,
                                          c_int, P, P]
@@ -105,14 +109,18 @@ def qfp4_dequantize(codes, scales, tscale, M, K, fmt, out_dt, out, stream):
     return lib().qfp4_dequantize(codes, scales, tscale, M, K, fmt, out_dt, out, stream)
 
 
+def qfp4_gemm_workspace_bytes(M, N, K, fmt):
+    return lib().qfp4_gemm_workspace_bytes(M, N, K, fmt)
+
+
 def qfp4_gemm_blockscaled(A_codes, A_scales, A_tscale, B_codes, B_scales, B_tscale, M, N, K, fmt, out_dt, out,
-                          stream):
+                          workspace, workspace_bytes, stream):
     return lib().qfp4_gemm_blockscaled(A_codes, A_scales, A_tscale, B_codes, B_scales, B_tscale, M, N, K, fmt,
-                                       out_dt, out, stream)
+                                       out_dt, out, workspace, workspace_bytes, stream)
 
 
-def qfp4_gemm_fused_rq_workspace_bytes(M, K, fmt):
-    return lib().qfp4_gemm_fused_rq_workspace_bytes(M, K, fmt)
+def qfp4_gemm_fused_rq_workspace_bytes(M, N, K, fmt):
+    return lib().qfp4_gemm_fused_rq_workspace_bytes(M, N, K, fmt)
 
 
 def qfp4_gemm_fused_rq(A_bf16, M, K, rotate, four6, fmt, B_codes, B_scales, B_tscale, N, workspace,
@@ -232,15 +240,19 @@ def dequantize(q, M, K, fmt, out_dtype=None, stream=None):
     return out
 
 
-def gemm(A, B, M, N, K, fmt, out_dtype=None, out=None, stream=None):
+def gemm(A, B, M, N, K, fmt, out_dtype=None, out=None, workspace=None, stream=None):
     """Y = deq(A) deq(B)^T for operands as returned by ``quantize``."""
     torch = _torch()
     out_dtype = torch.float32 if out_dtype is None else out_dtype
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=A["codes"].device)
+    wsb = qfp4_gemm_workspace_bytes(M, N, K, fmt)
+    if workspace is None:
+        workspace = torch.empty(max(wsb, 16), dtype=torch.uint8, device=A["codes"].device)
     st = qfp4_gemm_blockscaled(_ptr(A["codes"]), _ptr(A["scales"]), _ptr(A.get("tscale")), _ptr(B["codes"]),
                                _ptr(B["scales"]), _ptr(B.get("tscale")), M, N, K, fmt,
-                               F32 if out.dtype == torch.float32 else BF16, _ptr(out), _stream(stream))
+                               F32 if out.dtype == torch.float32 else BF16, _ptr(out), _ptr(workspace), wsb,
+                               _stream(stream))
     _check(st, "qfp4_gemm_blockscaled")
     return out
 
@@ -253,7 +265,7 @@ def gemm_fused_rq(A_bf16, B, N, fmt=NVFP4, rotate=True, four6=False, out_dtype=N
     out_dtype = torch.float32 if out_dtype is None else out_dtype
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=A_bf16.device)
-    wsb = qfp4_gemm_fused_rq_workspace_bytes(M, K, fmt)
+    wsb = qfp4_gemm_fused_rq_workspace_bytes(M, N, K, fmt)
     if workspace is None:
         workspace = torch.empty(max(wsb, 16), dtype=torch.uint8, device=A_bf16.device)
     st = qfp4_gemm_fused_rq(_ptr(A_bf16), M, K, int(rotate), int(four6), fmt, _ptr(B["codes"]), _ptr(B["scales"]),

@@ -18,11 +18,12 @@ int quantize_mxfp8(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_rou
                    uint8_t *codes, uint8_t *scales, uint8_t *codesT, uint8_t *scalesT, cudaStream_t stream);
 int gemm_blockscaled(const uint8_t *A_codes, const uint8_t *A_scales, const float *A_tscale, const uint8_t *B_codes,
                      const uint8_t *B_scales, const float *B_tscale, int64_t M, int64_t N, int64_t K, qfp4_fmt fmt,
-                     qfp4_dtype out_dt, void *out, cudaStream_t stream);
+                     qfp4_dtype out_dt, void *out, void *workspace, cudaStream_t stream);
+size_t gemm_workspace(int64_t M, int64_t N, int64_t K, qfp4_fmt fmt);
 int gemm_fused_rq(const void *A_bf16, int64_t M, int64_t K, int rotate, int four6, qfp4_fmt fmt,
                   const uint8_t *B_codes, const uint8_t *B_scales, const float *B_tscale, int64_t N, void *workspace,
                   qfp4_dtype out_dt, void *out, cudaStream_t stream);
-size_t gemm_fused_rq_workspace(int64_t M, int64_t K, qfp4_fmt fmt);
+size_t gemm_fused_rq_workspace(int64_t M, int64_t N, int64_t K, qfp4_fmt fmt);
 }  // namespace qfp4
 
 using namespace qfp4;
@@ -127,27 +128,46 @@ extern "C" int qfp4_dequantize(const uint8_t *codes, const uint8_t *scales, cons
     return dequantize(codes, scales, tscale, M * K, fmt, out_dt, out, reinterpret_cast<cudaStream_t>(stream));
 }
 
+extern "C" size_t qfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, qfp4_fmt fmt)
+{
+    return gemm_workspace(M, N, K, fmt);
+}
+
+// shape rules shared by both GEMM entry points
+static int gemm_shape_check(int64_t M, int64_t N, int64_t K, qfp4_dtype out_dt)
+{
+    if (M < 0 || N < 0 || K < 0) return QFP4_ERR_SHAPE;
+    if (K % 32) return QFP4_ERR_SHAPE;
+    if (N % (out_dt == QFP4_F32 ? 4 : 8)) return QFP4_ERR_SHAPE;
+    if (M > INT32_MAX / 2 || N > INT32_MAX / 2 || K > INT32_MAX / 2) return QFP4_ERR_SHAPE;
+    return QFP4_OK;
+}
+
 extern "C" int qfp4_gemm_blockscaled(const uint8_t *A_codes, const uint8_t *A_scales, const float *A_tscale,
                                      const uint8_t *B_codes, const uint8_t *B_scales, const float *B_tscale,
                                      int64_t M, int64_t N, int64_t K, qfp4_fmt fmt, qfp4_dtype out_dt, void *out,
-                                     qfp4_stream_t stream)
+                                     void *workspace, size_t workspace_bytes, qfp4_stream_t stream)
 {
-    if (M < 0 || N < 0 || K < 0) return QFP4_ERR_SHAPE;
     if (fmt != QFP4_MXFP4 && fmt != QFP4_NVFP4) return QFP4_ERR_ARG;
     if (out_dt != QFP4_BF16 && out_dt != QFP4_F32) return QFP4_ERR_ARG;
+    int st = gemm_shape_check(M, N, K, out_dt);
+    if (st != QFP4_OK) return st;
     if (M * N > 0 && (!A_codes || !A_scales || !B_codes || !B_scales || !out)) return QFP4_ERR_ARG;
-    if (fmt == QFP4_NVFP4 && (!A_tscale || !B_tscale)) return QFP4_ERR_ARG;
-    if (K % 32) return QFP4_ERR_SHAPE;
-    if (!ok_align(A_codes) || !ok_align(A_scales) || !ok_align(B_codes) || !ok_align(B_scales) || !ok_align(out))
+    if (fmt == QFP4_NVFP4 && M * N > 0 && (!A_tscale || !B_tscale)) return QFP4_ERR_ARG;
+    if (!ok_align(A_codes) || !ok_align(A_scales) || !ok_align(B_codes) || !ok_align(B_scales) || !ok_align(out) ||
+        !ok_align(workspace))
         return QFP4_ERR_ALIGN;
     if (M * N == 0) return QFP4_OK;
+    if (K == 0) return cudaMemsetAsync(out, 0, M * N * (out_dt == QFP4_F32 ? 4 : 2),
+                                       reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? QFP4_OK : QFP4_ERR_CUDA;
+    if (!workspace || workspace_bytes < gemm_workspace(M, N, K, fmt)) return QFP4_ERR_ARG;
     return gemm_blockscaled(A_codes, A_scales, A_tscale, B_codes, B_scales, B_tscale, M, N, K, fmt, out_dt, out,
-                            reinterpret_cast<cudaStream_t>(stream));
+                            workspace, reinterpret_cast<cudaStream_t>(stream));
 }
 
-extern "C" size_t qfp4_gemm_fused_rq_workspace_bytes(int64_t M, int64_t K, qfp4_fmt fmt)
+extern "C" size_t qfp4_gemm_fused_rq_workspace_bytes(int64_t M, int64_t N, int64_t K, qfp4_fmt fmt)
 {
-    return gemm_fused_rq_workspace(M, K, fmt);
+    return gemm_fused_rq_workspace(M, N, K, fmt);
 }
 
 extern "C" int qfp4_gemm_fused_rq(const void *A_bf16, int64_t M, int64_t K, int rotate, int four6, qfp4_fmt fmt,
@@ -155,18 +175,20 @@ extern "C" int qfp4_gemm_fused_rq(const void *A_bf16, int64_t M, int64_t K, int 
                                   void *workspace, size_t workspace_bytes, qfp4_dtype out_dt, void *out,
                                   qfp4_stream_t stream)
 {
-    if (M < 0 || N < 0 || K < 0) return QFP4_ERR_SHAPE;
     if (fmt != QFP4_MXFP4 && fmt != QFP4_NVFP4) return QFP4_ERR_ARG;
     if (out_dt != QFP4_BF16 && out_dt != QFP4_F32) return QFP4_ERR_ARG;
+    int st = gemm_shape_check(M, N, K, out_dt);
+    if (st != QFP4_OK) return st;
     if (M * N > 0 && (!A_bf16 || !B_codes || !B_scales || !out)) return QFP4_ERR_ARG;
-    if (fmt == QFP4_NVFP4 && !B_tscale) return QFP4_ERR_ARG;
+    if (fmt == QFP4_NVFP4 && M * N > 0 && !B_tscale) return QFP4_ERR_ARG;
     if (four6 && fmt != QFP4_NVFP4) return QFP4_ERR_UNSUPPORTED;
-    if (K % 32) return QFP4_ERR_SHAPE;
     if (rotate && K % 128) return QFP4_ERR_SHAPE;
     if (!ok_align(A_bf16) || !ok_align(B_codes) || !ok_align(B_scales) || !ok_align(out) || !ok_align(workspace))
         return QFP4_ERR_ALIGN;
     if (M * N == 0) return QFP4_OK;
-    if (!workspace || workspace_bytes < gemm_fused_rq_workspace(M, K, fmt)) return QFP4_ERR_ARG;
+    if (K == 0) return cudaMemsetAsync(out, 0, M * N * (out_dt == QFP4_F32 ? 4 : 2),
+                                       reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? QFP4_OK : QFP4_ERR_CUDA;
+    if (!workspace || workspace_bytes < gemm_fused_rq_workspace(M, N, K, fmt)) return QFP4_ERR_ARG;
     return gemm_fused_rq(A_bf16, M, K, rotate, four6, fmt, B_codes, B_scales, B_tscale, N, workspace, out_dt, out,
                          reinterpret_cast<cudaStream_t>(stream));
 }

@@ -3,5 +3,6 @@
 #include "runtime.cu"
 #include "quantize1d.cu"
 #include "dequant_fp32scale.cu"
+#include "gemm.cu"
 #include "pending.cu"
 #include "api.cu"

@@ -17,15 +17,4 @@ int quantize_mxfp8(const void *, qfp4_dtype, int64_t, int64_t, qfp4_round, uint6
 {
     return QFP4_ERR_UNSUPPORTED;
 }
-int gemm_blockscaled(const uint8_t *, const uint8_t *, const float *, const uint8_t *, const uint8_t *, const float *,
-                     int64_t, int64_t, int64_t, qfp4_fmt, qfp4_dtype, void *, cudaStream_t)
-{
-    return QFP4_ERR_UNSUPPORTED;
-}
-int gemm_fused_rq(const void *, int64_t, int64_t, int, int, qfp4_fmt, const uint8_t *, const uint8_t *, const float *,
-                  int64_t, void *, qfp4_dtype, void *, cudaStream_t)
-{
-    return QFP4_ERR_UNSUPPORTED;
-}
-size_t gemm_fused_rq_workspace(int64_t, int64_t, qfp4_fmt) { return 0; }
 }  // namespace qfp4

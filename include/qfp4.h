@@ -171,27 +171,38 @@ int qfp4_dequantize(const uint8_t *codes, const uint8_t *scales, const float *ts
  * NVFP4 operands, FP32 accumulation; [LB] §FP4: Blackwell FP4 tensor
  * cores).  A is M x K and B is N x K, both K-major (codes + scales exactly
  * as qfp4_quantize writes them); for NVFP4 the tensor scales multiply the
- * accumulated sum: Y = acc * s_tA * s_tB (A_tscale, B_tscale device
- * pointers; ignored for MXFP4).  out: M x N row-major, binary32 or bf16.
- * Runs on 5th-generation tensor cores (tcgen05 block-scaled MMA, fp32
- * accumulators in tensor memory).  Needs K % 256 == 0 (K may be padded
- * with zero codes and zero scales), M >= 1, N >= 1 and N % 4 == 0.
+ * accumulated sum: Y = acc * (s_tA * s_tB) (A_tscale, B_tscale device
+ * pointers; ignored for MXFP4).  out: M x N row-major, binary32 or bf16
+ * (round to nearest even).  Runs on 5th-generation tensor cores (tcgen05
+ * block-scaled MMA, fp32 accumulators in tensor memory).
+ * workspace: device scratch of at least qfp4_gemm_workspace_bytes(M, N, K,
+ *   fmt) bytes; it receives the scales rearranged for the tensor cores
+ *   (contents on entry do not matter, the call overwrites them).
+ * Needs K % 32 == 0 (a K tail short of the 256-element tile is zero-filled),
+ * N % 4 == 0 (binary32 out) or N % 8 == 0 (bf16 out), M, N, K < 2^30.
  * ---------------------------------------------------------------------- */
+size_t qfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, qfp4_fmt fmt);
+
 int qfp4_gemm_blockscaled(const uint8_t *A_codes, const uint8_t *A_scales, const float *A_tscale,
                           const uint8_t *B_codes, const uint8_t *B_scales, const float *B_tscale,
                           int64_t M, int64_t N, int64_t K, qfp4_fmt fmt,
-                          qfp4_dtype out_dt, void *out, qfp4_stream_t stream);
+                          qfp4_dtype out_dt, void *out,
+                          void *workspace, size_t workspace_bytes,
+                          qfp4_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * qfp4_gemm_fused_rq -- the same GEMM with A given in bf16: A is rotated
  * (rotate != 0, along K in 128 blocks) and quantized (fmt, RNE, four6 as in
  * qfp4_quantize) inside the call, then multiplied by the pre-quantized B
- * ([QN] §QuTLASS: fused rotation and online quantization in the prologue;
+ * ([QN] §QuTLASS: fused rotation and online quantization before the GEMM;
  * B is expected to be rotated the same way offline, so that
- * (xH)(WH)^T = xW^T).  workspace: qfp4_gemm_fused_rq_workspace_bytes bytes
- * of device scratch (quantized A and the partial maxima).
+ * (xH)(WH)^T = xW^T).  A is quantized once into the workspace (not once
+ * per output tile), then consumed by the tensor-core kernel.
+ * workspace: at least qfp4_gemm_fused_rq_workspace_bytes(M, N, K, fmt)
+ * bytes of device scratch.  Same shape rules as qfp4_gemm_blockscaled,
+ * plus K % 128 == 0 with rotate.
  * ---------------------------------------------------------------------- */
-size_t qfp4_gemm_fused_rq_workspace_bytes(int64_t M, int64_t K, qfp4_fmt fmt);
+size_t qfp4_gemm_fused_rq_workspace_bytes(int64_t M, int64_t N, int64_t K, qfp4_fmt fmt);
 
 int qfp4_gemm_fused_rq(const void *A_bf16, int64_t M, int64_t K, int rotate, int four6, qfp4_fmt fmt,
                        const uint8_t *B_codes, const uint8_t *B_scales, const float *B_tscale, int64_t N,

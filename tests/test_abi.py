@@ -44,5 +44,11 @@ def test_argument_errors_return_before_any_launch():
     assert st == q.ERR_ALIGN
     st = q.qfp4_quantize(fake, q.BF16, 4, 64, q.NVFP4, q.RNE, 0, 0, 0, 0, fake, fake, None, None, fake, None, 0, None)
     assert st == q.ERR_ARG                                  # NVFP4 without workspace
-    st = q.qfp4_gemm_blockscaled(fake, fake, None, fake, fake, None, 64, 64, 48, q.MXFP4, q.F32, fake, None)
+    st = q.qfp4_gemm_blockscaled(fake, fake, None, fake, fake, None, 64, 64, 48, q.MXFP4, q.F32, fake, fake, 1 << 20,
+                                 None)
     assert st == q.ERR_SHAPE
+    st = q.qfp4_gemm_blockscaled(fake, fake, None, fake, fake, None, 64, 66, 64, q.MXFP4, q.F32, fake, fake, 1 << 20,
+                                 None)
+    assert st == q.ERR_SHAPE                                # N % 4
+    st = q.qfp4_gemm_blockscaled(fake, fake, None, fake, fake, None, 64, 64, 64, q.MXFP4, q.F32, fake, fake, 16, None)
+    assert st == q.ERR_ARG                                  # workspace too small
