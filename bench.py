@@ -1,0 +1,416 @@
+#!/usr/bin/env python3
+"""Benchmark of the FP4 microscaling hot path on B200.
+
+Default workload (one GPU): activation quantize + rotate -- X bf16 4096 x 4096,
+entries N(0,1) with 40 seeded channels x20; each step runs FWHT-128 + MXFP4
+(group 32, truncation-free E8M0) once with round-to-nearest-even and once
+with Philox stochastic rounding (seed 7).  value = algorithmic bytes moved
+(one read of X plus codes and scales, 2.531 B/element per run) / step time.
+
+Also reported: the roofline of the dominant kernel (live CUDA-event
+durations, measured HBM peak), the block-scaled FP4 GEMM of the NVFP4
+forward linear (8192 x 11008 x 4096) in TFLOP/s against the dense FP4 peak,
+the end-to-end figure through host buffers, SM clocks sampled during the
+timed region, and the CPU oracle on the host cores.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+Under torchrun (N > 1) every rank runs the same per-GPU workload (weak
+scaling, no data-path collective); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "FP4 quantize GB/s (% of HBM peak); block-scaled FP4 GEMM TFLOPS (% of peak)"
+M2, K2 = 4096, 4096
+BYTES_PER_ELEM_MXFP4 = 2 + 0.5 + 1 / 32           # bf16 read + E2M1 codes + E8M0 scales
+N_BUFS = 8                                         # rotating input/output sets: 8 x 40.5 MB > L2 (126 MB)
+FP4_PER_BF16 = 4.0                                 # nominal dense FP4 : BF16 tensor throughput (9 : 2.25 PF)
+GEMM_SHAPE = (8192, 11008, 4096)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="libqfp4", choices=["libqfp4", "reference"])
+    ap.add_argument("--no-gemm", action="store_true", help="skip the GEMM sub-measurement")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--profile-case", choices=["quant", "gemm", "quant-nvfp4"], default=None,
+                    help="run a few untimed calls of one kernel family (for ncu captures) and exit")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained"), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def csrc_hash():
+    h = hashlib.sha1()
+    d = os.path.join(ROOT, "bit_fwht_hadamard_b200", "csrc")
+    for n in sorted(os.listdir(d)):
+        with open(os.path.join(d, n), "rb") as f:
+            h.update(n.encode() + f.read())
+    return h.hexdigest()[:12]
+
+
+def ncu_traffic(key):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    cur = csrc_hash()
+    with open(p) as f:
+        for line in f:
+            t = line.split()
+            if len(t) >= 3 and not line.startswith("#") and t[0] == key and t[2] == cur:
+                return float(t[1])
+    return None
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = [r for r in csv.reader(io.StringIO(self.out or "")) if len(r) >= 9]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[1]) for r in rows]
+        mx = max(float(r[2]) for r in rows)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(float(r[3]) for r in rows if r[3].strip() not in ("", "[N/A]"))}
+
+
+# ------------------------------------------------------------------ reference arm (CPU oracle)
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    import oracle
+    import synth
+    rows = 512                                           # bounded sample: 512 of the 4096 rows per step
+    x = synth.cfg2_X()[:rows].copy()
+    n = rows * K2
+    for _ in range(args.warmup):
+        oracle.quantize(x, oracle.MXFP4, oracle.RNE, rotate=True)
+        oracle.quantize(x, oracle.MXFP4, oracle.SR, rotate=True, seed=7)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.quantize(x, oracle.MXFP4, oracle.RNE, rotate=True)
+        oracle.quantize(x, oracle.MXFP4, oracle.SR, rotate=True, seed=7)
+    dt = (time.perf_counter() - t0) / max(args.steps, 1)
+    gbs = 2 * n * BYTES_PER_ELEM_MXFP4 / dt / 1e9
+    sample = f"rows 0..{rows - 1} of X (4096 x 4096 bf16), RNE + SR per step, single-threaded C oracle"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": workload_config(),
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+
+
+def workload_config():
+    return {"workload": "activation quantize + rotate: X bf16 4096x4096 N(0,1), 40 seeded channels x20; "
+                        "FWHT-128 then MXFP4 g32 truncation-free E8M0; one RNE run + one Philox SR run (seed 7)",
+            "global_batch": 1, "shape": [M2, K2], "parallelism": "replicas (weak scaling)",
+            "l2": f"{N_BUFS} rotating input/output sets (> L2)"}
+
+
+# ------------------------------------------------------------------ CPU baseline (oracle on the host)
+def cpu_baseline():
+    import oracle
+    import synth
+    x = synth.cfg2_X()
+    t0 = time.perf_counter()
+    oracle.quantize(x, oracle.MXFP4, oracle.RNE, rotate=True)
+    oracle.quantize(x, oracle.MXFP4, oracle.SR, rotate=True, seed=7)
+    dt = time.perf_counter() - t0
+    return {"value": 2 * x.size * BYTES_PER_ELEM_MXFP4 / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": "one full step (X 4096x4096, RNE + SR), single-threaded C oracle", "seconds": dt}
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_gpu(args, rank, world):
+    import torch
+
+    import bit_fwht_hadamard_b200 as q
+    import synth
+    from bit_fwht_hadamard_b200 import build as _build
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if int(os.environ.get("LOCAL_RANK", "0")) == 0:
+        _build.build()                                   # no-op when libqfp4.so is newer than its sources
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    hbm_peak, bf16_peak, bf16_sust, peak_src = measured_peaks()
+    x_host = synth.cfg2_X()
+    x0 = torch.from_numpy(x_host.view(np.int16)).view(torch.bfloat16)
+    xs = [x0.to(dev)]
+    for i in range(1, N_BUFS):
+        xs.append(xs[0].clone())                          # distinct buffers (same values)
+    outs = [[q.quantize(xs[0], q.MXFP4, q.RNE, rotate=True), q.quantize(xs[0], q.MXFP4, q.SR, rotate=True, seed=7)]
+            for _ in range(N_BUFS)]
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+    L = q.lib()
+    # pre-marshalled C-ABI arguments: the timed loop is two ctypes calls per step
+    args_rne = [(xs[b].data_ptr(), q.BF16, M2, K2, q.MXFP4, q.RNE, 1, 0, 0, 0, outs[b][0]["codes"].data_ptr(),
+                 outs[b][0]["scales"].data_ptr(), None, None, None, None, 0, sh) for b in range(N_BUFS)]
+    args_sr = [(xs[b].data_ptr(), q.BF16, M2, K2, q.MXFP4, q.SR, 1, 0, 0, 7, outs[b][1]["codes"].data_ptr(),
+                outs[b][1]["scales"].data_ptr(), None, None, None, None, 0, sh) for b in range(N_BUFS)]
+    status = []
+
+    def step(i, ev=None):
+        b = i % N_BUFS
+        if ev is not None:
+            ev[0].record(stream)
+        status.append(L.qfp4_quantize(*args_rne[b]))
+        if ev is not None:
+            ev[1].record(stream)
+        status.append(L.qfp4_quantize(*args_sr[b]))
+        if ev is not None:
+            ev[2].record(stream)
+
+    for i in range(max(args.warmup, 3)):
+        step(i)
+    torch.cuda.synchronize()
+
+    # ---- device-resident timed region (per-launch events inside it)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        soak_until = time.perf_counter() + 1.0           # load the GPU before the region so clocks are seen
+        i = 0
+        while time.perf_counter() < soak_until:
+            step(i)
+            i += 1
+            if i % 64 == 0:
+                torch.cuda.synchronize()
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        n_launch0 = q.qfp4_launch_count()
+        # a spin kernel ahead of the start event lets the host enqueue the whole
+        # region before the device reaches it, so host overhead leaves no gaps
+        torch.cuda._sleep(int(2e9 * min(0.5, 40e-6 * args.steps + 2e-3)))
+        start.record(stream)
+        for i in range(args.steps):
+            step(i, evs[i])
+        stop.record(stream)
+        torch.cuda.synchronize()
+        n_launch = q.qfp4_launch_count() - n_launch0
+        barrier()
+    if any(st != q.OK for st in status):
+        raise RuntimeError(f"qfp4_quantize failed: {set(status)}")
+    elapsed_ms = start.elapsed_time(stop)
+    if dist is not None:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    ms_per_step = elapsed_ms / args.steps
+    n = M2 * K2
+    step_bytes = 2 * n * BYTES_PER_ELEM_MXFP4
+    value = world * step_bytes / (ms_per_step * 1e-3) / 1e9
+
+    rne_ms = statistics.mean(evs[i][0].elapsed_time(evs[i][1]) for i in range(args.steps))
+    sr_ms = statistics.mean(evs[i][1].elapsed_time(evs[i][2]) for i in range(args.steps))
+    dom_name, dom_ms = ("quant1d_mxfp4_rot_sr", sr_ms) if sr_ms >= rne_ms else ("quant1d_mxfp4_rot_rne", rne_ms)
+    launch_bytes = n * BYTES_PER_ELEM_MXFP4
+    achieved = launch_bytes / (dom_ms * 1e-3) / 1e9
+    traffic = ncu_traffic(dom_name)
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
+                "traffic": traffic, "kernel": dom_name, "peak_source": f"{peak_src} hbm_gbs",
+                "algorithmic_bytes_per_launch": launch_bytes,
+                "launches": {"quant1d_mxfp4_rot_rne_ms": rne_ms, "quant1d_mxfp4_rot_sr_ms": sr_ms,
+                             "rne_gbs": launch_bytes / (rne_ms * 1e-3) / 1e9,
+                             "sr_gbs": launch_bytes / (sr_ms * 1e-3) / 1e9}}
+
+    # ---- end to end through host buffers (pinned), same metric
+    x_pin = x0.pin_memory()
+    xd = torch.empty_like(xs[0])
+    h_out = [{k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in o.items()} for o in outs[0]]
+    e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(3, min(args.steps, 50))
+    for it in range(e2e_steps + 2):
+        if it == 2:
+            torch.cuda.synchronize()
+            barrier()
+            e_start.record(stream)
+        xd.copy_(x_pin, non_blocking=True)
+        q.quantize(xd, q.MXFP4, q.RNE, rotate=True, out=outs[0][0])
+        q.quantize(xd, q.MXFP4, q.SR, rotate=True, seed=7, out=outs[0][1])
+        for k in ("codes", "scales"):
+            h_out[0][k].copy_(outs[0][0][k], non_blocking=True)
+            h_out[1][k].copy_(outs[0][1][k], non_blocking=True)
+    e_stop.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e_start.elapsed_time(e_stop) / e2e_steps
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = x0.numel() * 2
+    d2h = sum(v.numel() for o in outs[0] for k, v in o.items() if k in ("codes", "scales"))
+    e2e = {"value": world * step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    # ---- GEMM of the NVFP4 forward linear (tensor-core roofline)
+    gemm = None
+    if not args.no_gemm:
+        gemm = bench_gemm(q, synth, dev, stream, bf16_peak, peak_src, max(3, min(args.steps, 20)))
+
+    result = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": workload_config(),
+        "roofline": roofline, "e2e": e2e, "gpu_launches": int(n_launch), "clocks": clk.summary(),
+        "frac_of_hbm_peak": value / world / hbm_peak,
+    }
+    if gemm is not None:
+        result["gemm"] = gemm
+    if rank == 0 and world == 1 and not args.no_cpu:
+        result["cpu_baseline"] = cpu_baseline()
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result))
+
+
+def bench_gemm(q, synth, dev, stream, bf16_peak, peak_src, iters):
+    import torch
+    M, N, K = GEMM_SHAPE
+    x = torch.from_numpy(synth.cfg3_X().view(np.int16)).view(torch.bfloat16).to(dev)
+    w = torch.from_numpy(synth.cfg3_W().view(np.int16)).view(torch.bfloat16).to(dev)
+    X = q.quantize(x, q.NVFP4, four6=True)
+    W = q.quantize(w, q.NVFP4, four6=True)
+    out = torch.empty((M, N), dtype=torch.float32, device=dev)
+    ws = torch.empty(q.qfp4_gemm_workspace_bytes(M, N, K, q.NVFP4), dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        q.gemm(X, W, M, N, K, q.NVFP4, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+    for a, b in evs:
+        a.record(stream)
+        q.gemm(X, W, M, N, K, q.NVFP4, out=out, workspace=ws)
+        b.record(stream)
+    torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    tflops = 2.0 * M * N * K / (ms * 1e-3) / 1e12
+    peak = bf16_peak * FP4_PER_BF16
+    return {"workload": "NVFP4 forward linear GEMM Y = X W^T, 8192 x 11008 x 4096, four-over-six operands, fp32 out",
+            "value": tflops, "unit": "TFLOP/s", "ms_per_call": ms,
+            "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+                         "frac": tflops / peak, "traffic": ncu_traffic("gemm_nvfp4_f32"),
+                         "kernel": "gemm_nvfp4_f32 (scale rearrange prepass + tcgen05 main loop)",
+                         "peak_source": f"{peak_src} bf16_tflops x {FP4_PER_BF16} (nominal FP4:BF16 dense ratio)"}}
+
+
+def run_profile_case(case):
+    """Two warm-up and two measured calls of one kernel family, nothing timed:
+    the small cases that ncu captures (inputs of the benchmark's own sizes)."""
+    import torch
+
+    import bit_fwht_hadamard_b200 as q
+    import synth
+    from bit_fwht_hadamard_b200 import build as _build
+    _build.build()
+    dev = torch.device("cuda:0")
+    if case == "quant":
+        x = torch.from_numpy(synth.cfg2_X().view(np.int16)).view(torch.bfloat16).to(dev)
+        for _ in range(2):
+            q.quantize(x, q.MXFP4, q.RNE, rotate=True)
+            q.quantize(x, q.MXFP4, q.SR, rotate=True, seed=7)
+    elif case == "quant-nvfp4":
+        x = torch.from_numpy(synth.cfg3_X().view(np.int16)).view(torch.bfloat16).to(dev)
+        for _ in range(2):
+            q.quantize(x, q.NVFP4, q.RNE, four6=True)
+    else:
+        M, N, K = GEMM_SHAPE
+        X = q.quantize(torch.from_numpy(synth.cfg3_X().view(np.int16)).view(torch.bfloat16).to(dev), q.NVFP4,
+                       four6=True)
+        W = q.quantize(torch.from_numpy(synth.cfg3_W().view(np.int16)).view(torch.bfloat16).to(dev), q.NVFP4,
+                       four6=True)
+        out = torch.empty((M, N), dtype=torch.float32, device=dev)
+        for _ in range(2):
+            q.gemm(X, W, M, N, K, q.NVFP4, out=out)
+    torch.cuda.synchronize()
+    print(f"profile case {case}: ok")
+
+
+def main():
+    args = parse()
+    if args.profile_case:
+        run_profile_case(args.profile_case)
+        return
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    run_gpu(args, rank, world)
+
+
+if __name__ == "__main__":
+    main()

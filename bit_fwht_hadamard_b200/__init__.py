@@ -29,7 +29,7 @@ EXPORTS = [
     "qfp4_quantize_workspace_bytes", "qfp4_quantize", "qfp4_quantize_mxfp8", "qfp4_quantize_fp32scale",
     "qfp4_dequantize", "qfp4_gemm_workspace_bytes", "qfp4_gemm_blockscaled", "qfp4_gemm_fused_rq_workspace_bytes",
     "qfp4_gemm_fused_rq",
-    "qfp4_status_string", "qfp4_last_device_error", "qfp4_version",
+    "qfp4_status_string", "qfp4_last_device_error", "qfp4_version", "qfp4_launch_count",
 ]
 
 _lib = None
@@ -77,6 +77,8 @@ def lib():
         L.qfp4_last_device_error.argtypes = []
         L.qfp4_version.restype = c_int
         L.qfp4_version.argtypes = []
+        L.qfp4_launch_count.restype = c_uint64
+        L.qfp4_launch_count.argtypes = []
         _lib = L
     return _lib
 
@@ -139,6 +141,10 @@ def qfp4_last_device_error():
 
 def qfp4_version():
     return lib().qfp4_version()
+
+
+def qfp4_launch_count():
+    return lib().qfp4_launch_count()
 
 
 # ------------------------------------------------------------------ torch conveniences

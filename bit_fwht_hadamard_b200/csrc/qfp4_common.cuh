@@ -282,8 +282,14 @@ inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 }  // namespace qfp4
 
+namespace qfp4 {
+void count_launch();
+}
+
+// After every kernel launch: count it, and turn a launch error into a status.
 #define QFP4_LAUNCH_CHECK()                                                                        \
     do {                                                                                           \
+        qfp4::count_launch();                                                                      \
         if (cudaPeekAtLastError() != cudaSuccess) {                                                \
             (void)cudaGetLastError();                                                              \
             return QFP4_ERR_CUDA;                                                                  \

@@ -1,6 +1,7 @@
 // runtime.cu -- host runtime of libqfp4: the device error word, the
 // tensor-map encoder (driver entry point looked up once, no libcuda link),
 // SM counts, status strings.
+#include <atomic>
 #include <mutex>
 
 #include "qfp4_common.cuh"
@@ -41,6 +42,9 @@ int encode_tensor_map(CUtensorMap *map, CUtensorMapDataType dtype, int rank, voi
     return r == CUDA_SUCCESS ? QFP4_OK : QFP4_ERR_CUDA;
 }
 
+static std::atomic<unsigned long long> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
 int num_sms()
 {
     int dev = 0, n = 148;
@@ -74,3 +78,5 @@ extern "C" int qfp4_last_device_error(void)
 }
 
 extern "C" int qfp4_version(void) { return 100; }
+
+extern "C" uint64_t qfp4_launch_count(void) { return qfp4::g_launches.load(std::memory_order_relaxed); }

@@ -220,6 +220,10 @@ int qfp4_last_device_error(void);
 /* Library version, as MAJOR*10000 + MINOR*100 + PATCH. */
 int qfp4_version(void);
 
+/* Diagnostics: number of kernels this process has launched through the
+ * library so far (host-side counter, all devices). */
+uint64_t qfp4_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif
