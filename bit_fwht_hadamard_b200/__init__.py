@@ -28,7 +28,7 @@ OK, ERR_ARG, ERR_SHAPE, ERR_UNSUPPORTED, ERR_ALIGN, ERR_CUDA, ERR_TIMEOUT = 0, -
 EXPORTS = [
     "qfp4_quantize_workspace_bytes", "qfp4_quantize", "qfp4_quantize_mxfp8", "qfp4_quantize_fp32scale",
     "qfp4_dequantize", "qfp4_gemm_workspace_bytes", "qfp4_gemm_blockscaled", "qfp4_gemm_fused_rq_workspace_bytes",
-    "qfp4_gemm_fused_rq",
+    "qfp4_gemm_fused_rq", "qfp4_gemm_blockscaled_noalloc",
     "qfp4_status_string", "qfp4_last_device_error", "qfp4_version", "qfp4_launch_count",
 ]
 
@@ -66,6 +66,8 @@ def lib():
         L.qfp4_gemm_blockscaled.restype = c_int
         L.qfp4_gemm_blockscaled.argtypes = [P, P, P, P, P, P, c_int64, c_int64, c_int64, c_int, c_int, P, P,
                                             c_size_t, P]
+        L.qfp4_gemm_blockscaled_noalloc.restype = c_int
+        L.qfp4_gemm_blockscaled_noalloc.argtypes = [P, P, P, P, P, P, c_int64, c_int64, c_int64, c_int, c_int, P, P]
         L.qfp4_gemm_fused_rq_workspace_bytes.restype = c_size_t
         L.qfp4_gemm_fused_rq_workspace_bytes.argtypes = [c_int64, c_int64, c_int64, c_int]
         L.qfp4_gemm_fused_rq.restype = c_int
@@ -119,6 +121,14 @@ def qfp4_gemm_blockscaled(A_codes, A_scales, A_tscale, B_codes, B_scales, B_tsca
                           workspace, workspace_bytes, stream):
     return lib().qfp4_gemm_blockscaled(A_codes, A_scales, A_tscale, B_codes, B_scales, B_tscale, M, N, K, fmt,
                                        out_dt, out, workspace, workspace_bytes, stream)
+
+
+def qfp4_gemm_blockscaled_noalloc(A_codes, A_scales, A_tscale, B_codes, B_scales, B_tscale, M, N, K, fmt, out_dt,
+                                  out, stream):
+    """The GEMM without a workspace argument (built-in 16 MiB scratch), for
+    callers that may not allocate device memory."""
+    return lib().qfp4_gemm_blockscaled_noalloc(A_codes, A_scales, A_tscale, B_codes, B_scales, B_tscale, M, N, K,
+                                               fmt, out_dt, out, stream)
 
 
 def qfp4_gemm_fused_rq_workspace_bytes(M, N, K, fmt):

@@ -6,3 +6,4 @@
 #include "gemm.cu"
 #include "pending.cu"
 #include "api.cu"
+#include "gemm_noalloc.cu"

@@ -191,6 +191,28 @@ int qfp4_gemm_blockscaled(const uint8_t *A_codes, const uint8_t *A_scales, const
                           qfp4_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * qfp4_gemm_blockscaled_noalloc -- qfp4_gemm_blockscaled for callers that
+ * cannot allocate device memory (an op or plugin hook that forbids
+ * allocation while enqueuing, an allocation-free real-time loop, a library
+ * handed only its inputs and outputs).  No counterpart on the source pages:
+ * it is a packaging of the same GEMM.  Same arguments, semantics and
+ * results as qfp4_gemm_blockscaled, minus the workspace: the rearranged
+ * scales go to a 16 MiB scratch array built into the library, which every
+ * GPU that loads the library's kernels holds until the process exits.
+ * The first call on a device looks up the array's device address (with
+ * that device current); make it before any stream capture.  All calls share
+ * the array (nothing in it needs to start at zero); calls whose work
+ * overlaps on the GPU race on it.  Returns QFP4_ERR_SHAPE when the shape's
+ * rearranged scales, qfp4_gemm_workspace_bytes(M, N, K, fmt), exceed
+ * 16 MiB.  Allocates nothing (no cudaMalloc / cudaFree, no allocating
+ * library call).
+ * ---------------------------------------------------------------------- */
+int qfp4_gemm_blockscaled_noalloc(const uint8_t *A_codes, const uint8_t *A_scales, const float *A_tscale,
+                                  const uint8_t *B_codes, const uint8_t *B_scales, const float *B_tscale,
+                                  int64_t M, int64_t N, int64_t K, qfp4_fmt fmt,
+                                  qfp4_dtype out_dt, void *out, qfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * qfp4_gemm_fused_rq -- the same GEMM with A given in bf16: A is rotated
  * (rotate != 0, along K in 128 blocks) and quantized (fmt, RNE, four6 as in
  * qfp4_quantize) inside the call, then multiplied by the pre-quantized B
