@@ -3,6 +3,7 @@
 #include "runtime.cu"
 #include "quantize1d.cu"
 #include "dequant_fp32scale.cu"
+#include "quantize2d.cu"
 #include "gemm.cu"
 #include "pending.cu"
 #include "api.cu"

@@ -208,12 +208,17 @@ __device__ __forceinline__ float block_max(float m, float *red)
 }
 
 // s_t = amax_t / (6 * 448), amax_t the max of the partial maxima.
-__device__ __forceinline__ float tensor_scale(const QuantParams &p, float *red)
+__device__ __forceinline__ float tensor_scale_from(const float *partials, int n_partials, float *red)
 {
     float m = 0.0f;
-    for (int i = threadIdx.x; i < p.n_partials; i += blockDim.x) m = fmaxf(m, p.partials[i]);
+    for (int i = threadIdx.x; i < n_partials; i += blockDim.x) m = fmaxf(m, partials[i]);
     m = block_max(m, red);
     return __fdiv_rn(m, 2688.0f);
+}
+
+__device__ __forceinline__ float tensor_scale(const QuantParams &p, float *red)
+{
+    return tensor_scale_from(p.partials, p.n_partials, red);
 }
 
 template <int G>
@@ -472,6 +477,15 @@ static int run_pass(const void *x, qfp4_dtype xdt, int64_t n, QuantParams p, cud
     }
     if (n_parts) *n_parts = parts;
     return QFP4_OK;
+}
+
+// Partial maxima of |x| over a flat range (the NVFP4 tensor-amax pass, no rotation).
+int amax_partials(const void *x, qfp4_dtype xdt, int64_t n, float *partials, int *n_parts, cudaStream_t stream)
+{
+    QuantParams p{};
+    p.n = n;
+    p.partials_out = partials;
+    return run_pass<MODE_AMAX, QFP4_NVFP4, false, false, false>(x, xdt, n, p, stream, n_parts);
 }
 
 template <int FMT, bool ROT, bool SR, bool FOUR6>

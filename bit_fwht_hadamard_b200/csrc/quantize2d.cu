@@ -1,0 +1,411 @@
+// quantize2d.cu -- 2D transposition-invariant NVFP4 blocks (X and X^T from
+// one pass), the 1D column-wise quantization of X^T, and the MXFP8 (E4M3)
+// variant with its column-wise output.
+//
+// Method: [TI] (2D blocks give X and X^T one shared scale set; stochastic
+// rounding; MXFP8 for the sensitive projections), [46] (four-over-six on the
+// column groups of the 1D baseline), [LB] §2-§3 (group scales, E8M0).
+//
+// 2D kernel: a warp covers two horizontally adjacent 16x16 tiles of one
+// 16-row band; lane (h, r) loads row r of tile h (16 bf16 = 32 B, so every
+// 32-byte sector a warp touches is fully used).  The tile amax is a 16-lane
+// shuffle reduction; each lane quantizes its row (RNE or Philox SR keyed on
+// X's element index), stores its 8 code bytes, then a 4-level nibble
+// transpose across the 16 lanes (block swaps of 8, 4, 2, 1 nibbles) gives
+// each lane one column of the tile -- the codes of X^T, bit-identical by
+// construction because every element was rounded once.
+//
+// Column-wise kernels (1D X^T baseline, MXFP8): a warp covers a 32 x 32
+// tile, lane = column, so a column group of 32 (or two of 16) sits in one
+// lane's registers; row loads are 64 contiguous bytes per warp instruction.
+#include "qfp4_common.cuh"
+#include "quantize1d.cuh"
+
+namespace qfp4 {
+
+struct Q2DParams {
+    int64_t M, K;
+    uint8_t *codes, *scales, *codesT, *scalesT;
+    const float *partials;
+    int n_partials;
+    float *tscale_out;
+    uint64_t seed;
+};
+
+template <typename T>
+__device__ __forceinline__ void load16(const T *x, int64_t off, float *v)
+{
+    if (sizeof(T) == 4) {
+        const float4 *s = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(x) + off);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const float4 f = s[c];
+            v[4 * c] = f.x;
+            v[4 * c + 1] = f.y;
+            v[4 * c + 2] = f.z;
+            v[4 * c + 3] = f.w;
+        }
+    } else {
+        const uint4 *s = reinterpret_cast<const uint4 *>(reinterpret_cast<const uint16_t *>(x) + off);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            const uint4 w = s[c];
+            v[8 * c] = bf16lo(w.x);
+            v[8 * c + 1] = bf16hi(w.x);
+            v[8 * c + 2] = bf16lo(w.y);
+            v[8 * c + 3] = bf16hi(w.y);
+            v[8 * c + 4] = bf16lo(w.z);
+            v[8 * c + 5] = bf16hi(w.z);
+            v[8 * c + 6] = bf16lo(w.w);
+            v[8 * c + 7] = bf16hi(w.w);
+        }
+    }
+}
+
+template <typename T>
+__device__ __forceinline__ float ld1(const T *x, int64_t i)
+{
+    if (sizeof(T) == 4) return reinterpret_cast<const float *>(x)[i];
+    return __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const uint16_t *>(x)[i]) << 16);
+}
+
+// Transpose a 16 x 16 nibble matrix held as one 64-bit row per lane of a
+// 16-lane group (nibble j of lane r = element (r, j)); afterwards nibble j of
+// lane r is element (j, r).  Shuffle partners stay inside the group.
+__device__ __forceinline__ uint64_t transpose16x16_nibbles(uint64_t w, int r)
+{
+#pragma unroll
+    for (int s = 8; s >= 1; s >>= 1) {
+        // nibble positions j with (j & s) != 0
+        const uint64_t m = s == 8 ? 0xFFFFFFFF00000000ull
+                         : s == 4 ? 0xFFFF0000FFFF0000ull
+                         : s == 2 ? 0xFF00FF00FF00FF00ull
+                                  : 0xF0F0F0F0F0F0F0F0ull;
+        const uint32_t lo = __shfl_xor_sync(0xFFFFFFFFu, static_cast<uint32_t>(w), s);
+        const uint32_t hi = __shfl_xor_sync(0xFFFFFFFFu, static_cast<uint32_t>(w >> 32), s);
+        const uint64_t o = (static_cast<uint64_t>(hi) << 32) | lo;
+        if ((r & s) == 0) w = (w & ~m) | ((o & ~m) << (4 * s));
+        else w = (w & m) | ((o & m) >> (4 * s));
+    }
+    return w;
+}
+
+// ---------------------------------------------------------------- 2D NVFP4
+template <bool SR, typename T>
+__global__ void __launch_bounds__(256) k_quant2d(const T *__restrict__ x, Q2DParams p)
+{
+    __shared__ float red[32];
+    const float s_t = tensor_scale_from(p.partials, p.n_partials, red);
+    if (p.tscale_out && blockIdx.x == 0 && threadIdx.x == 0) *p.tscale_out = s_t;
+
+    const int lane = threadIdx.x & 31, half = lane >> 4, r = lane & 15;
+    const int64_t tiles_k = p.K / 16, pairs = (tiles_k + 1) / 2;
+    const int64_t tasks = (p.M / 16) * pairs;
+    const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    for (int64_t task = warp0; task < tasks; task += nwarps) {
+        const int64_t band = task / pairs, tc = (task % pairs) * 2 + half;
+        const bool valid = tc < tiles_k;
+        const int64_t i = band * 16 + r, j0 = tc * 16;
+        float v[16];
+        if (valid) load16(x, i * p.K + j0, v);
+        else
+#pragma unroll
+            for (int t = 0; t < 16; ++t) v[t] = 0.0f;
+        float amax = 0.0f;
+#pragma unroll
+        for (int t = 0; t < 16; ++t) amax = fmaxf(amax, fabsf(v[t]));
+#pragma unroll
+        for (int o = 8; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+        uint32_t enc = 0u;
+        float S = 0.0f;
+        if (s_t != 0.0f) {
+            enc = e4m3_rne(__fdiv_rn(__fdiv_rn(amax, 6.0f), s_t));
+            S = __fmul_rn(e4m3_value(enc), s_t);
+        }
+        uint32_t w[2] = {0u, 0u};
+        if (S != 0.0f) {
+            float q[16];
+#pragma unroll
+            for (int t = 0; t < 16; ++t) q[t] = __fdiv_rn(v[t], S);
+            if (SR) sr_group<16>(q, static_cast<uint64_t>(i * p.K + j0), p.seed, w);
+            else {
+                w[0] = e2m1x8_rne(q);
+                w[1] = e2m1x8_rne(q + 8);
+            }
+        }
+        if (valid) {
+            *reinterpret_cast<uint2 *>(p.codes + (i * p.K + j0) / 2) = make_uint2(w[0], w[1]);
+            p.scales[i * tiles_k + tc] = static_cast<uint8_t>(enc);
+        }
+        if (p.codesT) {
+            const uint64_t t = transpose16x16_nibbles((static_cast<uint64_t>(w[1]) << 32) | w[0], r);
+            if (valid) {
+                const int64_t jr = j0 + r;                  // column of X = row of X^T
+                *reinterpret_cast<uint2 *>(p.codesT + (jr * p.M + band * 16) / 2) =
+                    make_uint2(static_cast<uint32_t>(t), static_cast<uint32_t>(t >> 32));
+                p.scalesT[jr * (p.M / 16) + band] = static_cast<uint8_t>(enc);
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------- 1D column-wise (X^T baseline)
+template <int FMT, bool SR, bool FOUR6, typename T>
+__global__ void __launch_bounds__(256) k_quant_cols(const T *__restrict__ x, Q2DParams p)
+{
+    __shared__ float red[32];
+    float s_t = 0.0f;
+    if (FMT == QFP4_NVFP4) s_t = tensor_scale_from(p.partials, p.n_partials, red);
+    constexpr int G = FMT == QFP4_MXFP4 ? 32 : 16;
+    const int lane = threadIdx.x & 31;
+    const int64_t col_blocks = (p.K + 31) / 32, row_blocks = (p.M + 31) / 32;
+    const int64_t tasks = row_blocks * col_blocks;
+    const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    for (int64_t task = warp0; task < tasks; task += nwarps) {
+        const int64_t i0 = (task / col_blocks) * 32, j = (task % col_blocks) * 32 + lane;
+        const int rows = static_cast<int>(imin<int64_t>(32, p.M - i0));   // 32, or 16 (NVFP4 with M % 32 == 16)
+        if (j >= p.K) continue;                     // no shuffles below: lanes are independent
+        float v[32];
+#pragma unroll
+        for (int r = 0; r < 32; ++r) v[r] = r < rows ? ld1(x, (i0 + r) * p.K + j) : 0.0f;
+        uint32_t cw[4];
+        uint32_t sc = 0u;
+#pragma unroll
+        for (int g = 0; g < 32 / G; ++g) {
+            const float *xg = v + g * G;
+            uint32_t *wg = cw + g * (G / 8);
+            float amax = 0.0f;
+#pragma unroll
+            for (int t = 0; t < G; ++t) amax = fmaxf(amax, fabsf(xg[t]));
+            uint32_t sbyte = 0u;
+            float S = 0.0f, mul = 0.0f;
+            if (FMT == QFP4_MXFP4) {
+                if (amax != 0.0f) {
+                    const int k = scale_exp(amax, 0x400000u, 2);
+                    sbyte = static_cast<uint32_t>(k + 127);
+                    S = exp2i(k);
+                    mul = exp2i(-k);
+                }
+            } else if (s_t != 0.0f) {
+                sbyte = e4m3_rne(__fdiv_rn(__fdiv_rn(amax, 6.0f), s_t));
+                S = __fmul_rn(e4m3_value(sbyte), s_t);
+            }
+            if (FMT == QFP4_NVFP4 && FOUR6) {
+                uint32_t w6[2], w4[2], enc4 = 0u;
+                float sse6, sse4, S4 = 0.0f;
+                if (s_t != 0.0f) {
+                    enc4 = e4m3_rne(__fdiv_rn(__fdiv_rn(amax, 4.0f), s_t));
+                    S4 = __fmul_rn(e4m3_value(enc4), s_t);
+                }
+                nv_block_rne(xg, S, w6, &sse6);
+                nv_block_rne(xg, S4, w4, &sse4);
+                const bool pick4 = sse4 < sse6;
+                wg[0] = pick4 ? w4[0] : w6[0];
+                wg[1] = pick4 ? w4[1] : w6[1];
+                sbyte = pick4 ? enc4 : sbyte;
+            } else if (S == 0.0f) {
+#pragma unroll
+                for (int t = 0; t < G / 8; ++t) wg[t] = 0u;
+            } else {
+                float q[G];
+#pragma unroll
+                for (int t = 0; t < G; ++t) q[t] = FMT == QFP4_MXFP4 ? __fmul_rn(xg[t], mul) : __fdiv_rn(xg[t], S);
+                if (SR) {
+#pragma unroll
+                    for (int t = 0; t < G / 8; ++t) wg[t] = 0u;
+#pragma unroll
+                    for (int t = 0; t < G; ++t) {
+                        const uint64_t e = static_cast<uint64_t>((i0 + g * G + t) * p.K + j);
+                        const uint4 rw = sr_words4(p.seed, e >> 2);
+                        const uint32_t word = (e & 3) == 0 ? rw.x : (e & 3) == 1 ? rw.y : (e & 3) == 2 ? rw.z : rw.w;
+                        wg[t >> 3] |= e2m1_sr(q[t], word) << (4 * (t & 7));
+                    }
+                } else {
+#pragma unroll
+                    for (int t = 0; t < G / 8; ++t) wg[t] = e2m1x8_rne(q + 8 * t);
+                }
+            }
+            sc |= sbyte << (8 * g);
+        }
+        // codes of column j, rows i0 .. i0+rows-1 (8-byte aligned: M % 16 == 0)
+        uint2 *cdst = reinterpret_cast<uint2 *>(p.codesT + (j * p.M + i0) / 2);
+        cdst[0] = make_uint2(cw[0], cw[1]);
+        if (rows == 32) cdst[1] = make_uint2(cw[2], cw[3]);
+        if (G == 32) {
+            p.scalesT[j * (p.M / 32) + i0 / 32] = static_cast<uint8_t>(sc);
+        } else {
+            p.scalesT[j * (p.M / 16) + i0 / 16] = static_cast<uint8_t>(sc);
+            if (rows == 32) p.scalesT[j * (p.M / 16) + i0 / 16 + 1] = static_cast<uint8_t>(sc >> 8);
+        }
+    }
+}
+
+// ---------------------------------------------------------------- MXFP8 (E4M3, g32)
+// E4M3 stochastic rounding: lo <= |v| < hi adjacent E4M3 values (subnormal
+// spacing 2^-9 below 2^-6, else 2^(e-3)), up iff (w >> 8) * 2^-24 < (|v|-lo)/(hi-lo);
+// saturates at 448.  Returns the byte.
+__device__ __forceinline__ uint32_t e4m3_sr(float v, uint32_t w)
+{
+    const uint32_t sign = (__float_as_uint(v) >> 24) & 0x80u;
+    const float a = fabsf(v);
+    float lo, sp, inv_sp;
+    if (a >= 0.015625f) {                                    // 2^-6: normal binade
+        const uint32_t spb = (__float_as_uint(a) & 0x7F800000u) - (3u << 23);
+        lo = __uint_as_float(__float_as_uint(a) & 0x7FF00000u);
+        sp = __uint_as_float(spb);
+        inv_sp = __uint_as_float((254u << 23) - spb);
+    } else {
+        lo = __fmul_rn(truncf(__fmul_rn(a, 512.0f)), 0.001953125f);   // exact: multiples of 2^-9
+        sp = 0.001953125f;
+        inv_sp = 512.0f;
+    }
+    const float p = __fmul_rn(__fsub_rn(a, lo), inv_sp);
+    const float u = __fmul_rn(static_cast<float>(w >> 8), 5.9604644775390625e-08f);
+    float rr = (u < p) ? __fadd_rn(lo, sp) : lo;
+    rr = fminf(rr, 448.0f);
+    return e4m3_rne(rr) | sign;
+}
+
+template <bool SR, bool COLS, typename T>
+__global__ void __launch_bounds__(256) k_mxfp8(const T *__restrict__ x, Q2DParams p)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t col_blocks = p.K / 32, row_blocks = (p.M + 31) / 32;
+    const int64_t tasks = row_blocks * col_blocks;
+    const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    for (int64_t task = warp0; task < tasks; task += nwarps) {
+        const int64_t i0 = (task / col_blocks) * 32, j = (task % col_blocks) * 32 + lane;
+        const int rows = static_cast<int>(imin<int64_t>(32, p.M - i0));
+        float v[32];
+        uint32_t wd[32];
+#pragma unroll
+        for (int r = 0; r < 32; ++r) {
+            v[r] = r < rows ? ld1(x, (i0 + r) * p.K + j) : 0.0f;
+            if (SR) {
+                const uint64_t e = static_cast<uint64_t>((i0 + r) * p.K + j);
+                const uint4 rw = sr_words4(p.seed, e >> 2);
+                wd[r] = (e & 3) == 0 ? rw.x : (e & 3) == 1 ? rw.y : (e & 3) == 2 ? rw.z : rw.w;
+            }
+        }
+        // row groups: 32 lanes of one row
+        uint8_t my_scale = 0;
+#pragma unroll
+        for (int r = 0; r < 32; ++r) {
+            float amax = fabsf(v[r]);
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+            uint32_t byte = 0u, sbyte = 0u;
+            if (amax != 0.0f) {
+                const int k = scale_exp(amax, 0x600000u, 8);
+                sbyte = static_cast<uint32_t>(k + 127);
+                const float q = __fmul_rn(v[r], exp2i(-k));
+                byte = SR ? e4m3_sr(q, wd[r]) : e4m3_rne(q);
+            }
+            if (lane == r) my_scale = static_cast<uint8_t>(sbyte);
+            if (r < rows) p.codes[(i0 + r) * p.K + j] = static_cast<uint8_t>(byte);
+        }
+        if (lane < rows) p.scales[(i0 + lane) * (p.K / 32) + j / 32] = my_scale;
+        if (COLS) {                                   // column group: this lane's 32 rows
+            float amax = 0.0f;
+#pragma unroll
+            for (int r = 0; r < 32; ++r) amax = fmaxf(amax, fabsf(v[r]));
+            uint32_t bytes[8] = {0, 0, 0, 0, 0, 0, 0, 0}, sbyte = 0u;
+            if (amax != 0.0f) {
+                const int k = scale_exp(amax, 0x600000u, 8);
+                sbyte = static_cast<uint32_t>(k + 127);
+                const float m = exp2i(-k);
+#pragma unroll
+                for (int r = 0; r < 32; ++r) {
+                    const float q = __fmul_rn(v[r], m);
+                    bytes[r >> 2] |= (SR ? e4m3_sr(q, wd[r]) : e4m3_rne(q)) << (8 * (r & 3));
+                }
+            }
+            uint4 *dst = reinterpret_cast<uint4 *>(p.codesT + j * p.M + i0);
+            dst[0] = make_uint4(bytes[0], bytes[1], bytes[2], bytes[3]);
+            dst[1] = make_uint4(bytes[4], bytes[5], bytes[6], bytes[7]);
+            p.scalesT[j * (p.M / 32) + i0 / 32] = static_cast<uint8_t>(sbyte);
+        }
+    }
+}
+
+// ---------------------------------------------------------------- host
+static int grid_for_warps(int64_t warp_tasks)
+{
+    const int64_t blocks = (warp_tasks + 7) / 8;              // 8 warps per 256-thread block
+    return static_cast<int>(imax<int64_t>(1, imin<int64_t>(blocks, 16 * num_sms())));
+}
+
+int quantize2d(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_round rounding, uint64_t seed,
+               uint8_t *codes, uint8_t *scales, uint8_t *codesT, uint8_t *scalesT, float *tscale, float *partials,
+               cudaStream_t stream)
+{
+    int n_parts = 0;
+    int st = amax_partials(x, xdt, M * K, partials, &n_parts, stream);
+    if (st != QFP4_OK) return st;
+    Q2DParams p{M, K, codes, scales, codesT, scalesT, partials, n_parts, tscale, seed};
+    const int grid = grid_for_warps((M / 16) * ((K / 16 + 1) / 2));
+    const bool sr = rounding == QFP4_SR;
+    if (xdt == QFP4_BF16) {
+        if (sr) k_quant2d<true, uint16_t><<<grid, 256, 0, stream>>>(static_cast<const uint16_t *>(x), p);
+        else k_quant2d<false, uint16_t><<<grid, 256, 0, stream>>>(static_cast<const uint16_t *>(x), p);
+    } else {
+        if (sr) k_quant2d<true, float><<<grid, 256, 0, stream>>>(static_cast<const float *>(x), p);
+        else k_quant2d<false, float><<<grid, 256, 0, stream>>>(static_cast<const float *>(x), p);
+    }
+    QFP4_LAUNCH_CHECK();
+    return QFP4_OK;
+}
+
+template <int FMT, bool SR, bool FOUR6>
+static int launch_cols(const void *x, qfp4_dtype xdt, const Q2DParams &p, int grid, cudaStream_t stream)
+{
+    if (xdt == QFP4_BF16)
+        k_quant_cols<FMT, SR, FOUR6, uint16_t><<<grid, 256, 0, stream>>>(static_cast<const uint16_t *>(x), p);
+    else k_quant_cols<FMT, SR, FOUR6, float><<<grid, 256, 0, stream>>>(static_cast<const float *>(x), p);
+    QFP4_LAUNCH_CHECK();
+    return QFP4_OK;
+}
+
+int quantize_columns(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_fmt fmt, qfp4_round rounding, int four6,
+                     uint64_t seed, uint8_t *codesT, uint8_t *scalesT, const float *partials, int n_partials,
+                     cudaStream_t stream)
+{
+    Q2DParams p{M, K, nullptr, nullptr, codesT, scalesT, partials, n_partials, nullptr, seed};
+    const int grid = grid_for_warps(((M + 31) / 32) * ((K + 31) / 32));
+    const bool sr = rounding == QFP4_SR;
+    if (fmt == QFP4_MXFP4)
+        return sr ? launch_cols<QFP4_MXFP4, true, false>(x, xdt, p, grid, stream)
+                  : launch_cols<QFP4_MXFP4, false, false>(x, xdt, p, grid, stream);
+    if (four6) return launch_cols<QFP4_NVFP4, false, true>(x, xdt, p, grid, stream);
+    return sr ? launch_cols<QFP4_NVFP4, true, false>(x, xdt, p, grid, stream)
+              : launch_cols<QFP4_NVFP4, false, false>(x, xdt, p, grid, stream);
+}
+
+int quantize_mxfp8(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_round rounding, uint64_t seed,
+                   uint8_t *codes, uint8_t *scales, uint8_t *codesT, uint8_t *scalesT, cudaStream_t stream)
+{
+    Q2DParams p{M, K, codes, scales, codesT, scalesT, nullptr, 0, nullptr, seed};
+    const int grid = grid_for_warps(((M + 31) / 32) * (K / 32));
+    const bool sr = rounding == QFP4_SR, cols = codesT != nullptr;
+#define QFP4_MX8(SRV, COLV)                                                                                   \
+    do {                                                                                                      \
+        if (xdt == QFP4_BF16)                                                                                 \
+            k_mxfp8<SRV, COLV, uint16_t><<<grid, 256, 0, stream>>>(static_cast<const uint16_t *>(x), p);      \
+        else k_mxfp8<SRV, COLV, float><<<grid, 256, 0, stream>>>(static_cast<const float *>(x), p);           \
+    } while (0)
+    if (sr) {
+        if (cols) QFP4_MX8(true, true);
+        else QFP4_MX8(true, false);
+    } else {
+        if (cols) QFP4_MX8(false, true);
+        else QFP4_MX8(false, false);
+    }
+#undef QFP4_MX8
+    QFP4_LAUNCH_CHECK();
+    return QFP4_OK;
+}
+
+}  // namespace qfp4
