@@ -162,9 +162,11 @@ __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w <
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 // E2M1 round-to-nearest-even with saturation to +-6, eight values packed
-// into one 32-bit word (element t in nibble t).  Uses the sm_100 hardware
-// conversion; the code's sign bit is then forced to the sign of the input
-// so that values rounding to zero keep their sign (the oracle's rule).
+// into one 32-bit word (element t in nibble t), by the sm_100 hardware
+// conversion.  The conversion keeps the sign of zero (-0.0 and negative
+// values that round to zero give code 0x8), which is the rule this library
+// follows; an exhaustive sweep of all finite binary32 inputs on B200 agrees
+// with the nearest / ties-to-even / saturating definition bit for bit.
 __device__ __forceinline__ uint32_t e2m1x8_rne(const float *v)
 {
     uint32_t out;
@@ -176,10 +178,55 @@ __device__ __forceinline__ uint32_t e2m1x8_rne(const float *v)
         "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
         : "=r"(out)
         : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
-    uint32_t s = 0;
-#pragma unroll
-    for (int t = 0; t < 8; ++t) s |= (__float_as_uint(v[t]) >> 31) << (4 * t + 3);
-    return out | s;
+    return out;
+}
+
+// ------------------------------------------------------------------ packed binary32 pairs
+// Two binary32 values in one 64-bit register pair (low = the even element);
+// sm_100's f32x2 arithmetic does two IEEE round-to-nearest operations per
+// instruction.
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t p, float &lo, float &hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(p));
+}
+__device__ __forceinline__ uint64_t f2add(uint64_t a, uint64_t b)
+{
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2sub(uint64_t a, uint64_t b)
+{
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2mul(uint64_t a, uint64_t b)
+{
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+// two bf16 (one 32-bit word) -> a packed pair, exact
+__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w)
+{
+    return f2pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+// E2M1 RNE of four packed pairs (8 values) -> one word of nibbles
+__device__ __forceinline__ uint32_t e2m1x8_rne_pairs(uint64_t p0, uint64_t p1, uint64_t p2, uint64_t p3)
+{
+    float v[8];
+    f2unpack(p0, v[0], v[1]);
+    f2unpack(p1, v[2], v[3]);
+    f2unpack(p2, v[4], v[5]);
+    f2unpack(p3, v[6], v[7]);
+    return e2m1x8_rne(v);
 }
 
 // E2M1 stochastic rounding of one value (|v| <= 6 or saturating):

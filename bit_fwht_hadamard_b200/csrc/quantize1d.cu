@@ -9,23 +9,27 @@
 //
 // Layout: the input is a flat stream of n = M*K elements (groups never cross
 // rows because K % g == 0, and rotation blocks never cross rows because
-// K % 128 == 0).  A thread owns one 64-element unit (a 128-byte bf16 row of
-// the tile); the two threads of a 128-element rotation block exchange one
-// butterfly stage with a warp shuffle, every other stage runs in registers.
-// bf16 tiles of 512 units (64 KiB) are brought into shared memory by TMA
-// with 128-byte swizzle (so the per-thread 16-byte reads are bank-conflict
-// free) through a 3-stage mbarrier pipeline; the grid is persistent.
+// K % 128 == 0).  Main (bf16) kernel: one persistent CTA per SM, 8 warps,
+// each warp with its own 3-stage ring of 8 KiB tiles (64 rows of 64 bf16)
+// brought in by TMA with 128-byte swizzle; an SM takes a contiguous range of
+// tiles (balanced to one 4096-element tile) and its warps interleave over
+// it.  A thread owns one 128-element unit (two 128-byte rows), held as 64
+// packed binary32 pairs: the whole rotation block is in registers, and the
+// butterflies of stages h = 2..64 and the scaling run as f32x2 operations
+// (two IEEE additions per instruction).  The direct kernel (64-element
+// units, one shuffle stage) serves binary32 inputs and the ragged tail.
 #include "qfp4_common.cuh"
 #include "quantize1d.cuh"
 
 namespace qfp4 {
 
-constexpr int QT_THREADS = 512;                 // one 64-element unit per thread
-constexpr int QT_TILE_ROWS = QT_THREADS;        // 64-element rows per tile
-constexpr int QT_BOX_ROWS = 256;                // TMA box height (hardware limit 256)
-constexpr int QT_STAGES = 3;
+constexpr int QT_WARPS = 8;                     // per CTA; one CTA per SM
+constexpr int QT_THREADS = 32 * QT_WARPS;
+constexpr int QT_TILE_ROWS = 64;                // 64 rows of 64 bf16 = one warp's tile (2 rows per lane)
+constexpr int QT_TILE_ELEMS = QT_TILE_ROWS * 64;
+constexpr int QT_STAGES = 3;                    // per warp
 constexpr int QT_STAGE_BYTES = QT_TILE_ROWS * 128;
-constexpr int QT_SMEM_BYTES = QT_STAGES * QT_STAGE_BYTES + 1024;
+constexpr int QT_SMEM_BYTES = QT_WARPS * QT_STAGES * QT_STAGE_BYTES + 1024;
 
 // E2M1 code -> binary32 value (exact), from the bit fields.
 __device__ __forceinline__ float e2m1_value(uint32_t c)
@@ -246,89 +250,231 @@ __device__ __forceinline__ void store_unit(const UnitOut &o, const QuantParams &
     }
 }
 
+// ---------------------------------------------------------------- 128-element units (TMA kernel)
+// FWHT-128 of one unit held as packed pairs (pair k = elements 2k, 2k+1):
+// stage h = 1 inside each pair, stages h = 2..64 between pairs k and
+// k + h/2 as f32x2 add / sub, then one f32x2 multiply by 1/sqrt(128).
+__device__ __forceinline__ void fwht128_packed(uint64_t (&p)[64])
+{
+#pragma unroll
+    for (int k = 0; k < 64; ++k) {
+        float a, b;
+        f2unpack(p[k], a, b);
+        p[k] = f2pack(__fadd_rn(a, b), __fsub_rn(a, b));
+    }
+#pragma unroll
+    for (int hp = 1; hp < 64; hp <<= 1) {
+#pragma unroll
+        for (int k = 0; k < 64; ++k) {
+            if ((k & hp) == 0) {
+                const uint64_t a = p[k], b = p[k + hp];
+                p[k] = f2add(a, b);
+                p[k + hp] = f2sub(a, b);
+            }
+        }
+    }
+    const uint64_t c2 = f2pack(inv_sqrt128(), inv_sqrt128());
+#pragma unroll
+    for (int k = 0; k < 64; ++k) p[k] = f2mul(p[k], c2);
+}
+
+__device__ __forceinline__ float absmax_pairs(const uint64_t *p, int n)
+{
+    float m = 0.0f;
+#pragma unroll
+    for (int j = 0; j < n; ++j) {
+        float a, b;
+        f2unpack(p[j], a, b);
+        m = fmaxf(m, fmaxf(fabsf(a), fabsf(b)));
+    }
+    return m;
+}
+
+struct Unit128 {
+    uint32_t codes[16];     // 128 nibbles
+    uint32_t scales[2];     // up to 8 scale bytes
+};
+
+template <int FMT, bool SR, bool FOUR6>
+__device__ __forceinline__ void quant_unit128(uint64_t (&p)[64], uint64_t e0, float s_t, uint64_t seed, Unit128 &o)
+{
+    o.scales[0] = o.scales[1] = 0u;
+    if (FMT == QFP4_MXFP4) {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            uint64_t *pg = p + 16 * g;
+            uint32_t *w = o.codes + 4 * g;
+            const float amax = absmax_pairs(pg, 16);
+            if (amax == 0.0f) {                      // all-zero group: byte 0, +0 codes
+                w[0] = w[1] = w[2] = w[3] = 0u;
+                continue;
+            }
+            const int k = scale_exp(amax, 0x400000u, 2);
+            o.scales[0] |= static_cast<uint32_t>(k + 127) << (8 * g);
+            const uint64_t m2 = f2pack(exp2i(-k), exp2i(-k));   // x * 2^-k == x / 2^k exactly
+#pragma unroll
+            for (int j = 0; j < 16; ++j) pg[j] = f2mul(pg[j], m2);
+            if (SR) {
+                float q[32];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) f2unpack(pg[j], q[2 * j], q[2 * j + 1]);
+                sr_group<32>(q, e0 + 32 * g, seed, w);
+            } else {
+#pragma unroll
+                for (int t = 0; t < 4; ++t) w[t] = e2m1x8_rne_pairs(pg[4 * t], pg[4 * t + 1], pg[4 * t + 2], pg[4 * t + 3]);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+            float x[16];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) f2unpack(p[8 * b + j], x[2 * j], x[2 * j + 1]);
+            float amax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
+            uint32_t *w = o.codes + 2 * b;
+            uint32_t enc = 0u;
+            float S = 0.0f;
+            if (s_t != 0.0f) {
+                enc = e4m3_rne(__fdiv_rn(__fdiv_rn(amax, 6.0f), s_t));
+                S = __fmul_rn(e4m3_value(enc), s_t);
+            }
+            if (FOUR6) {
+                uint32_t w6[2], w4[2], enc4 = 0u;
+                float sse6, sse4, S4 = 0.0f;
+                if (s_t != 0.0f) {
+                    enc4 = e4m3_rne(__fdiv_rn(__fdiv_rn(amax, 4.0f), s_t));
+                    S4 = __fmul_rn(e4m3_value(enc4), s_t);
+                }
+                nv_block_rne(x, S, w6, &sse6);
+                nv_block_rne(x, S4, w4, &sse4);
+                const bool pick4 = sse4 < sse6;
+                w[0] = pick4 ? w4[0] : w6[0];
+                w[1] = pick4 ? w4[1] : w6[1];
+                enc = pick4 ? enc4 : enc;
+            } else if (SR) {
+                if (S == 0.0f) {
+                    w[0] = w[1] = 0u;
+                } else {
+                    float q[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) q[i] = __fdiv_rn(x[i], S);
+                    sr_group<16>(q, e0 + 16 * b, seed, w);
+                }
+            } else {
+                nv_block_rne(x, S, w, nullptr);
+            }
+            o.scales[b >> 2] |= enc << (8 * (b & 3));
+        }
+    }
+}
+
+template <int G>
+__device__ __forceinline__ void store_unit128(const Unit128 &o, const QuantParams &p, uint64_t e0, int64_t n_valid)
+{
+    // n_valid: 128, or 64 when the launch range ends half way through the unit
+    uint4 *c4 = reinterpret_cast<uint4 *>(p.codes + (e0 >> 1));
+    uint8_t *sdst = p.scales + e0 / G;
+    c4[0] = make_uint4(o.codes[0], o.codes[1], o.codes[2], o.codes[3]);
+    c4[1] = make_uint4(o.codes[4], o.codes[5], o.codes[6], o.codes[7]);
+    if (n_valid >= 128) {
+        c4[2] = make_uint4(o.codes[8], o.codes[9], o.codes[10], o.codes[11]);
+        c4[3] = make_uint4(o.codes[12], o.codes[13], o.codes[14], o.codes[15]);
+    }
+    if (G == 32) {
+        if (n_valid >= 128) *reinterpret_cast<uint32_t *>(sdst) = o.scales[0];
+        else *reinterpret_cast<uint16_t *>(sdst) = static_cast<uint16_t>(o.scales[0]);
+    } else {
+        if (n_valid >= 128) *reinterpret_cast<uint2 *>(sdst) = make_uint2(o.scales[0], o.scales[1]);
+        else *reinterpret_cast<uint32_t *>(sdst) = o.scales[0];
+    }
+}
+
 // ---------------------------------------------------------------- TMA kernel
 template <int MODE, int FMT, bool ROT, bool SR, bool FOUR6>
 __global__ void __launch_bounds__(QT_THREADS, 1) k_quant1d_tma(const __grid_constant__ CUtensorMap tm, QuantParams p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ __align__(8) uint64_t full[QT_STAGES];
+    __shared__ __align__(8) uint64_t full[QT_WARPS][QT_STAGES];
     __shared__ float red[32];
 
-    const int tid = threadIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t rows = p.n / 64;
     const int64_t ntiles = (rows + QT_TILE_ROWS - 1) / QT_TILE_ROWS;
+    // contiguous tile range of this CTA, balanced to one tile
+    const int64_t t_begin = ntiles * blockIdx.x / gridDim.x, t_end = ntiles * (blockIdx.x + 1) / gridDim.x;
     constexpr int G = FMT == QFP4_MXFP4 ? 32 : 16;
 
     float s_t = 0.0f;
     if (MODE == MODE_QUANT && FMT == QFP4_NVFP4) {
         s_t = tensor_scale(p, red);
-        if (p.write_tscale && blockIdx.x == 0 && tid == 0) *p.tscale_out = s_t;
+        if (p.write_tscale && blockIdx.x == 0 && threadIdx.x == 0) *p.tscale_out = s_t;
     }
-    if (tid == 0) {
-        for (int s = 0; s < QT_STAGES; ++s) mbar_init(&full[s], 1);
+    uint64_t *bars = full[warp];
+    uint8_t *ring = smem + warp * (QT_STAGES * QT_STAGE_BYTES);
+    if (lane == 0) {
+        for (int s = 0; s < QT_STAGES; ++s) mbar_init(&bars[s], 1);
         fence_mbar_init();
-        prefetch_tensormap(&tm);
+        if (warp == 0) prefetch_tensormap(&tm);
     }
-    __syncthreads();
+    __syncwarp();
 
     auto issue = [&](int64_t t, int s) {
-        uint8_t *dst = smem + s * QT_STAGE_BYTES;
-        mbar_arrive_expect_tx(&full[s], QT_STAGE_BYTES);
-        const int r0 = static_cast<int>(t * QT_TILE_ROWS);
-        tma_load_2d(dst, &tm, &full[s], 0, r0);
-        tma_load_2d(dst + QT_BOX_ROWS * 128, &tm, &full[s], 0, r0 + QT_BOX_ROWS);
+        mbar_arrive_expect_tx(&bars[s], QT_STAGE_BYTES);
+        tma_load_2d(ring + s * QT_STAGE_BYTES, &tm, &bars[s], 0, static_cast<int>(t * QT_TILE_ROWS));
     };
-    if (tid == 0)
+    if (lane == 0)
         for (int s = 0; s < QT_STAGES; ++s) {
-            const int64_t t = blockIdx.x + static_cast<int64_t>(s) * gridDim.x;
-            if (t < ntiles) issue(t, s);
+            const int64_t t = t_begin + warp + static_cast<int64_t>(s) * QT_WARPS;
+            if (t < t_end) issue(t, s);
         }
 
     float tmax = 0.0f;
     int it = 0;
-    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
+    for (int64_t t = t_begin + warp; t < t_end; t += QT_WARPS, ++it) {
         const int s = it % QT_STAGES;
         const uint32_t ph = (it / QT_STAGES) & 1u;
-        const bool ok = mbar_wait(&full[s], ph);
-        if (__syncthreads_or(!ok)) return;
+        const bool ok = mbar_wait(&bars[s], ph);
+        if (__any_sync(0xFFFFFFFFu, !ok)) break;
 
-        const uint8_t *st = smem + s * QT_STAGE_BYTES + tid * 128;
-        float v[64];
+        // this lane's unit: rows 2*lane and 2*lane+1 of the tile (128-byte swizzle)
+        const uint8_t *st = ring + s * QT_STAGE_BYTES;
+        uint64_t v[64];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            const uint4 w = *reinterpret_cast<const uint4 *>(st + ((c ^ (tid & 7)) << 4));
-            v[8 * c + 0] = bf16lo(w.x);
-            v[8 * c + 1] = bf16hi(w.x);
-            v[8 * c + 2] = bf16lo(w.y);
-            v[8 * c + 3] = bf16hi(w.y);
-            v[8 * c + 4] = bf16lo(w.z);
-            v[8 * c + 5] = bf16hi(w.z);
-            v[8 * c + 6] = bf16lo(w.w);
-            v[8 * c + 7] = bf16hi(w.w);
+        for (int h = 0; h < 2; ++h) {
+            const int r = 2 * lane + h;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint4 w = *reinterpret_cast<const uint4 *>(st + r * 128 + ((c ^ (r & 7)) << 4));
+                v[32 * h + 4 * c + 0] = bf16x2_to_f2(w.x);
+                v[32 * h + 4 * c + 1] = bf16x2_to_f2(w.y);
+                v[32 * h + 4 * c + 2] = bf16x2_to_f2(w.z);
+                v[32 * h + 4 * c + 3] = bf16x2_to_f2(w.w);
+            }
         }
-        __syncthreads();
-        if (tid == 0) {
-            const int64_t tn = t + static_cast<int64_t>(QT_STAGES) * gridDim.x;
-            if (tn < ntiles) issue(tn, s);
+        __syncwarp();
+        if (lane == 0) {
+            const int64_t tn = t + static_cast<int64_t>(QT_STAGES) * QT_WARPS;
+            if (tn < t_end) issue(tn, s);
         }
 
-        const int64_t row = t * QT_TILE_ROWS + tid;
-        const bool valid = row < rows;
-        if (ROT) fwht128_pair(v, (tid & 1) != 0);
+        const int64_t row0 = t * QT_TILE_ROWS + 2 * lane;          // first 64-element row of the unit
+        const int64_t n_valid = imin<int64_t>(128, (rows - row0) * 64);
+        if (ROT) fwht128_packed(v);
         if (MODE == MODE_AMAX) {
-#pragma unroll
-            for (int i = 0; i < 64; ++i) tmax = fmaxf(tmax, fabsf(v[i]));
-        } else if (valid) {
-            const uint64_t e0 = p.e_base + static_cast<uint64_t>(row) * 64u;
-            UnitOut o;
-            quant_unit<FMT, SR, FOUR6>(v, e0, s_t, p.seed, o);
-            store_unit<G>(o, p, e0, 64);
+            tmax = fmaxf(tmax, absmax_pairs(v, 64));      // rows past the end were zero-filled by TMA
+        } else if (n_valid > 0) {
+            const uint64_t e0 = p.e_base + static_cast<uint64_t>(row0) * 64u;
+            Unit128 o;
+            quant_unit128<FMT, SR, FOUR6>(v, e0, s_t, p.seed, o);
+            store_unit128<G>(o, p, e0, n_valid);
         }
     }
     if (MODE == MODE_AMAX) {
         tmax = block_max(tmax, red);
-        if (tid == 0) p.partials_out[blockIdx.x] = tmax;
+        if (threadIdx.x == 0) p.partials_out[blockIdx.x] = tmax;
     }
 }
 
@@ -443,12 +589,12 @@ static int run_pass(const void *x, qfp4_dtype xdt, int64_t n, QuantParams p, cud
             CUtensorMap tm;
             const uint64_t dims[2] = {64, static_cast<uint64_t>(body / 64)};
             const uint64_t strides[1] = {128};
-            const uint32_t box[2] = {64, QT_BOX_ROWS};
+            const uint32_t box[2] = {64, QT_TILE_ROWS};
             int st = encode_tensor_map(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x), dims, strides,
                                        box, CU_TENSOR_MAP_SWIZZLE_128B);
             if (st != QFP4_OK) return st;
             const int64_t ntiles = (body / 64 + QT_TILE_ROWS - 1) / QT_TILE_ROWS;
-            const int grid = static_cast<int>(imin<int64_t>(ntiles, nsm));
+            const int grid = static_cast<int>(imin<int64_t>((ntiles + QT_WARPS - 1) / QT_WARPS, nsm));
             QuantParams q = p;
             q.n = body;
             q.partials_out = p.partials_out;

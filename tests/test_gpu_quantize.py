@@ -105,6 +105,33 @@ def test_degenerate_inputs():
     q.quantize(e, q.MXFP4)
 
 
+@pytest.mark.parametrize("rounding", [q.RNE, q.SR], ids=["rne", "sr"])
+def test_every_bf16_value_up_to_6(rounding):
+    """Every finite bf16 value with |x| <= 6 (both signs, zeros and subnormals)
+    goes through an MXFP4 group whose first element is 6.0, so k = 0 and the
+    code is the rounding of x itself: pins the E2M1 conversion, its ties and
+    the sign of zero on the GPU against the oracle."""
+    h = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    f = synth.bf16_bits_to_f32(h)
+    vals = h[np.isfinite(f) & (np.abs(f) <= 6.0)]
+    per = 31
+    n_groups = -(-len(vals) // per)
+    x = np.zeros((n_groups, 32), np.uint16)
+    x[:, 0] = 0x40C0                                    # 6.0
+    flat = np.zeros(n_groups * per, np.uint16)
+    flat[:len(vals)] = vals
+    x[:, 1:] = flat.reshape(n_groups, per)
+    rows = -(-n_groups // 4)
+    X = np.zeros((rows * 4, 32), np.uint16)
+    X[:n_groups] = x
+    X[n_groups:, 0] = 0x40C0
+    X = X.reshape(rows, 128)
+    got = q.quantize(to_dev(X), q.MXFP4, rounding, seed=77)
+    ref = oracle.quantize(X, oracle.MXFP4, rounding, seed=77)
+    assert (ref["scales"] == 127).all()
+    _cmp(got, ref)
+
+
 def test_large_dynamic_range():
     rng = np.random.default_rng(5)
     z = rng.standard_normal(64 * 512) * np.exp(rng.uniform(-60, 60, 64 * 512))
