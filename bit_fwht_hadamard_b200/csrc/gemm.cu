@@ -112,6 +112,25 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r)
           "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
 }
+// 16 lanes x 128 consecutive fp32 columns (16x256b shape, 16 repetitions):
+// thread t gets, for repetition j, columns 8j + 2(t%4) + {0,1} of lane
+// base + t/4 (r[4j], r[4j+1]) and of lane base + 8 + t/4 (r[4j+2], r[4j+3]).
+__device__ __forceinline__ void tmem_ld16x256b_x16(uint32_t taddr, uint32_t *r)
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
+        "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,"
+        "%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+          "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]),
+          "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]),
+          "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]),
+          "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]),
+          "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        : "r"(taddr));
+}
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // Ties registers filled by tcgen05.ld to a point after tcgen05.wait::ld, so
@@ -316,45 +335,46 @@ __global__ void __launch_bounds__(GM_THREADS, 1)
             tile_coords(t, p.tiles_m, p.tiles_n, mb, nb);
             if (!mbar_wait(&acc_full, ti & 1)) { abort_flag = 1; break; }
             tc_fence_after();
+            // two 16-lane halves of this warp's quadrant, 128 columns each
             uint32_t r[128];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + 128 * h + 32 * c, r + 32 * c);
+            for (int hh = 0; hh < 2; ++hh)
+                tmem_ld16x256b_x16(tmem + (static_cast<uint32_t>(32 * q + 16 * hh) << 16) + 128 * h, r + 64 * hh);
             tmem_ld_wait();
             reg_fence<128>(r);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty);
 
-            const int row = mb * GM_BM + 32 * q + lane;
-            const int col0 = nb * GM_BN + 128 * h;
-            if (row < p.M) {
-                if (OUT == QFP4_F32) {
-                    float *o = static_cast<float *>(p.out) + static_cast<int64_t>(row) * p.N + col0;
+            // r[64hh + 4j + {0,1}]: row 32q + 16hh + lane/4, columns 8j + 2(lane%4) + {0,1};
+            // r[64hh + 4j + {2,3}]: the row 8 below.  Four lanes cover 32 contiguous bytes.
+            const int col0 = nb * GM_BN + 128 * h + 2 * (lane & 3);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (col0 + 4 * j < p.N)
-                            reinterpret_cast<float4 *>(o)[j] =
-                                make_float4(__fmul_rn(__uint_as_float(r[4 * j]), alpha),
-                                            __fmul_rn(__uint_as_float(r[4 * j + 1]), alpha),
-                                            __fmul_rn(__uint_as_float(r[4 * j + 2]), alpha),
-                                            __fmul_rn(__uint_as_float(r[4 * j + 3]), alpha));
-                } else {
-                    uint16_t *o = static_cast<uint16_t *>(p.out) + static_cast<int64_t>(row) * p.N + col0;
+            for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        if (col0 + 8 * j < p.N) {
-                            uint32_t w[4];
+                for (int e = 0; e < 2; ++e) {
+                    const int row = mb * GM_BM + 32 * q + 16 * hh + 8 * e + (lane >> 2);
+                    if (row >= p.M) continue;
+                    if (OUT == QFP4_F32) {
+                        float *o = static_cast<float *>(p.out) + static_cast<int64_t>(row) * p.N + col0;
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const __nv_bfloat162 b2 = __floats2bfloat162_rn(
-                                    __fmul_rn(__uint_as_float(r[8 * j + 2 * e]), alpha),
-                                    __fmul_rn(__uint_as_float(r[8 * j + 2 * e + 1]), alpha));
-                                w[e] = *reinterpret_cast<const uint32_t *>(&b2);
+                        for (int j = 0; j < 16; ++j)
+                            if (col0 + 8 * j < p.N)
+                                *reinterpret_cast<float2 *>(o + 8 * j) =
+                                    make_float2(__fmul_rn(__uint_as_float(r[64 * hh + 4 * j + 2 * e]), alpha),
+                                                __fmul_rn(__uint_as_float(r[64 * hh + 4 * j + 2 * e + 1]), alpha));
+                    } else {
+                        uint16_t *o = static_cast<uint16_t *>(p.out) + static_cast<int64_t>(row) * p.N + col0;
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            if (col0 + 8 * j < p.N) {
+                                const __nv_bfloat162 b2 =
+                                    __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[64 * hh + 4 * j + 2 * e]), alpha),
+                                                          __fmul_rn(__uint_as_float(r[64 * hh + 4 * j + 2 * e + 1]), alpha));
+                                *reinterpret_cast<__nv_bfloat162 *>(o + 8 * j) = b2;
                             }
-                            reinterpret_cast<uint4 *>(o)[j] = make_uint4(w[0], w[1], w[2], w[3]);
-                        }
+                    }
                 }
-            }
         }
     }
 

@@ -23,13 +23,6 @@
 
 namespace qfp4 {
 
-constexpr int QT_WARPS = 8;                     // per CTA; one CTA per SM
-constexpr int QT_THREADS = 32 * QT_WARPS;
-constexpr int QT_TILE_ROWS = 64;                // 64 rows of 64 bf16 = one warp's tile (2 rows per lane)
-constexpr int QT_TILE_ELEMS = QT_TILE_ROWS * 64;
-constexpr int QT_STAGES = 3;                    // per warp
-constexpr int QT_STAGE_BYTES = QT_TILE_ROWS * 128;
-constexpr int QT_SMEM_BYTES = QT_WARPS * QT_STAGES * QT_STAGE_BYTES + 1024;
 
 // E2M1 code -> binary32 value (exact), from the bit fields.
 __device__ __forceinline__ float e2m1_value(uint32_t c)
@@ -250,22 +243,26 @@ __device__ __forceinline__ void store_unit(const UnitOut &o, const QuantParams &
     }
 }
 
-// ---------------------------------------------------------------- 128-element units (TMA kernel)
-// FWHT-128 of one unit held as packed pairs (pair k = elements 2k, 2k+1):
-// stage h = 1 inside each pair, stages h = 2..64 between pairs k and
-// k + h/2 as f32x2 add / sub, then one f32x2 multiply by 1/sqrt(128).
-__device__ __forceinline__ void fwht128_packed(uint64_t (&p)[64])
+// ---------------------------------------------------------------- packed units (TMA kernel)
+// A unit is UP packed binary32 pairs (pair k = elements 2k, 2k+1): UP = 64
+// holds a whole 128-element rotation block, UP = 32 holds half of one and
+// exchanges the h = 64 stage with its partner lane (lane ^ 1, the even lane
+// holding the lower half).  Stage h = 1 runs inside each pair; stages
+// h = 2 .. 2*UP between pairs k and k + h/2 as f32x2 add / sub; then one f32x2
+// multiply by 1/sqrt(128).
+template <int UP>
+__device__ __forceinline__ void fwht_packed(uint64_t (&p)[UP], bool upper)
 {
 #pragma unroll
-    for (int k = 0; k < 64; ++k) {
+    for (int k = 0; k < UP; ++k) {
         float a, b;
         f2unpack(p[k], a, b);
         p[k] = f2pack(__fadd_rn(a, b), __fsub_rn(a, b));
     }
 #pragma unroll
-    for (int hp = 1; hp < 64; hp <<= 1) {
+    for (int hp = 1; hp < UP; hp <<= 1) {
 #pragma unroll
-        for (int k = 0; k < 64; ++k) {
+        for (int k = 0; k < UP; ++k) {
             if ((k & hp) == 0) {
                 const uint64_t a = p[k], b = p[k + hp];
                 p[k] = f2add(a, b);
@@ -273,38 +270,57 @@ __device__ __forceinline__ void fwht128_packed(uint64_t (&p)[64])
             }
         }
     }
+    if (UP == 32) {
+        // h = 64 across the lane pair: lower gets mine + other, upper gets
+        // other - mine = other + (-mine) (negation is exact)
+        const uint64_t flip = upper ? 0x8000000080000000ull : 0ull;
+#pragma unroll
+        for (int k = 0; k < UP; ++k) {
+            const uint32_t lo = __shfl_xor_sync(0xFFFFFFFFu, static_cast<uint32_t>(p[k]), 1);
+            const uint32_t hi = __shfl_xor_sync(0xFFFFFFFFu, static_cast<uint32_t>(p[k] >> 32), 1);
+            p[k] = f2add((static_cast<uint64_t>(hi) << 32) | lo, p[k] ^ flip);
+        }
+    }
     const uint64_t c2 = f2pack(inv_sqrt128(), inv_sqrt128());
 #pragma unroll
-    for (int k = 0; k < 64; ++k) p[k] = f2mul(p[k], c2);
+    for (int k = 0; k < UP; ++k) p[k] = f2mul(p[k], c2);
 }
 
-__device__ __forceinline__ float absmax_pairs(const uint64_t *p, int n)
+// max |x| over n packed pairs, as a balanced tree
+template <int N>
+__device__ __forceinline__ float absmax_pairs(const uint64_t *p)
 {
-    float m = 0.0f;
+    float m[N];
 #pragma unroll
-    for (int j = 0; j < n; ++j) {
+    for (int j = 0; j < N; ++j) {
         float a, b;
         f2unpack(p[j], a, b);
-        m = fmaxf(m, fmaxf(fabsf(a), fabsf(b)));
+        m[j] = fmaxf(fabsf(a), fabsf(b));
     }
-    return m;
+#pragma unroll
+    for (int h = N / 2; h >= 1; h >>= 1)
+#pragma unroll
+        for (int j = 0; j < h; ++j) m[j] = fmaxf(m[j], m[j + h]);
+    return m[0];
 }
 
-struct Unit128 {
-    uint32_t codes[16];     // 128 nibbles
-    uint32_t scales[2];     // up to 8 scale bytes
+template <int UP>
+struct UnitP {
+    uint32_t codes[UP / 4];     // 2*UP nibbles
+    uint32_t scales[2];         // up to 8 scale bytes
 };
 
-template <int FMT, bool SR, bool FOUR6>
-__device__ __forceinline__ void quant_unit128(uint64_t (&p)[64], uint64_t e0, float s_t, uint64_t seed, Unit128 &o)
+template <int UP, int FMT, bool SR, bool FOUR6>
+__device__ __forceinline__ void quant_unit_packed(uint64_t (&p)[UP], uint64_t e0, float s_t, uint64_t seed,
+                                                  UnitP<UP> &o)
 {
     o.scales[0] = o.scales[1] = 0u;
     if (FMT == QFP4_MXFP4) {
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
+        for (int g = 0; g < UP / 16; ++g) {
             uint64_t *pg = p + 16 * g;
             uint32_t *w = o.codes + 4 * g;
-            const float amax = absmax_pairs(pg, 16);
+            const float amax = absmax_pairs<16>(pg);
             if (amax == 0.0f) {                      // all-zero group: byte 0, +0 codes
                 w[0] = w[1] = w[2] = w[3] = 0u;
                 continue;
@@ -326,13 +342,11 @@ __device__ __forceinline__ void quant_unit128(uint64_t (&p)[64], uint64_t e0, fl
         }
     } else {
 #pragma unroll
-        for (int b = 0; b < 8; ++b) {
+        for (int b = 0; b < UP / 8; ++b) {
             float x[16];
 #pragma unroll
             for (int j = 0; j < 8; ++j) f2unpack(p[8 * b + j], x[2 * j], x[2 * j + 1]);
-            float amax = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
+            const float amax = absmax_pairs<8>(p + 8 * b);
             uint32_t *w = o.codes + 2 * b;
             uint32_t enc = 0u;
             float S = 0.0f;
@@ -370,39 +384,41 @@ __device__ __forceinline__ void quant_unit128(uint64_t (&p)[64], uint64_t e0, fl
     }
 }
 
-template <int G>
-__device__ __forceinline__ void store_unit128(const Unit128 &o, const QuantParams &p, uint64_t e0, int64_t n_valid)
+template <int UP, int G>
+__device__ __forceinline__ void store_unit_packed(const UnitP<UP> &o, const QuantParams &p, uint64_t e0,
+                                                  int64_t n_valid)
 {
-    // n_valid: 128, or 64 when the launch range ends half way through the unit
+    // n_valid: 2*UP, or 64 when the launch range ends half way through a 128-element unit
     uint4 *c4 = reinterpret_cast<uint4 *>(p.codes + (e0 >> 1));
     uint8_t *sdst = p.scales + e0 / G;
-    c4[0] = make_uint4(o.codes[0], o.codes[1], o.codes[2], o.codes[3]);
-    c4[1] = make_uint4(o.codes[4], o.codes[5], o.codes[6], o.codes[7]);
-    if (n_valid >= 128) {
-        c4[2] = make_uint4(o.codes[8], o.codes[9], o.codes[10], o.codes[11]);
-        c4[3] = make_uint4(o.codes[12], o.codes[13], o.codes[14], o.codes[15]);
-    }
-    if (G == 32) {
-        if (n_valid >= 128) *reinterpret_cast<uint32_t *>(sdst) = o.scales[0];
-        else *reinterpret_cast<uint16_t *>(sdst) = static_cast<uint16_t>(o.scales[0]);
-    } else {
-        if (n_valid >= 128) *reinterpret_cast<uint2 *>(sdst) = make_uint2(o.scales[0], o.scales[1]);
-        else *reinterpret_cast<uint32_t *>(sdst) = o.scales[0];
-    }
+    const bool full = n_valid >= 2 * UP;
+#pragma unroll
+    for (int c = 0; c < UP / 16; ++c)
+        if (full || c < 2) c4[c] = make_uint4(o.codes[4 * c], o.codes[4 * c + 1], o.codes[4 * c + 2], o.codes[4 * c + 3]);
+    constexpr int nsb = 2 * UP / G;                   // scale bytes of a full unit: 2, 4 or 8
+    const int nb = full ? nsb : 64 / G;
+    if (nb == 8) *reinterpret_cast<uint2 *>(sdst) = make_uint2(o.scales[0], o.scales[1]);
+    else if (nb == 4) *reinterpret_cast<uint32_t *>(sdst) = o.scales[0];
+    else *reinterpret_cast<uint16_t *>(sdst) = static_cast<uint16_t>(o.scales[0]);
 }
 
 // ---------------------------------------------------------------- TMA kernel
-template <int MODE, int FMT, bool ROT, bool SR, bool FOUR6>
-__global__ void __launch_bounds__(QT_THREADS, 1) k_quant1d_tma(const __grid_constant__ CUtensorMap tm, QuantParams p)
+// WARPS warps per CTA (one CTA per SM), each with a STAGES-deep ring of tiles
+// of 32 * (UP / 32) ... = UP rows of 64 bf16 (one unit of UP pairs per lane).
+template <int MODE, int FMT, bool ROT, bool SR, bool FOUR6, int WARPS, int STAGES, int UP>
+__global__ void __launch_bounds__(32 * WARPS, 1) k_quant1d_tma(const __grid_constant__ CUtensorMap tm, QuantParams p)
 {
+    constexpr int ROWS_PER_LANE = UP / 32;             // 64-element rows per unit
+    constexpr int TILE_ROWS = 32 * ROWS_PER_LANE;
+    constexpr int STAGE_BYTES = TILE_ROWS * 128;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ __align__(8) uint64_t full[QT_WARPS][QT_STAGES];
+    __shared__ __align__(8) uint64_t full[WARPS][STAGES];
     __shared__ float red[32];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t rows = p.n / 64;
-    const int64_t ntiles = (rows + QT_TILE_ROWS - 1) / QT_TILE_ROWS;
+    const int64_t ntiles = (rows + TILE_ROWS - 1) / TILE_ROWS;
     // contiguous tile range of this CTA, balanced to one tile
     const int64_t t_begin = ntiles * blockIdx.x / gridDim.x, t_end = ntiles * (blockIdx.x + 1) / gridDim.x;
     constexpr int G = FMT == QFP4_MXFP4 ? 32 : 16;
@@ -413,38 +429,38 @@ __global__ void __launch_bounds__(QT_THREADS, 1) k_quant1d_tma(const __grid_cons
         if (p.write_tscale && blockIdx.x == 0 && threadIdx.x == 0) *p.tscale_out = s_t;
     }
     uint64_t *bars = full[warp];
-    uint8_t *ring = smem + warp * (QT_STAGES * QT_STAGE_BYTES);
+    uint8_t *ring = smem + warp * (STAGES * STAGE_BYTES);
     if (lane == 0) {
-        for (int s = 0; s < QT_STAGES; ++s) mbar_init(&bars[s], 1);
+        for (int s = 0; s < STAGES; ++s) mbar_init(&bars[s], 1);
         fence_mbar_init();
         if (warp == 0) prefetch_tensormap(&tm);
     }
     __syncwarp();
 
     auto issue = [&](int64_t t, int s) {
-        mbar_arrive_expect_tx(&bars[s], QT_STAGE_BYTES);
-        tma_load_2d(ring + s * QT_STAGE_BYTES, &tm, &bars[s], 0, static_cast<int>(t * QT_TILE_ROWS));
+        mbar_arrive_expect_tx(&bars[s], STAGE_BYTES);
+        tma_load_2d(ring + s * STAGE_BYTES, &tm, &bars[s], 0, static_cast<int>(t * TILE_ROWS));
     };
     if (lane == 0)
-        for (int s = 0; s < QT_STAGES; ++s) {
-            const int64_t t = t_begin + warp + static_cast<int64_t>(s) * QT_WARPS;
+        for (int s = 0; s < STAGES; ++s) {
+            const int64_t t = t_begin + warp + static_cast<int64_t>(s) * WARPS;
             if (t < t_end) issue(t, s);
         }
 
     float tmax = 0.0f;
     int it = 0;
-    for (int64_t t = t_begin + warp; t < t_end; t += QT_WARPS, ++it) {
-        const int s = it % QT_STAGES;
-        const uint32_t ph = (it / QT_STAGES) & 1u;
+    for (int64_t t = t_begin + warp; t < t_end; t += WARPS, ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1u;
         const bool ok = mbar_wait(&bars[s], ph);
         if (__any_sync(0xFFFFFFFFu, !ok)) break;
 
-        // this lane's unit: rows 2*lane and 2*lane+1 of the tile (128-byte swizzle)
-        const uint8_t *st = ring + s * QT_STAGE_BYTES;
-        uint64_t v[64];
+        // this lane's unit: rows ROWS_PER_LANE*lane + h of the tile (128-byte swizzle)
+        const uint8_t *st = ring + s * STAGE_BYTES;
+        uint64_t v[UP];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int r = 2 * lane + h;
+        for (int h = 0; h < ROWS_PER_LANE; ++h) {
+            const int r = ROWS_PER_LANE * lane + h;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
                 const uint4 w = *reinterpret_cast<const uint4 *>(st + r * 128 + ((c ^ (r & 7)) << 4));
@@ -456,20 +472,20 @@ __global__ void __launch_bounds__(QT_THREADS, 1) k_quant1d_tma(const __grid_cons
         }
         __syncwarp();
         if (lane == 0) {
-            const int64_t tn = t + static_cast<int64_t>(QT_STAGES) * QT_WARPS;
+            const int64_t tn = t + static_cast<int64_t>(STAGES) * WARPS;
             if (tn < t_end) issue(tn, s);
         }
 
-        const int64_t row0 = t * QT_TILE_ROWS + 2 * lane;          // first 64-element row of the unit
-        const int64_t n_valid = imin<int64_t>(128, (rows - row0) * 64);
-        if (ROT) fwht128_packed(v);
+        const int64_t row0 = t * TILE_ROWS + ROWS_PER_LANE * lane;   // first 64-element row of the unit
+        const int64_t n_valid = imin<int64_t>(2 * UP, (rows - row0) * 64);
+        if (ROT) fwht_packed<UP>(v, (lane & 1) != 0);
         if (MODE == MODE_AMAX) {
-            tmax = fmaxf(tmax, absmax_pairs(v, 64));      // rows past the end were zero-filled by TMA
+            tmax = fmaxf(tmax, absmax_pairs<UP>(v));   // rows past the end were zero-filled by TMA
         } else if (n_valid > 0) {
             const uint64_t e0 = p.e_base + static_cast<uint64_t>(row0) * 64u;
-            Unit128 o;
-            quant_unit128<FMT, SR, FOUR6>(v, e0, s_t, p.seed, o);
-            store_unit128<G>(o, p, e0, n_valid);
+            UnitP<UP> o;
+            quant_unit_packed<UP, FMT, SR, FOUR6>(v, e0, s_t, p.seed, o);
+            store_unit_packed<UP, G>(o, p, e0, n_valid);
         }
     }
     if (MODE == MODE_AMAX) {
@@ -477,6 +493,11 @@ __global__ void __launch_bounds__(QT_THREADS, 1) k_quant1d_tma(const __grid_cons
         if (threadIdx.x == 0) p.partials_out[blockIdx.x] = tmax;
     }
 }
+
+// Production configuration of the TMA kernel.
+constexpr int QT_WARPS = 16, QT_STAGES = 2, QT_UP = 32;
+constexpr int QT_TILE_ROWS = QT_UP;
+constexpr int QT_SMEM_BYTES = QT_WARPS * QT_STAGES * QT_UP * 128 + 1024;
 
 // ---------------------------------------------------------------- direct kernel
 // Loads straight from global memory (bf16 or binary32), one unit per thread;
@@ -553,14 +574,14 @@ static int smem_configured[2][2][2][2][2] = {};
 template <int MODE, int FMT, bool ROT, bool SR, bool FOUR6>
 static int launch_tma(const CUtensorMap &tm, const QuantParams &p, int grid, cudaStream_t stream)
 {
-    auto kern = k_quant1d_tma<MODE, FMT, ROT, SR, FOUR6>;
+    auto kern = k_quant1d_tma<MODE, FMT, ROT, SR, FOUR6, QT_WARPS, QT_STAGES, QT_UP>;
     int &done = smem_configured[MODE][FMT][ROT][SR][FOUR6];
     if (!done) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, QT_SMEM_BYTES) != cudaSuccess)
             return QFP4_ERR_CUDA;
         done = 1;
     }
-    kern<<<grid, QT_THREADS, QT_SMEM_BYTES, stream>>>(tm, p);
+    kern<<<grid, 32 * QT_WARPS, QT_SMEM_BYTES, stream>>>(tm, p);
     QFP4_LAUNCH_CHECK();
     return QFP4_OK;
 }
