@@ -177,6 +177,13 @@ __host__ __device__ constexpr uint32_t idesc_blockscaled(int fmt, int M, int N, 
            ((fmt == QFP4_NVFP4 ? 0u : 1u) << 23) | (static_cast<uint32_t>(M >> 4) << 24) | (sf_id << 29);
 }
 
+// wait of a whole warp before a .sync.aligned tcgen05 instruction: either
+// every lane saw the phase complete or every lane gives up
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity)
+{
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity)) != 0;
+}
+
 __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int &mb, int &nb)
 {
     const int per_group = GM_GROUP_M * tiles_n;
@@ -189,30 +196,56 @@ __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int
 }
 
 // ------------------------------------------------------------------ scale prepass
-// One thread per 16-byte line of a chunk: rows rb*128 + r0 + 32*rr (rr = 0..3),
-// scale groups c*4 + j (j = 0..3); zero beyond R rows or Kg groups.
-__global__ void __launch_bounds__(256) k_sf_rearrange(const uint8_t *__restrict__ sc, int R, int Kg, int NC,
-                                                      int n_lines, uint8_t *__restrict__ dst)
+// The GEMM reads scales in 512-byte chunks, one per (128-row block rb, group
+// of four scale columns c), chunk index rb * NC + c: byte (r % 32) * 16 +
+// (r / 32) * 4 + j holds the scale of row rb * 128 + r, column 4c + j; zero
+// beyond R rows or Kg columns.  A block takes one 128-row block and eight
+// chunks: it reads the 128 x 32 scale bytes row by row (16-byte loads where
+// the rows allow them) into shared memory and writes the eight chunks, 4 KiB
+// that are contiguous in the output, as 16-byte stores.  Both operands go in
+// one launch: blockIdx.y runs over A's row blocks, then B's.
+struct SfJob {
+    const uint8_t *sc;
+    int R, nblk;
+    uint8_t *dst;
+};
+constexpr int SF_CHUNKS_PER_BLOCK = 8;
+
+__global__ void __launch_bounds__(256) k_sf_chunks(SfJob ja, SfJob jb, int Kg, int NC)
 {
-    const int line = blockIdx.x * blockDim.x + threadIdx.x;
-    if (line >= n_lines) return;
-    const int r0 = line & 31;
-    const int chunk = line >> 5;
-    const int c = chunk % NC, rb = chunk / NC;
-    uint32_t w[4];
-#pragma unroll
-    for (int rr = 0; rr < 4; ++rr) {
-        const int row = rb * 128 + r0 + 32 * rr;
-        uint32_t v = 0;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int grp = c * 4 + j;
-            const uint32_t b = (row < R && grp < Kg) ? sc[static_cast<int64_t>(row) * Kg + grp] : 0u;
-            v |= b << (8 * j);
+    __shared__ uint32_t tile[128 * 9];                    // 128 rows x 32 bytes, row stride 36 bytes
+    const bool is_a = static_cast<int>(blockIdx.y) < ja.nblk;
+    const SfJob j = is_a ? ja : jb;
+    const int rb = is_a ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.y) - ja.nblk;
+    const int c0 = static_cast<int>(blockIdx.x) * SF_CHUNKS_PER_BLOCK;
+    const int t = threadIdx.x;
+    {
+        const int row = t >> 1, gs = 4 * c0 + 16 * (t & 1);
+        const int64_t grow = static_cast<int64_t>(rb) * 128 + row;
+        uint32_t w[4] = {0u, 0u, 0u, 0u};
+        if (grow < j.R) {
+            const uint8_t *src = j.sc + grow * Kg + gs;
+            if (gs + 16 <= Kg && (reinterpret_cast<uintptr_t>(src) & 15u) == 0) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(src);
+                w[0] = v.x;
+                w[1] = v.y;
+                w[2] = v.z;
+                w[3] = v.w;
+            } else {
+                for (int i = 0; i < 16; ++i)
+                    if (gs + i < Kg) w[i >> 2] |= static_cast<uint32_t>(src[i]) << (8 * (i & 3));
+            }
         }
-        w[rr] = v;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) tile[row * 9 + 4 * (t & 1) + i] = w[i];
     }
-    *reinterpret_cast<uint4 *>(dst + static_cast<int64_t>(line) * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    __syncthreads();
+    const int ci = t >> 5, r0 = t & 31;
+    if (c0 + ci < NC) {
+        const uint4 o = make_uint4(tile[r0 * 9 + ci], tile[(r0 + 32) * 9 + ci], tile[(r0 + 64) * 9 + ci],
+                                   tile[(r0 + 96) * 9 + ci]);
+        *reinterpret_cast<uint4 *>(j.dst + (static_cast<int64_t>(rb) * NC + c0 + ci) * 512 + r0 * 16) = o;
+    }
 }
 
 // ------------------------------------------------------------------ main kernel
@@ -222,7 +255,7 @@ __global__ void __launch_bounds__(GM_THREADS, 1)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ __align__(8) uint64_t full[GM_STAGES], empty[GM_STAGES], acc_full, acc_empty;
+    __shared__ __align__(8) uint64_t full[GM_STAGES], empty[GM_STAGES], acc_full, acc_empty, drain;
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile int abort_flag;
 
@@ -237,6 +270,7 @@ __global__ void __launch_bounds__(GM_THREADS, 1)
         }
         mbar_init(&acc_full, 1);
         mbar_init(&acc_empty, GM_EPI_WARPS);
+        mbar_init(&drain, 1);
         abort_flag = 0;
         fence_mbar_init();
         prefetch_tensormap(&tmA);
@@ -279,6 +313,7 @@ __global__ void __launch_bounds__(GM_THREADS, 1)
                     bulk_g2s(stage_sfb(s) + CPS * 512, p.sfb + cb1, CPS * 512, &full[s]);
                 }
             }
+            if (abort_flag) settle_ns(kSettleNs);   // loads already issued may still be landing
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
@@ -322,6 +357,9 @@ __global__ void __launch_bounds__(GM_THREADS, 1)
                 }
                 umma_commit(&acc_full);
             }
+            // every MMA and scale copy this thread issued has finished before the CTA can leave
+            umma_commit(&drain);
+            if (!mbar_wait(&drain, 0)) abort_flag = 1;
         }
     } else {
         // ------------------------------------------------ epilogue
@@ -333,7 +371,7 @@ __global__ void __launch_bounds__(GM_THREADS, 1)
         for (int t = blockIdx.x; t < ntiles && !abort_flag; t += gridDim.x, ++ti) {
             int mb, nb;
             tile_coords(t, p.tiles_m, p.tiles_n, mb, nb);
-            if (!mbar_wait(&acc_full, ti & 1)) { abort_flag = 1; break; }
+            if (!warp_wait(&acc_full, ti & 1)) { abort_flag = 1; break; }
             tc_fence_after();
             // two 16-lane halves of this warp's quadrant, 128 columns each
             uint32_t r[128];
@@ -384,6 +422,420 @@ __global__ void __launch_bounds__(GM_THREADS, 1)
     if (warp == 1) tmem_dealloc(tmem, GM_TMEM_COLS);
 }
 
+// ------------------------------------------------------------------ 2-CTA kernel
+// A cluster of two CTAs on two SMs computes a 256 x 256 tile with
+// tcgen05.mma.cta_group::2 (M = 256: each CTA holds 128 rows of A and of the
+// accumulator, and half (128 rows) of the tile's B, which the pair shares).
+// Each CTA loads its A half and B half with cta_group::2 TMA loads that
+// complete on the leader CTA's barrier; the leader alone issues the MMAs and
+// its commits arrive in both CTAs.  Compared with the 1-CTA tile each SM
+// stages 38 KiB instead of 54 KiB per k-tile and issues half the MMAs per unit
+// of work.
+//
+// Scale factors do not go through tcgen05.cp: every copy instruction costs
+// about as much issue time as an MMA of a quarter k-tile, and the twelve an
+// NVFP4 k-tile needs would cap the tensor pipe near 60 %.  Instead a second
+// producer thread loads each k-tile's scale chunks (plain TMA into this CTA's
+// own ring of scale slots, which runs ahead of the operand stages) and four
+// scale warps (one per TMEM lane quadrant) write them into a ring of TMEM
+// buffers with tcgen05.st, concurrently with the MMAs.  The MMA for rows in
+// quadrant q reads the A scale of row r at lane r, column addr + q and the
+// B scale of column n at lane (n mod 32) + 32 q, column addr + n / 32, and
+// the MMA takes scale addresses on 4-column (A) and 8-column (B) boundaries:
+//   A: lane r, columns bufA + 4 w + (0..3) = scale word w of row r
+//   B: lane l + 32 q, column bufB + 8 w + m = scale word w of column l + 32 m
+// A k-tile takes 4 CPS columns of A scales and 8 CPS of B scales; the 256
+// columns after the accumulator hold g2_sf_bufs(FMT) such buffers (B buffers
+// first, then A), which is how far the scale warps may run ahead of the MMAs.
+// (word w holds the four scales of k-groups 4w .. 4w + 3 of the k-tile; only
+// column bufA + 4 w + q of a quadrant-q lane is read, the other three hold
+// copies so that one store writes a quadrant's A scales).  Every store starts
+// on a multiple of its own width.
+// No TMA multicast.
+constexpr int G2_BM = 256, G2_BN = 256;                   // cluster tile
+// warp roles by warpgroup: 0 operand producer, 1 MMA issuer, 2 scale producer
+// (3 idle); 4..7 scale warps; 8..15 epilogue.  setmaxnreg moves registers from the first two
+// warpgroups to the epilogue: 128 x 48 + 128 x 80 + 256 x 184 = 63488 of the
+// 512 x 128 = 65536 the block is launched with.
+constexpr int G2_SF_WARPS = 4;
+constexpr int G2_THREADS = 512;
+constexpr int G2_SF_WARP0 = 4, G2_EPI_WARP0 = 8;
+constexpr int G2_A_BYTES = 128 * GM_BKB;                  // this CTA's A rows
+constexpr int G2_B_BYTES = 128 * GM_BKB;                  // this CTA's half of B
+constexpr int G2_STAGE_BYTES = G2_A_BYTES + G2_B_BYTES;
+constexpr int G2_STAGES = 6;
+constexpr int G2_SF_SLOT_BYTES = 12 * 512;                // A: CPS chunks, B: 2 x CPS chunks (CPS <= 4)
+constexpr int G2_SF_SLOTS = 5;
+constexpr int G2_SMEM = G2_STAGES * G2_STAGE_BYTES + G2_SF_SLOTS * G2_SF_SLOT_BYTES + 1024;
+__host__ __device__ constexpr int g2_sf_bufs(int fmt) { return fmt == QFP4_NVFP4 ? 5 : 10; }
+constexpr int G2_SF_BUFS_MAX = 10;
+static_assert(256 + g2_sf_bufs(QFP4_NVFP4) * 12 * 4 <= GM_TMEM_COLS, "TMEM columns (NVFP4)");
+static_assert(256 + g2_sf_bufs(QFP4_MXFP4) * 12 * 2 <= GM_TMEM_COLS, "TMEM columns (MXFP4)");
+
+__device__ __forceinline__ uint32_t cluster_ctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// shared::cluster address of the same shared variable in CTA `rank`
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// arrive on a barrier given by its shared::cluster address (this CTA's or the
+// partner's).  Default semantics (release at CTA scope): what the arrival
+// publishes is tensor-memory state that tcgen05.wait + tcgen05.fence already
+// made complete, so no cluster-wide memory fence is needed, and one per
+// k-tile would stall the scale warps.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
+{
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ void tma_load_2d_cg2(void *smem_dst, const CUtensorMap *map, uint32_t leader_bar, int c0, int c1)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+        "[%2];" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_bar), "r"(c0), "r"(c1)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_cg2(uint32_t *dst, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_cg2()
+{
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_cg2(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// arrive on `bar` (same offset) in both CTAs once this thread's tcgen05 work completes
+__device__ __forceinline__ void umma_commit_cg2_both(uint64_t *bar)
+{
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"(static_cast<uint16_t>(3))
+        : "memory");
+}
+template <int FMT>
+__device__ __forceinline__ void umma_blockscaled_cg2(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa,
+                                                     uint32_t sfb, uint32_t accumulate)
+{
+    if (FMT == QFP4_NVFP4)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+            "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+            : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+            "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+            : "memory");
+}
+
+#define QFP4_R8(b) "r"(v[b]), "r"(v[b + 1]), "r"(v[b + 2]), "r"(v[b + 3]), "r"(v[b + 4]), "r"(v[b + 5]), "r"(v[b + 6]), "r"(v[b + 7])
+__device__ __forceinline__ void tmem_st_x8(uint32_t taddr, const uint32_t *v)
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr), QFP4_R8(0)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t *v)
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+                 "%14, %15, %16};" ::"r"(taddr),
+                 QFP4_R8(0), QFP4_R8(8)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t *v)
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+                 "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
+                     taddr),
+                 QFP4_R8(0), QFP4_R8(8), QFP4_R8(16), QFP4_R8(24)
+                 : "memory");
+}
+#undef QFP4_R8
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// end of every role of the 2-CTA kernel: no CTA leaves while its partner may
+// still signal it; the allocating warp then frees the pair's tensor memory
+__device__ __forceinline__ void g2_exit(uint32_t tmem, bool dealloc)
+{
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    if (dealloc) tmem_dealloc_cg2(tmem, GM_TMEM_COLS);
+}
+
+template <int FMT, int OUT>
+__global__ void __launch_bounds__(G2_THREADS, 1)
+    k_gemm_bs2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB, GemmParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ __align__(8) uint64_t full[G2_STAGES], empty[G2_STAGES], sfs_full[G2_SF_SLOTS], sfs_empty[G2_SF_SLOTS];
+    __shared__ __align__(8) uint64_t sf_full[G2_SF_BUFS_MAX], sf_empty[G2_SF_BUFS_MAX], acc_full, acc_empty, drain;
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ volatile int abort_flag;
+
+    constexpr int CPS = gm_cps(FMT);
+    constexpr int NBUF = g2_sf_bufs(FMT);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+    const int tiles_m = (p.M + G2_BM - 1) / G2_BM, tiles_n = (p.N + G2_BN - 1) / G2_BN;
+    const int ntiles = tiles_m * tiles_n;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < G2_STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int s = 0; s < G2_SF_SLOTS; ++s) {
+            mbar_init(&sfs_full[s], 1);
+            mbar_init(&sfs_empty[s], G2_SF_WARPS);
+        }
+        for (int b = 0; b < NBUF; ++b) {
+            mbar_init(&sf_full[b], 2 * G2_SF_WARPS);
+            mbar_init(&sf_empty[b], 1);
+        }
+        mbar_init(&acc_full, 1);
+        mbar_init(&acc_empty, 2 * GM_EPI_WARPS);
+        mbar_init(&drain, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tensormap(&tmA);
+        prefetch_tensormap(&tmB);
+        prefetch_tensormap(&tmSA);
+        prefetch_tensormap(&tmSB);
+    }
+    if (warp == 1) {
+        tmem_alloc_cg2(&tmem_base_sh, GM_TMEM_COLS);
+        tmem_relinquish_cg2();
+    }
+    tc_fence_before();
+    cluster_sync();                          // barriers of both CTAs initialised before any remote use
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_sh;
+
+    auto stage_a = [&](int s) { return smem + s * G2_STAGE_BYTES; };
+    auto stage_b = [&](int s) { return smem + s * G2_STAGE_BYTES + G2_A_BYTES; };
+    auto slot_sfa = [&](int s) { return smem + G2_STAGES * G2_STAGE_BYTES + s * G2_SF_SLOT_BYTES; };
+    auto slot_sfb = [&](int s) { return slot_sfa(s) + CPS * 512; };
+    auto buf_b = [&](int b) { return tmem + 256 + b * (8 * CPS); };
+    auto buf_a = [&](int b) { return tmem + 256 + NBUF * (8 * CPS) + b * (4 * CPS); };
+
+    // Each role ends with its own copy of the exit sequence, so that the
+    // register-count regions set by setmaxnreg never merge again.
+    if (warp < G2_SF_WARP0) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 48;");
+        if (warp == 0) {
+        // ------------------------------------------------ producer (both CTAs)
+        if (lane == 0) {
+            const uint32_t ab_bytes = G2_A_BYTES + G2_B_BYTES;
+            int it = 0;
+            for (int t = cluster; t < ntiles && !abort_flag; t += nclusters) {
+                int mb, nb;
+                tile_coords(t, tiles_m, tiles_n, mb, nb);
+                const int rb_a = 2 * mb + static_cast<int>(rank);   // this CTA's 128-row block of A
+                for (int kt = 0; kt < p.KT; ++kt, ++it) {
+                    const int s = it % G2_STAGES;
+                    const uint32_t ph = (it / G2_STAGES) & 1u;
+                    if (!mbar_wait(&empty[s], ph ^ 1u)) { abort_flag = 1; break; }
+                    const uint32_t lbar = mapa_shared(smem_u32(&full[s]), 0);
+                    if (leader) mbar_arrive_expect_tx(&full[s], 2 * ab_bytes);
+                    tma_load_2d_cg2(stage_a(s), &tmA, lbar, kt * GM_BKB, rb_a * 128);
+                    tma_load_2d_cg2(stage_b(s), &tmB, lbar, kt * GM_BKB, nb * G2_BN + 128 * static_cast<int>(rank));
+                }
+            }
+            // wait until the leader's commits have released every stage, so no
+            // arrival is still on its way to this CTA when it leaves
+            for (int i = 0; i < G2_STAGES && !abort_flag; ++i, ++it)
+                if (!mbar_wait(&empty[it % G2_STAGES], ((it / G2_STAGES) & 1u) ^ 1u)) abort_flag = 1;
+            if (abort_flag) settle_ns(kSettleNs);   // loads already issued may still be landing
+        }
+        } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer (leader CTA only)
+        if (leader && lane == 0) {
+            int it = 0, ti = 0;
+            for (int t = cluster; t < ntiles && !abort_flag; t += nclusters, ++ti) {
+                if (!mbar_wait(&acc_empty, (ti & 1) ^ 1u)) { abort_flag = 1; break; }
+                tc_fence_after();
+                for (int kt = 0; kt < p.KT; ++kt, ++it) {
+                    const int s = it % G2_STAGES, b = it % NBUF;
+                    if (!mbar_wait(&full[s], (it / G2_STAGES) & 1u)) { abort_flag = 1; break; }
+                    if (!mbar_wait(&sf_full[b], (it / NBUF) & 1u)) { abort_flag = 1; break; }
+                    tc_fence_after();
+                    const uint64_t adesc = desc_k_sw128(stage_a(s));
+                    const uint64_t bdesc = desc_k_sw128(stage_b(s));
+#pragma unroll
+                    for (int k = 0; k < GM_BK / 64; ++k) {
+                        uint32_t sfa, sfb, id;
+                        if (FMT == QFP4_NVFP4) {
+                            sfa = buf_a(b) + 4 * k;
+                            sfb = buf_b(b) + 8 * k;
+                            id = idesc_blockscaled(FMT, G2_BM, G2_BN, 0);
+                        } else {
+                            const uint32_t sel = 2u * (k & 1);
+                            sfa = (buf_a(b) + 4 * (k >> 1)) | (sel << 30);
+                            sfb = (buf_b(b) + 8 * (k >> 1)) | (sel << 30);
+                            id = idesc_blockscaled(FMT, G2_BM, G2_BN, sel);
+                        }
+                        umma_blockscaled_cg2<FMT>(tmem, adesc + 2 * k, bdesc + 2 * k, id, sfa, sfb, (kt | k) != 0);
+                    }
+                    umma_commit_cg2_both(&empty[s]);
+                    umma_commit_cg2_both(&sf_empty[b]);
+                }
+                umma_commit_cg2_both(&acc_full);
+            }
+            // every MMA this thread issued has finished before either CTA can leave
+            umma_commit_cg2_both(&drain);
+            if (!mbar_wait(&drain, 0)) abort_flag = 1;
+        }
+        } else if (warp == 2) {
+        // ------------------------------------------------ scale producer (both CTAs)
+        if (lane == 0) {
+            int it = 0;
+            for (int t = cluster; t < ntiles && !abort_flag; t += nclusters) {
+                int mb, nb;
+                tile_coords(t, tiles_m, tiles_n, mb, nb);
+                const int rb_a = 2 * mb + static_cast<int>(rank);
+                for (int kt = 0; kt < p.KT; ++kt, ++it) {
+                    const int s = it % G2_SF_SLOTS;
+                    if (!mbar_wait(&sfs_empty[s], ((it / G2_SF_SLOTS) & 1u) ^ 1u)) { abort_flag = 1; break; }
+                    // scale chunks (rows of 128 B, 4 per 512-byte chunk, CPS chunks per k-tile)
+                    mbar_arrive_expect_tx(&sfs_full[s], 3 * CPS * 512);
+                    tma_load_2d(slot_sfa(s), &tmSA, &sfs_full[s], 0, (rb_a * p.NC + kt * CPS) * 4);
+                    tma_load_2d(slot_sfb(s), &tmSB, &sfs_full[s], 0, ((2 * nb) * p.NC + kt * CPS) * 4);
+                    tma_load_2d(slot_sfb(s) + CPS * 512, &tmSB, &sfs_full[s], 0, ((2 * nb + 1) * p.NC + kt * CPS) * 4);
+                }
+            }
+            if (abort_flag) settle_ns(kSettleNs);   // loads already issued may still be landing
+        }
+        }
+        g2_exit(tmem, warp == 1);
+        return;
+    }
+    if (warp < G2_EPI_WARP0) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 80;");
+        // ------------------------------------------------ scale warps (both CTAs: own TMEM quadrant)
+        const int q = warp & 3;
+        const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
+        int it = 0;
+        for (int t = cluster; t < ntiles && !abort_flag; t += nclusters) {
+            for (int kt = 0; kt < p.KT; ++kt, ++it) {
+                const int s = it % G2_SF_SLOTS, b = it % NBUF;
+                if (!warp_wait(&sfs_full[s], (it / G2_SF_SLOTS) & 1u)) { abort_flag = 1; break; }
+                if (!warp_wait(&sf_empty[b], ((it / NBUF) & 1u) ^ 1u)) { abort_flag = 1; break; }
+                tc_fence_after();
+                uint32_t av[4 * CPS], bv[8 * CPS];
+                const uint8_t *sa = slot_sfa(s) + lane * 16 + q * 4;
+#pragma unroll
+                for (int w = 0; w < CPS; ++w) {
+                    const uint32_t word = *reinterpret_cast<const uint32_t *>(sa + 512 * w);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) av[4 * w + c] = word;
+                }
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int w = 0; w < CPS; ++w) {
+                        const uint4 u = *reinterpret_cast<const uint4 *>(slot_sfb(s) + 512 * (h * CPS + w) + lane * 16);
+                        bv[8 * w + 4 * h + 0] = u.x;
+                        bv[8 * w + 4 * h + 1] = u.y;
+                        bv[8 * w + 4 * h + 2] = u.z;
+                        bv[8 * w + 4 * h + 3] = u.w;
+                    }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sfs_empty[s]);   // the slot's bytes are in registers now
+                if (CPS == 4) {
+                    tmem_st_x16(buf_a(b) + lane_base, av);
+                    tmem_st_x32(buf_b(b) + lane_base, bv);
+                } else {
+                    tmem_st_x8(buf_a(b) + lane_base, av);
+                    tmem_st_x16(buf_b(b) + lane_base, bv);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&sf_full[b]), 0));
+            }
+        }
+        g2_exit(tmem, false);
+        return;
+    }
+    {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 184;");
+        // ------------------------------------------------ epilogue (both CTAs: own 128 rows)
+        const int q = warp & 3;
+        const int h = (warp - G2_EPI_WARP0) >> 2;
+        const uint32_t acc_empty_leader = mapa_shared(smem_u32(&acc_empty), 0);
+        float alpha = 1.0f;
+        if (FMT == QFP4_NVFP4) alpha = __fmul_rn(*p.tA, *p.tB);
+        int ti = 0;
+        for (int t = cluster; t < ntiles && !abort_flag; t += nclusters, ++ti) {
+            int mb, nb;
+            tile_coords(t, tiles_m, tiles_n, mb, nb);
+            if (!warp_wait(&acc_full, ti & 1)) { abort_flag = 1; break; }
+            tc_fence_after();
+            uint32_t r[128];
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+                tmem_ld16x256b_x16(tmem + (static_cast<uint32_t>(32 * q + 16 * hh) << 16) + 128 * h, r + 64 * hh);
+            tmem_ld_wait();
+            reg_fence<128>(r);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+
+            const int col0 = nb * G2_BN + 128 * h + 2 * (lane & 3);
+            const int row_base = mb * G2_BM + 128 * static_cast<int>(rank);
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int row = row_base + 32 * q + 16 * hh + 8 * e + (lane >> 2);
+                    if (row >= p.M) continue;
+                    if (OUT == QFP4_F32) {
+                        float *o = static_cast<float *>(p.out) + static_cast<int64_t>(row) * p.N + col0;
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            if (col0 + 8 * j < p.N)
+                                *reinterpret_cast<float2 *>(o + 8 * j) =
+                                    make_float2(__fmul_rn(__uint_as_float(r[64 * hh + 4 * j + 2 * e]), alpha),
+                                                __fmul_rn(__uint_as_float(r[64 * hh + 4 * j + 2 * e + 1]), alpha));
+                    } else {
+                        uint16_t *o = static_cast<uint16_t *>(p.out) + static_cast<int64_t>(row) * p.N + col0;
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            if (col0 + 8 * j < p.N) {
+                                const __nv_bfloat162 b2 =
+                                    __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[64 * hh + 4 * j + 2 * e]), alpha),
+                                                          __fmul_rn(__uint_as_float(r[64 * hh + 4 * j + 2 * e + 1]), alpha));
+                                *reinterpret_cast<__nv_bfloat162 *>(o + 8 * j) = b2;
+                            }
+                    }
+                }
+        }
+    }
+    g2_exit(tmem, false);
+}
+
 // ------------------------------------------------------------------ host
 struct GemmLayout {
     int MB, NT, KT, NC;
@@ -409,13 +861,15 @@ size_t gemm_workspace(int64_t M, int64_t N, int64_t K, qfp4_fmt fmt)
     return L.sfa_bytes + L.sfb_bytes;
 }
 
-int rearrange_scales(const uint8_t *scales, int64_t R, int64_t K, qfp4_fmt fmt, int n_blocks128, int NC, uint8_t *dst,
-                     cudaStream_t stream)
+// Scale chunks of A (n_blocks_a 128-row blocks) and B (n_blocks_b) in one launch.
+int rearrange_scales(const uint8_t *a_scales, int64_t M, int n_blocks_a, uint8_t *sfa, const uint8_t *b_scales,
+                     int64_t N, int n_blocks_b, uint8_t *sfb, int64_t K, qfp4_fmt fmt, int NC, cudaStream_t stream)
 {
     const int g = fmt == QFP4_MXFP4 ? 32 : 16;
-    const int n_lines = n_blocks128 * NC * 32;
-    k_sf_rearrange<<<(n_lines + 255) / 256, 256, 0, stream>>>(scales, static_cast<int>(R), static_cast<int>(K / g), NC,
-                                                             n_lines, dst);
+    const SfJob ja{a_scales, static_cast<int>(M), n_blocks_a, sfa};
+    const SfJob jb{b_scales, static_cast<int>(N), n_blocks_b, sfb};
+    const dim3 grid((NC + SF_CHUNKS_PER_BLOCK - 1) / SF_CHUNKS_PER_BLOCK, n_blocks_a + n_blocks_b);
+    k_sf_chunks<<<grid, 256, 0, stream>>>(ja, jb, static_cast<int>(K / g), NC);
     QFP4_LAUNCH_CHECK();
     return QFP4_OK;
 }
@@ -435,12 +889,43 @@ static int launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const GemmP
     return QFP4_OK;
 }
 
+template <int FMT, int OUT>
+static int launch_gemm2(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tsa, const CUtensorMap &tsb,
+                        const GemmParams &p, int grid, cudaStream_t s)
+{
+    static bool configured = false;
+    auto kern = k_gemm_bs2<FMT, OUT>;
+    if (!configured) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G2_SMEM) != cudaSuccess)
+            return QFP4_ERR_CUDA;
+        configured = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(G2_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = G2_SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, p);
+    QFP4_LAUNCH_CHECK();
+    return QFP4_OK;
+}
+
 // Main kernel on already rearranged scales (sfa / sfb in the chunk layout).
+// Problems taller than one 128-row block run on CTA pairs (256 x 256 tiles),
+// the rest on single CTAs (128 x 256 tiles).
 int gemm_core(const uint8_t *A_codes, const uint8_t *sfa, const float *A_tscale, const uint8_t *B_codes,
               const uint8_t *sfb, const float *B_tscale, int64_t M, int64_t N, int64_t K, qfp4_fmt fmt,
               qfp4_dtype out_dt, void *out, cudaStream_t stream)
 {
     const GemmLayout L = gemm_layout(M, N, K, fmt);
+    const bool pair = M > GM_BM;
     CUtensorMap ta, tb;
     {
         const uint64_t dims[2] = {static_cast<uint64_t>(K / 2), static_cast<uint64_t>(M)};
@@ -453,7 +938,7 @@ int gemm_core(const uint8_t *A_codes, const uint8_t *sfa, const float *A_tscale,
     {
         const uint64_t dims[2] = {static_cast<uint64_t>(K / 2), static_cast<uint64_t>(N)};
         const uint64_t strides[1] = {static_cast<uint64_t>(K / 2)};
-        const uint32_t box[2] = {GM_BKB, GM_BN};
+        const uint32_t box[2] = {GM_BKB, static_cast<uint32_t>(pair ? 128 : GM_BN)};
         int st = encode_tensor_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(B_codes), dims,
                                    strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
         if (st != QFP4_OK) return st;
@@ -471,6 +956,35 @@ int gemm_core(const uint8_t *A_codes, const uint8_t *sfa, const float *A_tscale,
     p.tA = A_tscale;
     p.tB = B_tscale;
     p.out = out;
+    if (pair) {
+        // scale chunks viewed as rows of 128 B (4 rows per 512-byte chunk)
+        const int cps = gm_cps(fmt);
+        CUtensorMap tsa, tsb;
+        // rows past the last 128-row block of A (odd block counts) read as zeros
+        {
+            const uint64_t dims[2] = {128, static_cast<uint64_t>(L.MB) * L.NC * 4};
+            const uint64_t strides[1] = {128};
+            const uint32_t box[2] = {128, static_cast<uint32_t>(4 * cps)};
+            int st = encode_tensor_map(&tsa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(sfa), dims,
+                                       strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+            if (st != QFP4_OK) return st;
+        }
+        {
+            const uint64_t dims[2] = {128, static_cast<uint64_t>(2 * L.NT) * L.NC * 4};
+            const uint64_t strides[1] = {128};
+            const uint32_t box[2] = {128, static_cast<uint32_t>(4 * cps)};
+            int st = encode_tensor_map(&tsb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(sfb), dims,
+                                       strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+            if (st != QFP4_OK) return st;
+        }
+        const int ntiles = static_cast<int>(((M + G2_BM - 1) / G2_BM) * ((N + G2_BN - 1) / G2_BN));
+        const int grid = 2 * imin<int>(ntiles, num_sms() / 2);
+        if (fmt == QFP4_NVFP4)
+            return out_dt == QFP4_F32 ? launch_gemm2<QFP4_NVFP4, QFP4_F32>(ta, tb, tsa, tsb, p, grid, stream)
+                                      : launch_gemm2<QFP4_NVFP4, QFP4_BF16>(ta, tb, tsa, tsb, p, grid, stream);
+        return out_dt == QFP4_F32 ? launch_gemm2<QFP4_MXFP4, QFP4_F32>(ta, tb, tsa, tsb, p, grid, stream)
+                                  : launch_gemm2<QFP4_MXFP4, QFP4_BF16>(ta, tb, tsa, tsb, p, grid, stream);
+    }
     const int grid = static_cast<int>(imin<int64_t>(static_cast<int64_t>(L.MB) * L.NT, num_sms()));
     if (fmt == QFP4_NVFP4)
         return out_dt == QFP4_F32 ? launch_gemm<QFP4_NVFP4, QFP4_F32>(ta, tb, p, grid, stream)
@@ -486,9 +1000,7 @@ int gemm_blockscaled(const uint8_t *A_codes, const uint8_t *A_scales, const floa
     const GemmLayout L = gemm_layout(M, N, K, fmt);
     uint8_t *sfa = static_cast<uint8_t *>(workspace);
     uint8_t *sfb = sfa + L.sfa_bytes;
-    int st = rearrange_scales(A_scales, M, K, fmt, L.MB, L.NC, sfa, stream);
-    if (st != QFP4_OK) return st;
-    st = rearrange_scales(B_scales, N, K, fmt, 2 * L.NT, L.NC, sfb, stream);
+    const int st = rearrange_scales(A_scales, M, L.MB, sfa, B_scales, N, 2 * L.NT, sfb, K, fmt, L.NC, stream);
     if (st != QFP4_OK) return st;
     return gemm_core(A_codes, sfa, A_tscale, B_codes, sfb, B_tscale, M, N, K, fmt, out_dt, out, stream);
 }
@@ -535,9 +1047,7 @@ int gemm_fused_rq(const void *A_bf16, int64_t M, int64_t K, int rotate, int four
     if (st != QFP4_OK) return st;
     const GemmLayout L = gemm_layout(M, N, K, fmt);
     uint8_t *sfa = ws + F.chunks, *sfb = sfa + L.sfa_bytes;
-    st = rearrange_scales(a_scales, M, K, fmt, L.MB, L.NC, sfa, stream);
-    if (st != QFP4_OK) return st;
-    st = rearrange_scales(B_scales, N, K, fmt, 2 * L.NT, L.NC, sfb, stream);
+    st = rearrange_scales(a_scales, M, L.MB, sfa, B_scales, N, 2 * L.NT, sfb, K, fmt, L.NC, stream);
     if (st != QFP4_OK) return st;
     return gemm_core(a_codes, sfa, a_tscale, B_codes, sfb, B_tscale, M, N, K, fmt, out_dt, out, stream);
 }

@@ -88,6 +88,16 @@ __device__ __forceinline__ uint64_t global_ns()
     return t;
 }
 
+// After a wait gave up: let copies this thread already started (TMA loads,
+// at most a few stages) land before the CTA leaves, for at most `ns`.
+__device__ __forceinline__ void settle_ns(uint64_t ns)
+{
+    const uint64_t t0 = global_ns();
+    while (global_ns() - t0 < ns) {
+    }
+}
+constexpr uint64_t kSettleNs = 100000ull;
+
 // Bounded wait: true when the phase completed, false (error recorded) when
 // kWaitLimitNs of wall time (or kSpinLimit polls) ran out.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;

@@ -449,11 +449,15 @@ __global__ void __launch_bounds__(32 * WARPS, 1) k_quant1d_tma(const __grid_cons
 
     float tmax = 0.0f;
     int it = 0;
+    bool gave_up = false;
     for (int64_t t = t_begin + warp; t < t_end; t += WARPS, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1u;
         const bool ok = mbar_wait(&bars[s], ph);
-        if (__any_sync(0xFFFFFFFFu, !ok)) break;
+        if (__any_sync(0xFFFFFFFFu, !ok)) {
+            gave_up = true;
+            break;
+        }
 
         // this lane's unit: rows ROWS_PER_LANE*lane + h of the tile (128-byte swizzle)
         const uint8_t *st = ring + s * STAGE_BYTES;
@@ -488,6 +492,7 @@ __global__ void __launch_bounds__(32 * WARPS, 1) k_quant1d_tma(const __grid_cons
             store_unit_packed<UP, G>(o, p, e0, n_valid);
         }
     }
+    if (gave_up && lane == 0) settle_ns(kSettleNs);   // loads of this warp's ring may still be landing
     if (MODE == MODE_AMAX) {
         tmax = block_max(tmax, red);
         if (threadIdx.x == 0) p.partials_out[blockIdx.x] = tmax;
