@@ -214,6 +214,8 @@ constexpr int SF_CHUNKS_PER_BLOCK = 8;
 __global__ void __launch_bounds__(256) k_sf_chunks(SfJob ja, SfJob jb, int Kg, int NC)
 {
     __shared__ uint32_t tile[128 * 9];                    // 128 rows x 32 bytes, row stride 36 bytes
+    pdl_wait();
+    pdl_trigger();
     const bool is_a = static_cast<int>(blockIdx.y) < ja.nblk;
     const SfJob j = is_a ? ja : jb;
     const int rb = is_a ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.y) - ja.nblk;
@@ -284,6 +286,8 @@ __global__ void __launch_bounds__(GM_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base_sh;
+    pdl_wait();
+    pdl_trigger();
 
     auto stage_a = [&](int s) { return smem + s * GM_STAGE_BYTES; };
     auto stage_b = [&](int s) { return smem + s * GM_STAGE_BYTES + GM_A_BYTES; };
@@ -632,6 +636,8 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
     cluster_sync();                          // barriers of both CTAs initialised before any remote use
     tc_fence_after();
     const uint32_t tmem = tmem_base_sh;
+    pdl_wait();
+    pdl_trigger();
 
     auto stage_a = [&](int s) { return smem + s * G2_STAGE_BYTES; };
     auto stage_b = [&](int s) { return smem + s * G2_STAGE_BYTES + G2_A_BYTES; };
@@ -869,7 +875,10 @@ int rearrange_scales(const uint8_t *a_scales, int64_t M, int n_blocks_a, uint8_t
     const SfJob ja{a_scales, static_cast<int>(M), n_blocks_a, sfa};
     const SfJob jb{b_scales, static_cast<int>(N), n_blocks_b, sfb};
     const dim3 grid((NC + SF_CHUNKS_PER_BLOCK - 1) / SF_CHUNKS_PER_BLOCK, n_blocks_a + n_blocks_b);
-    k_sf_chunks<<<grid, 256, 0, stream>>>(ja, jb, static_cast<int>(K / g), NC);
+    if (launch_pdl(k_sf_chunks, grid, dim3(256), 0, stream, ja, jb, static_cast<int>(K / g), NC) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return QFP4_ERR_CUDA;
+    }
     QFP4_LAUNCH_CHECK();
     return QFP4_OK;
 }
@@ -884,7 +893,10 @@ static int launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const GemmP
             return QFP4_ERR_CUDA;
         configured = true;
     }
-    kern<<<grid, GM_THREADS, GM_SMEM, s>>>(ta, tb, p);
+    if (launch_pdl(kern, dim3(grid), dim3(GM_THREADS), GM_SMEM, s, ta, tb, p) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return QFP4_ERR_CUDA;
+    }
     QFP4_LAUNCH_CHECK();
     return QFP4_OK;
 }
@@ -905,14 +917,19 @@ static int launch_gemm2(const CUtensorMap &ta, const CUtensorMap &tb, const CUte
     cfg.blockDim = dim3(G2_THREADS, 1, 1);
     cfg.dynamicSmemBytes = G2_SMEM;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, p);
+    cfg.numAttrs = 2;
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, p) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return QFP4_ERR_CUDA;
+    }
     QFP4_LAUNCH_CHECK();
     return QFP4_OK;
 }

@@ -113,6 +113,34 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
     return false;
 }
 
+// ------------------------------------------------------------------ dependent launches
+// Kernels are launched with programmatic stream serialization: a kernel may
+// start (run its prologue: barrier setup, tensor-map prefetch, tensor-memory
+// allocation) while the previous kernel in the stream is finishing.  Every
+// thread calls pdl_wait() before its first global-memory access; it returns
+// once the previous grid has completed and its writes are visible (at once
+// when there is no such grid).  pdl_trigger() lets the next kernel be
+// scheduled as soon as every CTA of this grid has issued it or exited.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<Args &&>(args)...);
+}
+
 // ------------------------------------------------------------------ PTX: TMA
 __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1)
 {
@@ -223,6 +251,18 @@ __device__ __forceinline__ uint64_t f2mul(uint64_t a, uint64_t b)
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
     return r;
 }
+__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
 // two bf16 (one 32-bit word) -> a packed pair, exact
 __device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w)
 {
@@ -242,9 +282,8 @@ __device__ __forceinline__ uint32_t e2m1x8_rne_pairs(uint64_t p0, uint64_t p1, u
 // E2M1 stochastic rounding of one value (|v| <= 6 or saturating):
 // lo <= |v| < hi adjacent grid values, up iff u < (|v| - lo) / (hi - lo)
 // with u = (w >> 8) * 2^-24.  Returns the 4-bit code.
-__device__ __forceinline__ uint32_t e2m1_sr(float v, uint32_t w)
+__device__ __forceinline__ float e2m1_sr_grid(float v, uint32_t w)
 {
-    const uint32_t sign = (__float_as_uint(v) >> 28) & 8u;
     const float a = fabsf(v);
     float lo, sp, inv_sp;              // lower grid value, spacing, 1/spacing
     if (a >= 1.0f) {
@@ -261,9 +300,16 @@ __device__ __forceinline__ uint32_t e2m1_sr(float v, uint32_t w)
     const float u = __fmul_rn(static_cast<float>(w >> 8), 5.9604644775390625e-08f);  // 2^-24
     float r = (u < p) ? __fadd_rn(lo, sp) : lo;
     r = fminf(r, 6.0f);
+    return __uint_as_float(__float_as_uint(r) | (__float_as_uint(v) & 0x80000000u));   // sign kept, also on zero
+}
+
+// The same rule as a 4-bit code.
+__device__ __forceinline__ uint32_t e2m1_sr(float v, uint32_t w)
+{
+    const float r = e2m1_sr_grid(v, w);
     uint32_t code;
     asm("{\n\t.reg .b8 b;\n\tcvt.rn.satfinite.e2m1x2.f32 b, %1, %1;\n\tcvt.u32.u8 %0, b;\n\t}" : "=r"(code) : "f"(r));
-    return (code & 7u) | sign;
+    return code & 0xFu;
 }
 
 // E4M3 (OCP) round-to-nearest-even, saturating to +-448: returns the byte.

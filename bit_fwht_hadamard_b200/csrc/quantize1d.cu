@@ -98,17 +98,23 @@ __device__ __forceinline__ void nv_block_rne(const float *x, float S, uint32_t *
 
 // Stochastic rounding of 16 (NVFP4) or 32 (MXFP4) values v (already divided
 // by the scale) whose first element has logical index e (e % 4 == 0).
+// Each value goes to its signed E2M1 grid value in binary32; eight of those
+// then take one packed hardware conversion (exact: they are grid values).
 template <int G>
 __device__ __forceinline__ void sr_group(const float *v, uint64_t e, uint64_t seed, uint32_t *words)
 {
 #pragma unroll
-    for (int w = 0; w < G / 8; ++w) words[w] = 0u;
+    for (int w = 0; w < G / 8; ++w) {
+        float r[8];
 #pragma unroll
-    for (int q = 0; q < G / 4; ++q) {
-        const uint4 r = sr_words4(seed, (e >> 2) + q);
-        const uint32_t c0 = e2m1_sr(v[4 * q + 0], r.x), c1 = e2m1_sr(v[4 * q + 1], r.y);
-        const uint32_t c2 = e2m1_sr(v[4 * q + 2], r.z), c3 = e2m1_sr(v[4 * q + 3], r.w);
-        words[q >> 1] |= (c0 | (c1 << 4) | (c2 << 8) | (c3 << 12)) << (16 * (q & 1));
+        for (int h = 0; h < 2; ++h) {
+            const uint4 rw = sr_words4(seed, (e >> 2) + 2 * w + h);
+            r[4 * h + 0] = e2m1_sr_grid(v[8 * w + 4 * h + 0], rw.x);
+            r[4 * h + 1] = e2m1_sr_grid(v[8 * w + 4 * h + 1], rw.y);
+            r[4 * h + 2] = e2m1_sr_grid(v[8 * w + 4 * h + 2], rw.z);
+            r[4 * h + 3] = e2m1_sr_grid(v[8 * w + 4 * h + 3], rw.w);
+        }
+        words[w] = e2m1x8_rne(r);
     }
 }
 
@@ -248,9 +254,10 @@ __device__ __forceinline__ void store_unit(const UnitOut &o, const QuantParams &
 // holds a whole 128-element rotation block, UP = 32 holds half of one and
 // exchanges the h = 64 stage with its partner lane (lane ^ 1, the even lane
 // holding the lower half).  Stage h = 1 runs inside each pair; stages
-// h = 2 .. 2*UP between pairs k and k + h/2 as f32x2 add / sub; then one f32x2
-// multiply by 1/sqrt(128).
-template <int UP>
+// h = 2 .. 2*UP between pairs k and k + h/2 as f32x2 add / sub; then, when
+// NORM, one f32x2 multiply by 1/sqrt(128) (callers that fold the
+// normalisation into their scale multiply pass NORM = false).
+template <int UP, bool NORM>
 __device__ __forceinline__ void fwht_packed(uint64_t (&p)[UP], bool upper)
 {
 #pragma unroll
@@ -271,22 +278,25 @@ __device__ __forceinline__ void fwht_packed(uint64_t (&p)[UP], bool upper)
         }
     }
     if (UP == 32) {
-        // h = 64 across the lane pair: lower gets mine + other, upper gets
-        // other - mine = other + (-mine) (negation is exact)
-        const uint64_t flip = upper ? 0x8000000080000000ull : 0ull;
+        // h = 64 across the lane pair: lower gets other + mine, upper gets
+        // other - mine, both as one rounding of other + (+-1) * mine
+        const float sg = upper ? -1.0f : 1.0f;
+        const uint64_t sg2 = f2pack(sg, sg);
 #pragma unroll
         for (int k = 0; k < UP; ++k) {
             const uint32_t lo = __shfl_xor_sync(0xFFFFFFFFu, static_cast<uint32_t>(p[k]), 1);
             const uint32_t hi = __shfl_xor_sync(0xFFFFFFFFu, static_cast<uint32_t>(p[k] >> 32), 1);
-            p[k] = f2add((static_cast<uint64_t>(hi) << 32) | lo, p[k] ^ flip);
+            p[k] = f2fma(p[k], sg2, (static_cast<uint64_t>(hi) << 32) | lo);
         }
     }
-    const uint64_t c2 = f2pack(inv_sqrt128(), inv_sqrt128());
+    if (NORM) {
+        const uint64_t c2 = f2pack(inv_sqrt128(), inv_sqrt128());
 #pragma unroll
-    for (int k = 0; k < UP; ++k) p[k] = f2mul(p[k], c2);
+        for (int k = 0; k < UP; ++k) p[k] = f2mul(p[k], c2);
+    }
 }
 
-// max |x| over n packed pairs, as a balanced tree
+// max |x| over n packed pairs (n a power of two), three-input maxima
 template <int N>
 __device__ __forceinline__ float absmax_pairs(const uint64_t *p)
 {
@@ -297,10 +307,19 @@ __device__ __forceinline__ float absmax_pairs(const uint64_t *p)
         f2unpack(p[j], a, b);
         m[j] = fmaxf(fabsf(a), fabsf(b));
     }
+    int n = N;
 #pragma unroll
-    for (int h = N / 2; h >= 1; h >>= 1)
+    while (n > 1) {
+        const int t = (n + 2) / 3;                  // ceil(n / 3)
 #pragma unroll
-        for (int j = 0; j < h; ++j) m[j] = fmaxf(m[j], m[j + h]);
+        for (int j = 0; j < t; ++j) {
+            const float a = m[3 * j];
+            const float b = 3 * j + 1 < n ? m[3 * j + 1] : a;
+            const float c = 3 * j + 2 < n ? m[3 * j + 2] : a;
+            m[j] = fmax3(a, b, c);
+        }
+        n = t;
+    }
     return m[0];
 }
 
@@ -310,24 +329,38 @@ struct UnitP {
     uint32_t scales[2];         // up to 8 scale bytes
 };
 
-template <int UP, int FMT, bool SR, bool FOUR6>
+// RAW: the rotation left out its 1/sqrt(128) (fwht_packed<UP, false>); only
+// the MXFP4 round-to-nearest path takes raw values.  With c = 1/sqrt(128) the
+// normalised group maximum is fl(amax_raw * c) (rounding is monotone), and
+// fl(x * (c * 2^-k)) equals fl(fl(x * c) * 2^-k) whenever the latter is a
+// normal number; when it is subnormal both encode to a zero of x's sign.
+// c * 2^-k itself is normal for k <= 120; larger k (groups near the top of
+// the binary32 range) take the two multiplies.
+template <int UP, int FMT, bool SR, bool FOUR6, bool RAW = false>
 __device__ __forceinline__ void quant_unit_packed(uint64_t (&p)[UP], uint64_t e0, float s_t, uint64_t seed,
                                                   UnitP<UP> &o)
 {
+    static_assert(!RAW || (FMT == QFP4_MXFP4 && !SR), "raw values only on the MXFP4 round-to-nearest path");
     o.scales[0] = o.scales[1] = 0u;
     if (FMT == QFP4_MXFP4) {
 #pragma unroll
         for (int g = 0; g < UP / 16; ++g) {
             uint64_t *pg = p + 16 * g;
             uint32_t *w = o.codes + 4 * g;
-            const float amax = absmax_pairs<16>(pg);
+            const float amax = RAW ? __fmul_rn(absmax_pairs<16>(pg), inv_sqrt128()) : absmax_pairs<16>(pg);
             if (amax == 0.0f) {                      // all-zero group: byte 0, +0 codes
                 w[0] = w[1] = w[2] = w[3] = 0u;
                 continue;
             }
             const int k = scale_exp(amax, 0x400000u, 2);
             o.scales[0] |= static_cast<uint32_t>(k + 127) << (8 * g);
-            const uint64_t m2 = f2pack(exp2i(-k), exp2i(-k));   // x * 2^-k == x / 2^k exactly
+            if (RAW && k > 120) {
+                const uint64_t c2 = f2pack(inv_sqrt128(), inv_sqrt128());
+#pragma unroll
+                for (int j = 0; j < 16; ++j) pg[j] = f2mul(pg[j], c2);
+            }
+            const float mk = (RAW && k <= 120) ? __fmul_rn(inv_sqrt128(), exp2i(-k)) : exp2i(-k);
+            const uint64_t m2 = f2pack(mk, mk);      // x * 2^-k == x / 2^k exactly
 #pragma unroll
             for (int j = 0; j < 16; ++j) pg[j] = f2mul(pg[j], m2);
             if (SR) {
@@ -423,11 +456,6 @@ __global__ void __launch_bounds__(32 * WARPS, 1) k_quant1d_tma(const __grid_cons
     const int64_t t_begin = ntiles * blockIdx.x / gridDim.x, t_end = ntiles * (blockIdx.x + 1) / gridDim.x;
     constexpr int G = FMT == QFP4_MXFP4 ? 32 : 16;
 
-    float s_t = 0.0f;
-    if (MODE == MODE_QUANT && FMT == QFP4_NVFP4) {
-        s_t = tensor_scale(p, red);
-        if (p.write_tscale && blockIdx.x == 0 && threadIdx.x == 0) *p.tscale_out = s_t;
-    }
     uint64_t *bars = full[warp];
     uint8_t *ring = smem + warp * (STAGES * STAGE_BYTES);
     if (lane == 0) {
@@ -436,6 +464,13 @@ __global__ void __launch_bounds__(32 * WARPS, 1) k_quant1d_tma(const __grid_cons
         if (warp == 0) prefetch_tensormap(&tm);
     }
     __syncwarp();
+    pdl_wait();
+    pdl_trigger();
+    float s_t = 0.0f;
+    if (MODE == MODE_QUANT && FMT == QFP4_NVFP4) {
+        s_t = tensor_scale(p, red);
+        if (p.write_tscale && blockIdx.x == 0 && threadIdx.x == 0) *p.tscale_out = s_t;
+    }
 
     auto issue = [&](int64_t t, int s) {
         mbar_arrive_expect_tx(&bars[s], STAGE_BYTES);
@@ -482,13 +517,14 @@ __global__ void __launch_bounds__(32 * WARPS, 1) k_quant1d_tma(const __grid_cons
 
         const int64_t row0 = t * TILE_ROWS + ROWS_PER_LANE * lane;   // first 64-element row of the unit
         const int64_t n_valid = imin<int64_t>(2 * UP, (rows - row0) * 64);
-        if (ROT) fwht_packed<UP>(v, (lane & 1) != 0);
+        constexpr bool RAW = ROT && MODE == MODE_QUANT && FMT == QFP4_MXFP4 && !SR;
+        if (ROT) fwht_packed<UP, !RAW>(v, (lane & 1) != 0);
         if (MODE == MODE_AMAX) {
             tmax = fmaxf(tmax, absmax_pairs<UP>(v));   // rows past the end were zero-filled by TMA
         } else if (n_valid > 0) {
             const uint64_t e0 = p.e_base + static_cast<uint64_t>(row0) * 64u;
             UnitP<UP> o;
-            quant_unit_packed<UP, FMT, SR, FOUR6>(v, e0, s_t, p.seed, o);
+            quant_unit_packed<UP, FMT, SR, FOUR6, RAW>(v, e0, s_t, p.seed, o);
             store_unit_packed<UP, G>(o, p, e0, n_valid);
         }
     }
@@ -511,6 +547,8 @@ template <int MODE, int FMT, bool ROT, bool SR, bool FOUR6, typename T>
 __global__ void __launch_bounds__(128) k_quant1d_direct(const T *__restrict__ x, QuantParams p)
 {
     __shared__ float red[32];
+    pdl_wait();
+    pdl_trigger();
     constexpr int G = FMT == QFP4_MXFP4 ? 32 : 16;
     float s_t = 0.0f;
     if (MODE == MODE_QUANT && FMT == QFP4_NVFP4) {
@@ -586,7 +624,10 @@ static int launch_tma(const CUtensorMap &tm, const QuantParams &p, int grid, cud
             return QFP4_ERR_CUDA;
         done = 1;
     }
-    kern<<<grid, 32 * QT_WARPS, QT_SMEM_BYTES, stream>>>(tm, p);
+    if (launch_pdl(kern, dim3(grid), dim3(32 * QT_WARPS), QT_SMEM_BYTES, stream, tm, p) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return QFP4_ERR_CUDA;
+    }
     QFP4_LAUNCH_CHECK();
     return QFP4_OK;
 }
@@ -594,7 +635,11 @@ static int launch_tma(const CUtensorMap &tm, const QuantParams &p, int grid, cud
 template <int MODE, int FMT, bool ROT, bool SR, bool FOUR6, typename T>
 static int launch_direct(const T *x, const QuantParams &p, int grid, cudaStream_t stream)
 {
-    k_quant1d_direct<MODE, FMT, ROT, SR, FOUR6, T><<<grid, 128, 0, stream>>>(x, p);
+    if (launch_pdl(k_quant1d_direct<MODE, FMT, ROT, SR, FOUR6, T>, dim3(grid), dim3(128), 0, stream, x, p) !=
+        cudaSuccess) {
+        (void)cudaGetLastError();
+        return QFP4_ERR_CUDA;
+    }
     QFP4_LAUNCH_CHECK();
     return QFP4_OK;
 }
