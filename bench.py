@@ -368,7 +368,7 @@ def bench_gemm(q, synth, dev, stream, bf16_peak, peak_src, iters):
             "value": tflops, "unit": "TFLOP/s", "ms_per_call": ms,
             "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
                          "frac": tflops / peak, "traffic": ncu_traffic("gemm_nvfp4_f32"),
-                         "kernel": "gemm_nvfp4_f32 (scale rearrange prepass + tcgen05 main loop)",
+                         "kernel": "gemm_nvfp4_f32 (scale-chunk prepass + 2-CTA tcgen05 main loop)",
                          "peak_source": f"{peak_src} bf16_tflops x {FP4_PER_BF16} (nominal FP4:BF16 dense ratio)"}}
 
 

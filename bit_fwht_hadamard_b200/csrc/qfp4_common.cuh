@@ -284,22 +284,23 @@ __device__ __forceinline__ uint32_t e2m1x8_rne_pairs(uint64_t p0, uint64_t p1, u
 // with u = (w >> 8) * 2^-24.  Returns the 4-bit code.
 __device__ __forceinline__ float e2m1_sr_grid(float v, uint32_t w)
 {
+    // Grid spacing sp = 2^(m - 128) with m = clamp(biased exponent of |v|, 127, 129):
+    // 0.5 below 2, 1 in [2, 4), 2 from 4 on.  Everything below is exact binary32:
+    //   q24 = |v| / sp * 2^24                      (scaling by a power of two)
+    //   fl24 = floor(q24 / 2^24) * 2^24            (round-toward-zero add of 1.5 * 2^47,
+    //                                               whose ulp is 2^24, then its removal)
+    //   frac24 = q24 - fl24 = ((|v| - lo) / sp) * 2^24
+    // so u < (|v| - lo) / sp with u = (w >> 8) * 2^-24 is (w >> 8) < frac24, and the
+    // result is (fl24 or fl24 + 2^24) * sp * 2^-24, saturated at 6.
     const float a = fabsf(v);
-    float lo, sp, inv_sp;              // lower grid value, spacing, 1/spacing
-    if (a >= 1.0f) {
-        const uint32_t spb = (__float_as_uint(a) & 0x7F800000u) - 0x00800000u;   // 2^(exp-1)
-        lo = __uint_as_float(__float_as_uint(a) & 0x7FC00000u);                 // 1 mantissa bit
-        sp = __uint_as_float(spb);
-        inv_sp = __uint_as_float((254u << 23) - spb);
-    } else {
-        lo = a >= 0.5f ? 0.5f : 0.0f;
-        sp = 0.5f;
-        inv_sp = 2.0f;
-    }
-    const float p = __fmul_rn(__fsub_rn(a, lo), inv_sp);   // exact: power-of-two spacing
-    const float u = __fmul_rn(static_cast<float>(w >> 8), 5.9604644775390625e-08f);  // 2^-24
-    float r = (u < p) ? __fadd_rn(lo, sp) : lo;
-    r = fminf(r, 6.0f);
+    const int m = imin(imax(static_cast<int>(__float_as_uint(a) >> 23), 127), 129);
+    const float inv24 = __uint_as_float(static_cast<uint32_t>(279 - m) << 23);   // 2^24 / sp
+    const float sp24 = __uint_as_float(static_cast<uint32_t>(m - 25) << 23);     // sp / 2^24
+    const float q24 = __fmul_rn(a, inv24);
+    const float fl24 = __fsub_rn(__fadd_rz(q24, 211106232532992.0f), 211106232532992.0f);   // 1.5 * 2^47
+    const float frac24 = __fsub_rn(q24, fl24);
+    const float r24 = (static_cast<float>(w >> 8) < frac24) ? __fadd_rn(fl24, 16777216.0f) : fl24;
+    const float r = fminf(__fmul_rn(r24, sp24), 6.0f);
     return __uint_as_float(__float_as_uint(r) | (__float_as_uint(v) & 0x80000000u));   // sign kept, also on zero
 }
 
