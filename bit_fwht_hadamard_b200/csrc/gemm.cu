@@ -384,9 +384,6 @@ __global__ void __launch_bounds__(GM_THREADS, 1)
                 tmem_ld16x256b_x16(tmem + (static_cast<uint32_t>(32 * q + 16 * hh) << 16) + 128 * h, r + 64 * hh);
             tmem_ld_wait();
             reg_fence<128>(r);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty);
 
             // r[64hh + 4j + {0,1}]: row 32q + 16hh + lane/4, columns 8j + 2(lane%4) + {0,1};
             // r[64hh + 4j + {2,3}]: the row 8 below.  Four lanes cover 32 contiguous bytes.
@@ -417,6 +414,10 @@ __global__ void __launch_bounds__(GM_THREADS, 1)
                             }
                     }
                 }
+            // handed back after the stores, as in the 2-CTA kernel
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty);
         }
     }
 
@@ -445,16 +446,17 @@ __global__ void __launch_bounds__(GM_THREADS, 1)
 // buffers with tcgen05.st, concurrently with the MMAs.  The MMA for rows in
 // quadrant q reads the A scale of row r at lane r, column addr + q and the
 // B scale of column n at lane (n mod 32) + 32 q, column addr + n / 32, and
-// the MMA takes scale addresses on 4-column (A) and 8-column (B) boundaries:
-//   A: lane r, columns bufA + 4 w + (0..3) = scale word w of row r
-//   B: lane l + 32 q, column bufB + 8 w + m = scale word w of column l + 32 m
-// A k-tile takes 4 CPS columns of A scales and 8 CPS of B scales; the 256
-// columns after the accumulator hold g2_sf_bufs(FMT) such buffers (B buffers
-// first, then A), which is how far the scale warps may run ahead of the MMAs.
-// (word w holds the four scales of k-groups 4w .. 4w + 3 of the k-tile; only
-// column bufA + 4 w + q of a quadrant-q lane is read, the other three hold
-// copies so that one store writes a quadrant's A scales).  Every store starts
-// on a multiple of its own width.
+// the MMA takes scale addresses on 4-column (A) and 8-column (B) boundaries.
+// Each of a k-tile's four MMAs (K = 64) gets a scale word of its own: the
+// four E4M3 scales of its K (NVFP4), or its two E8M0 scales in bytes 0-1
+// (MXFP4, so no MMA reads a word through the byte selector):
+//   A: lane r, columns bufA + 4 k + (0..3) = scale word of MMA k for row r
+//   B: lane l + 32 q, column bufB + 8 k + m = scale word of MMA k for column l + 32 m
+// Only column bufA + 4 k + q of a quadrant-q lane is read; the other three
+// hold copies so that one store writes a quadrant's A scales.  A k-tile takes
+// 16 + 32 columns; the 256 columns after the accumulator hold 5 such buffers,
+// which is how far the scale warps may run ahead of the MMAs.  Every store
+// starts on a multiple of its own width.
 // No TMA multicast.
 constexpr int G2_BM = 256, G2_BN = 256;                   // cluster tile
 // warp roles by warpgroup: 0 operand producer, 1 MMA issuer, 2 scale producer
@@ -471,10 +473,9 @@ constexpr int G2_STAGES = 6;
 constexpr int G2_SF_SLOT_BYTES = 12 * 512;                // A: CPS chunks, B: 2 x CPS chunks (CPS <= 4)
 constexpr int G2_SF_SLOTS = 5;
 constexpr int G2_SMEM = G2_STAGES * G2_STAGE_BYTES + G2_SF_SLOTS * G2_SF_SLOT_BYTES + 1024;
-__host__ __device__ constexpr int g2_sf_bufs(int fmt) { return fmt == QFP4_NVFP4 ? 5 : 10; }
-constexpr int G2_SF_BUFS_MAX = 10;
-static_assert(256 + g2_sf_bufs(QFP4_NVFP4) * 12 * 4 <= GM_TMEM_COLS, "TMEM columns (NVFP4)");
-static_assert(256 + g2_sf_bufs(QFP4_MXFP4) * 12 * 2 <= GM_TMEM_COLS, "TMEM columns (MXFP4)");
+__host__ __device__ constexpr int g2_sf_bufs(int) { return 5; }
+constexpr int G2_SF_BUFS_MAX = 5;
+static_assert(256 + G2_SF_BUFS_MAX * 48 <= GM_TMEM_COLS, "TMEM columns");
 
 __device__ __forceinline__ uint32_t cluster_ctarank()
 {
@@ -551,11 +552,6 @@ __device__ __forceinline__ void umma_blockscaled_cg2(uint32_t d, uint64_t a, uin
 }
 
 #define QFP4_R8(b) "r"(v[b]), "r"(v[b + 1]), "r"(v[b + 2]), "r"(v[b + 3]), "r"(v[b + 4]), "r"(v[b + 5]), "r"(v[b + 6]), "r"(v[b + 7])
-__device__ __forceinline__ void tmem_st_x8(uint32_t taddr, const uint32_t *v)
-{
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr), QFP4_R8(0)
-                 : "memory");
-}
 __device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t *v)
 {
     asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
@@ -643,8 +639,8 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
     auto stage_b = [&](int s) { return smem + s * G2_STAGE_BYTES + G2_A_BYTES; };
     auto slot_sfa = [&](int s) { return smem + G2_STAGES * G2_STAGE_BYTES + s * G2_SF_SLOT_BYTES; };
     auto slot_sfb = [&](int s) { return slot_sfa(s) + CPS * 512; };
-    auto buf_b = [&](int b) { return tmem + 256 + b * (8 * CPS); };
-    auto buf_a = [&](int b) { return tmem + 256 + NBUF * (8 * CPS) + b * (4 * CPS); };
+    auto buf_b = [&](int b) { return tmem + 256 + b * 32; };
+    auto buf_a = [&](int b) { return tmem + 256 + NBUF * 32 + b * 16; };
 
     // Each role ends with its own copy of the exit sequence, so that the
     // register-count regions set by setmaxnreg never merge again.
@@ -691,18 +687,9 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
                     const uint64_t bdesc = desc_k_sw128(stage_b(s));
 #pragma unroll
                     for (int k = 0; k < GM_BK / 64; ++k) {
-                        uint32_t sfa, sfb, id;
-                        if (FMT == QFP4_NVFP4) {
-                            sfa = buf_a(b) + 4 * k;
-                            sfb = buf_b(b) + 8 * k;
-                            id = idesc_blockscaled(FMT, G2_BM, G2_BN, 0);
-                        } else {
-                            const uint32_t sel = 2u * (k & 1);
-                            sfa = (buf_a(b) + 4 * (k >> 1)) | (sel << 30);
-                            sfb = (buf_b(b) + 8 * (k >> 1)) | (sel << 30);
-                            id = idesc_blockscaled(FMT, G2_BM, G2_BN, sel);
-                        }
-                        umma_blockscaled_cg2<FMT>(tmem, adesc + 2 * k, bdesc + 2 * k, id, sfa, sfb, (kt | k) != 0);
+                        umma_blockscaled_cg2<FMT>(tmem, adesc + 2 * k, bdesc + 2 * k,
+                                                  idesc_blockscaled(FMT, G2_BM, G2_BN, 0), buf_a(b) + 4 * k,
+                                                  buf_b(b) + 8 * k, (kt | k) != 0);
                     }
                     umma_commit_cg2_both(&empty[s]);
                     umma_commit_cg2_both(&sf_empty[b]);
@@ -711,6 +698,9 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
             }
             // every MMA this thread issued has finished before either CTA can leave
             umma_commit_cg2_both(&drain);
+            if (!mbar_wait(&drain, 0)) abort_flag = 1;
+        } else if (!leader && lane == 0) {
+            // the partner waits for the leader's drain arrival (multicast into this CTA)
             if (!mbar_wait(&drain, 0)) abort_flag = 1;
         }
         } else if (warp == 2) {
@@ -749,39 +739,53 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
                 if (!warp_wait(&sfs_full[s], (it / G2_SF_SLOTS) & 1u)) { abort_flag = 1; break; }
                 if (!warp_wait(&sf_empty[b], ((it / NBUF) & 1u) ^ 1u)) { abort_flag = 1; break; }
                 tc_fence_after();
-                uint32_t av[4 * CPS], bv[8 * CPS];
+                // raw scale words of this k-tile: word w = the four scales of
+                // k-groups 4w .. 4w + 3 (CPS words per row)
+                uint32_t ra[CPS], rb[2][CPS][4];
                 const uint8_t *sa = slot_sfa(s) + lane * 16 + q * 4;
 #pragma unroll
-                for (int w = 0; w < CPS; ++w) {
-                    const uint32_t word = *reinterpret_cast<const uint32_t *>(sa + 512 * w);
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) av[4 * w + c] = word;
-                }
+                for (int w = 0; w < CPS; ++w) ra[w] = *reinterpret_cast<const uint32_t *>(sa + 512 * w);
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
 #pragma unroll
                     for (int w = 0; w < CPS; ++w) {
                         const uint4 u = *reinterpret_cast<const uint4 *>(slot_sfb(s) + 512 * (h * CPS + w) + lane * 16);
-                        bv[8 * w + 4 * h + 0] = u.x;
-                        bv[8 * w + 4 * h + 1] = u.y;
-                        bv[8 * w + 4 * h + 2] = u.z;
-                        bv[8 * w + 4 * h + 3] = u.w;
+                        rb[h][w][0] = u.x;
+                        rb[h][w][1] = u.y;
+                        rb[h][w][2] = u.z;
+                        rb[h][w][3] = u.w;
                     }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sfs_empty[s]);   // the slot's bytes are in registers now
-                if (CPS == 4) {
-                    tmem_st_x16(buf_a(b) + lane_base, av);
-                    tmem_st_x32(buf_b(b) + lane_base, bv);
-                } else {
-                    tmem_st_x8(buf_a(b) + lane_base, av);
-                    tmem_st_x16(buf_b(b) + lane_base, bv);
+                // one TMEM word per MMA k (K = 64): NVFP4 uses a whole raw word,
+                // MXFP4 the half of one (its two block-32 scales, in bytes 0-1)
+                auto mma_word = [&](uint32_t raw4, uint32_t raw2, int k) -> uint32_t {
+                    return FMT == QFP4_NVFP4 ? raw4 : (raw2 >> (16 * (k & 1))) & 0xFFFFu;
+                };
+                uint32_t av[16], bv[32];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint32_t wa = mma_word(ra[k % CPS], ra[k >> 1], k);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) av[4 * k + c] = wa;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+#pragma unroll
+                        for (int mm = 0; mm < 4; ++mm)
+                            bv[8 * k + 4 * h + mm] = mma_word(rb[h][k % CPS][mm], rb[h][k >> 1][mm], k);
                 }
+                tmem_st_x16(buf_a(b) + lane_base, av);
+                tmem_st_x32(buf_b(b) + lane_base, bv);
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&sf_full[b]), 0));
             }
         }
+        // the leader's last releases of the scale buffers are multicast into
+        // this CTA too: let them land before the CTA can leave
+        for (int i = 0; i < NBUF && !abort_flag; ++i, ++it)
+            if (!warp_wait(&sf_empty[it % NBUF], ((it / NBUF) & 1u) ^ 1u)) abort_flag = 1;
         g2_exit(tmem, false);
         return;
     }
@@ -805,9 +809,6 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
                 tmem_ld16x256b_x16(tmem + (static_cast<uint32_t>(32 * q + 16 * hh) << 16) + 128 * h, r + 64 * hh);
             tmem_ld_wait();
             reg_fence<128>(r);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
 
             const int col0 = nb * G2_BN + 128 * h + 2 * (lane & 3);
             const int row_base = mb * G2_BM + 128 * static_cast<int>(rank);
@@ -837,6 +838,14 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
                             }
                     }
                 }
+            // The accumulator is handed back only after this warp's stores are
+            // issued.  Handing it back right after the tcgen05.ld / wait::ld
+            // pair (so the next tile's MMAs overlap these stores) gave
+            // occasional wrong 32 x 128 blocks on B200: one warp's values
+            // partly from the next tile, seen as run-to-run differences.
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
         }
     }
     g2_exit(tmem, false);

@@ -109,6 +109,26 @@ def test_gemm_full_size_forward_linear():
 
 
 @pytest.mark.parametrize("fmt", FMTS, ids=["mxfp4", "nvfp4"])
+@pytest.mark.parametrize("out", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_gemm_bitwise_deterministic(fmt, out):
+    """Every output element is accumulated in one fixed order (k-tiles in
+    sequence, one CTA pair per tile), so repeated calls must agree bit for
+    bit.  Several tiles per CTA pair, so the accumulator hand-off between
+    tiles and the wrap-around of every stage, scale-slot and scale-buffer ring
+    are exercised; a hand-off race would show up as differing elements."""
+    M, N, K = 4096, 9216, 2048          # 16 x 36 = 576 tiles of 256 x 256 on 74 pairs, 8 k-tiles each
+    X = q.quantize(to_dev(synth.cfg3_X(M, K, seed=11)), fmt[0])
+    W = q.quantize(to_dev(synth.cfg3_W(N, K, seed=12)), fmt[0])
+    ys = [q.gemm(X, W, M, N, K, fmt[0], out_dtype=out) for _ in range(4)]
+    torch.cuda.synchronize()
+    ref = ys[0].view(torch.int32 if out == torch.float32 else torch.int16)
+    for y in ys[1:]:
+        diff = int((y.view(ref.dtype) != ref).sum())
+        assert diff == 0, f"{diff} elements differ between calls"
+    assert q.qfp4_last_device_error() == 0
+
+
+@pytest.mark.parametrize("fmt", FMTS, ids=["mxfp4", "nvfp4"])
 @pytest.mark.parametrize("four6", [False, True])
 def test_fused_rotate_quantize_gemm(fmt, four6):
     if four6 and fmt[1] == oracle.MXFP4:
