@@ -296,7 +296,25 @@ __device__ __forceinline__ void fwht_packed(uint64_t (&p)[UP], bool upper)
     }
 }
 
-// max |x| over n packed pairs (n a power of two), three-input maxima
+// in-place reduction of m[0 .. N) to m[0] with three-input maxima
+// (compile-time sizes, so m stays in registers)
+template <int N>
+__device__ __forceinline__ void max3_reduce(float *m)
+{
+    if constexpr (N > 1) {
+        constexpr int T = (N + 2) / 3;
+#pragma unroll
+        for (int j = 0; j < T; ++j) {
+            const float a = m[3 * j];
+            const float b = 3 * j + 1 < N ? m[3 * j + 1] : a;
+            const float c = 3 * j + 2 < N ? m[3 * j + 2] : a;
+            m[j] = fmax3(a, b, c);
+        }
+        max3_reduce<T>(m);
+    }
+}
+
+// max |x| over N packed pairs
 template <int N>
 __device__ __forceinline__ float absmax_pairs(const uint64_t *p)
 {
@@ -307,19 +325,7 @@ __device__ __forceinline__ float absmax_pairs(const uint64_t *p)
         f2unpack(p[j], a, b);
         m[j] = fmaxf(fabsf(a), fabsf(b));
     }
-    int n = N;
-#pragma unroll
-    while (n > 1) {
-        const int t = (n + 2) / 3;                  // ceil(n / 3)
-#pragma unroll
-        for (int j = 0; j < t; ++j) {
-            const float a = m[3 * j];
-            const float b = 3 * j + 1 < n ? m[3 * j + 1] : a;
-            const float c = 3 * j + 2 < n ? m[3 * j + 2] : a;
-            m[j] = fmax3(a, b, c);
-        }
-        n = t;
-    }
+    max3_reduce<N>(m);
     return m[0];
 }
 
@@ -536,9 +542,12 @@ __global__ void __launch_bounds__(32 * WARPS, 1) k_quant1d_tma(const __grid_cons
 }
 
 // Production configuration of the TMA kernel.
-constexpr int QT_WARPS = 16, QT_STAGES = 2, QT_UP = 32;
+// 20 warps (<= 96 registers a thread) except four-over-six, which needs the
+// registers of 16 warps
+__host__ __device__ constexpr int qt_warps(bool four6) { return four6 ? 16 : 20; }
+constexpr int QT_STAGES = 2, QT_UP = 32;
 constexpr int QT_TILE_ROWS = QT_UP;
-constexpr int QT_SMEM_BYTES = QT_WARPS * QT_STAGES * QT_UP * 128 + 1024;
+__host__ __device__ constexpr int qt_smem_bytes(bool four6) { return qt_warps(four6) * QT_STAGES * QT_UP * 128 + 1024; }
 
 // ---------------------------------------------------------------- direct kernel
 // Loads straight from global memory (bf16 or binary32), one unit per thread;
@@ -617,14 +626,15 @@ static int smem_configured[2][2][2][2][2] = {};
 template <int MODE, int FMT, bool ROT, bool SR, bool FOUR6>
 static int launch_tma(const CUtensorMap &tm, const QuantParams &p, int grid, cudaStream_t stream)
 {
-    auto kern = k_quant1d_tma<MODE, FMT, ROT, SR, FOUR6, QT_WARPS, QT_STAGES, QT_UP>;
+    constexpr int W = qt_warps(FOUR6), SMEM = qt_smem_bytes(FOUR6);
+    auto kern = k_quant1d_tma<MODE, FMT, ROT, SR, FOUR6, W, QT_STAGES, QT_UP>;
     int &done = smem_configured[MODE][FMT][ROT][SR][FOUR6];
     if (!done) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, QT_SMEM_BYTES) != cudaSuccess)
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess)
             return QFP4_ERR_CUDA;
         done = 1;
     }
-    if (launch_pdl(kern, dim3(grid), dim3(32 * QT_WARPS), QT_SMEM_BYTES, stream, tm, p) != cudaSuccess) {
+    if (launch_pdl(kern, dim3(grid), dim3(32 * W), SMEM, stream, tm, p) != cudaSuccess) {
         (void)cudaGetLastError();
         return QFP4_ERR_CUDA;
     }
@@ -665,7 +675,7 @@ static int run_pass(const void *x, qfp4_dtype xdt, int64_t n, QuantParams p, cud
                                        box, CU_TENSOR_MAP_SWIZZLE_128B);
             if (st != QFP4_OK) return st;
             const int64_t ntiles = (body / 64 + QT_TILE_ROWS - 1) / QT_TILE_ROWS;
-            const int grid = static_cast<int>(imin<int64_t>((ntiles + QT_WARPS - 1) / QT_WARPS, nsm));
+            const int grid = static_cast<int>(imin<int64_t>((ntiles + qt_warps(FOUR6) - 1) / qt_warps(FOUR6), nsm));
             QuantParams q = p;
             q.n = body;
             q.partials_out = p.partials_out;
