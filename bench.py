@@ -180,6 +180,17 @@ def cpu_baseline():
             "sample": "one full step (X 4096x4096, RNE + SR), single-threaded C oracle", "seconds": dt}
 
 
+def max_over_ranks(x, dist, device):
+    """The largest x over all ranks, returned on every rank (x itself without a
+    process group): timings are reported for the slowest rank."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ------------------------------------------------------------------ GPU arm
 def run_gpu(args, rank, world):
     import torch
@@ -268,11 +279,7 @@ def run_gpu(args, rank, world):
         barrier()
     if any(st != q.OK for st in status):
         raise RuntimeError(f"qfp4_quantize failed: {set(status)}")
-    elapsed_ms = start.elapsed_time(stop)
-    if dist is not None:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(start.elapsed_time(stop), dist, dev)
     ms_per_step = elapsed_ms / args.steps
     n = M2 * K2
     step_bytes = 2 * n * BYTES_PER_ELEM_MXFP4
@@ -291,32 +298,53 @@ def run_gpu(args, rank, world):
                              "rne_gbs": launch_bytes / (rne_ms * 1e-3) / 1e9,
                              "sr_gbs": launch_bytes / (sr_ms * 1e-3) / 1e9}}
 
-    # ---- end to end through host buffers (pinned), same metric
+    # ---- end to end through host buffers (pinned), same metric.  Every step
+    # copies its input in from pinned host memory, runs both quantizes and
+    # copies its codes and scales back; steps are pipelined over two buffer
+    # slots (upload, compute and download on three streams), so step i+1's
+    # upload overlaps step i's compute and download (PCIe is full duplex).
     x_pin = x0.pin_memory()
-    xd = torch.empty_like(xs[0])
-    h_out = [{k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in o.items()} for o in outs[0]]
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    xd = [torch.empty_like(xs[0]) for _ in range(2)]
+    od = [[q.quantize(xs[0], q.MXFP4, q.RNE, rotate=True), q.quantize(xs[0], q.MXFP4, q.SR, rotate=True, seed=7)]
+          for _ in range(2)]
+    h_out = [[{k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in o.items()} for o in od[0]]
+             for _ in range(2)]
+    ev = lambda: torch.cuda.Event()                         # noqa: E731
+    in_done, comp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
     e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e2e_steps = max(3, min(args.steps, 50))
-    for it in range(e2e_steps + 2):
-        if it == 2:
-            torch.cuda.synchronize()
-            barrier()
-            e_start.record(stream)
-        xd.copy_(x_pin, non_blocking=True)
-        q.quantize(xd, q.MXFP4, q.RNE, rotate=True, out=outs[0][0])
-        q.quantize(xd, q.MXFP4, q.SR, rotate=True, seed=7, out=outs[0][1])
-        for k in ("codes", "scales"):
-            h_out[0][k].copy_(outs[0][0][k], non_blocking=True)
-            h_out[1][k].copy_(outs[0][1][k], non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    e_start.record(stream)
+    s_in.wait_event(e_start)
+    s_out.wait_event(e_start)
+    for i in range(e2e_steps):
+        b = i % 2
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(comp_done[b])               # slot's device input no longer read
+            xd[b].copy_(x_pin, non_blocking=True)
+            in_done[b].record(s_in)
+        stream.wait_event(in_done[b])
+        if i >= 2:
+            stream.wait_event(out_done[b])                  # slot's device outputs already copied out
+        q.quantize(xd[b], q.MXFP4, q.RNE, rotate=True, out=od[b][0])
+        q.quantize(xd[b], q.MXFP4, q.SR, rotate=True, seed=7, out=od[b][1])
+        comp_done[b].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(comp_done[b])
+            for j in range(2):
+                for k in ("codes", "scales"):
+                    h_out[b][j][k].copy_(od[b][j][k], non_blocking=True)
+            out_done[b].record(s_out)
+    stream.wait_event(out_done[(e2e_steps - 1) % 2])
+    stream.wait_event(out_done[(e2e_steps - 2) % 2])
     e_stop.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e_start.elapsed_time(e_stop) / e2e_steps
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_stop) / e2e_steps, dist, dev)
     h2d = x0.numel() * 2
-    d2h = sum(v.numel() for o in outs[0] for k, v in o.items() if k in ("codes", "scales"))
+    d2h = sum(v.numel() for o in od[0] for k, v in o.items() if k in ("codes", "scales"))
     e2e = {"value": world * step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
