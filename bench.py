@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--profile-case", choices=["quant", "gemm", "quant-nvfp4"], default=None,
                     help="run a few untimed calls of one kernel family (for ncu captures) and exit")
+    ap.add_argument("--rows", action="store_true",
+                    help="time every entry point of the path on its own full-size workload (one JSON line each)")
     return ap.parse_args()
 
 
@@ -432,10 +434,199 @@ def run_profile_case(case):
     print(f"profile case {case}: ok")
 
 
+# ------------------------------------------------------------------ every entry point on its own workload
+def time_calls(torch, stream, call, iters=20, warm=3):
+    """Mean device time (ms) of call(i): CUDA events on the launching stream
+    around each call, after a device-side head start so that host overhead
+    leaves no gaps inside a bracket."""
+    for i in range(warm):
+        call(i)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+    torch.cuda._sleep(int(2e9 * 5e-3))
+    for i, (a, b) in enumerate(evs):
+        a.record(stream)
+        call(warm + i)
+        b.record(stream)
+    torch.cuda.synchronize()
+    return statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+
+def run_rows():
+    """One JSON line per entry point of the path, each on the full-size
+    synthetic workload it serves: quantize variants in GB/s of algorithmic
+    bytes against the measured HBM peak, GEMMs in TFLOP/s against the dense
+    FP4 peak.  Quantize inputs rotate over enough copies that consecutive
+    calls never find their input in L2."""
+    import torch
+
+    import bit_fwht_hadamard_b200 as q
+    import synth
+    from bit_fwht_hadamard_b200 import build as _build
+    _build.build()
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+    hbm_peak, bf16_peak, _, peak_src = measured_peaks()
+    fp4_peak = bf16_peak * FP4_PER_BF16
+    L = q.lib()
+    bad = []
+    bf16 = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)   # noqa: E731
+
+    def ok(st):
+        if st != q.OK:
+            bad.append(st)
+
+    def emit(row, workload, ms, nbytes=None, flops=None, **extra):
+        d = {"row": row, "workload": workload, "ms_per_call": ms}
+        if nbytes is not None:
+            a = nbytes / (ms * 1e-3) / 1e9
+            d.update(bound="hbm", algorithmic_bytes=nbytes, achieved=a, unit="GB/s", peak=hbm_peak,
+                     frac=a / hbm_peak, peak_source=f"{peak_src} hbm_gbs")
+        else:
+            a = flops / (ms * 1e-3) / 1e12
+            d.update(bound="tensor", flops=flops, achieved=a, unit="TFLOP/s", peak=fp4_peak, frac=a / fp4_peak,
+                     peak_source=f"{peak_src} bf16_tflops x {FP4_PER_BF16}")
+        d.update(extra)
+        print(json.dumps(d), flush=True)
+
+    def n_sets(nbytes):
+        return max(1, -(-(512 << 20) // nbytes))            # > 4x L2 between two calls on the same set
+
+    def fp4_row(row, workload, x, fmt, rounding, bpe, rotate=False, block2d=False, four6=False, transposed=False,
+                seed=0):
+        M, K = x.shape
+        ns = n_sets(x.numel() * 2)
+        xs = [x] + [x.clone() for _ in range(ns - 1)]
+        outs = [q.quantize(x, fmt, rounding, rotate=rotate, block2d=block2d, four6=four6, seed=seed,
+                           transposed=transposed) for _ in range(ns)]
+        wsb = q.qfp4_quantize_workspace_bytes(M, K, fmt, rotate, block2d)
+        ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
+        av = [(xs[b].data_ptr(), q.BF16, M, K, fmt, rounding, int(rotate), int(block2d), int(four6), seed,
+               o["codes"].data_ptr(), o["scales"].data_ptr(), q._ptr(o.get("codesT")), q._ptr(o.get("scalesT")),
+               q._ptr(o.get("tscale")), ws.data_ptr(), wsb, sh) for b, o in enumerate(outs)]
+        ms = time_calls(torch, stream, lambda i: ok(L.qfp4_quantize(*av[i % ns])))
+        emit(row, workload, ms, nbytes=bpe * M * K, bytes_per_element=bpe, input_sets=ns)
+
+    def mxfp8_row(row, workload, x, rounding, transposed, seed=0):
+        M, K = x.shape
+        bpe = 2 + (1 + 1 / 32) * (2 if transposed else 1)
+        ns = n_sets(x.numel() * 2)
+        xs = [x] + [x.clone() for _ in range(ns - 1)]
+        outs = [q.quantize_mxfp8(x, rounding, seed=seed, transposed=transposed) for _ in range(ns)]
+        av = [(xs[b].data_ptr(), q.BF16, M, K, rounding, seed, o["codes"].data_ptr(), o["scales"].data_ptr(),
+               q._ptr(o.get("codesT")), q._ptr(o.get("scalesT")), sh) for b, o in enumerate(outs)]
+        ms = time_calls(torch, stream, lambda i: ok(L.qfp4_quantize_mxfp8(*av[i % ns])))
+        emit(row, workload, ms, nbytes=bpe * M * K, bytes_per_element=bpe, input_sets=ns)
+
+    def dequant_row(row, workload, x, fmt, out_dtype):
+        M, K = x.shape
+        g = 32 if fmt == q.MXFP4 else 16
+        bpe = 0.5 + 1 / g + (4 if out_dtype == torch.float32 else 2)
+        ns = n_sets(M * K // 2)
+        src = [q.quantize(x, fmt) for _ in range(ns)]
+        outs = [torch.empty((M, K), dtype=out_dtype, device=dev) for _ in range(ns)]
+        odt = q.F32 if out_dtype == torch.float32 else q.BF16
+        av = [(s["codes"].data_ptr(), s["scales"].data_ptr(), q._ptr(s.get("tscale")), M, K, fmt, odt,
+               outs[b].data_ptr(), sh) for b, s in enumerate(src)]
+        ms = time_calls(torch, stream, lambda i: ok(L.qfp4_dequantize(*av[i % ns])))
+        emit(row, workload, ms, nbytes=bpe * M * K, bytes_per_element=bpe, input_sets=ns)
+
+    def gemm_row(row, workload, A, B, M, N, K, fmt, out_dtype):
+        out = torch.empty((M, N), dtype=out_dtype, device=dev)
+        wsb = q.qfp4_gemm_workspace_bytes(M, N, K, fmt)
+        ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
+        odt = q.F32 if out_dtype == torch.float32 else q.BF16
+        av = (A["codes"].data_ptr(), A["scales"].data_ptr(), q._ptr(A.get("tscale")), B["codes"].data_ptr(),
+              B["scales"].data_ptr(), q._ptr(B.get("tscale")), M, N, K, fmt, odt, out.data_ptr(), ws.data_ptr(), wsb,
+              sh)
+        ms = time_calls(torch, stream, lambda i: ok(L.qfp4_gemm_blockscaled(*av)))
+        emit(row, workload, ms, flops=2.0 * M * N * K)
+
+    def fused_row(row, workload, A_bf16, B, N, fmt, out_dtype):
+        M, K = A_bf16.shape
+        out = torch.empty((M, N), dtype=out_dtype, device=dev)
+        wsb = q.qfp4_gemm_fused_rq_workspace_bytes(M, N, K, fmt)
+        ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
+        odt = q.F32 if out_dtype == torch.float32 else q.BF16
+        av = (A_bf16.data_ptr(), M, K, 1, 0, fmt, B["codes"].data_ptr(), B["scales"].data_ptr(),
+              q._ptr(B.get("tscale")), N, ws.data_ptr(), wsb, odt, out.data_ptr(), sh)
+        ms = time_calls(torch, stream, lambda i: ok(L.qfp4_gemm_fused_rq(*av)))
+        emit(row, workload, ms, flops=2.0 * M * N * K)
+
+    F32, BF = torch.float32, torch.bfloat16
+    with ClockSampler(0) as clk:
+        # rotation + MXFP4 (the default bench step's two launches, one at a time)
+        x2 = bf16(synth.cfg2_X())
+        for r, name in ((q.RNE, "RNE"), (q.SR, "SR")):
+            fp4_row("a0 a1 a3 a5", f"X bf16 4096x4096 (N(0,1), 40 channels x20): FWHT-128 + MXFP4 {name}", x2,
+                    q.MXFP4, r, 2 + 0.5 + 1 / 32, rotate=True, seed=7)
+        # NVFP4 forward-linear operands: tensor amax, E4M3 scales, four-over-six
+        x3, w3 = bf16(synth.cfg3_X()), bf16(synth.cfg3_W())
+        nv = 2 + 0.5 + 1 / 16
+        fp4_row("a2 a3 a4 a5", "X bf16 8192x4096 Student-t(3)*0.5: NVFP4 four-over-six RNE", x3, q.NVFP4, q.RNE, nv,
+                four6=True)
+        fp4_row("a2 a3 a4 a5", "W bf16 11008x4096 N(0,0.02^2): NVFP4 four-over-six RNE", w3, q.NVFP4, q.RNE, nv,
+                four6=True)
+        fp4_row("a2 a3 a5", "X bf16 8192x4096 Student-t(3)*0.5: NVFP4 RNE", x3, q.NVFP4, q.RNE, nv)
+        fp4_row("a2 a3 a5", "X bf16 8192x4096 Student-t(3)*0.5: NVFP4 Philox SR", x3, q.NVFP4, q.SR, nv, seed=7)
+        dequant_row("decode", "NVFP4 codes of X 8192x4096 -> bf16", x3, q.NVFP4, BF)
+        dequant_row("decode", "NVFP4 codes of X 8192x4096 -> fp32", x3, q.NVFP4, F32)
+        # Quartet-style backward: 2D blocks, MXFP8, column-wise 1D
+        g4 = bf16(synth.cfg4_G())
+        fp4_row("a6", "G bf16 8192x4096 (N(0,1e-6), 0.1% x100): 2D 16x16 NVFP4 Philox SR, G and G^T", g4, q.NVFP4,
+                q.SR, 2 + 2 * (0.5 + 1 / 16), block2d=True, transposed=True, seed=11)
+        fp4_row("a6", "G bf16 8192x4096: 2D 16x16 NVFP4 RNE, G and G^T", g4, q.NVFP4, q.RNE,
+                2 + 2 * (0.5 + 1 / 16), block2d=True, transposed=True)
+        fp4_row("column-wise", "G bf16 8192x4096: 1D MXFP4 RNE rows + independent column-wise groups", g4, q.MXFP4,
+                q.RNE, 2 + 2 * (0.5 + 1 / 32), transposed=True)
+        for r, name in ((q.RNE, "RNE"), (q.SR, "SR")):
+            mxfp8_row("a7", f"G bf16 8192x4096: MXFP8 E4M3 g32 {name}", g4, r, False, seed=11)
+        mxfp8_row("a7", "G bf16 8192x4096: MXFP8 E4M3 g32 RNE, rows + column-wise", g4, q.RNE, True)
+        # backward GEMMs on 2D-quantized operands: dX = G W, dW = G^T X
+        x4, w4 = bf16(synth.cfg4_X()), bf16(synth.cfg4_W())
+        G2 = q.quantize(g4, q.NVFP4, q.SR, block2d=True, transposed=True, seed=11)
+        W2 = q.quantize(w4, q.NVFP4, q.RNE, block2d=True, transposed=True)
+        X2 = q.quantize(x4, q.NVFP4, q.RNE, block2d=True, transposed=True)
+        T = lambda o: {"codes": o["codesT"], "scales": o["scalesT"], "tscale": o["tscale"]}   # noqa: E731
+        gemm_row("a8", "dX = G W: NVFP4 8192x4096x4096, fp32 out", G2, T(W2), 8192, 4096, 4096, q.NVFP4, F32)
+        gemm_row("a8", "dW = G^T X: NVFP4 4096x4096x8192, fp32 out", T(G2), T(X2), 4096, 4096, 8192, q.NVFP4, F32)
+        del G2, W2, X2, x4, w4, g4, x3, w3
+        # 7B-class linear shapes: the GEMM alone and the fused rotate + quantize + GEMM
+        for (M, N, K) in ((16384, 4096, 4096), (16384, 14336, 4096), (16384, 4096, 14336)):
+            a5 = bf16(synth.cfg5_A(M, K))
+            B5 = q.quantize(bf16(synth.cfg5_B(N, K)), q.NVFP4, q.RNE, rotate=True)
+            A5 = q.quantize(a5, q.NVFP4, q.RNE, rotate=True)
+            gemm_row("a8", f"NVFP4 GEMM {M}x{N}x{K} (A pre-quantized), bf16 out", A5, B5, M, N, K, q.NVFP4, BF)
+            fused_row("a9", f"fused FWHT-128 + NVFP4 RNE of A bf16 + GEMM {M}x{N}x{K}, bf16 out", a5, B5, N, q.NVFP4,
+                      BF)
+            del a5, B5, A5
+        # standalone quantize bandwidth over 2^20 .. 2^30 bf16 elements (K = 4096):
+        # rows of the 16384 x 4096 outlier-channel input, repeated past 2^26 elements
+        base = bf16(synth.cfg5_A(16384, 4096))
+        for e in range(20, 31, 2):
+            M = (1 << e) // 4096
+            x = base[:M].clone() if M <= 16384 else base.repeat(M // 16384, 1)
+            fp4_row("sweep", f"2^{e} bf16 elements ({M}x4096): NVFP4 RNE", x, q.NVFP4, q.RNE, nv)
+            fp4_row("sweep", f"2^{e} bf16 elements ({M}x4096): FWHT-128 + MXFP4 RNE", x, q.MXFP4, q.RNE,
+                    2 + 0.5 + 1 / 32, rotate=True)
+            del x
+    torch.cuda.synchronize()
+    err = q.qfp4_last_device_error()
+    print(json.dumps({"rows_done": True, "clocks": clk.summary(), "device_error": err, "bad_status": sorted(set(bad)),
+                      "csrc": csrc_hash()}), flush=True)
+    if bad or err:
+        raise RuntimeError(f"status {sorted(set(bad))}, device error {err}")
+
+
 def main():
     args = parse()
     if args.profile_case:
         run_profile_case(args.profile_case)
+        return
+    if args.rows:
+        run_rows()
         return
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -20,49 +20,112 @@ __device__ __forceinline__ uint16_t f64_to_bf16_rn(double v)
     return static_cast<uint16_t>((u >> 16) | (signbit(v) ? 0x8000u : 0u));
 }
 
-__device__ __forceinline__ double e2m1_value_f64(uint32_t c)
+// bfloat16 bits of the exact product m * s, given p = fl(m * s) (binary32)
+// and its exact error e = m * s - p (one FMA).  Rounding p to bfloat16 by
+// ties-to-even gives the rounding of m * s except when p is itself a
+// bfloat16 midpoint, where the sign of e says on which side m * s lies.
+// Needs |p| >= 2^-100 (the error of the product is then representable) or
+// m * s exactly zero.
+__device__ __forceinline__ uint32_t bf16_from_split(float p, float e)
 {
-    const uint32_t E = (c >> 1) & 3u, m = c & 1u;
-    const double mag = (E == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, static_cast<int>(E) - 1);
-    return (c & 8u) ? -mag : mag;
+    const uint32_t u = __float_as_uint(p);
+    if ((u & 0xFFFFu) == 0x8000u && e != 0.0f) {
+        const bool away = (e > 0.0f) == (p > 0.0f);      // m * s beyond the midpoint in magnitude
+        return (away ? u + 0x8000u : u - 0x8000u) >> 16;
+    }
+    return (u + 0x7FFFu + ((u >> 16) & 1u)) >> 16;
 }
 
-// One thread: 16 consecutive elements (one NVFP4 block, half an MXFP4 group).
+// 2^(b - 128) for a byte b, as binary32 (2^-128 and 2^-127 are subnormal).
+__device__ __forceinline__ float exp2_b128(uint32_t b)
+{
+    return __uint_as_float(b >= 2u ? (b - 1u) << 23 : 0x00200000u << b);
+}
+
+// One 16-element chunk (one NVFP4 block, half an MXFP4 group) from its code
+// word pair w and scale byte sb.  Every output is the exact value
+// g * scale (* s_t) rounded once:
+// - MXFP4: g * 2^(b-127) = (2 g) * 2^(b-128) has at most two significant bits
+//   and an exponent >= -129, so it is exact in binary32 and in bfloat16.
+// - NVFP4: m = g * dec(enc) is exact (at most 6 significant bits, inside the
+//   normal range), and fl(m * s_t) is the one rounding (binary32 out); for
+//   bfloat16 out the rounding uses the split above, or binary64 for products
+//   below 2^-100 or beyond the binary32 range.
+// A scale byte that encodes NaN (E8M0 0xFF, E4M3 0x7F / 0xFF) gives NaN.
+template <int FMT, int OUT>
+__device__ __forceinline__ void dequant_chunk(uint2 w, uint32_t sb, float st, int64_t e0, void *out)
+{
+    const uint64_t st2 = f2pack(st, st);
+    uint64_t g[8], m[8], v[8];
+    e2m1x8_values(w.x, g);
+    e2m1x8_values(w.y, g + 4);
+    if (FMT == QFP4_MXFP4) {
+        const float h = sb == 255u ? __uint_as_float(0x7FC00000u) : exp2_b128(sb);   // E8M0 0xFF: NaN
+        const uint64_t two = f2pack(2.0f, 2.0f), h2 = f2pack(h, h);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = f2mul(f2mul(g[j], two), h2);
+    } else {
+        const float d = (sb & 0x7Fu) == 0x7Fu ? __uint_as_float(0x7FC00000u) : e4m3_value(sb);   // E4M3 NaN
+        const uint64_t d2 = f2pack(d, d);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            m[j] = f2mul(g[j], d2);
+            v[j] = f2mul(m[j], st2);
+        }
+    }
+    if (OUT == QFP4_F32) {
+        float4 *o = reinterpret_cast<float4 *>(static_cast<float *>(out) + e0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            float a, b, c, d;
+            f2unpack(v[2 * q], a, b);
+            f2unpack(v[2 * q + 1], c, d);
+            o[q] = make_float4(a, b, c, d);
+        }
+    } else {
+        uint32_t h[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            float p[2], mm[2];
+            f2unpack(v[j], p[0], p[1]);
+            uint32_t b16[2];
+            if (FMT == QFP4_MXFP4) {
+                b16[0] = __float_as_uint(p[0]) >> 16;          // exact in bfloat16
+                b16[1] = __float_as_uint(p[1]) >> 16;
+            } else {
+                f2unpack(m[j], mm[0], mm[1]);
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    const float a = fabsf(p[t]);
+                    if ((a >= 0x1p-100f && a <= 3.0e38f) || mm[t] == 0.0f)
+                        b16[t] = bf16_from_split(p[t], __fmaf_rn(mm[t], st, -p[t]));
+                    else if (a != a)
+                        b16[t] = 0x7FC0u;
+                    else
+                        b16[t] = f64_to_bf16_rn(static_cast<double>(mm[t]) * static_cast<double>(st));
+                }
+            }
+            h[j] = b16[0] | (b16[1] << 16);
+        }
+        uint4 *o = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(out) + e0);
+        o[0] = make_uint4(h[0], h[1], h[2], h[3]);
+        o[1] = make_uint4(h[4], h[5], h[6], h[7]);
+    }
+}
+
+// One thread per 16-element chunk (grid-stride loop).
 template <int FMT, int OUT>
 __global__ void __launch_bounds__(256) k_dequant(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scales,
                                                  const float *__restrict__ tscale, int64_t n, void *out)
 {
     const int64_t chunks = n / 16;
-    const double st = FMT == QFP4_NVFP4 ? static_cast<double>(*tscale) : 1.0;
+    const float st = FMT == QFP4_NVFP4 ? *tscale : 1.0f;
     for (int64_t c = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; c < chunks;
          c += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const int64_t e0 = c * 16;
         const uint2 w = *reinterpret_cast<const uint2 *>(codes + e0 / 2);
         const uint32_t sb = scales[FMT == QFP4_MXFP4 ? e0 / 32 : e0 / 16];
-        const double sc = FMT == QFP4_MXFP4 ? ldexp(1.0, static_cast<int>(sb) - 127)
-                                            : static_cast<double>(e4m3_value(sb)) * st;
-        double d[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const uint32_t code = ((i < 8 ? w.x : w.y) >> (4 * (i & 7))) & 15u;
-            d[i] = e2m1_value_f64(code) * sc;                 // exact: <= 31 significant bits
-        }
-        if (OUT == QFP4_F32) {
-            float4 *o = reinterpret_cast<float4 *>(static_cast<float *>(out) + e0);
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                o[q] = make_float4(__double2float_rn(d[4 * q]), __double2float_rn(d[4 * q + 1]),
-                                   __double2float_rn(d[4 * q + 2]), __double2float_rn(d[4 * q + 3]));
-        } else {
-            uint32_t h[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-                h[q] = static_cast<uint32_t>(f64_to_bf16_rn(d[2 * q])) |
-                       (static_cast<uint32_t>(f64_to_bf16_rn(d[2 * q + 1])) << 16);
-            uint4 *o = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(out) + e0);
-            o[0] = make_uint4(h[0], h[1], h[2], h[3]);
-            o[1] = make_uint4(h[4], h[5], h[6], h[7]);
-        }
+        dequant_chunk<FMT, OUT>(w, sb, st, e0, out);
     }
 }
 

@@ -9,6 +9,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -279,6 +280,26 @@ __device__ __forceinline__ uint32_t e2m1x8_rne_pairs(uint64_t p0, uint64_t p1, u
     return e2m1x8_rne(v);
 }
 
+// The eight E2M1 values of a word of nibbles as binary32 (exact: binary16
+// holds every E2M1 value, and the widening is exact).
+__device__ __forceinline__ void e2m1x8_values(uint32_t w, uint64_t *g4)
+{
+    uint32_t h[4];
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+        : "r"(w));
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h[q]));
+        g4[q] = f2pack(f.x, f.y);
+    }
+}
+
 // E2M1 stochastic rounding of one value (|v| <= 6 or saturating):
 // lo <= |v| < hi adjacent grid values, up iff u < (|v| - lo) / (hi - lo)
 // with u = (w >> 8) * 2^-24.  Returns the 4-bit code.
@@ -327,6 +348,31 @@ __device__ __forceinline__ uint32_t e4m3x2_rne(float a, float b)
     uint16_t out;
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(b), "f"(a));
     return out;
+}
+
+// E4M3 stochastic rounding: lo <= |v| < hi adjacent E4M3 values (subnormal
+// spacing 2^-9 below 2^-6, else 2^(e-3)), up iff (w >> 8) * 2^-24 < (|v|-lo)/(hi-lo);
+// saturates at 448.  Returns the byte.
+__device__ __forceinline__ uint32_t e4m3_sr(float v, uint32_t w)
+{
+    const uint32_t sign = (__float_as_uint(v) >> 24) & 0x80u;
+    const float a = fabsf(v);
+    float lo, sp, inv_sp;
+    if (a >= 0.015625f) {                                    // 2^-6: normal binade
+        const uint32_t spb = (__float_as_uint(a) & 0x7F800000u) - (3u << 23);
+        lo = __uint_as_float(__float_as_uint(a) & 0x7FF00000u);
+        sp = __uint_as_float(spb);
+        inv_sp = __uint_as_float((254u << 23) - spb);
+    } else {
+        lo = __fmul_rn(truncf(__fmul_rn(a, 512.0f)), 0.001953125f);   // exact: multiples of 2^-9
+        sp = 0.001953125f;
+        inv_sp = 512.0f;
+    }
+    const float p = __fmul_rn(__fsub_rn(a, lo), inv_sp);
+    const float u = __fmul_rn(static_cast<float>(w >> 8), 5.9604644775390625e-08f);
+    float rr = (u < p) ? __fadd_rn(lo, sp) : lo;
+    rr = fminf(rr, 448.0f);
+    return e4m3_rne(rr) | sign;
 }
 
 // E4M3 byte -> binary32 (exact), from the bit fields.

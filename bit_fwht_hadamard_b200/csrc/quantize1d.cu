@@ -64,29 +64,83 @@ struct UnitOut {
     uint32_t scales;        // byte g = scale of group g within the unit
 };
 
-// Quantize 16 values under effective scale S (RNE): codes (2 words), and
-// when `sse` is given the binary32 squared error summed as a fixed tree.
-__device__ __forceinline__ void nv_block_rne(const float *x, float S, uint32_t *w2, float *sse)
+// ---------------------------------------------------------------- NVFP4 without a division per element
+// fl(a / b) (b > 0) from y = fl(1/b), correctly rounded, and two FMA
+// corrections: q0 = fl(a y) is within 1.5 ulp of a / b; q1 = fl(q0 + r0 y),
+// r0 = fl(a - b q0), is within one ulp (faithful); and with q1 faithful the
+// remainder r1 = a - b q1 is exact and q2 = fl(q1 + r1 y) is fl(a / b)
+// (P. Markstein, IBM J. Res. Dev. 34(1), 1990: a reciprocal within half an
+// ulp plus a faithful quotient give the correctly rounded one).  This needs
+// normal intermediate values; quotients below the normal range only decide
+// a zero code, whose sign is taken from a.  nb = -b.
+__device__ __forceinline__ float div_rn_by(float a, float y, float nb)
 {
-    float q[16];
-    if (S == 0.0f) {
-        w2[0] = w2[1] = 0u;
+    float q = __fmul_rn(a, y);
+    q = __fmaf_rn(__fmaf_rn(q, nb, a), y, q);
+    return __fmaf_rn(__fmaf_rn(q, nb, a), y, q);
+}
+
+// The same on packed pairs; the sign of each a is put on its quotient.
+__device__ __forceinline__ uint64_t div_rn_by2(uint64_t a, uint64_t y2, uint64_t nb2)
+{
+    uint64_t q = f2mul(a, y2);
+    q = f2fma(f2fma(q, nb2, a), y2, q);
+    q = f2fma(f2fma(q, nb2, a), y2, q);
+    return q | (a & 0x8000000080000000ull);
+}
+
+// fl(x_i / S) for 16 values held as 8 packed pairs, S > 0.  Outside
+// [2^-125, 2^125] (1/S not normal) the IEEE division.
+__device__ __forceinline__ void nv_quot16_pairs(const uint64_t *pp, float S, uint64_t *q)
+{
+    if (S >= 0x1p-125f && S <= 0x1p125f) {
+        const float y = __frcp_rn(S);
+        const uint64_t y2 = f2pack(y, y), nS2 = f2pack(-S, -S);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) q[i] = 0.0f;
+        for (int j = 0; j < 8; ++j) q[j] = div_rn_by2(pp[j], y2, nS2);
     } else {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) q[i] = __fdiv_rn(x[i], S);
-        w2[0] = e2m1x8_rne(q);
-        w2[1] = e2m1x8_rne(q + 8);
+        for (int j = 0; j < 8; ++j) {
+            float a, b;
+            f2unpack(pp[j], a, b);
+            q[j] = f2pack(__fdiv_rn(a, S), __fdiv_rn(b, S));
+        }
     }
+}
+
+// E2M1 round-to-nearest-even codes of fl(x_i / S): two words of nibbles.
+__device__ __forceinline__ void nv_codes16_pairs(const uint64_t *pp, float S, uint32_t *w2)
+{
+    uint64_t q[8];
+    nv_quot16_pairs(pp, S, q);
+    w2[0] = e2m1x8_rne_pairs(q[0], q[1], q[2], q[3]);
+    w2[1] = e2m1x8_rne_pairs(q[4], q[5], q[6], q[7]);
+}
+
+// Quantize 16 values (8 packed pairs) under effective scale S (RNE): codes
+// (2 words), and when `sse` is given the binary32 squared error of the
+// dequantized values, sum(fl(fl(fl(g_i S) - x_i)^2)) as a fixed tree
+// (i + 8 into i, then i + 4, i + 2, i + 1).
+__device__ __forceinline__ void nv_block_rne_pairs(const uint64_t *pp, float S, uint32_t *w2, float *sse)
+{
+    if (S == 0.0f) w2[0] = w2[1] = 0u;
+    else nv_codes16_pairs(pp, S, w2);
     if (sse) {
+        // Scalar IEEE operations: the multiply feeding the subtraction must
+        // stay two roundings (the packed forms gave occasional one-ulp
+        // differences in these sums), and the sums decide the selection.
+        uint64_t g[8];
+        e2m1x8_values(w2[0], g);
+        e2m1x8_values(w2[1], g + 4);
         float e[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const uint32_t code = (w2[i >> 3] >> (4 * (i & 7))) & 15u;
-            const float deq = __fmul_rn(e2m1_value(code), S);
-            const float d = __fsub_rn(deq, x[i]);
-            e[i] = __fmul_rn(d, d);
+        for (int j = 0; j < 8; ++j) {
+            float g0, g1, x0, x1;
+            f2unpack(g[j], g0, g1);
+            f2unpack(pp[j], x0, x1);
+            const float d0 = __fsub_rn(__fmul_rn(g0, S), x0), d1 = __fsub_rn(__fmul_rn(g1, S), x1);
+            e[2 * j] = __fmul_rn(d0, d0);
+            e[2 * j + 1] = __fmul_rn(d1, d1);
         }
 #pragma unroll
         for (int h = 8; h >= 1; h >>= 1)
@@ -94,6 +148,44 @@ __device__ __forceinline__ void nv_block_rne(const float *x, float S, uint32_t *
             for (int i = 0; i < h; ++i) e[i] = __fadd_rn(e[i], e[i + h]);
         *sse = e[0];
     }
+}
+
+// The same for 16 unpacked values.
+__device__ __forceinline__ void nv_block_rne(const float *x, float S, uint32_t *w2, float *sse)
+{
+    uint64_t pp[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) pp[j] = f2pack(x[2 * j], x[2 * j + 1]);
+    nv_block_rne_pairs(pp, S, w2, sse);
+}
+
+// NVFP4 block scale bytes enc = E4M3_RNE(fl(fl(amax / d) / s_t)), d = 6 or 4,
+// with the quotients from div_rn_by: fl(amax / 6) by y = fl(1/6), fl(amax / 4)
+// is exact, and fl(t / s_t) by fl(1/s_t), worked out once per thread.  The
+// fast path needs amax / d and 1/s_t normal; otherwise IEEE divisions.
+struct NvScale {
+    float s_t, y_t;
+    bool fast;
+};
+
+__device__ __forceinline__ NvScale nv_scale_setup(float s_t)
+{
+    NvScale z;
+    z.s_t = s_t;
+    z.fast = s_t >= 0x1p-120f && s_t <= 0x1p120f;
+    z.y_t = z.fast ? __frcp_rn(s_t) : 0.0f;
+    return z;
+}
+
+template <bool D6>
+__device__ __forceinline__ uint32_t nv_scale_byte(float amax, const NvScale &z)
+{
+    if (z.fast && amax >= 0x1p-120f) {
+        const float t = D6 ? div_rn_by(amax, __uint_as_float(0x3E2AAAABu), -6.0f)   // fl(1/6)
+                           : __fmul_rn(amax, 0.25f);
+        return e4m3_rne(div_rn_by(t, z.y_t, -z.s_t));
+    }
+    return e4m3_rne(__fdiv_rn(__fdiv_rn(amax, D6 ? 6.0f : 4.0f), z.s_t));
 }
 
 // Stochastic rounding of 16 (NVFP4) or 32 (MXFP4) values v (already divided
@@ -119,7 +211,8 @@ __device__ __forceinline__ void sr_group(const float *v, uint64_t e, uint64_t se
 }
 
 template <int FMT, bool SR, bool FOUR6>
-__device__ __forceinline__ void quant_unit(const float (&v)[64], uint64_t e0, float s_t, uint64_t seed, UnitOut &o)
+__device__ __forceinline__ void quant_unit(const float (&v)[64], uint64_t e0, const NvScale &nz, uint64_t seed,
+                                           UnitOut &o)
 {
     o.scales = 0u;
     if (FMT == QFP4_MXFP4) {
@@ -156,18 +249,18 @@ __device__ __forceinline__ void quant_unit(const float (&v)[64], uint64_t e0, fl
             uint32_t *w = o.codes + 2 * b;
             uint32_t enc = 0u;
             float S = 0.0f;
-            if (s_t != 0.0f) {
-                enc = e4m3_rne(__fdiv_rn(__fdiv_rn(amax, 6.0f), s_t));
-                S = __fmul_rn(e4m3_value(enc), s_t);
+            if (nz.s_t != 0.0f) {
+                enc = nv_scale_byte<true>(amax, nz);
+                S = __fmul_rn(e4m3_value(enc), nz.s_t);
             }
             if (FOUR6) {
                 uint32_t w6[2], w4[2];
                 float sse6, sse4;
                 uint32_t enc4 = 0u;
                 float S4 = 0.0f;
-                if (s_t != 0.0f) {
-                    enc4 = e4m3_rne(__fdiv_rn(__fdiv_rn(amax, 4.0f), s_t));
-                    S4 = __fmul_rn(e4m3_value(enc4), s_t);
+                if (nz.s_t != 0.0f) {
+                    enc4 = nv_scale_byte<false>(amax, nz);
+                    S4 = __fmul_rn(e4m3_value(enc4), nz.s_t);
                 }
                 nv_block_rne(x, S, w6, &sse6);
                 nv_block_rne(x, S4, w4, &sse4);
@@ -179,9 +272,13 @@ __device__ __forceinline__ void quant_unit(const float (&v)[64], uint64_t e0, fl
                 if (S == 0.0f) {
                     w[0] = w[1] = 0u;
                 } else {
+                    uint64_t pp[8], qq[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) pp[j] = f2pack(x[2 * j], x[2 * j + 1]);
+                    nv_quot16_pairs(pp, S, qq);
                     float q[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) q[i] = __fdiv_rn(x[i], S);
+                    for (int j = 0; j < 8; ++j) f2unpack(qq[j], q[2 * j], q[2 * j + 1]);
                     sr_group<16>(q, e0 + 16 * b, seed, w);
                 }
             } else {
@@ -343,7 +440,7 @@ struct UnitP {
 // c * 2^-k itself is normal for k <= 120; larger k (groups near the top of
 // the binary32 range) take the two multiplies.
 template <int UP, int FMT, bool SR, bool FOUR6, bool RAW = false>
-__device__ __forceinline__ void quant_unit_packed(uint64_t (&p)[UP], uint64_t e0, float s_t, uint64_t seed,
+__device__ __forceinline__ void quant_unit_packed(uint64_t (&p)[UP], uint64_t e0, const NvScale &nz, uint64_t seed,
                                                   UnitP<UP> &o)
 {
     static_assert(!RAW || (FMT == QFP4_MXFP4 && !SR), "raw values only on the MXFP4 round-to-nearest path");
@@ -389,19 +486,19 @@ __device__ __forceinline__ void quant_unit_packed(uint64_t (&p)[UP], uint64_t e0
             uint32_t *w = o.codes + 2 * b;
             uint32_t enc = 0u;
             float S = 0.0f;
-            if (s_t != 0.0f) {
-                enc = e4m3_rne(__fdiv_rn(__fdiv_rn(amax, 6.0f), s_t));
-                S = __fmul_rn(e4m3_value(enc), s_t);
+            if (nz.s_t != 0.0f) {
+                enc = nv_scale_byte<true>(amax, nz);
+                S = __fmul_rn(e4m3_value(enc), nz.s_t);
             }
             if (FOUR6) {
                 uint32_t w6[2], w4[2], enc4 = 0u;
                 float sse6, sse4, S4 = 0.0f;
-                if (s_t != 0.0f) {
-                    enc4 = e4m3_rne(__fdiv_rn(__fdiv_rn(amax, 4.0f), s_t));
-                    S4 = __fmul_rn(e4m3_value(enc4), s_t);
+                if (nz.s_t != 0.0f) {
+                    enc4 = nv_scale_byte<false>(amax, nz);
+                    S4 = __fmul_rn(e4m3_value(enc4), nz.s_t);
                 }
-                nv_block_rne(x, S, w6, &sse6);
-                nv_block_rne(x, S4, w4, &sse4);
+                nv_block_rne_pairs(p + 8 * b, S, w6, &sse6);
+                nv_block_rne_pairs(p + 8 * b, S4, w4, &sse4);
                 const bool pick4 = sse4 < sse6;
                 w[0] = pick4 ? w4[0] : w6[0];
                 w[1] = pick4 ? w4[1] : w6[1];
@@ -410,13 +507,15 @@ __device__ __forceinline__ void quant_unit_packed(uint64_t (&p)[UP], uint64_t e0
                 if (S == 0.0f) {
                     w[0] = w[1] = 0u;
                 } else {
+                    uint64_t qq[8];
+                    nv_quot16_pairs(p + 8 * b, S, qq);
                     float q[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) q[i] = __fdiv_rn(x[i], S);
+                    for (int j = 0; j < 8; ++j) f2unpack(qq[j], q[2 * j], q[2 * j + 1]);
                     sr_group<16>(q, e0 + 16 * b, seed, w);
                 }
             } else {
-                nv_block_rne(x, S, w, nullptr);
+                nv_block_rne_pairs(p + 8 * b, S, w, nullptr);
             }
             o.scales[b >> 2] |= enc << (8 * (b & 3));
         }
@@ -441,6 +540,66 @@ __device__ __forceinline__ void store_unit_packed(const UnitP<UP> &o, const Quan
     else *reinterpret_cast<uint16_t *>(sdst) = static_cast<uint16_t>(o.scales[0]);
 }
 
+// MXFP8 of UP packed pairs (2*UP values, groups of 32): E8M0 scale with
+// 448 * 2^k >= amax (least k), elements fl(v * 2^-k) to E4M3 by
+// round-to-nearest-even or by the stochastic rule on the E4M3 grid (one
+// Philox call per 4 elements, counter = index / 4).  An all-zero group gives
+// scale byte 0 and zero codes.  2*UP code bytes in UP/2 words.
+template <int UP, bool SR>
+__device__ __forceinline__ void mxfp8_unit_packed(uint64_t (&p)[UP], uint64_t e0, uint64_t seed, uint32_t *codes,
+                                                  uint32_t &scales)
+{
+    scales = 0u;
+#pragma unroll
+    for (int g = 0; g < UP / 16; ++g) {
+        uint64_t *pg = p + 16 * g;
+        uint32_t *w = codes + 8 * g;
+        const float amax = absmax_pairs<16>(pg);
+        if (amax == 0.0f) {
+#pragma unroll
+            for (int t = 0; t < 8; ++t) w[t] = 0u;
+            continue;
+        }
+        const int k = scale_exp(amax, 0x600000u, 8);
+        scales |= static_cast<uint32_t>(k + 127) << (8 * g);
+        const float mk = exp2i(-k);
+        const uint64_t m2 = f2pack(mk, mk);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) pg[j] = f2mul(pg[j], m2);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            float a, b, c, d;
+            f2unpack(pg[2 * t], a, b);
+            f2unpack(pg[2 * t + 1], c, d);
+            if (SR) {
+                const uint4 rw = sr_words4(seed, ((e0 + 32 * g) >> 2) + t);
+                w[t] = e4m3_sr(a, rw.x) | (e4m3_sr(b, rw.y) << 8) | (e4m3_sr(c, rw.z) << 16) | (e4m3_sr(d, rw.w) << 24);
+            } else {
+                w[t] = e4m3x2_rne(a, b) | (e4m3x2_rne(c, d) << 16);
+            }
+        }
+    }
+}
+
+// 2*UP MXFP8 code bytes and UP/16 scale bytes of a unit starting at element
+// e0 (n_valid: 2*UP, or 64 when the launch range ends half way through).
+template <int UP>
+__device__ __forceinline__ void mxfp8_store_unit(const uint32_t *codes, uint32_t scales, const QuantParams &p,
+                                                 uint64_t e0, int64_t n_valid)
+{
+    uint4 *c4 = reinterpret_cast<uint4 *>(p.codes + e0);
+    const int nc = n_valid >= 2 * UP ? UP / 8 : 4;         // 16-byte chunks
+#pragma unroll
+    for (int c = 0; c < UP / 8; ++c)
+        if (c < nc) c4[c] = make_uint4(codes[4 * c], codes[4 * c + 1], codes[4 * c + 2], codes[4 * c + 3]);
+    uint8_t *sdst = p.scales + e0 / 32;
+    if (n_valid >= 2 * UP && UP == 32) *reinterpret_cast<uint16_t *>(sdst) = static_cast<uint16_t>(scales);
+    else
+#pragma unroll
+        for (int g = 0; g < UP / 16; ++g)
+            if (32 * g < n_valid) sdst[g] = static_cast<uint8_t>(scales >> (8 * g));
+}
+
 // ---------------------------------------------------------------- TMA kernel
 // WARPS warps per CTA (one CTA per SM), each with a STAGES-deep ring of tiles
 // of 32 * (UP / 32) ... = UP rows of 64 bf16 (one unit of UP pairs per lane).
@@ -460,7 +619,7 @@ __global__ void __launch_bounds__(32 * WARPS, 1) k_quant1d_tma(const __grid_cons
     const int64_t ntiles = (rows + TILE_ROWS - 1) / TILE_ROWS;
     // contiguous tile range of this CTA, balanced to one tile
     const int64_t t_begin = ntiles * blockIdx.x / gridDim.x, t_end = ntiles * (blockIdx.x + 1) / gridDim.x;
-    constexpr int G = FMT == QFP4_MXFP4 ? 32 : 16;
+    constexpr int G = FMT == QFP4_NVFP4 ? 16 : 32;
 
     uint64_t *bars = full[warp];
     uint8_t *ring = smem + warp * (STAGES * STAGE_BYTES);
@@ -477,6 +636,7 @@ __global__ void __launch_bounds__(32 * WARPS, 1) k_quant1d_tma(const __grid_cons
         s_t = tensor_scale(p, red);
         if (p.write_tscale && blockIdx.x == 0 && threadIdx.x == 0) *p.tscale_out = s_t;
     }
+    const NvScale nz = nv_scale_setup(s_t);
 
     auto issue = [&](int64_t t, int s) {
         mbar_arrive_expect_tx(&bars[s], STAGE_BYTES);
@@ -515,6 +675,11 @@ __global__ void __launch_bounds__(32 * WARPS, 1) k_quant1d_tma(const __grid_cons
                 v[32 * h + 4 * c + 3] = bf16x2_to_f2(w.w);
             }
         }
+        // The refill below is an async-proxy write to the stage these
+        // generic-proxy reads come from: without the proxy fence in every
+        // lane the two are unordered, and late reads (the last row chunks,
+        // which a short computation needs last) could see the next tile.
+        fence_proxy_async();
         __syncwarp();
         if (lane == 0) {
             const int64_t tn = t + static_cast<int64_t>(STAGES) * WARPS;
@@ -529,9 +694,15 @@ __global__ void __launch_bounds__(32 * WARPS, 1) k_quant1d_tma(const __grid_cons
             tmax = fmaxf(tmax, absmax_pairs<UP>(v));   // rows past the end were zero-filled by TMA
         } else if (n_valid > 0) {
             const uint64_t e0 = p.e_base + static_cast<uint64_t>(row0) * 64u;
-            UnitP<UP> o;
-            quant_unit_packed<UP, FMT, SR, FOUR6, RAW>(v, e0, s_t, p.seed, o);
-            store_unit_packed<UP, G>(o, p, e0, n_valid);
+            if constexpr (FMT == FMT_MXFP8) {
+                uint32_t cw[UP / 2], sc;
+                mxfp8_unit_packed<UP, SR>(v, e0, p.seed, cw, sc);
+                mxfp8_store_unit<UP>(cw, sc, p, e0, n_valid);
+            } else {
+                UnitP<UP> o;
+                quant_unit_packed<UP, FMT, SR, FOUR6, RAW>(v, e0, nz, p.seed, o);
+                store_unit_packed<UP, G>(o, p, e0, n_valid);
+            }
         }
     }
     if (gave_up && lane == 0) settle_ns(kSettleNs);   // loads of this warp's ring may still be landing
@@ -564,6 +735,7 @@ __global__ void __launch_bounds__(128) k_quant1d_direct(const T *__restrict__ x,
         s_t = tensor_scale(p, red);
         if (p.write_tscale && blockIdx.x == 0 && threadIdx.x == 0) *p.tscale_out = s_t;
     }
+    const NvScale nz = nv_scale_setup(s_t);
     const int64_t units = (p.n + 63) / 64;
     float tmax = 0.0f;
     for (int64_t u0 = static_cast<int64_t>(blockIdx.x) * blockDim.x; u0 < units;
@@ -610,7 +782,7 @@ __global__ void __launch_bounds__(128) k_quant1d_direct(const T *__restrict__ x,
         } else if (n_valid > 0) {
             const uint64_t e0 = p.e_base + static_cast<uint64_t>(off);
             UnitOut o;
-            quant_unit<FMT, SR, FOUR6>(v, e0, s_t, p.seed, o);
+            quant_unit<FMT, SR, FOUR6>(v, e0, nz, p.seed, o);
             store_unit<G>(o, p, e0, n_valid);
         }
     }
@@ -621,7 +793,7 @@ __global__ void __launch_bounds__(128) k_quant1d_direct(const T *__restrict__ x,
 }
 
 // ---------------------------------------------------------------- host launchers
-static int smem_configured[2][2][2][2][2] = {};
+static int smem_configured[2][3][2][2][2] = {};
 
 template <int MODE, int FMT, bool ROT, bool SR, bool FOUR6>
 static int launch_tma(const CUtensorMap &tm, const QuantParams &p, int grid, cudaStream_t stream)
@@ -707,6 +879,28 @@ static int run_pass(const void *x, qfp4_dtype xdt, int64_t n, QuantParams p, cud
 }
 
 // Partial maxima of |x| over a flat range (the NVFP4 tensor-amax pass, no rotation).
+int mxfp8_rows(const void *x, int64_t n, bool sr, uint64_t seed, uint8_t *codes, uint8_t *scales, cudaStream_t stream)
+{
+    if (n <= 0) return QFP4_OK;
+    CUtensorMap tm;
+    const uint64_t dims[2] = {64, static_cast<uint64_t>(n / 64)};
+    const uint64_t strides[1] = {128};
+    const uint32_t box[2] = {64, QT_TILE_ROWS};
+    int st = encode_tensor_map(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x), dims, strides, box,
+                               CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != QFP4_OK) return st;
+    QuantParams q{};
+    q.n = n;
+    q.e_base = 0;
+    q.codes = codes;
+    q.scales = scales;
+    q.seed = seed;
+    const int64_t ntiles = (n / 64 + QT_TILE_ROWS - 1) / QT_TILE_ROWS;
+    const int grid = static_cast<int>(imin<int64_t>((ntiles + qt_warps(false) - 1) / qt_warps(false), num_sms()));
+    return sr ? launch_tma<MODE_QUANT, FMT_MXFP8, false, true, false>(tm, q, grid, stream)
+              : launch_tma<MODE_QUANT, FMT_MXFP8, false, false, false>(tm, q, grid, stream);
+}
+
 int amax_partials(const void *x, qfp4_dtype xdt, int64_t n, float *partials, int *n_parts, cudaStream_t stream)
 {
     QuantParams p{};

@@ -6,6 +6,10 @@ namespace qfp4 {
 
 enum { MODE_AMAX = 0, MODE_QUANT = 1 };
 
+// Element format of the 1D kernels besides QFP4_MXFP4 / QFP4_NVFP4: MXFP8
+// (E4M3 elements, E8M0 scale per 32), row-wise.
+constexpr int FMT_MXFP8 = 2;
+
 // Upper bound on the number of partial tensor maxima a pass writes.
 constexpr int kMaxPartials = 1024;
 
@@ -24,6 +28,11 @@ struct QuantParams {
 
 int quantize1d(const void *x, qfp4_dtype xdt, int64_t n, qfp4_fmt fmt, qfp4_round rounding, int rotate, int four6,
                uint64_t seed, uint8_t *codes, uint8_t *scales, float *tscale, float *partials, int *n_parts_out,
+               cudaStream_t stream);
+
+// MXFP8 row-wise over a bf16 stream of n elements (n % 64 == 0) through the
+// TMA kernel.
+int mxfp8_rows(const void *x, int64_t n, bool sr, uint64_t seed, uint8_t *codes, uint8_t *scales,
                cudaStream_t stream);
 
 int amax_partials(const void *x, qfp4_dtype xdt, int64_t n, float *partials, int *n_parts, cudaStream_t stream);

@@ -32,24 +32,38 @@ struct Q2DParams {
     uint64_t seed;
 };
 
+// 16 consecutive elements as raw words (bf16: 32 bytes, binary32: 64 bytes),
+// so that the next task's loads can be in flight during this task's work.
 template <typename T>
-__device__ __forceinline__ void load16(const T *x, int64_t off, float *v)
+struct Raw16 {
+    uint4 w[sizeof(T) == 4 ? 4 : 2];
+};
+
+template <typename T>
+__device__ __forceinline__ void raw_load16(const T *x, int64_t off, bool valid, Raw16<T> &r)
 {
-    if (sizeof(T) == 4) {
-        const float4 *s = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(x) + off);
+    if (valid) {
+        const uint4 *s = reinterpret_cast<const uint4 *>(x + off);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const float4 f = s[c];
-            v[4 * c] = f.x;
-            v[4 * c + 1] = f.y;
-            v[4 * c + 2] = f.z;
-            v[4 * c + 3] = f.w;
-        }
+        for (int c = 0; c < (sizeof(T) == 4 ? 4 : 2); ++c) r.w[c] = s[c];
     } else {
-        const uint4 *s = reinterpret_cast<const uint4 *>(reinterpret_cast<const uint16_t *>(x) + off);
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            const uint4 w = s[c];
+        for (int c = 0; c < (sizeof(T) == 4 ? 4 : 2); ++c) r.w[c] = make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+
+template <typename T>
+__device__ __forceinline__ void raw_to_f32(const Raw16<T> &r, float *v)
+{
+#pragma unroll
+    for (int c = 0; c < (sizeof(T) == 4 ? 4 : 2); ++c) {
+        const uint4 w = r.w[c];
+        if (sizeof(T) == 4) {
+            v[4 * c] = __uint_as_float(w.x);
+            v[4 * c + 1] = __uint_as_float(w.y);
+            v[4 * c + 2] = __uint_as_float(w.z);
+            v[4 * c + 3] = __uint_as_float(w.w);
+        } else {
             v[8 * c] = bf16lo(w.x);
             v[8 * c + 1] = bf16hi(w.x);
             v[8 * c + 2] = bf16lo(w.y);
@@ -97,21 +111,29 @@ __global__ void __launch_bounds__(256) k_quant2d(const T *__restrict__ x, Q2DPar
     __shared__ float red[32];
     const float s_t = tensor_scale_from(p.partials, p.n_partials, red);
     if (p.tscale_out && blockIdx.x == 0 && threadIdx.x == 0) *p.tscale_out = s_t;
+    const NvScale nz = nv_scale_setup(s_t);
 
     const int lane = threadIdx.x & 31, half = lane >> 4, r = lane & 15;
     const int64_t tiles_k = p.K / 16, pairs = (tiles_k + 1) / 2;
     const int64_t tasks = (p.M / 16) * pairs;
     const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    // this lane's row of a task: row band*16 + r, columns tc*16 .. +15
+    auto fetch = [&](int64_t task, Raw16<T> &dst) {
+        const int64_t band = task / pairs, tc = (task % pairs) * 2 + half;
+        raw_load16(x, (band * 16 + r) * p.K + tc * 16, tc < tiles_k, dst);
+    };
+    Raw16<T> cur;
+    if (warp0 < tasks) fetch(warp0, cur);
     for (int64_t task = warp0; task < tasks; task += nwarps) {
+        Raw16<T> nxt{};
+        if (task + nwarps < tasks) fetch(task + nwarps, nxt);      // in flight during this task
         const int64_t band = task / pairs, tc = (task % pairs) * 2 + half;
         const bool valid = tc < tiles_k;
         const int64_t i = band * 16 + r, j0 = tc * 16;
         float v[16];
-        if (valid) load16(x, i * p.K + j0, v);
-        else
-#pragma unroll
-            for (int t = 0; t < 16; ++t) v[t] = 0.0f;
+        raw_to_f32(cur, v);
+        cur = nxt;
         float amax = 0.0f;
 #pragma unroll
         for (int t = 0; t < 16; ++t) amax = fmaxf(amax, fabsf(v[t]));
@@ -120,18 +142,22 @@ __global__ void __launch_bounds__(256) k_quant2d(const T *__restrict__ x, Q2DPar
         uint32_t enc = 0u;
         float S = 0.0f;
         if (s_t != 0.0f) {
-            enc = e4m3_rne(__fdiv_rn(__fdiv_rn(amax, 6.0f), s_t));
+            enc = nv_scale_byte<true>(amax, nz);
             S = __fmul_rn(e4m3_value(enc), s_t);
         }
         uint32_t w[2] = {0u, 0u};
         if (S != 0.0f) {
-            float q[16];
+            if (SR) {
+                uint64_t pp[8], qq[8];
 #pragma unroll
-            for (int t = 0; t < 16; ++t) q[t] = __fdiv_rn(v[t], S);
-            if (SR) sr_group<16>(q, static_cast<uint64_t>(i * p.K + j0), p.seed, w);
-            else {
-                w[0] = e2m1x8_rne(q);
-                w[1] = e2m1x8_rne(q + 8);
+                for (int t = 0; t < 8; ++t) pp[t] = f2pack(v[2 * t], v[2 * t + 1]);
+                nv_quot16_pairs(pp, S, qq);
+                float q[16];
+#pragma unroll
+                for (int t = 0; t < 8; ++t) f2unpack(qq[t], q[2 * t], q[2 * t + 1]);
+                sr_group<16>(q, static_cast<uint64_t>(i * p.K + j0), p.seed, w);
+            } else {
+                nv_block_rne(v, S, w, nullptr);
             }
         }
         if (valid) {
@@ -157,6 +183,7 @@ __global__ void __launch_bounds__(256) k_quant_cols(const T *__restrict__ x, Q2D
     __shared__ float red[32];
     float s_t = 0.0f;
     if (FMT == QFP4_NVFP4) s_t = tensor_scale_from(p.partials, p.n_partials, red);
+    const NvScale nz = nv_scale_setup(s_t);
     constexpr int G = FMT == QFP4_MXFP4 ? 32 : 16;
     const int lane = threadIdx.x & 31;
     const int64_t col_blocks = (p.K + 31) / 32, row_blocks = (p.M + 31) / 32;
@@ -189,14 +216,14 @@ __global__ void __launch_bounds__(256) k_quant_cols(const T *__restrict__ x, Q2D
                     mul = exp2i(-k);
                 }
             } else if (s_t != 0.0f) {
-                sbyte = e4m3_rne(__fdiv_rn(__fdiv_rn(amax, 6.0f), s_t));
+                sbyte = nv_scale_byte<true>(amax, nz);
                 S = __fmul_rn(e4m3_value(sbyte), s_t);
             }
             if (FMT == QFP4_NVFP4 && FOUR6) {
                 uint32_t w6[2], w4[2], enc4 = 0u;
                 float sse6, sse4, S4 = 0.0f;
                 if (s_t != 0.0f) {
-                    enc4 = e4m3_rne(__fdiv_rn(__fdiv_rn(amax, 4.0f), s_t));
+                    enc4 = nv_scale_byte<false>(amax, nz);
                     S4 = __fmul_rn(e4m3_value(enc4), s_t);
                 }
                 nv_block_rne(xg, S, w6, &sse6);
@@ -208,10 +235,21 @@ __global__ void __launch_bounds__(256) k_quant_cols(const T *__restrict__ x, Q2D
             } else if (S == 0.0f) {
 #pragma unroll
                 for (int t = 0; t < G / 8; ++t) wg[t] = 0u;
+            } else if (FMT == QFP4_NVFP4 && !SR) {
+                nv_block_rne(xg, S, wg, nullptr);
             } else {
                 float q[G];
+                if (FMT == QFP4_MXFP4) {
 #pragma unroll
-                for (int t = 0; t < G; ++t) q[t] = FMT == QFP4_MXFP4 ? __fmul_rn(xg[t], mul) : __fdiv_rn(xg[t], S);
+                    for (int t = 0; t < G; ++t) q[t] = __fmul_rn(xg[t], mul);
+                } else {
+                    uint64_t pp[G / 2], qq[G / 2];
+#pragma unroll
+                    for (int t = 0; t < G / 2; ++t) pp[t] = f2pack(xg[2 * t], xg[2 * t + 1]);
+                    nv_quot16_pairs(pp, S, qq);
+#pragma unroll
+                    for (int t = 0; t < G / 2; ++t) f2unpack(qq[t], q[2 * t], q[2 * t + 1]);
+                }
                 if (SR) {
 #pragma unroll
                     for (int t = 0; t < G / 8; ++t) wg[t] = 0u;
@@ -243,32 +281,8 @@ __global__ void __launch_bounds__(256) k_quant_cols(const T *__restrict__ x, Q2D
 }
 
 // ---------------------------------------------------------------- MXFP8 (E4M3, g32)
-// E4M3 stochastic rounding: lo <= |v| < hi adjacent E4M3 values (subnormal
-// spacing 2^-9 below 2^-6, else 2^(e-3)), up iff (w >> 8) * 2^-24 < (|v|-lo)/(hi-lo);
-// saturates at 448.  Returns the byte.
-__device__ __forceinline__ uint32_t e4m3_sr(float v, uint32_t w)
-{
-    const uint32_t sign = (__float_as_uint(v) >> 24) & 0x80u;
-    const float a = fabsf(v);
-    float lo, sp, inv_sp;
-    if (a >= 0.015625f) {                                    // 2^-6: normal binade
-        const uint32_t spb = (__float_as_uint(a) & 0x7F800000u) - (3u << 23);
-        lo = __uint_as_float(__float_as_uint(a) & 0x7FF00000u);
-        sp = __uint_as_float(spb);
-        inv_sp = __uint_as_float((254u << 23) - spb);
-    } else {
-        lo = __fmul_rn(truncf(__fmul_rn(a, 512.0f)), 0.001953125f);   // exact: multiples of 2^-9
-        sp = 0.001953125f;
-        inv_sp = 512.0f;
-    }
-    const float p = __fmul_rn(__fsub_rn(a, lo), inv_sp);
-    const float u = __fmul_rn(static_cast<float>(w >> 8), 5.9604644775390625e-08f);
-    float rr = (u < p) ? __fadd_rn(lo, sp) : lo;
-    rr = fminf(rr, 448.0f);
-    return e4m3_rne(rr) | sign;
-}
-
-template <bool SR, bool COLS, typename T>
+// ROWS / COLS: emit the row-wise and / or the column-wise output.
+template <bool SR, bool ROWS, bool COLS, typename T>
 __global__ void __launch_bounds__(256) k_mxfp8(const T *__restrict__ x, Q2DParams p)
 {
     const int lane = threadIdx.x & 31;
@@ -293,7 +307,7 @@ __global__ void __launch_bounds__(256) k_mxfp8(const T *__restrict__ x, Q2DParam
         // row groups: 32 lanes of one row
         uint8_t my_scale = 0;
 #pragma unroll
-        for (int r = 0; r < 32; ++r) {
+        for (int r = 0; r < (ROWS ? 32 : 0); ++r) {
             float amax = fabsf(v[r]);
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
@@ -307,7 +321,7 @@ __global__ void __launch_bounds__(256) k_mxfp8(const T *__restrict__ x, Q2DParam
             if (lane == r) my_scale = static_cast<uint8_t>(sbyte);
             if (r < rows) p.codes[(i0 + r) * p.K + j] = static_cast<uint8_t>(byte);
         }
-        if (lane < rows) p.scales[(i0 + lane) * (p.K / 32) + j / 32] = my_scale;
+        if (ROWS && lane < rows) p.scales[(i0 + lane) * (p.K / 32) + j / 32] = my_scale;
         if (COLS) {                                   // column group: this lane's 32 rows
             float amax = 0.0f;
 #pragma unroll
@@ -390,11 +404,22 @@ int quantize_mxfp8(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_rou
     Q2DParams p{M, K, codes, scales, codesT, scalesT, nullptr, 0, nullptr, seed};
     const int grid = grid_for_warps(((M + 31) / 32) * (K / 32));
     const bool sr = rounding == QFP4_SR, cols = codesT != nullptr;
+    if (xdt == QFP4_BF16 && (M * K) % 64 == 0) {
+        // row-wise output through the TMA-fed 1D kernel; the column-wise one
+        // (if asked for) by the tile kernel without its row part
+        int st = mxfp8_rows(x, M * K, sr, seed, codes, scales, stream);
+        if (st != QFP4_OK || !cols) return st;
+        const uint16_t *xb = static_cast<const uint16_t *>(x);
+        if (sr) k_mxfp8<true, false, true, uint16_t><<<grid, 256, 0, stream>>>(xb, p);
+        else k_mxfp8<false, false, true, uint16_t><<<grid, 256, 0, stream>>>(xb, p);
+        QFP4_LAUNCH_CHECK();
+        return QFP4_OK;
+    }
 #define QFP4_MX8(SRV, COLV)                                                                                   \
     do {                                                                                                      \
         if (xdt == QFP4_BF16)                                                                                 \
-            k_mxfp8<SRV, COLV, uint16_t><<<grid, 256, 0, stream>>>(static_cast<const uint16_t *>(x), p);      \
-        else k_mxfp8<SRV, COLV, float><<<grid, 256, 0, stream>>>(static_cast<const float *>(x), p);           \
+            k_mxfp8<SRV, true, COLV, uint16_t><<<grid, 256, 0, stream>>>(static_cast<const uint16_t *>(x), p); \
+        else k_mxfp8<SRV, true, COLV, float><<<grid, 256, 0, stream>>>(static_cast<const float *>(x), p);    \
     } while (0)
     if (sr) {
         if (cols) QFP4_MX8(true, true);

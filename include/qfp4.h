@@ -160,7 +160,9 @@ int qfp4_quantize_fp32scale(const void *x, qfp4_dtype xdt, int64_t M, int64_t K,
 /* ------------------------------------------------------------------------
  * qfp4_dequantize -- out[i][j] = value(code) * scale (* s_t for NVFP4),
  * formed exactly and rounded once to out_dt (nearest even).  tscale:
- * NVFP4 device pointer to s_t, MXFP4 ignored.  Needs K % g == 0.
+ * NVFP4 device pointer to s_t, MXFP4 ignored.  Needs K % g == 0.  A scale
+ * byte that encodes NaN (E8M0 0xFF; E4M3 0x7F, 0xFF -- the quantize calls
+ * never write one) gives NaN outputs for its group.
  * ---------------------------------------------------------------------- */
 int qfp4_dequantize(const uint8_t *codes, const uint8_t *scales, const float *tscale,
                     int64_t M, int64_t K, qfp4_fmt fmt, qfp4_dtype out_dt, void *out,

@@ -11,7 +11,7 @@ import torch
 import bit_fwht_hadamard_b200 as q
 import oracle
 import synth
-from gpu_util import host, mismatch_report, to_dev
+from gpu_util import blocks_to_rows, encode_input, host, mismatch_report, nvfp4_boundary_blocks, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -141,6 +141,20 @@ def test_large_dynamic_range():
             _cmp(q.quantize(to_dev(x), fmt[0], rounding, seed=2), oracle.quantize(x, fmt[1], rounding, seed=2))
 
 
+@pytest.mark.parametrize("kind", ["bf16", "f32"])
+@pytest.mark.parametrize("four6", [False, True], ids=["rne", "four6"])
+def test_nvfp4_rounding_boundaries(kind, four6):
+    """Quotients x / S exactly on (bf16 input) or within 3 ulps of (float32
+    input) every E2M1 midpoint, and block maxima on or next to the E4M3
+    midpoints (normal and subnormal): codes and scales agree with the
+    oracle's IEEE divisions bit for bit, through the TMA kernel (bf16) and
+    the direct kernel (float32)."""
+    x = encode_input(blocks_to_rows(nvfp4_boundary_blocks(kind)), kind)
+    got = q.quantize(to_dev(x), q.NVFP4, q.RNE, four6=four6)
+    ref = oracle.quantize(x, oracle.NVFP4, oracle.RNE, four6=four6)
+    _cmp(got, ref)
+
+
 def test_misaligned_pointer_is_rejected():
     x = torch.zeros(64 * 128 + 8, dtype=torch.bfloat16, device="cuda")
     codes = torch.empty(64 * 64, dtype=torch.uint8, device="cuda")
@@ -179,3 +193,60 @@ def test_fp32_scale_modes_match_oracle(gran):
     ref = oracle.quantize_fp32scale(W, gran)
     assert np.array_equal(host(got["codes"]), ref["codes"])
     assert np.array_equal(host(got["scales"]).view(np.uint32), ref["scales"].view(np.uint32))
+
+
+# every code under every scale byte, tensor scales that reach each rounding case
+_CODES16 = np.array([0x10, 0x32, 0x54, 0x76, 0x98, 0xBA, 0xDC, 0xFE], np.uint8)   # codes 0..15 in order
+_TSCALES = [1.0, 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, (1 + 2.0 ** -8) / 3, (1 + 2.0 ** -8) / 5,
+            (1 + 2.0 ** -7) / 7, 2.0 ** -130, 1.0e35]
+
+
+@pytest.mark.parametrize("out", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_dequantize_every_code_and_scale(out):
+    """All 16 codes under each of the 256 scale bytes, NVFP4 (one block per
+    byte) under tensor scales whose products land on bfloat16 midpoints --
+    exactly, and with a nonzero remainder -- below 2^-100 and near the top
+    of the range; MXFP4 likewise over its 256 bytes.  NaN scale bytes give
+    NaN; every other output equals the exact value rounded once."""
+    midpoint_with_remainder = 0
+    cases = [(q.NVFP4, oracle.NVFP4, 16, np.float32(t)) for t in _TSCALES] + [(q.MXFP4, oracle.MXFP4, 32, None)]
+    for fmt, ofmt, K, ts in cases:
+        M = 256
+        codes = np.tile(_CODES16, (M, K // 16))                    # K / 2 bytes a row
+        scales = np.arange(256, dtype=np.uint8).reshape(M, 1)      # row r: scale byte r
+        dq = {"codes": torch.from_numpy(codes).cuda(), "scales": torch.from_numpy(scales).cuda()}
+        if ts is not None:
+            dq["tscale"] = torch.tensor([float(ts)], dtype=torch.float32, device="cuda")
+        got = host(q.dequantize(dq, M, K, fmt, out))
+        exact = oracle.dequantize(codes, scales, None if ts is None else np.float32(ts), M, K, ofmt)
+        nan = np.isnan(exact)
+        assert nan.any()                                           # E8M0 0xFF / E4M3 0x7F, 0xFF
+        fin = ~nan
+        if out == torch.float32:
+            assert np.isnan(got[nan]).all()
+            assert np.array_equal(got[fin].view(np.uint32), oracle.f64_to_f32_array(exact[fin]).view(np.uint32))
+        else:
+            g16 = got.view(np.uint16)
+            assert (((g16[nan] & 0x7F80) == 0x7F80) & ((g16[nan] & 0x7F) != 0)).all()
+            assert np.array_equal(g16[fin], oracle.f64_to_bf16_array(exact[fin]))
+            p = oracle.f64_to_f32_array(exact[fin])
+            midpoint_with_remainder += int(np.sum(((p.view(np.uint32) & 0xFFFF) == 0x8000) &
+                                                  (p.astype(np.float64) != exact[fin])))
+    if out == torch.bfloat16:
+        assert midpoint_with_remainder > 0
+
+
+def test_quantize_repeatable_full_size():
+    """Repeated calls on one full-size input (G 8192 x 4096) give bit-identical
+    outputs for every format of the TMA-fed kernel: guards its shared-memory
+    ring against a refill landing before the reads of a stage are done."""
+    x = to_dev(synth.cfg4_G())
+    calls = [lambda: q.quantize(x, q.MXFP4, q.RNE), lambda: q.quantize(x, q.MXFP4, q.RNE, rotate=True),
+             lambda: q.quantize(x, q.NVFP4, q.RNE), lambda: q.quantize(x, q.NVFP4, q.SR, seed=3),
+             lambda: q.quantize_mxfp8(x, q.RNE), lambda: q.quantize_mxfp8(x, q.SR, seed=3)]
+    for f in calls:
+        first = {k: host(v) for k, v in f().items()}
+        for _ in range(3):
+            again = f()
+            for k, v in first.items():
+                assert np.array_equal(host(again[k]).view(np.uint8), v.view(np.uint8)), k

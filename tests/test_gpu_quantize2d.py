@@ -9,7 +9,8 @@ import torch
 import bit_fwht_hadamard_b200 as q
 import oracle
 import synth
-from gpu_util import host, mismatch_report, to_dev
+from gpu_util import (blocks_to_rows, blocks_to_tiles, encode_input, host, mismatch_report, nvfp4_boundary_blocks,
+                      to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -57,6 +58,18 @@ def test_2d_full_size_gradient_sr():
     _cmp(got, ref)
 
 
+@pytest.mark.parametrize("kind", ["bf16", "f32"])
+def test_2d_rounding_boundaries(kind):
+    """16 x 16 tiles whose quotients sit on (bf16) or next to (float32) the
+    E2M1 midpoints and whose maxima put the scale on or next to E4M3
+    midpoints: X and X^T codes and scales bit-exact."""
+    x = encode_input(blocks_to_tiles(nvfp4_boundary_blocks(kind)), kind)
+    for transposed in (False, True):
+        got = q.quantize(to_dev(x), q.NVFP4, q.RNE, block2d=True, transposed=transposed)
+        ref = oracle.quantize(x, oracle.NVFP4, oracle.RNE, block2d=True, transposed=transposed)
+        _cmp(got, ref)
+
+
 # ------------------------------------------------------------------ 1D column-wise
 @pytest.mark.parametrize("M,K", [(32, 32), (64, 96), (48, 64), (96, 80), (256, 512)])
 @pytest.mark.parametrize("fmt", [(q.MXFP4, oracle.MXFP4), (q.NVFP4, oracle.NVFP4)], ids=["mxfp4", "nvfp4"])
@@ -69,6 +82,20 @@ def test_1d_columnwise_matches_oracle(M, K, fmt, mode):
     rounding = q.SR if mode == "sr" else q.RNE
     got = q.quantize(to_dev(x), fmt[0], rounding, four6=(mode == "four6"), seed=99, transposed=True)
     ref = oracle.quantize(x, fmt[1], rounding, four6=(mode == "four6"), seed=99, transposed=True)
+    _cmp(got, ref)
+
+
+@pytest.mark.parametrize("kind", ["bf16", "f32"])
+@pytest.mark.parametrize("four6", [False, True], ids=["rne", "four6"])
+def test_columnwise_rounding_boundaries(kind, four6):
+    """The rounding-boundary blocks laid down the columns (groups along M)."""
+    rows = blocks_to_rows(nvfp4_boundary_blocks(kind))            # (R, 128), blocks along K
+    R = -(-rows.shape[0] // 16) * 16
+    padded = np.zeros((R, rows.shape[1]))
+    padded[:rows.shape[0]] = rows
+    x = encode_input(np.ascontiguousarray(padded.T), kind)        # (128, R), blocks along M
+    got = q.quantize(to_dev(x), q.NVFP4, q.RNE, four6=four6, transposed=True)
+    ref = oracle.quantize(x, oracle.NVFP4, oracle.RNE, four6=four6, transposed=True)
     _cmp(got, ref)
 
 
