@@ -560,46 +560,46 @@ def run_rows():
         # rotation + MXFP4 (the default bench step's two launches, one at a time)
         x2 = bf16(synth.cfg2_X())
         for r, name in ((q.RNE, "RNE"), (q.SR, "SR")):
-            fp4_row("a0 a1 a3 a5", f"X bf16 4096x4096 (N(0,1), 40 channels x20): FWHT-128 + MXFP4 {name}", x2,
+            fp4_row("rotate + mxfp4", f"X bf16 4096x4096 (N(0,1), 40 channels x20): FWHT-128 + MXFP4 {name}", x2,
                     q.MXFP4, r, 2 + 0.5 + 1 / 32, rotate=True, seed=7)
         # NVFP4 forward-linear operands: tensor amax, E4M3 scales, four-over-six
         x3, w3 = bf16(synth.cfg3_X()), bf16(synth.cfg3_W())
         nv = 2 + 0.5 + 1 / 16
-        fp4_row("a2 a3 a4 a5", "X bf16 8192x4096 Student-t(3)*0.5: NVFP4 four-over-six RNE", x3, q.NVFP4, q.RNE, nv,
+        fp4_row("nvfp4 four-over-six", "X bf16 8192x4096 Student-t(3)*0.5: NVFP4 four-over-six RNE", x3, q.NVFP4, q.RNE, nv,
                 four6=True)
-        fp4_row("a2 a3 a4 a5", "W bf16 11008x4096 N(0,0.02^2): NVFP4 four-over-six RNE", w3, q.NVFP4, q.RNE, nv,
+        fp4_row("nvfp4 four-over-six", "W bf16 11008x4096 N(0,0.02^2): NVFP4 four-over-six RNE", w3, q.NVFP4, q.RNE, nv,
                 four6=True)
-        fp4_row("a2 a3 a5", "X bf16 8192x4096 Student-t(3)*0.5: NVFP4 RNE", x3, q.NVFP4, q.RNE, nv)
-        fp4_row("a2 a3 a5", "X bf16 8192x4096 Student-t(3)*0.5: NVFP4 Philox SR", x3, q.NVFP4, q.SR, nv, seed=7)
-        dequant_row("decode", "NVFP4 codes of X 8192x4096 -> bf16", x3, q.NVFP4, BF)
-        dequant_row("decode", "NVFP4 codes of X 8192x4096 -> fp32", x3, q.NVFP4, F32)
+        fp4_row("nvfp4", "X bf16 8192x4096 Student-t(3)*0.5: NVFP4 RNE", x3, q.NVFP4, q.RNE, nv)
+        fp4_row("nvfp4", "X bf16 8192x4096 Student-t(3)*0.5: NVFP4 Philox SR", x3, q.NVFP4, q.SR, nv, seed=7)
+        dequant_row("dequantize", "NVFP4 codes of X 8192x4096 -> bf16", x3, q.NVFP4, BF)
+        dequant_row("dequantize", "NVFP4 codes of X 8192x4096 -> fp32", x3, q.NVFP4, F32)
         # Quartet-style backward: 2D blocks, MXFP8, column-wise 1D
         g4 = bf16(synth.cfg4_G())
-        fp4_row("a6", "G bf16 8192x4096 (N(0,1e-6), 0.1% x100): 2D 16x16 NVFP4 Philox SR, G and G^T", g4, q.NVFP4,
+        fp4_row("2d blocks", "G bf16 8192x4096 (N(0,1e-6), 0.1% x100): 2D 16x16 NVFP4 Philox SR, G and G^T", g4, q.NVFP4,
                 q.SR, 2 + 2 * (0.5 + 1 / 16), block2d=True, transposed=True, seed=11)
-        fp4_row("a6", "G bf16 8192x4096: 2D 16x16 NVFP4 RNE, G and G^T", g4, q.NVFP4, q.RNE,
+        fp4_row("2d blocks", "G bf16 8192x4096: 2D 16x16 NVFP4 RNE, G and G^T", g4, q.NVFP4, q.RNE,
                 2 + 2 * (0.5 + 1 / 16), block2d=True, transposed=True)
         fp4_row("column-wise", "G bf16 8192x4096: 1D MXFP4 RNE rows + independent column-wise groups", g4, q.MXFP4,
                 q.RNE, 2 + 2 * (0.5 + 1 / 32), transposed=True)
         for r, name in ((q.RNE, "RNE"), (q.SR, "SR")):
-            mxfp8_row("a7", f"G bf16 8192x4096: MXFP8 E4M3 g32 {name}", g4, r, False, seed=11)
-        mxfp8_row("a7", "G bf16 8192x4096: MXFP8 E4M3 g32 RNE, rows + column-wise", g4, q.RNE, True)
+            mxfp8_row("mxfp8", f"G bf16 8192x4096: MXFP8 E4M3 g32 {name}", g4, r, False, seed=11)
+        mxfp8_row("mxfp8", "G bf16 8192x4096: MXFP8 E4M3 g32 RNE, rows + column-wise", g4, q.RNE, True)
         # backward GEMMs on 2D-quantized operands: dX = G W, dW = G^T X
         x4, w4 = bf16(synth.cfg4_X()), bf16(synth.cfg4_W())
         G2 = q.quantize(g4, q.NVFP4, q.SR, block2d=True, transposed=True, seed=11)
         W2 = q.quantize(w4, q.NVFP4, q.RNE, block2d=True, transposed=True)
         X2 = q.quantize(x4, q.NVFP4, q.RNE, block2d=True, transposed=True)
         T = lambda o: {"codes": o["codesT"], "scales": o["scalesT"], "tscale": o["tscale"]}   # noqa: E731
-        gemm_row("a8", "dX = G W: NVFP4 8192x4096x4096, fp32 out", G2, T(W2), 8192, 4096, 4096, q.NVFP4, F32)
-        gemm_row("a8", "dW = G^T X: NVFP4 4096x4096x8192, fp32 out", T(G2), T(X2), 4096, 4096, 8192, q.NVFP4, F32)
+        gemm_row("gemm", "dX = G W: NVFP4 8192x4096x4096, fp32 out", G2, T(W2), 8192, 4096, 4096, q.NVFP4, F32)
+        gemm_row("gemm", "dW = G^T X: NVFP4 4096x4096x8192, fp32 out", T(G2), T(X2), 4096, 4096, 8192, q.NVFP4, F32)
         del G2, W2, X2, x4, w4, g4, x3, w3
         # 7B-class linear shapes: the GEMM alone and the fused rotate + quantize + GEMM
         for (M, N, K) in ((16384, 4096, 4096), (16384, 14336, 4096), (16384, 4096, 14336)):
             a5 = bf16(synth.cfg5_A(M, K))
             B5 = q.quantize(bf16(synth.cfg5_B(N, K)), q.NVFP4, q.RNE, rotate=True)
             A5 = q.quantize(a5, q.NVFP4, q.RNE, rotate=True)
-            gemm_row("a8", f"NVFP4 GEMM {M}x{N}x{K} (A pre-quantized), bf16 out", A5, B5, M, N, K, q.NVFP4, BF)
-            fused_row("a9", f"fused FWHT-128 + NVFP4 RNE of A bf16 + GEMM {M}x{N}x{K}, bf16 out", a5, B5, N, q.NVFP4,
+            gemm_row("gemm", f"NVFP4 GEMM {M}x{N}x{K} (A pre-quantized), bf16 out", A5, B5, M, N, K, q.NVFP4, BF)
+            fused_row("fused rotate + quantize + gemm", f"fused FWHT-128 + NVFP4 RNE of A bf16 + GEMM {M}x{N}x{K}, bf16 out", a5, B5, N, q.NVFP4,
                       BF)
             del a5, B5, A5
         # standalone quantize bandwidth over 2^20 .. 2^30 bf16 elements (K = 4096):
@@ -608,8 +608,8 @@ def run_rows():
         for e in range(20, 31, 2):
             M = (1 << e) // 4096
             x = base[:M].clone() if M <= 16384 else base.repeat(M // 16384, 1)
-            fp4_row("sweep", f"2^{e} bf16 elements ({M}x4096): NVFP4 RNE", x, q.NVFP4, q.RNE, nv)
-            fp4_row("sweep", f"2^{e} bf16 elements ({M}x4096): FWHT-128 + MXFP4 RNE", x, q.MXFP4, q.RNE,
+            fp4_row("quantize sweep", f"2^{e} bf16 elements ({M}x4096): NVFP4 RNE", x, q.NVFP4, q.RNE, nv)
+            fp4_row("quantize sweep", f"2^{e} bf16 elements ({M}x4096): FWHT-128 + MXFP4 RNE", x, q.MXFP4, q.RNE,
                     2 + 0.5 + 1 / 32, rotate=True)
             del x
     torch.cuda.synchronize()

@@ -346,10 +346,29 @@ __global__ void __launch_bounds__(256) k_mxfp8(const T *__restrict__ x, Q2DParam
 }
 
 // ---------------------------------------------------------------- host
+// One resident wave of 256-thread blocks (8 warps each, one task per warp at
+// a time): each block pays its prologue (the tensor-scale reduction) once,
+// and its warps loop over their tasks.
+template <auto Kern>
 static int grid_for_warps(int64_t warp_tasks)
 {
-    const int64_t blocks = (warp_tasks + 7) / 8;              // 8 warps per 256-thread block
-    return static_cast<int>(imax<int64_t>(1, imin<int64_t>(blocks, 16 * num_sms())));
+    static const int per_sm = [] {
+        int b = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, Kern, 256, 0) != cudaSuccess || b < 1) {
+            (void)cudaGetLastError();
+            b = 1;
+        }
+        return b;
+    }();
+    const int64_t blocks = (warp_tasks + 7) / 8;
+    return static_cast<int>(imax<int64_t>(1, imin<int64_t>(blocks, static_cast<int64_t>(per_sm) * num_sms())));
+}
+
+// Launch one of the tile kernels with its resident-wave grid.
+template <auto Kern, typename T>
+static void launch_tiles(int64_t warp_tasks, const void *x, const Q2DParams &p, cudaStream_t stream)
+{
+    Kern<<<grid_for_warps<Kern>(warp_tasks), 256, 0, stream>>>(static_cast<const T *>(x), p);
 }
 
 int quantize2d(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_round rounding, uint64_t seed,
@@ -360,25 +379,24 @@ int quantize2d(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_round r
     int st = amax_partials(x, xdt, M * K, partials, &n_parts, stream);
     if (st != QFP4_OK) return st;
     Q2DParams p{M, K, codes, scales, codesT, scalesT, partials, n_parts, tscale, seed};
-    const int grid = grid_for_warps((M / 16) * ((K / 16 + 1) / 2));
+    const int64_t tasks = (M / 16) * ((K / 16 + 1) / 2);
     const bool sr = rounding == QFP4_SR;
     if (xdt == QFP4_BF16) {
-        if (sr) k_quant2d<true, uint16_t><<<grid, 256, 0, stream>>>(static_cast<const uint16_t *>(x), p);
-        else k_quant2d<false, uint16_t><<<grid, 256, 0, stream>>>(static_cast<const uint16_t *>(x), p);
+        if (sr) launch_tiles<k_quant2d<true, uint16_t>, uint16_t>(tasks, x, p, stream);
+        else launch_tiles<k_quant2d<false, uint16_t>, uint16_t>(tasks, x, p, stream);
     } else {
-        if (sr) k_quant2d<true, float><<<grid, 256, 0, stream>>>(static_cast<const float *>(x), p);
-        else k_quant2d<false, float><<<grid, 256, 0, stream>>>(static_cast<const float *>(x), p);
+        if (sr) launch_tiles<k_quant2d<true, float>, float>(tasks, x, p, stream);
+        else launch_tiles<k_quant2d<false, float>, float>(tasks, x, p, stream);
     }
     QFP4_LAUNCH_CHECK();
     return QFP4_OK;
 }
 
 template <int FMT, bool SR, bool FOUR6>
-static int launch_cols(const void *x, qfp4_dtype xdt, const Q2DParams &p, int grid, cudaStream_t stream)
+static int launch_cols(const void *x, qfp4_dtype xdt, const Q2DParams &p, int64_t tasks, cudaStream_t stream)
 {
-    if (xdt == QFP4_BF16)
-        k_quant_cols<FMT, SR, FOUR6, uint16_t><<<grid, 256, 0, stream>>>(static_cast<const uint16_t *>(x), p);
-    else k_quant_cols<FMT, SR, FOUR6, float><<<grid, 256, 0, stream>>>(static_cast<const float *>(x), p);
+    if (xdt == QFP4_BF16) launch_tiles<k_quant_cols<FMT, SR, FOUR6, uint16_t>, uint16_t>(tasks, x, p, stream);
+    else launch_tiles<k_quant_cols<FMT, SR, FOUR6, float>, float>(tasks, x, p, stream);
     QFP4_LAUNCH_CHECK();
     return QFP4_OK;
 }
@@ -388,38 +406,36 @@ int quantize_columns(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_f
                      cudaStream_t stream)
 {
     Q2DParams p{M, K, nullptr, nullptr, codesT, scalesT, partials, n_partials, nullptr, seed};
-    const int grid = grid_for_warps(((M + 31) / 32) * ((K + 31) / 32));
+    const int64_t tasks = ((M + 31) / 32) * ((K + 31) / 32);
     const bool sr = rounding == QFP4_SR;
     if (fmt == QFP4_MXFP4)
-        return sr ? launch_cols<QFP4_MXFP4, true, false>(x, xdt, p, grid, stream)
-                  : launch_cols<QFP4_MXFP4, false, false>(x, xdt, p, grid, stream);
-    if (four6) return launch_cols<QFP4_NVFP4, false, true>(x, xdt, p, grid, stream);
-    return sr ? launch_cols<QFP4_NVFP4, true, false>(x, xdt, p, grid, stream)
-              : launch_cols<QFP4_NVFP4, false, false>(x, xdt, p, grid, stream);
+        return sr ? launch_cols<QFP4_MXFP4, true, false>(x, xdt, p, tasks, stream)
+                  : launch_cols<QFP4_MXFP4, false, false>(x, xdt, p, tasks, stream);
+    if (four6) return launch_cols<QFP4_NVFP4, false, true>(x, xdt, p, tasks, stream);
+    return sr ? launch_cols<QFP4_NVFP4, true, false>(x, xdt, p, tasks, stream)
+              : launch_cols<QFP4_NVFP4, false, false>(x, xdt, p, tasks, stream);
 }
 
 int quantize_mxfp8(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_round rounding, uint64_t seed,
                    uint8_t *codes, uint8_t *scales, uint8_t *codesT, uint8_t *scalesT, cudaStream_t stream)
 {
     Q2DParams p{M, K, codes, scales, codesT, scalesT, nullptr, 0, nullptr, seed};
-    const int grid = grid_for_warps(((M + 31) / 32) * (K / 32));
+    const int64_t tasks = ((M + 31) / 32) * (K / 32);
     const bool sr = rounding == QFP4_SR, cols = codesT != nullptr;
     if (xdt == QFP4_BF16 && (M * K) % 64 == 0) {
         // row-wise output through the TMA-fed 1D kernel; the column-wise one
         // (if asked for) by the tile kernel without its row part
         int st = mxfp8_rows(x, M * K, sr, seed, codes, scales, stream);
         if (st != QFP4_OK || !cols) return st;
-        const uint16_t *xb = static_cast<const uint16_t *>(x);
-        if (sr) k_mxfp8<true, false, true, uint16_t><<<grid, 256, 0, stream>>>(xb, p);
-        else k_mxfp8<false, false, true, uint16_t><<<grid, 256, 0, stream>>>(xb, p);
+        if (sr) launch_tiles<k_mxfp8<true, false, true, uint16_t>, uint16_t>(tasks, x, p, stream);
+        else launch_tiles<k_mxfp8<false, false, true, uint16_t>, uint16_t>(tasks, x, p, stream);
         QFP4_LAUNCH_CHECK();
         return QFP4_OK;
     }
-#define QFP4_MX8(SRV, COLV)                                                                                   \
-    do {                                                                                                      \
-        if (xdt == QFP4_BF16)                                                                                 \
-            k_mxfp8<SRV, true, COLV, uint16_t><<<grid, 256, 0, stream>>>(static_cast<const uint16_t *>(x), p); \
-        else k_mxfp8<SRV, true, COLV, float><<<grid, 256, 0, stream>>>(static_cast<const float *>(x), p);    \
+#define QFP4_MX8(SRV, COLV)                                                                     \
+    do {                                                                                        \
+        if (xdt == QFP4_BF16) launch_tiles<k_mxfp8<SRV, true, COLV, uint16_t>, uint16_t>(tasks, x, p, stream); \
+        else launch_tiles<k_mxfp8<SRV, true, COLV, float>, float>(tasks, x, p, stream);          \
     } while (0)
     if (sr) {
         if (cols) QFP4_MX8(true, true);
