@@ -52,7 +52,7 @@ def parse():
     ap.add_argument("--impl", default="libqfp4", choices=["libqfp4", "reference"])
     ap.add_argument("--no-gemm", action="store_true", help="skip the GEMM sub-measurement")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    ap.add_argument("--profile-case", choices=["quant", "gemm", "quant-nvfp4"], default=None,
+    ap.add_argument("--profile-case", choices=["quant", "gemm", "quant-nvfp4", "backward"], default=None,
                     help="run a few untimed calls of one kernel family (for ncu captures) and exit")
     ap.add_argument("--rows", action="store_true",
                     help="time every entry point of the path on its own full-size workload (one JSON line each)")
@@ -417,6 +417,15 @@ def run_profile_case(case):
         for _ in range(2):
             q.quantize(x, q.MXFP4, q.RNE, rotate=True)
             q.quantize(x, q.MXFP4, q.SR, rotate=True, seed=7)
+    elif case == "backward":
+        # gradient G 8192 x 4096: 2D NVFP4 with G^T, MXFP8 rows + columns,
+        # 1D MXFP4 rows + independent columns (one launch of each tile kernel
+        # per iteration, in that order)
+        g = torch.from_numpy(synth.cfg4_G().view(np.int16)).view(torch.bfloat16).to(dev)
+        for _ in range(2):
+            q.quantize(g, q.NVFP4, q.RNE, block2d=True, transposed=True)
+            q.quantize_mxfp8(g, q.RNE, transposed=True)
+            q.quantize(g, q.MXFP4, q.RNE, transposed=True)
     elif case == "quant-nvfp4":
         x = torch.from_numpy(synth.cfg3_X().view(np.int16)).view(torch.bfloat16).to(dev)
         for _ in range(2):
