@@ -54,8 +54,9 @@ def parse():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--profile-case", choices=["quant", "gemm", "quant-nvfp4", "backward"], default=None,
                     help="run a few untimed calls of one kernel family (for ncu captures) and exit")
-    ap.add_argument("--rows", action="store_true",
-                    help="time every entry point of the path on its own full-size workload (one JSON line each)")
+    ap.add_argument("--rows", nargs="?", const="", default=None, metavar="FILTER",
+                    help="time every entry point of the path on its own full-size workload (one JSON line each); "
+                         "FILTER keeps only the rows whose label contains it")
     return ap.parse_args()
 
 
@@ -68,10 +69,20 @@ def measured_peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-def csrc_hash():
+# the source files each profiled kernel is built from (its ncu figures stay
+# valid while these are unchanged)
+KERNEL_SOURCES = {
+    "quant1d_mxfp4_rot_rne": ("qfp4_common.cuh", "quantize1d.cuh", "quantize1d.cu"),
+    "quant1d_mxfp4_rot_sr": ("qfp4_common.cuh", "quantize1d.cuh", "quantize1d.cu"),
+    "gemm_nvfp4_f32": ("qfp4_common.cuh", "gemm.cu"),
+}
+
+
+def csrc_hash(files=None):
+    """Hash of the library sources (all of them, or the named files)."""
     h = hashlib.sha1()
     d = os.path.join(ROOT, "bit_fwht_hadamard_b200", "csrc")
-    for n in sorted(os.listdir(d)):
+    for n in sorted(files if files is not None else os.listdir(d)):
         with open(os.path.join(d, n), "rb") as f:
             h.update(n.encode() + f.read())
     return h.hexdigest()[:12]
@@ -79,11 +90,11 @@ def csrc_hash():
 
 def ncu_traffic(key):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel sources (else None)."""
+    the kernel's current sources (else None)."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
-    if not os.path.exists(p):
+    if not os.path.exists(p) or key not in KERNEL_SOURCES:
         return None
-    cur = csrc_hash()
+    cur = csrc_hash(KERNEL_SOURCES[key])
     with open(p) as f:
         for line in f:
             t = line.split()
@@ -461,7 +472,7 @@ def time_calls(torch, stream, call, iters=20, warm=3):
     return statistics.mean(a.elapsed_time(b) for a, b in evs)
 
 
-def run_rows():
+def run_rows(only=""):
     """One JSON line per entry point of the path, each on the full-size
     synthetic workload it serves: quantize variants in GB/s of algorithmic
     bytes against the measured HBM peak, GEMMs in TFLOP/s against the dense
@@ -566,61 +577,85 @@ def run_rows():
 
     F32, BF = torch.float32, torch.bfloat16
     with ClockSampler(0) as clk:
+        want = lambda *labels: any(only in lb for lb in labels)                   # noqa: E731
         # rotation + MXFP4 (the default bench step's two launches, one at a time)
-        x2 = bf16(synth.cfg2_X())
-        for r, name in ((q.RNE, "RNE"), (q.SR, "SR")):
-            fp4_row("rotate + mxfp4", f"X bf16 4096x4096 (N(0,1), 40 channels x20): FWHT-128 + MXFP4 {name}", x2,
-                    q.MXFP4, r, 2 + 0.5 + 1 / 32, rotate=True, seed=7)
+        if want("rotate + mxfp4"):
+            x2 = bf16(synth.cfg2_X())
+            for r, name in ((q.RNE, "RNE"), (q.SR, "SR")):
+                fp4_row("rotate + mxfp4", f"X bf16 4096x4096 (N(0,1), 40 channels x20): FWHT-128 + MXFP4 {name}", x2,
+                        q.MXFP4, r, 2 + 0.5 + 1 / 32, rotate=True, seed=7)
+            del x2
         # NVFP4 forward-linear operands: tensor amax, E4M3 scales, four-over-six
-        x3, w3 = bf16(synth.cfg3_X()), bf16(synth.cfg3_W())
         nv = 2 + 0.5 + 1 / 16
-        fp4_row("nvfp4 four-over-six", "X bf16 8192x4096 Student-t(3)*0.5: NVFP4 four-over-six RNE", x3, q.NVFP4, q.RNE, nv,
-                four6=True)
-        fp4_row("nvfp4 four-over-six", "W bf16 11008x4096 N(0,0.02^2): NVFP4 four-over-six RNE", w3, q.NVFP4, q.RNE, nv,
-                four6=True)
-        fp4_row("nvfp4", "X bf16 8192x4096 Student-t(3)*0.5: NVFP4 RNE", x3, q.NVFP4, q.RNE, nv)
-        fp4_row("nvfp4", "X bf16 8192x4096 Student-t(3)*0.5: NVFP4 Philox SR", x3, q.NVFP4, q.SR, nv, seed=7)
-        dequant_row("dequantize", "NVFP4 codes of X 8192x4096 -> bf16", x3, q.NVFP4, BF)
-        dequant_row("dequantize", "NVFP4 codes of X 8192x4096 -> fp32", x3, q.NVFP4, F32)
-        # Quartet-style backward: 2D blocks, MXFP8, column-wise 1D
-        g4 = bf16(synth.cfg4_G())
-        fp4_row("2d blocks", "G bf16 8192x4096 (N(0,1e-6), 0.1% x100): 2D 16x16 NVFP4 Philox SR, G and G^T", g4, q.NVFP4,
-                q.SR, 2 + 2 * (0.5 + 1 / 16), block2d=True, transposed=True, seed=11)
-        fp4_row("2d blocks", "G bf16 8192x4096: 2D 16x16 NVFP4 RNE, G and G^T", g4, q.NVFP4, q.RNE,
-                2 + 2 * (0.5 + 1 / 16), block2d=True, transposed=True)
-        fp4_row("column-wise", "G bf16 8192x4096: 1D MXFP4 RNE rows + independent column-wise groups", g4, q.MXFP4,
-                q.RNE, 2 + 2 * (0.5 + 1 / 32), transposed=True)
-        for r, name in ((q.RNE, "RNE"), (q.SR, "SR")):
-            mxfp8_row("mxfp8", f"G bf16 8192x4096: MXFP8 E4M3 g32 {name}", g4, r, False, seed=11)
-        mxfp8_row("mxfp8", "G bf16 8192x4096: MXFP8 E4M3 g32 RNE, rows + column-wise", g4, q.RNE, True)
-        # backward GEMMs on 2D-quantized operands: dX = G W, dW = G^T X
-        x4, w4 = bf16(synth.cfg4_X()), bf16(synth.cfg4_W())
-        G2 = q.quantize(g4, q.NVFP4, q.SR, block2d=True, transposed=True, seed=11)
-        W2 = q.quantize(w4, q.NVFP4, q.RNE, block2d=True, transposed=True)
-        X2 = q.quantize(x4, q.NVFP4, q.RNE, block2d=True, transposed=True)
-        T = lambda o: {"codes": o["codesT"], "scales": o["scalesT"], "tscale": o["tscale"]}   # noqa: E731
-        gemm_row("gemm", "dX = G W: NVFP4 8192x4096x4096, fp32 out", G2, T(W2), 8192, 4096, 4096, q.NVFP4, F32)
-        gemm_row("gemm", "dW = G^T X: NVFP4 4096x4096x8192, fp32 out", T(G2), T(X2), 4096, 4096, 8192, q.NVFP4, F32)
-        del G2, W2, X2, x4, w4, g4, x3, w3
+        if want("nvfp4 four-over-six", "nvfp4", "dequantize"):
+            x3, w3 = bf16(synth.cfg3_X()), bf16(synth.cfg3_W())
+            if want("nvfp4 four-over-six"):
+                fp4_row("nvfp4 four-over-six", "X bf16 8192x4096 Student-t(3)*0.5: NVFP4 four-over-six RNE", x3, q.NVFP4,
+                        q.RNE, nv, four6=True)
+                fp4_row("nvfp4 four-over-six", "W bf16 11008x4096 N(0,0.02^2): NVFP4 four-over-six RNE", w3, q.NVFP4,
+                        q.RNE, nv, four6=True)
+            if want("nvfp4"):
+                fp4_row("nvfp4", "X bf16 8192x4096 Student-t(3)*0.5: NVFP4 RNE", x3, q.NVFP4, q.RNE, nv)
+                fp4_row("nvfp4", "X bf16 8192x4096 Student-t(3)*0.5: NVFP4 Philox SR", x3, q.NVFP4, q.SR, nv, seed=7)
+            if want("dequantize"):
+                dequant_row("dequantize", "NVFP4 codes of X 8192x4096 -> bf16", x3, q.NVFP4, BF)
+                dequant_row("dequantize", "NVFP4 codes of X 8192x4096 -> fp32", x3, q.NVFP4, F32)
+            del x3, w3
+        # Quartet-style backward: 2D blocks, MXFP8, column-wise 1D, backward GEMMs
+        if want("2d blocks", "column-wise", "mxfp8", "gemm"):
+            g4 = bf16(synth.cfg4_G())
+            if want("2d blocks"):
+                fp4_row("2d blocks", "G bf16 8192x4096 (N(0,1e-6), 0.1% x100): 2D 16x16 NVFP4 Philox SR, G and G^T", g4,
+                        q.NVFP4, q.SR, 2 + 2 * (0.5 + 1 / 16), block2d=True, transposed=True, seed=11)
+                fp4_row("2d blocks", "G bf16 8192x4096: 2D 16x16 NVFP4 RNE, G and G^T", g4, q.NVFP4, q.RNE,
+                        2 + 2 * (0.5 + 1 / 16), block2d=True, transposed=True)
+            if want("column-wise"):
+                fp4_row("column-wise", "G bf16 8192x4096: 1D MXFP4 RNE rows + independent column-wise groups", g4,
+                        q.MXFP4, q.RNE, 2 + 2 * (0.5 + 1 / 32), transposed=True)
+                fp4_row("column-wise", "G bf16 8192x4096: 1D NVFP4 Philox SR rows + independent column-wise groups", g4,
+                        q.NVFP4, q.SR, 2 + 2 * (0.5 + 1 / 16), transposed=True, seed=11)
+            if want("mxfp8"):
+                for r, name in ((q.RNE, "RNE"), (q.SR, "SR")):
+                    mxfp8_row("mxfp8", f"G bf16 8192x4096: MXFP8 E4M3 g32 {name}", g4, r, False, seed=11)
+                mxfp8_row("mxfp8", "G bf16 8192x4096: MXFP8 E4M3 g32 RNE, rows + column-wise", g4, q.RNE, True)
+                mxfp8_row("mxfp8", "G bf16 8192x4096: MXFP8 E4M3 g32 SR, rows + column-wise", g4, q.SR, True, seed=11)
+            if want("gemm"):
+                # backward GEMMs on 2D-quantized operands: dX = G W, dW = G^T X
+                x4, w4 = bf16(synth.cfg4_X()), bf16(synth.cfg4_W())
+                G2 = q.quantize(g4, q.NVFP4, q.SR, block2d=True, transposed=True, seed=11)
+                W2 = q.quantize(w4, q.NVFP4, q.RNE, block2d=True, transposed=True)
+                X2 = q.quantize(x4, q.NVFP4, q.RNE, block2d=True, transposed=True)
+                T = lambda o: {"codes": o["codesT"], "scales": o["scalesT"], "tscale": o["tscale"]}   # noqa: E731
+                gemm_row("gemm", "dX = G W: NVFP4 8192x4096x4096, fp32 out", G2, T(W2), 8192, 4096, 4096, q.NVFP4, F32)
+                gemm_row("gemm", "dW = G^T X: NVFP4 4096x4096x8192, fp32 out", T(G2), T(X2), 4096, 4096, 8192, q.NVFP4,
+                         F32)
+                del G2, W2, X2, x4, w4
+            del g4
         # 7B-class linear shapes: the GEMM alone and the fused rotate + quantize + GEMM
-        for (M, N, K) in ((16384, 4096, 4096), (16384, 14336, 4096), (16384, 4096, 14336)):
-            a5 = bf16(synth.cfg5_A(M, K))
-            B5 = q.quantize(bf16(synth.cfg5_B(N, K)), q.NVFP4, q.RNE, rotate=True)
-            A5 = q.quantize(a5, q.NVFP4, q.RNE, rotate=True)
-            gemm_row("gemm", f"NVFP4 GEMM {M}x{N}x{K} (A pre-quantized), bf16 out", A5, B5, M, N, K, q.NVFP4, BF)
-            fused_row("fused rotate + quantize + gemm", f"fused FWHT-128 + NVFP4 RNE of A bf16 + GEMM {M}x{N}x{K}, bf16 out", a5, B5, N, q.NVFP4,
-                      BF)
-            del a5, B5, A5
+        if want("gemm", "fused rotate + quantize + gemm"):
+            for (M, N, K) in ((16384, 4096, 4096), (16384, 14336, 4096), (16384, 4096, 14336)):
+                a5 = bf16(synth.cfg5_A(M, K))
+                B5 = q.quantize(bf16(synth.cfg5_B(N, K)), q.NVFP4, q.RNE, rotate=True)
+                A5 = q.quantize(a5, q.NVFP4, q.RNE, rotate=True)
+                if want("gemm"):
+                    gemm_row("gemm", f"NVFP4 GEMM {M}x{N}x{K} (A pre-quantized), bf16 out", A5, B5, M, N, K, q.NVFP4,
+                             BF)
+                if want("fused rotate + quantize + gemm"):
+                    fused_row("fused rotate + quantize + gemm",
+                              f"fused FWHT-128 + NVFP4 RNE of A bf16 + GEMM {M}x{N}x{K}, bf16 out", a5, B5, N, q.NVFP4,
+                              BF)
+                del a5, B5, A5
         # standalone quantize bandwidth over 2^20 .. 2^30 bf16 elements (K = 4096):
         # rows of the 16384 x 4096 outlier-channel input, repeated past 2^26 elements
-        base = bf16(synth.cfg5_A(16384, 4096))
-        for e in range(20, 31, 2):
-            M = (1 << e) // 4096
-            x = base[:M].clone() if M <= 16384 else base.repeat(M // 16384, 1)
-            fp4_row("quantize sweep", f"2^{e} bf16 elements ({M}x4096): NVFP4 RNE", x, q.NVFP4, q.RNE, nv)
-            fp4_row("quantize sweep", f"2^{e} bf16 elements ({M}x4096): FWHT-128 + MXFP4 RNE", x, q.MXFP4, q.RNE,
-                    2 + 0.5 + 1 / 32, rotate=True)
-            del x
+        if want("quantize sweep"):
+            base = bf16(synth.cfg5_A(16384, 4096))
+            for e in range(20, 31, 2):
+                M = (1 << e) // 4096
+                x = base[:M].clone() if M <= 16384 else base.repeat(M // 16384, 1)
+                fp4_row("quantize sweep", f"2^{e} bf16 elements ({M}x4096): NVFP4 RNE", x, q.NVFP4, q.RNE, nv)
+                fp4_row("quantize sweep", f"2^{e} bf16 elements ({M}x4096): FWHT-128 + MXFP4 RNE", x, q.MXFP4, q.RNE,
+                        2 + 0.5 + 1 / 32, rotate=True)
+                del x
     torch.cuda.synchronize()
     err = q.qfp4_last_device_error()
     print(json.dumps({"rows_done": True, "clocks": clk.summary(), "device_error": err, "bad_status": sorted(set(bad)),
@@ -634,8 +669,8 @@ def main():
     if args.profile_case:
         run_profile_case(args.profile_case)
         return
-    if args.rows:
-        run_rows()
+    if args.rows is not None:
+        run_rows(args.rows)
         return
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

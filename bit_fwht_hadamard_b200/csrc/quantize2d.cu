@@ -345,6 +345,177 @@ __global__ void __launch_bounds__(256) k_mxfp8(const T *__restrict__ x, Q2DParam
     }
 }
 
+// ---------------------------------------------------------------- column-wise outputs, 4 columns a lane
+// bf16 input: a warp covers 32 rows x 128 columns, lane l the 4 adjacent
+// columns jb = j0 + 4 l .. jb + 3, loaded as one 8-byte word per row (256
+// bytes per warp instruction).  The 32 rows stay as raw bf16 pairs (64
+// registers).  Per column: the group maxima, the scales, then the codes of
+// X^T row jb + c (E2M1 nibbles, or E4M3 bytes for FMT_MXFP8).  Stochastic
+// rounding runs row by row: the 4 columns of a row are one Philox counter
+// ((i0 + r) K + jb) / 4, so each call serves four elements.  Groups along M:
+// 32 (MXFP4, MXFP8) or 16 (NVFP4, where the last row block may have 16 rows).
+__device__ __forceinline__ float nv_quot1(float x, float S, float y, bool fast)
+{
+    if (!fast) return __fdiv_rn(x, S);
+    const float q = div_rn_by(x, y, -S);
+    return __uint_as_float(__float_as_uint(q) | (__float_as_uint(x) & 0x80000000u));   // sign of x, also on zero
+}
+
+template <int FMT, bool SR, bool FOUR6>
+__global__ void __launch_bounds__(256) k_cols4(const uint16_t *__restrict__ x, Q2DParams p)
+{
+    constexpr bool MX8 = FMT == FMT_MXFP8, NV = FMT == QFP4_NVFP4;
+    constexpr int G = NV ? 16 : 32, NG = 32 / G;
+    __shared__ float red[32];
+    float s_t = 0.0f;
+    if (NV) s_t = tensor_scale_from(p.partials, p.n_partials, red);
+    const NvScale nz = nv_scale_setup(s_t);
+    const int lane = threadIdx.x & 31;
+    const int64_t col_blocks = (p.K + 127) / 128, row_blocks = (p.M + 31) / 32;
+    const int64_t tasks = row_blocks * col_blocks;
+    const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    for (int64_t task = warp0; task < tasks; task += nwarps) {
+        const int64_t i0 = (task / col_blocks) * 32, jb = (task % col_blocks) * 128 + 4 * lane;
+        const int rows = static_cast<int>(imin<int64_t>(32, p.M - i0));   // 32, or 16 (NVFP4, M % 32 == 16)
+        if (jb >= p.K) continue;                    // K % 4 == 0: a lane's columns are all in or all out
+        uint32_t raw[32][2];
+#pragma unroll
+        for (int r = 0; r < 32; ++r) {
+            if (r < rows) {
+                const uint2 w = *reinterpret_cast<const uint2 *>(x + (i0 + r) * p.K + jb);
+                raw[r][0] = w.x;
+                raw[r][1] = w.y;
+            } else {
+                raw[r][0] = raw[r][1] = 0u;
+            }
+        }
+        auto val = [&](int r, int c) -> float { return (c & 1) ? bf16hi(raw[r][c >> 1]) : bf16lo(raw[r][c >> 1]); };
+
+        // scales per (group, column)
+        float S[NG][4], Y[NG][4], mul[4];
+        bool fast[NG][4];
+        uint32_t sb[NG][4], w[4][MX8 ? 8 : 4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int t = 0; t < (MX8 ? 8 : 4); ++t) w[c][t] = 0u;
+#pragma unroll
+        for (int g = 0; g < NG; ++g)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                float amax = 0.0f;
+#pragma unroll
+                for (int r = 0; r < G; ++r) amax = fmaxf(amax, fabsf(val(G * g + r, c)));
+                sb[g][c] = 0u;
+                S[g][c] = 0.0f;
+                Y[g][c] = 0.0f;
+                fast[g][c] = false;
+                if (!NV) {
+                    mul[c] = 0.0f;
+                    if (amax != 0.0f) {
+                        const int k = MX8 ? scale_exp(amax, 0x600000u, 8) : scale_exp(amax, 0x400000u, 2);
+                        sb[g][c] = static_cast<uint32_t>(k + 127);
+                        S[g][c] = 1.0f;                      // marks a nonzero group
+                        mul[c] = exp2i(-k);
+                    }
+                } else if (s_t != 0.0f) {
+                    uint32_t enc = nv_scale_byte<true>(amax, nz);
+                    float Sv = __fmul_rn(e4m3_value(enc), s_t);
+                    if (FOUR6) {
+                        float xg[16];
+#pragma unroll
+                        for (int r = 0; r < 16; ++r) xg[r] = val(16 * g + r, c);
+                        const uint32_t enc4 = nv_scale_byte<false>(amax, nz);
+                        const float S4 = __fmul_rn(e4m3_value(enc4), s_t);
+                        uint32_t w6[2], w4[2];
+                        float sse6, sse4;
+                        nv_block_rne(xg, Sv, w6, &sse6);
+                        nv_block_rne(xg, S4, w4, &sse4);
+                        const bool pick4 = sse4 < sse6;
+                        w[c][2 * g] = pick4 ? w4[0] : w6[0];
+                        w[c][2 * g + 1] = pick4 ? w4[1] : w6[1];
+                        enc = pick4 ? enc4 : enc;
+                    }
+                    sb[g][c] = enc;
+                    S[g][c] = Sv;
+                    fast[g][c] = Sv >= 0x1p-125f && Sv <= 0x1p125f;
+                    Y[g][c] = fast[g][c] ? __frcp_rn(Sv) : 0.0f;
+                }
+            }
+
+        // codes
+        if (SR) {
+#pragma unroll
+            for (int r = 0; r < 32; ++r) {
+                if (r < rows) {
+                    const uint4 rw = sr_words4(p.seed, static_cast<uint64_t>((i0 + r) * p.K + jb) >> 2);
+                    const uint32_t wd[4] = {rw.x, rw.y, rw.z, rw.w};
+                    const int g = r / G;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        if (S[g][c] == 0.0f) continue;       // zero group (or S = 0): code 0
+                        const float v = val(r, c);
+                        const float q = NV ? nv_quot1(v, S[g][c], Y[g][c], fast[g][c]) : __fmul_rn(v, mul[c]);
+                        if (MX8) w[c][r >> 2] |= e4m3_sr(q, wd[c]) << (8 * (r & 3));
+                        else w[c][r >> 3] |= e2m1_sr(q, wd[c]) << (4 * (r & 7));
+                    }
+                }
+            }
+        } else if (!FOUR6) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+#pragma unroll
+                for (int g = 0; g < NG; ++g) {
+                    if (S[g][c] == 0.0f) continue;
+                    if (NV) {
+                        float xg[16];
+#pragma unroll
+                        for (int r = 0; r < 16; ++r) xg[r] = val(16 * g + r, c);
+                        nv_block_rne(xg, S[g][c], &w[c][2 * g], nullptr);
+                    } else if (MX8) {
+#pragma unroll
+                        for (int t = 0; t < 8; ++t)
+                            w[c][t] = e4m3x2_rne(__fmul_rn(val(4 * t, c), mul[c]), __fmul_rn(val(4 * t + 1, c), mul[c])) |
+                                      (e4m3x2_rne(__fmul_rn(val(4 * t + 2, c), mul[c]),
+                                                  __fmul_rn(val(4 * t + 3, c), mul[c])) << 16);
+                    } else {
+#pragma unroll
+                        for (int t = 0; t < 4; ++t) {
+                            float q8[8];
+#pragma unroll
+                            for (int u = 0; u < 8; ++u) q8[u] = __fmul_rn(val(8 * t + u, c), mul[c]);
+                            w[c][t] = e2m1x8_rne(q8);
+                        }
+                    }
+                }
+            }
+        }
+
+        // stores: X^T rows jb .. jb + 3, elements i0 .. i0 + rows - 1
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int64_t j = jb + c;
+            if (MX8) {
+                uint4 *dst = reinterpret_cast<uint4 *>(p.codesT + j * p.M + i0);
+                dst[0] = make_uint4(w[c][0], w[c][1], w[c][2], w[c][3]);
+                dst[1] = make_uint4(w[c][4], w[c][5], w[c][6], w[c][7]);
+                p.scalesT[j * (p.M / 32) + i0 / 32] = static_cast<uint8_t>(sb[0][c]);
+            } else {
+                uint2 *dst = reinterpret_cast<uint2 *>(p.codesT + (j * p.M + i0) / 2);
+                dst[0] = make_uint2(w[c][0], w[c][1]);
+                if (rows == 32) dst[1] = make_uint2(w[c][2], w[c][3]);
+                if (G == 32) {
+                    p.scalesT[j * (p.M / 32) + i0 / 32] = static_cast<uint8_t>(sb[0][c]);
+                } else {
+                    p.scalesT[j * (p.M / 16) + i0 / 16] = static_cast<uint8_t>(sb[0][c]);
+                    if (rows == 32) p.scalesT[j * (p.M / 16) + i0 / 16 + 1] = static_cast<uint8_t>(sb[NG - 1][c]);
+                }
+            }
+        }
+    }
+}
+
 // ---------------------------------------------------------------- host
 // One resident wave of 256-thread blocks (8 warps each, one task per warp at
 // a time): each block pays its prologue (the tensor-scale reduction) once,
@@ -392,11 +563,14 @@ int quantize2d(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_round r
     return QFP4_OK;
 }
 
+// bf16: the 4-columns-a-lane kernel (32 x 128 tasks); binary32: one column a lane.
 template <int FMT, bool SR, bool FOUR6>
-static int launch_cols(const void *x, qfp4_dtype xdt, const Q2DParams &p, int64_t tasks, cudaStream_t stream)
+static int launch_cols(const void *x, qfp4_dtype xdt, const Q2DParams &p, cudaStream_t stream)
 {
-    if (xdt == QFP4_BF16) launch_tiles<k_quant_cols<FMT, SR, FOUR6, uint16_t>, uint16_t>(tasks, x, p, stream);
-    else launch_tiles<k_quant_cols<FMT, SR, FOUR6, float>, float>(tasks, x, p, stream);
+    if (xdt == QFP4_BF16)
+        launch_tiles<k_cols4<FMT, SR, FOUR6>, uint16_t>(((p.M + 31) / 32) * ((p.K + 127) / 128), x, p, stream);
+    else
+        launch_tiles<k_quant_cols<FMT, SR, FOUR6, float>, float>(((p.M + 31) / 32) * ((p.K + 31) / 32), x, p, stream);
     QFP4_LAUNCH_CHECK();
     return QFP4_OK;
 }
@@ -406,14 +580,13 @@ int quantize_columns(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_f
                      cudaStream_t stream)
 {
     Q2DParams p{M, K, nullptr, nullptr, codesT, scalesT, partials, n_partials, nullptr, seed};
-    const int64_t tasks = ((M + 31) / 32) * ((K + 31) / 32);
     const bool sr = rounding == QFP4_SR;
     if (fmt == QFP4_MXFP4)
-        return sr ? launch_cols<QFP4_MXFP4, true, false>(x, xdt, p, tasks, stream)
-                  : launch_cols<QFP4_MXFP4, false, false>(x, xdt, p, tasks, stream);
-    if (four6) return launch_cols<QFP4_NVFP4, false, true>(x, xdt, p, tasks, stream);
-    return sr ? launch_cols<QFP4_NVFP4, true, false>(x, xdt, p, tasks, stream)
-              : launch_cols<QFP4_NVFP4, false, false>(x, xdt, p, tasks, stream);
+        return sr ? launch_cols<QFP4_MXFP4, true, false>(x, xdt, p, stream)
+                  : launch_cols<QFP4_MXFP4, false, false>(x, xdt, p, stream);
+    if (four6) return launch_cols<QFP4_NVFP4, false, true>(x, xdt, p, stream);
+    return sr ? launch_cols<QFP4_NVFP4, true, false>(x, xdt, p, stream)
+              : launch_cols<QFP4_NVFP4, false, false>(x, xdt, p, stream);
 }
 
 int quantize_mxfp8(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_round rounding, uint64_t seed,
@@ -427,8 +600,9 @@ int quantize_mxfp8(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_rou
         // (if asked for) by the tile kernel without its row part
         int st = mxfp8_rows(x, M * K, sr, seed, codes, scales, stream);
         if (st != QFP4_OK || !cols) return st;
-        if (sr) launch_tiles<k_mxfp8<true, false, true, uint16_t>, uint16_t>(tasks, x, p, stream);
-        else launch_tiles<k_mxfp8<false, false, true, uint16_t>, uint16_t>(tasks, x, p, stream);
+        const int64_t tasks4 = ((M + 31) / 32) * ((K + 127) / 128);
+        if (sr) launch_tiles<k_cols4<FMT_MXFP8, true, false>, uint16_t>(tasks4, x, p, stream);
+        else launch_tiles<k_cols4<FMT_MXFP8, false, false>, uint16_t>(tasks4, x, p, stream);
         QFP4_LAUNCH_CHECK();
         return QFP4_OK;
     }
