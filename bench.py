@@ -25,6 +25,7 @@ import hashlib
 import io
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -78,13 +79,21 @@ KERNEL_SOURCES = {
 }
 
 
+def _code_only(text):
+    """Source text without comments and with whitespace runs collapsed, so
+    that the hash follows code changes only."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return re.sub(r"\s+", " ", text).strip()
+
+
 def csrc_hash(files=None):
-    """Hash of the library sources (all of them, or the named files)."""
+    """Hash of the library sources' code (all files, or the named ones)."""
     h = hashlib.sha1()
     d = os.path.join(ROOT, "bit_fwht_hadamard_b200", "csrc")
     for n in sorted(files if files is not None else os.listdir(d)):
-        with open(os.path.join(d, n), "rb") as f:
-            h.update(n.encode() + f.read())
+        with open(os.path.join(d, n), encoding="utf-8") as f:
+            h.update(n.encode() + _code_only(f.read()).encode())
     return h.hexdigest()[:12]
 
 

@@ -1,6 +1,7 @@
 // quantize1d.cu -- 1D FP4 microscaling quantize (MXFP4 / NVFP4), optional
 // 128-point Walsh-Hadamard rotation, RNE or Philox stochastic rounding,
-// optional four-over-six; plus the NVFP4 tensor-amax pass.
+// optional four-over-six; the NVFP4 tensor-amax pass; and the row-wise MXFP8
+// quantize, which shares the same kernel.
 //
 // Method ([QN] Hadamard rotation + QuTLASS online quantization; [LB] §FP4,
 // §2, §3, §7; [46] Methodology): per 128 block along K an optional
@@ -9,15 +10,14 @@
 //
 // Layout: the input is a flat stream of n = M*K elements (groups never cross
 // rows because K % g == 0, and rotation blocks never cross rows because
-// K % 128 == 0).  Main (bf16) kernel: one persistent CTA per SM, 8 warps,
-// each warp with its own 3-stage ring of 8 KiB tiles (64 rows of 64 bf16)
-// brought in by TMA with 128-byte swizzle; an SM takes a contiguous range of
-// tiles (balanced to one 4096-element tile) and its warps interleave over
-// it.  A thread owns one 128-element unit (two 128-byte rows), held as 64
-// packed binary32 pairs: the whole rotation block is in registers, and the
-// butterflies of stages h = 2..64 and the scaling run as f32x2 operations
-// (two IEEE additions per instruction).  The direct kernel (64-element
-// units, one shuffle stage) serves binary32 inputs and the ragged tail.
+// K % 128 == 0).  Main (bf16) kernel: one persistent CTA per SM, 20 warps
+// (16 with four-over-six), each warp with its own 2-stage ring of 4 KiB
+// tiles (32 rows of 64 bf16) brought in by TMA with 128-byte swizzle; an SM
+// takes a contiguous range of tiles and its warps interleave over it.  A
+// thread owns one 64-element row as 32 packed binary32 pairs; the
+// rotation's stages h = 2..32 run as f32x2 operations inside the thread and
+// h = 64 pairs it with the neighbouring lane.  The direct kernel serves
+// binary32 inputs and the ragged tail (n % 64) of bf16 inputs.
 #include "qfp4_common.cuh"
 #include "quantize1d.cuh"
 

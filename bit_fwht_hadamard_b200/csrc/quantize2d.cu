@@ -15,9 +15,12 @@
 // each lane one column of the tile -- the codes of X^T, bit-identical by
 // construction because every element was rounded once.
 //
-// Column-wise kernels (1D X^T baseline, MXFP8): a warp covers a 32 x 32
-// tile, lane = column, so a column group of 32 (or two of 16) sits in one
-// lane's registers; row loads are 64 contiguous bytes per warp instruction.
+// Column-wise outputs (1D X^T baseline, MXFP8 columns): for bf16 input a warp
+// covers 32 rows x 128 columns with 4 adjacent columns a lane (`k_cols4`,
+// 256-byte row loads per warp instruction); binary32 inputs use a 32 x 32
+// tile with one column a lane.  Either way a column group of 32 (or two of
+// 16) sits in one lane's registers.  The row-wise MXFP8 output of a bf16
+// input comes from the TMA kernel of the 1D quantize.
 #include "qfp4_common.cuh"
 #include "quantize1d.cuh"
 
