@@ -233,3 +233,18 @@ def test_f64_to_bf16_rounding():
     ref = torch.from_numpy(v).to(torch.bfloat16).view(torch.uint16).numpy()
     ours = np.array([oracle.f64_to_bf16(float(t)) for t in v], np.uint16)
     assert (ours == ref).all()
+
+
+def test_dequantize_nan_scale_bytes():
+    """E8M0 0xFF and E4M3 0x7F / 0xFF are the OCP NaN encodings: a group under
+    such a byte dequantizes to NaN, every other byte to finite values."""
+    codes16 = np.array([0x10, 0x32, 0x54, 0x76, 0x98, 0xBA, 0xDC, 0xFE], np.uint8)   # codes 0..15
+    for fmt, K, nan_bytes in ((oracle.NVFP4, 16, {0x7F, 0xFF}), (oracle.MXFP4, 32, {0xFF})):
+        codes = np.tile(codes16, (256, K // 16))
+        scales = np.arange(256, dtype=np.uint8).reshape(256, 1)
+        ts = np.float32(0.5) if fmt == oracle.NVFP4 else None
+        out = oracle.dequantize(codes, scales, ts, 256, K, fmt)
+        for b in range(256):
+            assert np.isnan(out[b]).all() == (b in nan_bytes), b
+            if b not in nan_bytes:
+                assert np.isfinite(out[b]).all()
