@@ -52,3 +52,36 @@ def test_argument_errors_return_before_any_launch():
     assert st == q.ERR_SHAPE                                # N % 4
     st = q.qfp4_gemm_blockscaled(fake, fake, None, fake, fake, None, 64, 64, 64, q.MXFP4, q.F32, fake, fake, 16, None)
     assert st == q.ERR_ARG                                  # workspace too small
+
+
+def test_more_argument_errors_follow_the_header():
+    """The remaining documented rejections, all decided on the host."""
+    f = 1 << 20
+    Q = q.qfp4_quantize
+    # four-over-six only with NVFP4, 1D, round-to-nearest
+    assert Q(f, q.BF16, 16, 64, q.NVFP4, q.SR, 0, 0, 1, 0, f, f, None, None, f, f, 4096, None) == q.ERR_UNSUPPORTED
+    assert Q(f, q.BF16, 16, 64, q.NVFP4, q.RNE, 0, 1, 1, 0, f, f, None, None, f, f, 4096, None) == q.ERR_UNSUPPORTED
+    # 2D blocks only with NVFP4 and without rotation
+    assert Q(f, q.BF16, 16, 128, q.MXFP4, q.RNE, 0, 1, 0, 0, f, f, None, None, None, None, 0, None) == q.ERR_UNSUPPORTED
+    assert Q(f, q.BF16, 16, 128, q.NVFP4, q.RNE, 1, 1, 0, 0, f, f, None, None, f, f, 4096, None) == q.ERR_UNSUPPORTED
+    # 1D column-wise output not with rotation; codesT and scalesT together
+    assert Q(f, q.BF16, 32, 128, q.MXFP4, q.RNE, 1, 0, 0, 0, f, f, f, f, None, None, 0, None) == q.ERR_UNSUPPORTED
+    assert Q(f, q.BF16, 32, 128, q.MXFP4, q.RNE, 0, 0, 0, 0, f, f, f, None, None, None, 0, None) == q.ERR_ARG
+    # shapes: rotation needs K % 128, 2D needs M % 16, 1D columns need M % g
+    assert Q(f, q.BF16, 16, 96, q.MXFP4, q.RNE, 1, 0, 0, 0, f, f, None, None, None, None, 0, None) == q.ERR_SHAPE
+    assert Q(f, q.BF16, 24, 64, q.NVFP4, q.RNE, 0, 1, 0, 0, f, f, f, f, f, f, 4096, None) == q.ERR_SHAPE
+    assert Q(f, q.BF16, 48, 64, q.MXFP4, q.RNE, 0, 0, 0, 0, f, f, f, f, None, None, 0, None) == q.ERR_SHAPE
+    # enum values
+    assert Q(f, q.BF16, 16, 64, 7, q.RNE, 0, 0, 0, 0, f, f, None, None, None, None, 0, None) == q.ERR_ARG
+    assert Q(f, 9, 16, 64, q.MXFP4, q.RNE, 0, 0, 0, 0, f, f, None, None, None, None, 0, None) == q.ERR_ARG
+    # MXFP8: K % 32; column output needs M % 32
+    M8 = q.qfp4_quantize_mxfp8
+    assert M8(f, q.BF16, 32, 48, q.RNE, 0, f, f, None, None, None) == q.ERR_SHAPE
+    assert M8(f, q.BF16, 48, 64, q.RNE, 0, f, f, f, f, None) == q.ERR_SHAPE
+    assert M8(f, q.BF16, 32, 64, 5, 0, f, f, None, None, None) == q.ERR_ARG
+    # dequantize: K % g, NVFP4 needs the tensor scale, output type
+    D = q.qfp4_dequantize
+    assert D(f, f, None, 4, 48, q.MXFP4, q.F32, f, None) == q.ERR_SHAPE
+    assert D(f, f, None, 4, 64, q.NVFP4, q.F32, f, None) == q.ERR_ARG
+    assert D(f, f, None, 4, 64, q.MXFP4, 3, f, None) == q.ERR_ARG
+    assert D(f + 4, f, None, 4, 64, q.MXFP4, q.F32, f, None) == q.ERR_ALIGN
