@@ -24,12 +24,14 @@ RNE, SR = 0, 1
 BF16, F32 = 0, 1
 GRAN_TENSOR, GRAN_ROW, GRAN_GROUP16, GRAN_GROUP32 = 0, 1, 2, 3
 OK, ERR_ARG, ERR_SHAPE, ERR_UNSUPPORTED, ERR_ALIGN, ERR_CUDA, ERR_TIMEOUT = 0, -1, -2, -3, -4, -5, -6
+DEV_ERR_TIMEOUT = 1
 
 EXPORTS = [
     "qfp4_quantize_workspace_bytes", "qfp4_quantize", "qfp4_quantize_mxfp8", "qfp4_quantize_fp32scale",
     "qfp4_dequantize", "qfp4_gemm_workspace_bytes", "qfp4_gemm_blockscaled", "qfp4_gemm_fused_rq_workspace_bytes",
     "qfp4_gemm_fused_rq", "qfp4_gemm_blockscaled_noalloc",
-    "qfp4_status_string", "qfp4_last_device_error", "qfp4_version", "qfp4_launch_count",
+    "qfp4_status_string", "qfp4_last_device_error", "qfp4_selftest_wait_timeout", "qfp4_version",
+    "qfp4_launch_count",
 ]
 
 _lib = None
@@ -77,6 +79,8 @@ def lib():
         L.qfp4_status_string.argtypes = [c_int]
         L.qfp4_last_device_error.restype = c_int
         L.qfp4_last_device_error.argtypes = []
+        L.qfp4_selftest_wait_timeout.restype = c_int
+        L.qfp4_selftest_wait_timeout.argtypes = [c_int64, P]
         L.qfp4_version.restype = c_int
         L.qfp4_version.argtypes = []
         L.qfp4_launch_count.restype = c_uint64
@@ -149,6 +153,10 @@ def qfp4_last_device_error():
     return lib().qfp4_last_device_error()
 
 
+def qfp4_selftest_wait_timeout(limit_us, stream):
+    return lib().qfp4_selftest_wait_timeout(limit_us, stream)
+
+
 def qfp4_version():
     return lib().qfp4_version()
 
@@ -216,28 +224,31 @@ def quantize(x, fmt=MXFP4, rounding=RNE, rotate=False, block2d=False, four6=Fals
     return o
 
 
-def quantize_mxfp8(x, rounding=RNE, seed=0, transposed=False, stream=None):
+def quantize_mxfp8(x, rounding=RNE, seed=0, transposed=False, stream=None, out=None):
     torch = _torch()
     M, K = x.shape
     dev = x.device
-    o = {"codes": torch.empty((M, K), dtype=torch.uint8, device=dev),
-         "scales": torch.empty((M, K // 32), dtype=torch.uint8, device=dev)}
-    if transposed:
-        o["codesT"] = torch.empty((K, M), dtype=torch.uint8, device=dev)
-        o["scalesT"] = torch.empty((K, M // 32), dtype=torch.uint8, device=dev)
+    o = dict(out) if out is not None else {}
+    if "codes" not in o:
+        o["codes"] = torch.empty((M, K), dtype=torch.uint8, device=dev)
+        o["scales"] = torch.empty((M, K // 32), dtype=torch.uint8, device=dev)
+        if transposed:
+            o["codesT"] = torch.empty((K, M), dtype=torch.uint8, device=dev)
+            o["scalesT"] = torch.empty((K, M // 32), dtype=torch.uint8, device=dev)
     st = qfp4_quantize_mxfp8(_ptr(x), _xdt(x), M, K, rounding, seed, _ptr(o["codes"]), _ptr(o["scales"]),
                              _ptr(o.get("codesT")), _ptr(o.get("scalesT")), _stream(stream))
     _check(st, "qfp4_quantize_mxfp8")
     return o
 
 
-def quantize_fp32scale(x, gran, stream=None):
+def quantize_fp32scale(x, gran, stream=None, out=None):
     torch = _torch()
     M, K = x.shape
     dev = x.device
     n_scales = {GRAN_TENSOR: 1, GRAN_ROW: M, GRAN_GROUP16: M * K // 16, GRAN_GROUP32: M * K // 32}[gran]
-    o = {"codes": torch.empty((M, K // 2), dtype=torch.uint8, device=dev),
-         "scales": torch.empty(n_scales, dtype=torch.float32, device=dev)}
+    o = dict(out) if out is not None else {
+        "codes": torch.empty((M, K // 2), dtype=torch.uint8, device=dev),
+        "scales": torch.empty(n_scales, dtype=torch.float32, device=dev)}
     wsb = qfp4_quantize_workspace_bytes(M, K, NVFP4)
     ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
     st = qfp4_quantize_fp32scale(_ptr(x), _xdt(x), M, K, gran, _ptr(o["codes"]), _ptr(o["scales"]), _ptr(ws), wsb,
@@ -246,10 +257,12 @@ def quantize_fp32scale(x, gran, stream=None):
     return o
 
 
-def dequantize(q, M, K, fmt, out_dtype=None, stream=None):
+def dequantize(q, M, K, fmt, out_dtype=None, stream=None, out=None):
     torch = _torch()
-    out_dtype = torch.float32 if out_dtype is None else out_dtype
-    out = torch.empty((M, K), dtype=out_dtype, device=q["codes"].device)
+    if out is None:
+        out_dtype = torch.float32 if out_dtype is None else out_dtype
+        out = torch.empty((M, K), dtype=out_dtype, device=q["codes"].device)
+    out_dtype = out.dtype
     st = qfp4_dequantize(_ptr(q["codes"]), _ptr(q["scales"]), _ptr(q.get("tscale")), M, K, fmt,
                          F32 if out_dtype == torch.float32 else BF16, _ptr(out), _stream(stream))
     _check(st, "qfp4_dequantize")

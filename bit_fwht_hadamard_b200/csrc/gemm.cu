@@ -3,21 +3,22 @@
 // packed E2M1 codes with row-major scales as qfp4_quantize writes them).
 //
 // Method: [QN] §QuTLASS (MXFP4 / NVFP4 operands, FP32 accumulation);
-// [LB] §FP4 (Blackwell FP4 tensor cores).  Hardware path (sm_100a):
-//   * tcgen05.mma.cta_group::1 kind::mxf4 (E8M0 scale per 32, MXFP4) or
-//     kind::mxf4nvf4 (E4M3 scale per 16, NVFP4), M=128 x N=256 x K=64 per
-//     instruction, fp32 accumulators in tensor memory (TMEM);
-//   * operands staged in shared memory by TMA (128-byte swizzle, no
-//     multicast), scale factors staged by 1D bulk copies and moved to TMEM
-//     with tcgen05.cp (32x128b, replicated to the four lane quadrants);
-//   * persistent, warp-specialised CTA: warp 0 produces (TMA), warp 1
-//     issues MMAs (one elected lane), warps 2-9 drain the accumulator
-//     (tcgen05.ld) and store; the accumulator is released as soon as the
-//     tile is in registers, so the next tile's MMAs overlap the stores.
-// The row-major scales are first rearranged by a small prepass into
-// 512-byte chunks in the tcgen05.cp source layout (128 rows x 4 scales:
-// byte (r%32)*16 + (r/32)*4 + j), so the main loop loads them with plain
-// contiguous bulk copies; the chunks live in the caller's workspace.
+// [LB] §FP4 (Blackwell FP4 tensor cores).  Two persistent, warp-specialised
+// kernels on sm_100a, both with fp32 accumulators in tensor memory (TMEM),
+// operands staged by TMA with 128-byte swizzle and no multicast:
+//   * k_gemm_bs2 (M > 128): a cluster of two CTAs computes a 256 x 256 tile
+//     with tcgen05.mma.cta_group::2 (kind::mxf4 block32 for MXFP4,
+//     kind::mxf4nvf4 block16 for NVFP4).  The leader's one MMA lane issues;
+//     a scale producer and four scale warps per CTA move each k-tile's scale
+//     words into a ring of TMEM buffers with tcgen05.st; eight epilogue warps
+//     per CTA read the accumulator (tcgen05.ld), hand it back, then store.
+//   * k_gemm_blockscaled (M <= 128): one CTA per 128 x 256 tile; the MMA lane
+//     moves the scale chunks to TMEM with tcgen05.cp (32x128b.warpx4).
+// Both hand the accumulator back as soon as it is in registers, so the next
+// tile's MMAs overlap the stores.  The row-major scales are first rearranged
+// by a small prepass into 512-byte chunks (128 rows x 4 scales: byte
+// (r%32)*16 + (r/32)*4 + j), which the main loops load with plain TMA or
+// bulk copies; the chunks live in the caller's workspace.
 #include "qfp4_common.cuh"
 #include "quantize1d.cuh"
 
@@ -384,6 +385,10 @@ __global__ void __launch_bounds__(GM_THREADS, 1)
                 tmem_ld16x256b_x16(tmem + (static_cast<uint32_t>(32 * q + 16 * hh) << 16) + 128 * h, r + 64 * hh);
             tmem_ld_wait();
             reg_fence<128>(r);
+            // the accumulator is in registers: hand it back before the stores
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty);
 
             // r[64hh + 4j + {0,1}]: row 32q + 16hh + lane/4, columns 8j + 2(lane%4) + {0,1};
             // r[64hh + 4j + {2,3}]: the row 8 below.  Four lanes cover 32 contiguous bytes.
@@ -414,10 +419,6 @@ __global__ void __launch_bounds__(GM_THREADS, 1)
                             }
                     }
                 }
-            // handed back after the stores, as in the 2-CTA kernel
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty);
         }
     }
 
@@ -494,14 +495,17 @@ __device__ __forceinline__ void cluster_sync()
 {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-// arrive on a barrier given by its shared::cluster address (this CTA's or the
-// partner's).  Default semantics (release at CTA scope): what the arrival
-// publishes is tensor-memory state that tcgen05.wait + tcgen05.fence already
-// made complete, so no cluster-wide memory fence is needed, and one per
-// k-tile would stall the scale warps.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
+// Arrive on a barrier of the leader CTA, given by its shared::cluster address.
+// The leader's own threads arrive with the default release at CTA scope.  The
+// partner's arrivals cross CTAs, so they release at cluster scope: that orders
+// the partner's completed tensor-memory accesses (tcgen05.wait + fence) before
+// the leader's acquire in the memory model, not only in practice.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr, bool remote)
 {
-    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+    if (remote)
+        asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+    else
+        asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 __device__ __forceinline__ void tma_load_2d_cg2(void *smem_dst, const CUtensorMap *map, uint32_t leader_bar, int c0, int c1)
 {
@@ -676,12 +680,12 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
         if (leader && lane == 0) {
             int it = 0, ti = 0;
             for (int t = cluster; t < ntiles && !abort_flag; t += nclusters, ++ti) {
-                if (!mbar_wait(&acc_empty, (ti & 1) ^ 1u)) { abort_flag = 1; break; }
+                if (!mbar_wait_cluster(&acc_empty, (ti & 1) ^ 1u)) { abort_flag = 1; break; }
                 tc_fence_after();
                 for (int kt = 0; kt < p.KT; ++kt, ++it) {
                     const int s = it % G2_STAGES, b = it % NBUF;
                     if (!mbar_wait(&full[s], (it / G2_STAGES) & 1u)) { abort_flag = 1; break; }
-                    if (!mbar_wait(&sf_full[b], (it / NBUF) & 1u)) { abort_flag = 1; break; }
+                    if (!mbar_wait_cluster(&sf_full[b], (it / NBUF) & 1u)) { abort_flag = 1; break; }
                     tc_fence_after();
                     const uint64_t adesc = desc_k_sw128(stage_a(s));
                     const uint64_t bdesc = desc_k_sw128(stage_b(s));
@@ -755,8 +759,13 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
                         rb[h][w][2] = u.z;
                         rb[h][w][3] = u.w;
                     }
+                // The slot is refilled by the scale producer's next TMA load (an
+                // async-proxy write); the reads above are generic-proxy accesses
+                // that may still be outstanding when the release below issues.
+                // The proxy fence in every lane orders them before the refill.
+                fence_proxy_async();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sfs_empty[s]);   // the slot's bytes are in registers now
+                if (lane == 0) mbar_arrive(&sfs_empty[s]);
                 // one TMEM word per MMA k (K = 64): NVFP4 uses a whole raw word,
                 // MXFP4 the half of one (its two block-32 scales, in bytes 0-1)
                 auto mma_word = [&](uint32_t raw4, uint32_t raw2, int k) -> uint32_t {
@@ -779,7 +788,7 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&sf_full[b]), 0));
+                if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&sf_full[b]), 0), !leader);
             }
         }
         // the leader's last releases of the scale buffers are multicast into
@@ -809,6 +818,11 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
                 tmem_ld16x256b_x16(tmem + (static_cast<uint32_t>(32 * q + 16 * hh) << 16) + 128 * h, r + 64 * hh);
             tmem_ld_wait();
             reg_fence<128>(r);
+            // the accumulator is in registers: hand it back at once, so the
+            // next tile's MMAs overlap these stores
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(acc_empty_leader, !leader);
 
             const int col0 = nb * G2_BN + 128 * h + 2 * (lane & 3);
             const int row_base = mb * G2_BM + 128 * static_cast<int>(rank);
@@ -838,14 +852,6 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
                             }
                     }
                 }
-            // The accumulator is handed back only after this warp's stores are
-            // issued.  Handing it back right after the tcgen05.ld / wait::ld
-            // pair (so the next tile's MMAs overlap these stores) gave
-            // occasional wrong 32 x 128 blocks on B200: one warp's values
-            // partly from the next tile, seen as run-to-run differences.
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
         }
     }
     g2_exit(tmem, false);
@@ -895,13 +901,8 @@ int rearrange_scales(const uint8_t *a_scales, int64_t M, int n_blocks_a, uint8_t
 template <int FMT, int OUT>
 static int launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p, int grid, cudaStream_t s)
 {
-    static bool configured = false;
     auto kern = k_gemm_blockscaled<FMT, OUT>;
-    if (!configured) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GM_SMEM) != cudaSuccess)
-            return QFP4_ERR_CUDA;
-        configured = true;
-    }
+    if (ensure_dyn_smem<k_gemm_blockscaled<FMT, OUT>>(GM_SMEM) != QFP4_OK) return QFP4_ERR_CUDA;
     if (launch_pdl(kern, dim3(grid), dim3(GM_THREADS), GM_SMEM, s, ta, tb, p) != cudaSuccess) {
         (void)cudaGetLastError();
         return QFP4_ERR_CUDA;
@@ -914,13 +915,8 @@ template <int FMT, int OUT>
 static int launch_gemm2(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tsa, const CUtensorMap &tsb,
                         const GemmParams &p, int grid, cudaStream_t s)
 {
-    static bool configured = false;
     auto kern = k_gemm_bs2<FMT, OUT>;
-    if (!configured) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G2_SMEM) != cudaSuccess)
-            return QFP4_ERR_CUDA;
-        configured = true;
-    }
+    if (ensure_dyn_smem<k_gemm_bs2<FMT, OUT>>(G2_SMEM) != QFP4_OK) return QFP4_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid, 1, 1);
     cfg.blockDim = dim3(G2_THREADS, 1, 1);

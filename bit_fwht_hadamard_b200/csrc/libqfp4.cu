@@ -5,6 +5,5 @@
 #include "dequant_fp32scale.cu"
 #include "quantize2d.cu"
 #include "gemm.cu"
-#include "pending.cu"
 #include "api.cu"
 #include "gemm_noalloc.cu"

@@ -13,6 +13,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/qfp4.h"
 
 #if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ != 1000)
@@ -27,8 +29,9 @@ template <class T>
 __host__ __device__ __forceinline__ T imax(T a, T b) { return a < b ? b : a; }
 
 // ------------------------------------------------------------------ errors
-// Device-side sticky error word (bounded waits that gave up, bounds checks).
-enum : int { DEV_ERR_NONE = 0, DEV_ERR_TIMEOUT = 1, DEV_ERR_BOUNDS = 2 };
+// Device-side sticky error word: the code of the first bounded wait that gave
+// up (QFP4_DEV_ERR_TIMEOUT), read and cleared by qfp4_last_device_error.
+enum : int { DEV_ERR_NONE = 0, DEV_ERR_TIMEOUT = QFP4_DEV_ERR_TIMEOUT };
 static __device__ int g_dev_error = 0;   // one copy: the library is a single translation unit
 
 // A spin on an mbarrier gives up after this many polls (seconds of wall
@@ -99,19 +102,44 @@ __device__ __forceinline__ void settle_ns(uint64_t ns)
 }
 constexpr uint64_t kSettleNs = 100000ull;
 
-// Bounded wait: true when the phase completed, false (error recorded) when
-// kWaitLimitNs of wall time (or kSpinLimit polls) ran out.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
+// The same poll with acquire at cluster scope, for a barrier that threads of
+// the partner CTA arrive on with release at cluster scope.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity)
 {
-    if (mbar_try_wait(bar, parity)) return true;
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait: true when the phase completed, false (error recorded) when
+// limit_ns of wall time (or kSpinLimit polls) ran out.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+template <bool CLUSTER = false>
+__device__ __forceinline__ bool mbar_wait_for(uint64_t *bar, uint32_t parity, uint64_t limit_ns)
+{
+    auto poll = [&] { return CLUSTER ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+    if (poll()) return true;
     const uint64_t t0 = global_ns();
     for (uint32_t i = 0; i < kSpinLimit; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 255u) == 255u && global_ns() - t0 > kWaitLimitNs) break;
+        if (poll()) return true;
+        if ((i & 255u) == 255u && global_ns() - t0 > limit_ns) break;
     }
     record_error(DEV_ERR_TIMEOUT);
     return false;
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
+{
+    return mbar_wait_for<false>(bar, parity, kWaitLimitNs);
+}
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity)
+{
+    return mbar_wait_for<true>(bar, parity, kWaitLimitNs);
 }
 
 // ------------------------------------------------------------------ dependent launches
@@ -429,6 +457,30 @@ int encode_tensor_map(CUtensorMap *map, CUtensorMapDataType dtype, int rank, voi
 int num_sms();
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Raise kernel Kern's dynamic shared-memory limit to `bytes` on the current
+// device.  The attribute is per device, so it is recorded per device (and
+// per kernel: one set of flags per template instance); devices beyond the
+// table set it on every call.
+template <auto Kern>
+int ensure_dyn_smem(int bytes)
+{
+    constexpr int kMaxDevices = 64;
+    static std::atomic<int> done[kMaxDevices];       // static storage: starts at zero
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return QFP4_ERR_CUDA;
+    }
+    const bool tracked = dev >= 0 && dev < kMaxDevices;
+    if (tracked && done[dev].load(std::memory_order_acquire) >= bytes) return QFP4_OK;
+    if (cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return QFP4_ERR_CUDA;
+    }
+    if (tracked) done[dev].store(bytes, std::memory_order_release);
+    return QFP4_OK;
+}
 
 }  // namespace qfp4
 

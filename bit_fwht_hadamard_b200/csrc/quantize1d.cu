@@ -793,19 +793,13 @@ __global__ void __launch_bounds__(128) k_quant1d_direct(const T *__restrict__ x,
 }
 
 // ---------------------------------------------------------------- host launchers
-static int smem_configured[2][3][2][2][2] = {};
-
 template <int MODE, int FMT, bool ROT, bool SR, bool FOUR6>
 static int launch_tma(const CUtensorMap &tm, const QuantParams &p, int grid, cudaStream_t stream)
 {
     constexpr int W = qt_warps(FOUR6), SMEM = qt_smem_bytes(FOUR6);
     auto kern = k_quant1d_tma<MODE, FMT, ROT, SR, FOUR6, W, QT_STAGES, QT_UP>;
-    int &done = smem_configured[MODE][FMT][ROT][SR][FOUR6];
-    if (!done) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess)
-            return QFP4_ERR_CUDA;
-        done = 1;
-    }
+    if (ensure_dyn_smem<k_quant1d_tma<MODE, FMT, ROT, SR, FOUR6, W, QT_STAGES, QT_UP>>(SMEM) != QFP4_OK)
+        return QFP4_ERR_CUDA;
     if (launch_pdl(kern, dim3(grid), dim3(32 * W), SMEM, stream, tm, p) != cudaSuccess) {
         (void)cudaGetLastError();
         return QFP4_ERR_CUDA;

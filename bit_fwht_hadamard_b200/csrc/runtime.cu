@@ -77,6 +77,25 @@ extern "C" int qfp4_last_device_error(void)
     return v;
 }
 
-extern "C" int qfp4_version(void) { return 100; }
+// One thread waits on an mbarrier that expects an arrival nobody makes, with
+// no copy or MMA in flight, so only the bounded wait's give-up path runs.
+__global__ void k_wait_timeout(uint64_t limit_ns)
+{
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x != 0) return;
+    qfp4::mbar_init(&bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    (void)qfp4::mbar_wait_for<false>(&bar, 0, limit_ns);
+}
+
+extern "C" int qfp4_selftest_wait_timeout(int64_t limit_us, qfp4_stream_t stream)
+{
+    if (limit_us < 1 || limit_us > 1000000) return QFP4_ERR_ARG;
+    k_wait_timeout<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(static_cast<uint64_t>(limit_us) * 1000u);
+    QFP4_LAUNCH_CHECK();
+    return QFP4_OK;
+}
+
+extern "C" int qfp4_version(void) { return 200; }
 
 extern "C" uint64_t qfp4_launch_count(void) { return qfp4::g_launches.load(std::memory_order_relaxed); }

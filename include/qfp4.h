@@ -237,9 +237,21 @@ int qfp4_gemm_fused_rq(const void *A_bf16, int64_t M, int64_t K, int rotate, int
 const char *qfp4_status_string(int status);
 
 /* Sticky device-side error word of the current device: 0 when clean, else
- * the code a bounded wait or a bounds check recorded (cleared by the read).
- * Synchronizes the current device. */
+ * the code of the first device-side failure since the last read (cleared by
+ * the read); -1 if the device could not be read.  Synchronizes the current
+ * device.  Codes: */
+enum {
+    QFP4_DEV_ERR_TIMEOUT = 1    /* a bounded wait inside a kernel gave up (the kernel returned early) */
+};
 int qfp4_last_device_error(void);
+
+/* Diagnostics: launch a one-thread kernel whose only action is a bounded
+ * wait on a barrier that nothing completes, giving up after limit_us
+ * microseconds (1 .. 10^6).  Nothing else is in flight, so it exercises the
+ * give-up path every other kernel's waits share: afterwards
+ * qfp4_last_device_error() returns QFP4_DEV_ERR_TIMEOUT and the context
+ * stays usable.  No counterpart on the source pages (a library self-test). */
+int qfp4_selftest_wait_timeout(int64_t limit_us, qfp4_stream_t stream);
 
 /* Library version, as MAJOR*10000 + MINOR*100 + PATCH. */
 int qfp4_version(void);

@@ -25,3 +25,13 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(autouse=True)
+def _output_guard_bands():
+    """After each test, the guard bands around every guarded GPU output
+    (tests/gpu_util.guarded) must be intact."""
+    yield
+    gu = sys.modules.get("gpu_util")
+    if gu is not None:
+        gu.check_guards()

@@ -88,3 +88,91 @@ def blocks_to_tiles(blocks: np.ndarray, tiles_per_row: int = 4) -> np.ndarray:
     tiles = np.repeat(b[:, None, :], 16, axis=1)                  # (n, 16, 16)
     R = n // tiles_per_row
     return tiles.reshape(R, tiles_per_row, 16, 16).transpose(0, 2, 1, 3).reshape(R * 16, tiles_per_row * 16)
+
+
+# ------------------------------------------------------------------ guarded outputs
+# Every output a GPU test hands to the library sits between two 256-byte
+# guard bands filled with a pattern; after each test (an autouse fixture in
+# conftest.py) the bands must be intact, so a kernel that writes past either
+# end of an output buffer fails the test that made it.  The output itself
+# starts out holding the pattern too, so elements a kernel forgets to write
+# differ from the oracle.
+GUARD_BYTES = 256
+GUARD_PATTERN = 0xA5
+_guards = []
+
+
+def guarded(shape, dtype, device="cuda"):
+    shape = tuple(int(s) for s in shape)
+    n = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
+    raw = torch.full((n + 2 * GUARD_BYTES,), GUARD_PATTERN, dtype=torch.uint8, device=device)
+    _guards.append((raw, n))
+    return raw[GUARD_BYTES:GUARD_BYTES + n].view(dtype).view(shape)
+
+
+def check_guards():
+    """Assert every guard band since the last check is intact, then forget them."""
+    if not _guards:
+        return
+    torch.cuda.synchronize()
+    bad = []
+    for raw, n in _guards:
+        pre, post = raw[:GUARD_BYTES], raw[GUARD_BYTES + n:]
+        if not bool((pre == GUARD_PATTERN).all()) or not bool((post == GUARD_PATTERN).all()):
+            bad.append((n, int((pre != GUARD_PATTERN).sum()), int((post != GUARD_PATTERN).sum())))
+    _guards.clear()
+    assert not bad, f"writes outside output buffers (bytes, bytes changed before, after): {bad}"
+
+
+def _fmt_g(fmt):
+    import bit_fwht_hadamard_b200 as q
+    return 32 if fmt == q.MXFP4 else 16
+
+
+def quantize(x, fmt, rounding=0, rotate=False, block2d=False, four6=False, seed=0, transposed=False):
+    """q.quantize with every output in a guarded buffer."""
+    import bit_fwht_hadamard_b200 as q
+    M, K = x.shape
+    g = _fmt_g(fmt)
+    o = {"codes": guarded((M, K // 2), torch.uint8), "scales": guarded((M, K // g), torch.uint8)}
+    if transposed:
+        o["codesT"] = guarded((K, M // 2), torch.uint8)
+        o["scalesT"] = guarded((K, M // g), torch.uint8)
+    if fmt == q.NVFP4:
+        o["tscale"] = guarded((1,), torch.float32)
+    return q.quantize(x, fmt, rounding, rotate=rotate, block2d=block2d, four6=four6, seed=seed,
+                      transposed=transposed, out=o)
+
+
+def quantize_mxfp8(x, rounding=0, seed=0, transposed=False):
+    import bit_fwht_hadamard_b200 as q
+    M, K = x.shape
+    o = {"codes": guarded((M, K), torch.uint8), "scales": guarded((M, K // 32), torch.uint8)}
+    if transposed:
+        o["codesT"] = guarded((K, M), torch.uint8)
+        o["scalesT"] = guarded((K, M // 32), torch.uint8)
+    return q.quantize_mxfp8(x, rounding, seed=seed, transposed=transposed, out=o)
+
+
+def quantize_fp32scale(x, gran):
+    import bit_fwht_hadamard_b200 as q
+    M, K = x.shape
+    n = {q.GRAN_TENSOR: 1, q.GRAN_ROW: M, q.GRAN_GROUP16: M * K // 16, q.GRAN_GROUP32: M * K // 32}[gran]
+    return q.quantize_fp32scale(x, gran, out={"codes": guarded((M, K // 2), torch.uint8),
+                                              "scales": guarded((n,), torch.float32)})
+
+
+def dequantize(qd, M, K, fmt, out_dtype=None):
+    import bit_fwht_hadamard_b200 as q
+    return q.dequantize(qd, M, K, fmt, out=guarded((M, K), out_dtype or torch.float32))
+
+
+def gemm(A, B, M, N, K, fmt, out_dtype=None):
+    import bit_fwht_hadamard_b200 as q
+    return q.gemm(A, B, M, N, K, fmt, out=guarded((M, N), out_dtype or torch.float32))
+
+
+def gemm_fused_rq(A_bf16, B, N, fmt, rotate=True, four6=False, out_dtype=None):
+    import bit_fwht_hadamard_b200 as q
+    return q.gemm_fused_rq(A_bf16, B, N, fmt=fmt, rotate=rotate, four6=four6,
+                           out=guarded((A_bf16.shape[0], N), out_dtype or torch.float32))

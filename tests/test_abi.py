@@ -85,3 +85,8 @@ def test_more_argument_errors_follow_the_header():
     assert D(f, f, None, 4, 64, q.NVFP4, q.F32, f, None) == q.ERR_ARG
     assert D(f, f, None, 4, 64, q.MXFP4, 3, f, None) == q.ERR_ARG
     assert D(f + 4, f, None, 4, 64, q.MXFP4, q.F32, f, None) == q.ERR_ALIGN
+
+
+def test_selftest_wait_limit_is_checked_on_the_host():
+    assert q.qfp4_selftest_wait_timeout(0, None) == q.ERR_ARG
+    assert q.qfp4_selftest_wait_timeout(1_000_001, None) == q.ERR_ARG

@@ -92,3 +92,36 @@ def test_one_correction_is_not_always_enough_in_theory():
         if rn32(x * rn32(1 / S)) != rn32(x / S):
             misses += 1
     assert misses > 0
+
+
+def _sr_up(v: Fraction, u24: int) -> bool:
+    """The stochastic decision between 0 and 0.5 for |v| < 0.5: up iff
+    u < |v| / 0.5 with u = u24 * 2^-24."""
+    return Fraction(u24, 1 << 24) < abs(v) / Fraction(1, 2)
+
+
+def test_underflowing_quotients_decide_the_same_codes():
+    """Markstein's theorem assumes no underflow, but the kernels use the chain
+    for every S in [2^-125, 2^125], so x / S may be subnormal (a block whose
+    values span more than 2^126).  There the chain can miss fl(x / S) by an
+    ulp; this pins that every such miss is harmless: both results have the
+    same sign and the same zero-ness, and both lie far below 2^-25, where the
+    E2M1 nearest code is a signed zero and the stochastic decision between 0
+    and 0.5 depends only on whether v is zero (u is a multiple of 2^-24)."""
+    rng = random.Random(31)
+    n = misses = 0
+    for _ in range(6000):
+        S = f32(rng.uniform(1, 2) * 2.0 ** rng.randint(-125, 125))
+        e = rng.randint(-172, -110)
+        x = rn32(Fraction(rng.uniform(1, 2)) * Fraction(2) ** e * S) * rng.choice([1, -1])
+        want = rn32(x / S)
+        got = quotient_chain(x, S)
+        n += 1
+        if got == want:
+            continue
+        misses += 1
+        assert (got == 0) == (want == 0) and (got < 0) == (want < 0), (float(x), float(S))
+        assert max(abs(got), abs(want)) < Fraction(1, 1 << 100), (float(x), float(S))
+        for u24 in (0, 1, (1 << 24) - 1):
+            assert _sr_up(got, u24) == _sr_up(want, u24)
+    assert n > 5000 and misses > 0           # the underflow range really is exercised

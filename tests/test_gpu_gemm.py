@@ -12,6 +12,7 @@ import torch
 import bit_fwht_hadamard_b200 as q
 import oracle
 import synth
+import gpu_util as G
 from gpu_util import host, to_dev
 
 pytestmark = pytest.mark.gpu
@@ -64,7 +65,7 @@ def test_gemm_matches_oracle(M, N, K, fmt, out):
     b = synth.cfg3_W(N, K, seed=N + 5 * K)
     A, B = oracle.quantize(a, fmt[1]), oracle.quantize(b, fmt[1])
     od = torch.float32 if out == "f32" else torch.bfloat16
-    y = q.gemm(_upload(A), _upload(B), M, N, K, fmt[0], out_dtype=od)
+    y = G.gemm(_upload(A), _upload(B), M, N, K, fmt[0], out_dtype=od)
     yh = host(y)
     if out == "bf16":
         yh = synth.bf16_bits_to_f32(yh)
@@ -87,7 +88,7 @@ def test_gemm_exact_on_representable_inputs(fmt):
     if fmt[1] == oracle.NVFP4:
         A["tscale"] = np.array([1.0], np.float32)
         B["tscale"] = np.array([1.0], np.float32)
-    y = host(q.gemm(_upload(A), _upload(B), M, N, K, fmt[0]))
+    y = host(G.gemm(_upload(A), _upload(B), M, N, K, fmt[0]))
     rows, cols = _all_pairs(M, N)
     ref, _ = oracle.gemm_sampled(A, B, M, N, K, fmt[1], rows, cols)
     assert np.array_equal(y[rows, cols].astype(np.float64), ref)
@@ -99,9 +100,9 @@ def test_gemm_full_size_forward_linear():
     128 x 128 corner tiles."""
     M, N, K = 8192, 11008, 4096
     x, w = synth.cfg3_X(), synth.cfg3_W()
-    X = q.quantize(to_dev(x), q.NVFP4, four6=True)
-    W = q.quantize(to_dev(w), q.NVFP4, four6=True)
-    y = host(q.gemm(X, W, M, N, K, q.NVFP4))
+    X = G.quantize(to_dev(x), q.NVFP4, four6=True)
+    W = G.quantize(to_dev(w), q.NVFP4, four6=True)
+    y = host(G.gemm(X, W, M, N, K, q.NVFP4))
     A = {k: host(v) for k, v in X.items()}
     B = {k: host(v) for k, v in W.items()}
     rows, cols = _sample_pairs(M, N, 20_000, seed=3)
@@ -117,9 +118,9 @@ def test_gemm_bitwise_deterministic(fmt, out):
     tiles and the wrap-around of every stage, scale-slot and scale-buffer ring
     are exercised; a hand-off race would show up as differing elements."""
     M, N, K = 4096, 9216, 2048          # 16 x 36 = 576 tiles of 256 x 256 on 74 pairs, 8 k-tiles each
-    X = q.quantize(to_dev(synth.cfg3_X(M, K, seed=11)), fmt[0])
-    W = q.quantize(to_dev(synth.cfg3_W(N, K, seed=12)), fmt[0])
-    ys = [q.gemm(X, W, M, N, K, fmt[0], out_dtype=out) for _ in range(4)]
+    X = G.quantize(to_dev(synth.cfg3_X(M, K, seed=11)), fmt[0])
+    W = G.quantize(to_dev(synth.cfg3_W(N, K, seed=12)), fmt[0])
+    ys = [G.gemm(X, W, M, N, K, fmt[0], out_dtype=out) for _ in range(4)]
     torch.cuda.synchronize()
     ref = ys[0].view(torch.int32 if out == torch.float32 else torch.int16)
     for y in ys[1:]:
@@ -137,7 +138,7 @@ def test_fused_rotate_quantize_gemm(fmt, four6):
     a = synth.cfg5_A(M, K, seed=21)
     b = synth.cfg5_B(N, K, seed=22)
     B = oracle.quantize(b, fmt[1], rotate=True)                  # weights rotated offline
-    y = host(q.gemm_fused_rq(to_dev(a), _upload(B), N, fmt=fmt[0], rotate=True, four6=four6))
+    y = host(G.gemm_fused_rq(to_dev(a), _upload(B), N, fmt=fmt[0], rotate=True, four6=four6))
     A = oracle.quantize(a, fmt[1], rotate=True, four6=four6)
     rows, cols = _all_pairs(M, N)
     _check(y, A, B, M, N, K, fmt[1], rows, cols)
@@ -147,6 +148,6 @@ def test_gemm_argument_errors():
     A = {"codes": torch.zeros((128, 128), dtype=torch.uint8, device="cuda"),
          "scales": torch.zeros((128, 8), dtype=torch.uint8, device="cuda")}
     with pytest.raises(q.QFP4Error) as e:
-        q.gemm(A, A, 128, 130, 256, q.MXFP4)                      # N % 4
+        G.gemm(A, A, 128, 130, 256, q.MXFP4)                      # N % 4
     assert e.value.status == q.ERR_SHAPE
     assert q.qfp4_last_device_error() == 0

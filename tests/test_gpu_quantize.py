@@ -11,6 +11,7 @@ import torch
 import bit_fwht_hadamard_b200 as q
 import oracle
 import synth
+import gpu_util as G
 from gpu_util import blocks_to_rows, encode_input, host, mismatch_report, nvfp4_boundary_blocks, to_dev
 
 pytestmark = pytest.mark.gpu
@@ -40,7 +41,7 @@ def test_quantize_1d_matches_oracle(M, K, fmt, rounding, rotate):
     if K % g or (rotate and K % 128):
         pytest.skip("shape not valid for this mode")
     x = synth.cfg2_X(M, K, seed=M * 1000 + K)
-    got = q.quantize(to_dev(x), fmt[0], rounding, rotate=rotate, seed=0xDEADBEEF12345)
+    got = G.quantize(to_dev(x), fmt[0], rounding, rotate=rotate, seed=0xDEADBEEF12345)
     ref = oracle.quantize(x, fmt[1], rounding, rotate=rotate, seed=0xDEADBEEF12345)
     _cmp(got, ref)
 
@@ -51,7 +52,7 @@ def test_four_over_six_matches_oracle(M, K, rotate):
     if rotate and K % 128:
         pytest.skip()
     x = synth.cfg3_X(M, K, seed=M + K)
-    got = q.quantize(to_dev(x), q.NVFP4, q.RNE, rotate=rotate, four6=True)
+    got = G.quantize(to_dev(x), q.NVFP4, q.RNE, rotate=rotate, four6=True)
     ref = oracle.quantize(x, oracle.NVFP4, oracle.RNE, rotate=rotate, four6=True)
     _cmp(got, ref)
 
@@ -62,7 +63,7 @@ def test_float32_input(fmt, rounding):
     W = np.zeros((256, 800), np.float32)
     W[:, :784] = synth.cfg1_W()
     W[17, 300] = 50 * np.abs(W).max()
-    got = q.quantize(to_dev(W), fmt[0], rounding, seed=3)
+    got = G.quantize(to_dev(W), fmt[0], rounding, seed=3)
     ref = oracle.quantize(W, fmt[1], rounding, seed=3)
     _cmp(got, ref)
 
@@ -72,7 +73,7 @@ def test_full_size_activation_quantize_rne_and_sr():
     x = synth.cfg2_X()
     xd = to_dev(x)
     for rounding, seed in ((q.RNE, 0), (q.SR, 7)):
-        got = q.quantize(xd, q.MXFP4, rounding, rotate=True, seed=seed)
+        got = G.quantize(xd, q.MXFP4, rounding, rotate=True, seed=seed)
         ref = oracle.quantize(x, oracle.MXFP4, rounding, rotate=True, seed=seed)
         _cmp(got, ref)
 
@@ -80,7 +81,7 @@ def test_full_size_activation_quantize_rne_and_sr():
 def test_full_size_nvfp4_four6_forward_operands():
     """X 8192 x 4096 Student-t(3)*0.5 and W 11008 x 4096 N(0, 0.02^2), NVFP4 + four-over-six."""
     for x in (synth.cfg3_X(), synth.cfg3_W()):
-        got = q.quantize(to_dev(x), q.NVFP4, q.RNE, four6=True)
+        got = G.quantize(to_dev(x), q.NVFP4, q.RNE, four6=True)
         ref = oracle.quantize(x, oracle.NVFP4, oracle.RNE, four6=True)
         _cmp(got, ref)
 
@@ -88,7 +89,7 @@ def test_full_size_nvfp4_four6_forward_operands():
 def test_degenerate_inputs():
     z = np.zeros((64, 256), np.uint16)
     for fmt in FMTS:
-        got = q.quantize(to_dev(z), fmt[0], q.RNE)
+        got = G.quantize(to_dev(z), fmt[0], q.RNE)
         _cmp(got, oracle.quantize(z, fmt[1], oracle.RNE))
     z[3, 5] = 0x8000                                   # a negative zero
     x = synth.cfg2_X(64, 256, seed=9)
@@ -98,11 +99,11 @@ def test_degenerate_inputs():
     for fmt in FMTS:
         for rounding in (q.RNE, q.SR):
             for arr in (z, x):
-                _cmp(q.quantize(to_dev(arr), fmt[0], rounding, seed=1),
+                _cmp(G.quantize(to_dev(arr), fmt[0], rounding, seed=1),
                      oracle.quantize(arr, fmt[1], rounding, seed=1))
     # M = 0 is a no-op that succeeds
     e = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
-    q.quantize(e, q.MXFP4)
+    G.quantize(e, q.MXFP4)
 
 
 @pytest.mark.parametrize("rounding", [q.RNE, q.SR], ids=["rne", "sr"])
@@ -126,7 +127,7 @@ def test_every_bf16_value_up_to_6(rounding):
     X[:n_groups] = x
     X[n_groups:, 0] = 0x40C0
     X = X.reshape(rows, 128)
-    got = q.quantize(to_dev(X), q.MXFP4, rounding, seed=77)
+    got = G.quantize(to_dev(X), q.MXFP4, rounding, seed=77)
     ref = oracle.quantize(X, oracle.MXFP4, rounding, seed=77)
     assert (ref["scales"] == 127).all()
     _cmp(got, ref)
@@ -138,7 +139,7 @@ def test_large_dynamic_range():
     x = synth.to_bf16(z, (64, 512))
     for fmt in FMTS:
         for rounding in (q.RNE, q.SR):
-            _cmp(q.quantize(to_dev(x), fmt[0], rounding, seed=2), oracle.quantize(x, fmt[1], rounding, seed=2))
+            _cmp(G.quantize(to_dev(x), fmt[0], rounding, seed=2), oracle.quantize(x, fmt[1], rounding, seed=2))
 
 
 @pytest.mark.parametrize("kind", ["bf16", "f32"])
@@ -150,7 +151,7 @@ def test_nvfp4_rounding_boundaries(kind, four6):
     oracle's IEEE divisions bit for bit, through the TMA kernel (bf16) and
     the direct kernel (float32)."""
     x = encode_input(blocks_to_rows(nvfp4_boundary_blocks(kind)), kind)
-    got = q.quantize(to_dev(x), q.NVFP4, q.RNE, four6=four6)
+    got = G.quantize(to_dev(x), q.NVFP4, q.RNE, four6=four6)
     ref = oracle.quantize(x, oracle.NVFP4, oracle.RNE, four6=four6)
     _cmp(got, ref)
 
@@ -172,8 +173,8 @@ def test_dequantize_matches_oracle(fmt, out):
     M, K = 300, 512
     x = synth.cfg3_X(M, K, seed=77)
     ref_q = oracle.quantize(x, fmt[1])
-    gq = q.quantize(to_dev(x), fmt[0])
-    got = host(q.dequantize(gq, M, K, fmt[0], out))
+    gq = G.quantize(to_dev(x), fmt[0])
+    got = host(G.dequantize(gq, M, K, fmt[0], out))
     exact = oracle.dequantize(ref_q["codes"], ref_q["scales"], ref_q.get("tscale"), M, K, fmt[1])
     if out == torch.float32:
         assert np.array_equal(got, oracle.f64_to_f32_array(exact))
@@ -189,7 +190,7 @@ def test_fp32_scale_modes_match_oracle(gran):
     W = np.zeros((256, 800), np.float32)
     W[:, :784] = synth.cfg1_W()
     W[17, 300] = 50 * np.abs(W).max()
-    got = q.quantize_fp32scale(to_dev(W), gran)
+    got = G.quantize_fp32scale(to_dev(W), gran)
     ref = oracle.quantize_fp32scale(W, gran)
     assert np.array_equal(host(got["codes"]), ref["codes"])
     assert np.array_equal(host(got["scales"]).view(np.uint32), ref["scales"].view(np.uint32))
@@ -217,7 +218,7 @@ def test_dequantize_every_code_and_scale(out):
         dq = {"codes": torch.from_numpy(codes).cuda(), "scales": torch.from_numpy(scales).cuda()}
         if ts is not None:
             dq["tscale"] = torch.tensor([float(ts)], dtype=torch.float32, device="cuda")
-        got = host(q.dequantize(dq, M, K, fmt, out))
+        got = host(G.dequantize(dq, M, K, fmt, out))
         exact = oracle.dequantize(codes, scales, None if ts is None else np.float32(ts), M, K, ofmt)
         nan = np.isnan(exact)
         assert nan.any()                                           # E8M0 0xFF / E4M3 0x7F, 0xFF
@@ -241,9 +242,9 @@ def test_quantize_repeatable_full_size():
     outputs for every format of the TMA-fed kernel: guards its shared-memory
     ring against a refill landing before the reads of a stage are done."""
     x = to_dev(synth.cfg4_G())
-    calls = [lambda: q.quantize(x, q.MXFP4, q.RNE), lambda: q.quantize(x, q.MXFP4, q.RNE, rotate=True),
-             lambda: q.quantize(x, q.NVFP4, q.RNE), lambda: q.quantize(x, q.NVFP4, q.SR, seed=3),
-             lambda: q.quantize_mxfp8(x, q.RNE), lambda: q.quantize_mxfp8(x, q.SR, seed=3)]
+    calls = [lambda: G.quantize(x, q.MXFP4, q.RNE), lambda: G.quantize(x, q.MXFP4, q.RNE, rotate=True),
+             lambda: G.quantize(x, q.NVFP4, q.RNE), lambda: G.quantize(x, q.NVFP4, q.SR, seed=3),
+             lambda: G.quantize_mxfp8(x, q.RNE), lambda: G.quantize_mxfp8(x, q.SR, seed=3)]
     for f in calls:
         first = {k: host(v) for k, v in f().items()}
         for _ in range(3):

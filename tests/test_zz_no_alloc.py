@@ -9,10 +9,11 @@ the library instead of asking for a workspace.
 
 These checks call it through the C ABI and compare it with the workspace
 entry point, qfp4_gemm_blockscaled, on two calls in a row (different shapes
-and formats, so the second call reuses scratch the first one filled), within
-the GEMM tolerance of the other GPU tests: |diff| <= 1e-5 * sum_k |a||b|.
-The file name makes pytest collect it last; it builds all of its own inputs,
-so it also passes alone in a fresh process.
+and formats, so the second call reuses scratch the first one filled).  Both
+run the same kernels in the same order, so the outputs must agree bit for
+bit; a scratch-reuse bug that only perturbed values would show.  A third
+case fills the 16 MiB exactly.  The file name makes pytest collect it last;
+it builds all of its own inputs, so it also passes alone in a fresh process.
 """
 import numpy as np
 import pytest
@@ -40,30 +41,47 @@ def _noalloc(A, B, M, N, K, fmt):
     return out
 
 
-def _bound(A, B, M, N, K, fmt):
-    """1e-5 * sum_k |a_k||b_k| from the library's own dequantized operands."""
-    da = q.dequantize(A, M, K, fmt).double().abs()
-    db = q.dequantize(B, N, K, fmt).double().abs()
-    return 1e-5 * (da @ db.T)
+def _same_bits(got, want):
+    diff = int((got.view(torch.int32) != want.view(torch.int32)).sum())
+    assert diff == 0, f"{diff} of {want.numel()} outputs differ from the workspace GEMM"
 
 
 def test_noalloc_gemm_matches_workspace_gemm_on_two_calls():
     cases = [(384, 512, 1024, q.NVFP4, 101), (256, 768, 2048, q.MXFP4, 202)]
     for M, N, K, fmt, seed in cases:
         A, B = _operands(M, N, K, fmt, seed)
-        want = q.gemm(A, B, M, N, K, fmt).double()
-        got = _noalloc(A, B, M, N, K, fmt).double()
+        want = q.gemm(A, B, M, N, K, fmt)
+        got = _noalloc(A, B, M, N, K, fmt)
         torch.cuda.synchronize()
-        diff = (got - want).abs()
-        assert bool((diff <= _bound(A, B, M, N, K, fmt)).all()), float(diff.max())
+        _same_bits(got, want)
+    assert q.qfp4_last_device_error() == 0
+
+
+def test_noalloc_gemm_with_scales_filling_the_scratch_exactly():
+    # 4096 x 4096 x 32768 NVFP4: (32 A blocks + 2 x 16 B blocks) x 128 k-tiles x
+    # 4 chunks x 512 B = 16 MiB, the largest shape class the scratch admits
+    M, N, K = 4096, 4096, 32768
+    assert q.qfp4_gemm_workspace_bytes(M, N, K, q.NVFP4) == 16 << 20
+    A, B = _operands(M, N, K, q.NVFP4, 303)
+    want = q.gemm(A, B, M, N, K, q.NVFP4)
+    got = _noalloc(A, B, M, N, K, q.NVFP4)
+    torch.cuda.synchronize()
+    _same_bits(got, want)
     assert q.qfp4_last_device_error() == 0
 
 
 def test_noalloc_gemm_rejects_shapes_beyond_its_scratch():
-    # (16384 x 4096 x 14336, NVFP4) needs more than the built-in 16 MiB for its
-    # rearranged scales; the call refuses before touching any buffer
-    assert q.qfp4_gemm_workspace_bytes(16384, 4096, 14336, q.NVFP4) > 16 << 20
+    # one more 128-row block of A than the exact fit above, and the
+    # 16384 x 4096 x 14336 NVFP4 shape: both need more than the built-in
+    # 16 MiB for their rearranged scales; the call refuses before touching
+    # any buffer
     fake = 1 << 20
-    st = q.qfp4_gemm_blockscaled_noalloc(fake, fake, fake, fake, fake, fake, 16384, 4096, 14336, q.NVFP4, q.F32,
-                                         fake, None)
-    assert st == q.ERR_SHAPE
+    for M, N, K in ((4097, 4096, 32768), (16384, 4096, 14336)):
+        assert q.qfp4_gemm_workspace_bytes(M, N, K, q.NVFP4) > 16 << 20
+        st = q.qfp4_gemm_blockscaled_noalloc(fake, fake, fake, fake, fake, fake, M, N, K, q.NVFP4, q.F32, fake,
+                                             None)
+        assert st == q.ERR_SHAPE
+    # argument errors come first, as in the workspace entry point
+    st = q.qfp4_gemm_blockscaled_noalloc(fake, fake, fake, fake, fake, fake, 1 << 40, 4096, 4096, 7, q.F32, fake,
+                                         None)
+    assert st == q.ERR_ARG
