@@ -21,7 +21,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "qfp4_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
-MXFP4, NVFP4 = 0, 1
+MXFP4, NVFP4, MXFP8 = 0, 1, 2
+RULE_DEFAULT, RULE_OCP_FLOOR, RULE_E4M3_UP = 0, 1, 2
 RNE, SR = 0, 1
 BF16, F32 = 0, 1
 GRAN_TENSOR, GRAN_ROW, GRAN_GROUP16, GRAN_GROUP32 = 0, 1, 2, 3
@@ -75,6 +76,18 @@ def lib():
         L.or_quantize.restype = c_int
         L.or_quantize.argtypes = [c_void_p, c_int, c_int64, c_int64, c_int, c_int, c_int, c_int, c_int,
                                   c_uint64, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]
+        L.or_scale_exp_floor.restype = c_int
+        L.or_scale_exp_floor.argtypes = [c_float, c_int]
+        L.or_e4m3_up.restype = c_uint8
+        L.or_e4m3_up.argtypes = [c_float]
+        L.or_quantize_ex.restype = c_int
+        L.or_quantize_ex.argtypes = [c_void_p, c_int, c_int64, c_int64, c_int, c_int, c_int, c_int, c_int, c_int,
+                                     c_uint64, c_int64, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                     c_void_p, c_void_p]
+        L.or_tensor_amax.restype = c_float
+        L.or_tensor_amax.argtypes = [c_void_p, c_int, c_int64, c_int64, c_int]
+        L.or_mxfp4_group.restype = c_int
+        L.or_mxfp4_group.argtypes = [c_void_p, c_void_p, c_int, c_int, c_int, c_uint64, c_void_p, c_void_p]
         L.or_four6_pick.restype = c_int
         L.or_four6_pick.argtypes = [c_void_p, c_float, c_void_p, c_void_p]
         L.or_quantize_mxfp8.restype = c_int
@@ -217,6 +230,74 @@ def quantize_status(x, fmt, rounding=RNE, rotate=False, block2d=False, four6=Fal
                              _p(codes), _p(scales), _p(codesT), _p(scalesT), _p(tscale))
 
 
+def scale_exp_floor(amax: float, emax: int = 2) -> int:
+    return lib().or_scale_exp_floor(amax, emax)
+
+
+def e4m3_up(v: float) -> int:
+    return lib().or_e4m3_up(v)
+
+
+def quantize_ex(x: np.ndarray, fmt: int, rounding: int = RNE, rotate: bool = False, block2d: bool = False,
+                four6: bool = False, rule: int = RULE_DEFAULT, seed: int = 0, row0: int = 0, amax_in=None,
+                want_amax: bool = False, transposed: bool = False):
+    """or_quantize_ex: scale-rule variants, a given tensor amax (NVFP4) and
+    a first-row offset.  Returns dict(codes, scales, [codesT, scalesT],
+    [tscale], [amax])."""
+    x = np.ascontiguousarray(x)
+    M, K = x.shape
+    g = 32 if fmt == MXFP4 else 16
+    codes = np.zeros((M, K // 2), np.uint8)
+    scales = np.zeros((M, K // g), np.uint8)
+    codesT = scalesT = None
+    if transposed:
+        codesT = np.zeros((K, M // 2), np.uint8)
+        scalesT = np.zeros((K, M // g), np.uint8)
+    tscale = np.zeros(1, np.float32)
+    ain = None if amax_in is None else np.asarray([amax_in], np.float32)
+    aout = np.zeros(1, np.float32) if want_amax else None
+    _check(lib().or_quantize_ex(_p(x), _xdt(x), M, K, fmt, rounding, int(rotate), int(block2d), int(four6), rule,
+                                seed, row0, _p(ain), _p(codes), _p(scales), _p(codesT), _p(scalesT), _p(tscale),
+                                _p(aout)))
+    out = {"codes": codes, "scales": scales}
+    if transposed:
+        out["codesT"], out["scalesT"] = codesT, scalesT
+    if fmt == NVFP4:
+        out["tscale"] = tscale
+    if want_amax:
+        out["amax"] = aout
+    return out
+
+
+def quantize_ex_status(x, fmt, rounding=RNE, rotate=False, block2d=False, four6=False, rule=RULE_DEFAULT, seed=0,
+                       row0=0, amax_in=None, transposed=False) -> int:
+    x = np.ascontiguousarray(x)
+    M, K = x.shape
+    n = max(M * K, 2)
+    bufs = [np.zeros(n, np.uint8) for _ in range(4)]
+    tscale = np.zeros(1, np.float32)
+    ain = None if amax_in is None else np.asarray([amax_in], np.float32)
+    return lib().or_quantize_ex(_p(x), _xdt(x), M, K, fmt, rounding, int(rotate), int(block2d), int(four6), rule,
+                                seed, row0, _p(ain), _p(bufs[0]), _p(bufs[1]),
+                                _p(bufs[2]) if transposed else None, _p(bufs[3]) if transposed else None,
+                                _p(tscale), None)
+
+
+def tensor_amax(x: np.ndarray, rotate: bool = False) -> float:
+    x = np.ascontiguousarray(x)
+    return float(lib().or_tensor_amax(_p(x), _xdt(x), x.shape[0], x.shape[1], int(rotate)))
+
+
+def mxfp4_group(x32: np.ndarray, rounding: int = RNE, four6: bool = False, rule: int = RULE_DEFAULT,
+                seed: int = 0, e=None):
+    x32 = np.ascontiguousarray(x32, dtype=np.float32)
+    e = np.ascontiguousarray(np.arange(32, dtype=np.uint64) if e is None else e, dtype=np.uint64)
+    sb = np.zeros(1, np.uint8)
+    codes = np.zeros(32, np.uint8)
+    pick = lib().or_mxfp4_group(_p(x32), _p(e), rounding, int(four6), rule, seed, _p(sb), _p(codes))
+    return pick, int(sb[0]), codes
+
+
 def four6_pick(x16: np.ndarray, s_t: float):
     x16 = np.ascontiguousarray(x16, dtype=np.float32)
     enc = np.zeros(1, np.uint8)
@@ -273,8 +354,8 @@ def gemm_sampled(A: dict, B: dict, M: int, N: int, K: int, fmt: int, rows, cols)
     cols = np.ascontiguousarray(cols, np.int64)
     out = np.zeros(rows.shape[0], np.float64)
     mag = np.zeros(rows.shape[0], np.float64)
-    tA = None if fmt == MXFP4 else np.ascontiguousarray(np.asarray(A["tscale"], np.float32).reshape(1))
-    tB = None if fmt == MXFP4 else np.ascontiguousarray(np.asarray(B["tscale"], np.float32).reshape(1))
+    tA = None if fmt != NVFP4 else np.ascontiguousarray(np.asarray(A["tscale"], np.float32).reshape(1))
+    tB = None if fmt != NVFP4 else np.ascontiguousarray(np.asarray(B["tscale"], np.float32).reshape(1))
     _check(lib().or_gemm_sampled(_p(np.ascontiguousarray(A["codes"])), _p(np.ascontiguousarray(A["scales"])),
                                  _p(tA), _p(np.ascontiguousarray(B["codes"])), _p(np.ascontiguousarray(B["scales"])),
                                  _p(tB), M, N, K, fmt, _p(rows), _p(cols), rows.shape[0], _p(out), _p(mag)))

@@ -118,6 +118,19 @@ uint8_t or_e4m3_sr(float v, uint32_t r)
     return (uint8_t)(sign | (u < p ? lo + 1 : lo));
 }
 
+/* E4M3 rounded up: the least finite E4M3 value >= |v| (the truncation-free
+ * rule of [TI] applied to the NVFP4 block scale, so that S >= amax_b / 6 and
+ * no element of the block clips), saturating at 448; sign copied from v. */
+uint8_t or_e4m3_up(float v)
+{
+    assert(isfinite(v));
+    uint8_t sign = signbit(v) ? 0x80 : 0;
+    double a = fabs((double)v);
+    if (a >= 448.0) return (uint8_t)(sign | 0x7E);
+    int lo = e4m3_floor_byte(a);
+    return (uint8_t)(sign | ((double)or_e4m3_value((uint8_t)lo) == a ? lo : lo + 1));
+}
+
 /* E8M0 ([LB] §3: an 8-bit exponent, scale 2^k only) */
 double or_e8m0_value(uint8_t b)
 {
@@ -135,6 +148,21 @@ int or_scale_exp(float amax, double top)
     for (int k = -127; k <= 127; ++k)
         if (ldexp(top, k) >= (double)amax) return k;
     return 127;
+}
+
+/* The OCP MX rule for the shared exponent (the "2^k scale" of [LB] §3 with
+ * its rounding direction taken from the OCP microscaling definition, as the
+ * ablation next to [TI]'s truncation-free rule): k = floor(log2(amax)) -
+ * emax, emax = 2 for E2M1 (largest value 6 = 1.5 * 2^2), i.e. the largest k
+ * with 2^(k + emax) <= amax, clamped to [-127, 127].  amax / 2^k lies in
+ * [4, 8), so values above 6 * 2^k are clipped to 6 (saturation).  amax = 0
+ * gives -127. */
+int or_scale_exp_floor(float amax, int emax)
+{
+    assert(isfinite(amax) && amax >= 0.0f);
+    for (int k = 127; k >= -127; --k)
+        if (ldexp(1.0, k + emax) <= (double)amax) return k;
+    return -127;
 }
 
 /* ========================================================================
@@ -240,20 +268,30 @@ static uint8_t fp4_round(float v, int rounding, uint64_t seed, uint64_t e)
  * NVFP4 two-level scale.  The pages give the idea (a fine group scale under
  * one per-tensor FP scale, [LB] §3 VS-Quant; NVFP4 named in [QN], [46]);
  * the formula taken: per-tensor s_t = amax_t / (6*448) in binary32, and the
- * block scale byte enc = E4M3_RNE_satfinite((amax_b / d) / s_t) with d = 6
- * (d = 4 for the four-over-six candidate).  The effective block scale used
+ * block scale byte enc = E4M3((amax_b / d) / s_t) with d = 6 (d = 4 for the
+ * four-over-six candidate), rounded to nearest (default rule) or up (the
+ * truncation-free rule), saturating at 448.  The effective block scale used
  * to divide is S = dec(enc) * s_t in binary32.
  * ====================================================================== */
-static uint8_t nv_enc(float amax_b, float s_t, float d)
+static uint8_t nv_enc(float amax_b, float s_t, float d, int rule)
 {
     float q = amax_b / d;
     float r = q / s_t;
-    return or_e4m3_rne(r);
+    if (!(r < 448.0f)) return 0x7E;               /* 448 and beyond, incl. +inf */
+    return rule == OR_RULE_E4M3_UP ? or_e4m3_up(r) : or_e4m3_rne(r);
 }
 
 static float nv_seff(uint8_t enc, float s_t)
 {
     return or_e4m3_value(enc) * s_t;
+}
+
+/* E2M1 code of v = x / S; a quotient that overflowed binary32 (a tiny S)
+ * saturates like any magnitude beyond 6. */
+static uint8_t fp4_code(float v, int rounding, uint64_t seed, uint64_t e)
+{
+    if (isinf(v)) return (uint8_t)((signbit(v) ? 8 : 0) | 7);
+    return fp4_round(v, rounding, seed, e);
 }
 
 /* quantize n values x[] (logical indices e[]) under effective scale S;
@@ -264,43 +302,89 @@ static void quant_block(const float *x, const uint64_t *e, int n, float S,
     for (int t = 0; t < n; ++t) {
         if (S == 0.0f) { codes[t] = 0; continue; }
         float v = x[t] / S;
-        codes[t] = fp4_round(v, rounding, seed, e[t]);
+        codes[t] = fp4_code(v, rounding, seed, e[t]);
     }
 }
 
 /* Four-over-six ([46] Methodology 1-3): two candidate scales per block, the
  * standard one (amax/6) and a smaller-range one (amax/4); quantize with each
  * (round to nearest) and keep the one with the lower block squared error.
- * Readings: block = the NVFP4 16-element block; error = sum over the block
- * of (deq - x)^2 in binary32 with deq = value(code) * S, summed as a fixed
- * tree (pairs i, i+8; then +4; +2; +1); a tie keeps amax/6. */
-static float block_sse16(const float *x, const uint8_t *codes, float S)
+ * Readings: block = the NVFP4 16-element block (the MXFP4 32-element group
+ * for the MXFP4 variant); error = sum over the block of (deq - x)^2 in
+ * binary32 with deq = value(code) * S, summed as a fixed tree (pairs i,
+ * i + n/2; then halves again down to 1); a tie keeps the standard scale. */
+static float block_sse(const float *x, const uint8_t *codes, float S, int n)
 {
-    float e[16];
-    for (int i = 0; i < 16; ++i) {
+    float e[32];
+    for (int i = 0; i < n; ++i) {
         float deq = or_e2m1_value(codes[i]) * S;
         float d = deq - x[i];
         e[i] = d * d;
     }
-    for (int h = 8; h >= 1; h >>= 1)
+    for (int h = n / 2; h >= 1; h >>= 1)
         for (int i = 0; i < h; ++i) e[i] = e[i] + e[i + h];
     return e[0];
 }
 
-int or_four6_pick(const float *x16, float s_t, uint8_t *enc_out, uint8_t codes_out[16])
+static int nv_four6(const float *x16, float s_t, int rule, uint8_t *enc_out, uint8_t codes_out[16])
 {
     float amax = 0.0f;
     for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x16[i]));
     uint64_t e[16] = {0};                         /* unused by RNE */
-    uint8_t enc6 = nv_enc(amax, s_t, 6.0f), enc4 = nv_enc(amax, s_t, 4.0f);
+    uint8_t enc6 = nv_enc(amax, s_t, 6.0f, rule), enc4 = nv_enc(amax, s_t, 4.0f, rule);
     float S6 = nv_seff(enc6, s_t), S4 = nv_seff(enc4, s_t);
     uint8_t c6[16], c4[16];
     quant_block(x16, e, 16, S6, OR_RNE, 0, c6);
     quant_block(x16, e, 16, S4, OR_RNE, 0, c4);
-    float sse6 = block_sse16(x16, c6, S6), sse4 = block_sse16(x16, c4, S4);
+    float sse6 = block_sse(x16, c6, S6, 16), sse4 = block_sse(x16, c4, S4, 16);
     int pick4 = sse4 < sse6;
     *enc_out = pick4 ? enc4 : enc6;
     memcpy(codes_out, pick4 ? c4 : c6, 16);
+    return pick4;
+}
+
+int or_four6_pick(const float *x16, float s_t, uint8_t *enc_out, uint8_t codes_out[16])
+{
+    return nv_four6(x16, s_t, OR_RULE_DEFAULT, enc_out, codes_out);
+}
+
+/* MXFP4 group exponent under a scale rule: truncation-free ([TI]) by
+ * default, the OCP floor rule as the ablation. */
+static int mx_exp(float amax, int rule)
+{
+    return rule == OR_RULE_OCP_FLOOR ? or_scale_exp_floor(amax, 2) : or_scale_exp(amax, 6.0);
+}
+
+/* One MXFP4 group of 32: scale byte and codes.  With four6, the second
+ * candidate is the least k4 with 4 * 2^k4 >= amax ([46]'s amax/4 scale
+ * carried to power-of-two scales); the group keeps the candidate with the
+ * lower block squared error (RNE), a tie keeps the rule's exponent.  An
+ * all-zero group gives byte 0 and +0 codes. */
+int or_mxfp4_group(const float *xg, const uint64_t *eg, int rounding, int four6, int rule,
+                   uint64_t seed, uint8_t *sbyte, uint8_t cg[32])
+{
+    float amax = 0.0f;
+    for (int t = 0; t < 32; ++t) amax = fmaxf(amax, fabsf(xg[t]));
+    if (amax == 0.0f) {
+        *sbyte = 0;
+        memset(cg, 0, 32);
+        return 0;
+    }
+    int k = mx_exp(amax, rule), pick4 = 0;
+    quant_block(xg, eg, 32, (float)ldexp(1.0, k), rounding, seed, cg);
+    if (four6) {
+        int k4 = or_scale_exp(amax, 4.0);
+        uint8_t c4[32];
+        quant_block(xg, eg, 32, (float)ldexp(1.0, k4), OR_RNE, 0, c4);
+        float sse = block_sse(xg, cg, (float)ldexp(1.0, k), 32);
+        float sse4 = block_sse(xg, c4, (float)ldexp(1.0, k4), 32);
+        if (sse4 < sse) {
+            k = k4;
+            memcpy(cg, c4, 32);
+            pick4 = 1;
+        }
+    }
+    *sbyte = (uint8_t)(k + 127);
     return pick4;
 }
 
@@ -308,7 +392,8 @@ int or_four6_pick(const float *x16, float s_t, uint8_t *enc_out, uint8_t codes_o
  * qfp4_quantize semantics.
  * ====================================================================== */
 static int check_quantize_args(const void *x, int xdt, int64_t M, int64_t K, int fmt,
-                               int rounding, int rotate, int block2d, int four6,
+                               int rounding, int rotate, int block2d, int four6, int rule,
+                               int64_t row0, const float *amax_in, const float *amax_out,
                                const uint8_t *codes, const uint8_t *scales,
                                const uint8_t *codesT, const uint8_t *scalesT,
                                const float *tscale)
@@ -317,34 +402,51 @@ static int check_quantize_args(const void *x, int xdt, int64_t M, int64_t K, int
     if (fmt != OR_MXFP4 && fmt != OR_NVFP4) return OR_ERR_ARG;
     if (rounding != OR_RNE && rounding != OR_SR) return OR_ERR_ARG;
     if (xdt != OR_BF16 && xdt != OR_F32) return OR_ERR_ARG;
+    if (rule < OR_RULE_DEFAULT || rule > OR_RULE_E4M3_UP || row0 < 0) return OR_ERR_ARG;
     if ((M * K > 0) && (!x || !codes || !scales)) return OR_ERR_ARG;
     if ((codesT == NULL) != (scalesT == NULL)) return OR_ERR_ARG;
     if (fmt == OR_NVFP4 && !tscale) return OR_ERR_ARG;
     int g = fmt == OR_MXFP4 ? 32 : 16;
-    if (four6 && (fmt != OR_NVFP4 || block2d || rounding != OR_RNE)) return OR_ERR_UNSUPPORTED;
-    if (block2d && (fmt != OR_NVFP4 || rotate)) return OR_ERR_UNSUPPORTED;
+    if (rule == OR_RULE_OCP_FLOOR && fmt != OR_MXFP4) return OR_ERR_UNSUPPORTED;
+    if (rule == OR_RULE_E4M3_UP && fmt != OR_NVFP4) return OR_ERR_UNSUPPORTED;
+    if ((amax_in || amax_out) && fmt != OR_NVFP4) return OR_ERR_UNSUPPORTED;
+    if (four6 && (block2d || rounding != OR_RNE)) return OR_ERR_UNSUPPORTED;
+    if (block2d && rotate) return OR_ERR_UNSUPPORTED;
     if (!block2d && rotate && codesT) return OR_ERR_UNSUPPORTED;
+    if (row0 && (block2d || codesT)) return OR_ERR_UNSUPPORTED;
     if (K % g) return OR_ERR_SHAPE;
     if (rotate && K % 128) return OR_ERR_SHAPE;
-    if (block2d && (M % 16 || K % 16)) return OR_ERR_SHAPE;
+    if (block2d && (M % g || K % g)) return OR_ERR_SHAPE;
     if (!block2d && codesT && M % g) return OR_ERR_SHAPE;
     return OR_OK;
 }
 
-/* per-tensor amax of the (rotated) input, then s_t in binary32 */
-static float tensor_scale(const void *x, int xdt, int64_t M, int64_t K, int rotate, float *row)
+/* per-tensor amax of the (rotated) input */
+static float tensor_amax(const void *x, int xdt, int64_t M, int64_t K, int rotate, float *row)
 {
     float amax_t = 0.0f;
     for (int64_t i = 0; i < M; ++i) {
         load_row(x, xdt, K, i, rotate, row);
         for (int64_t j = 0; j < K; ++j) amax_t = fmaxf(amax_t, fabsf(row[j]));
     }
-    return amax_t / 2688.0f;                       /* 6 * 448 */
+    return amax_t;
 }
 
-/* 1D groups of g along K for one row (MXFP4 or NVFP4, optional 4/6) */
-static void quantize_row_1d(const float *row, int64_t i, int64_t K, int fmt, int rounding,
-                            int four6, uint64_t seed, float s_t,
+float or_tensor_amax(const void *x, int xdt, int64_t M, int64_t K, int rotate)
+{
+    if (M <= 0 || K <= 0) return 0.0f;
+    float *row = (float *)malloc(sizeof(float) * (size_t)K);
+    if (!row) return NAN;
+    float a = tensor_amax(x, xdt, M, K, rotate, row);
+    free(row);
+    return a;
+}
+
+/* 1D groups of g along K for one row (MXFP4 or NVFP4, optional 4/6); the
+ * row's logical index is i (random words keyed on i*K + j), its outputs go
+ * to local row il of codes / scales */
+static void quantize_row_1d(const float *row, int64_t i, int64_t il, int64_t K, int fmt, int rounding,
+                            int four6, int rule, uint64_t seed, float s_t,
                             uint8_t *codes, uint8_t *scales)
 {
     int g = fmt == OR_MXFP4 ? 32 : 16;
@@ -360,37 +462,31 @@ static void quantize_row_1d(const float *row, int64_t i, int64_t K, int fmt, int
         }
         uint8_t sbyte;
         if (fmt == OR_MXFP4) {
-            if (amax == 0.0f) {                       /* all-zero group: +0 codes */
-                sbyte = 0;
-                memset(cg, 0, sizeof cg);
-            } else {
-                int k = or_scale_exp(amax, 6.0);
-                sbyte = (uint8_t)(k + 127);
-                quant_block(xg, eg, g, (float)ldexp(1.0, k), rounding, seed, cg);
-            }
+            or_mxfp4_group(xg, eg, rounding, four6, rule, seed, &sbyte, cg);
         } else if (four6) {
-            or_four6_pick(xg, s_t, &sbyte, cg);
+            nv_four6(xg, s_t, rule, &sbyte, cg);
         } else {
-            sbyte = nv_enc(amax, s_t, 6.0f);
+            sbyte = nv_enc(amax, s_t, 6.0f, rule);
             quant_block(xg, eg, g, nv_seff(sbyte, s_t), rounding, seed, cg);
         }
-        scales[i * (K / g) + j0 / g] = sbyte;
-        for (int t = 0; t < g; ++t) put_nibble(codes, i * K + j0 + t, cg[t]);
+        scales[il * (K / g) + j0 / g] = sbyte;
+        for (int t = 0; t < g; ++t) put_nibble(codes, il * K + j0 + t, cg[t]);
     }
 }
 
-int or_quantize(const void *x, int xdt, int64_t M, int64_t K,
-                int fmt, int rounding, int rotate, int block2d, int four6,
-                uint64_t seed,
-                uint8_t *codes, uint8_t *scales,
-                uint8_t *codesT, uint8_t *scalesT,
-                float *tscale)
+int or_quantize_ex(const void *x, int xdt, int64_t M, int64_t K,
+                   int fmt, int rounding, int rotate, int block2d, int four6, int rule,
+                   uint64_t seed, int64_t row0, const float *amax_in,
+                   uint8_t *codes, uint8_t *scales,
+                   uint8_t *codesT, uint8_t *scalesT,
+                   float *tscale, float *amax_out)
 {
-    int st = check_quantize_args(x, xdt, M, K, fmt, rounding, rotate, block2d, four6,
-                                 codes, scales, codesT, scalesT, tscale);
+    int st = check_quantize_args(x, xdt, M, K, fmt, rounding, rotate, block2d, four6, rule, row0,
+                                 amax_in, amax_out, codes, scales, codesT, scalesT, tscale);
     if (st != OR_OK) return st;
     if (M == 0 || K == 0) {
-        if (fmt == OR_NVFP4) *tscale = 0.0f;
+        if (fmt == OR_NVFP4) *tscale = amax_in ? *amax_in / 2688.0f : 0.0f;
+        if (amax_out) *amax_out = 0.0f;
         return OR_OK;
     }
     int g = fmt == OR_MXFP4 ? 32 : 16;
@@ -399,9 +495,17 @@ int or_quantize(const void *x, int xdt, int64_t M, int64_t K,
 
     float s_t = 0.0f;
     if (fmt == OR_NVFP4) {
-        s_t = tensor_scale(x, xdt, M, K, rotate, row);
+        /* the tensor scale from this tensor's own amax, or (delayed scaling,
+         * [QN] open questions: an EMA / history of activation scales) from an
+         * amax the caller supplies */
+        if (!amax_in || amax_out) {
+            float own = tensor_amax(x, xdt, M, K, rotate, row);
+            if (amax_out) *amax_out = own;
+            s_t = own / 2688.0f;                   /* 6 * 448 */
+        }
+        if (amax_in) s_t = *amax_in / 2688.0f;
         *tscale = s_t;
-        if (s_t == 0.0f) {                /* all-zero (or underflowed) tensor */
+        if (s_t == 0.0f) {                /* all-zero (or underflowed) tensor scale */
             memset(codes, 0, (size_t)(M * K / 2));
             memset(scales, 0, (size_t)(M * (K / g)));
             if (codesT) {
@@ -414,40 +518,54 @@ int or_quantize(const void *x, int xdt, int64_t M, int64_t K,
     }
 
     if (block2d) {
-        /* [TI]: 2D blocks (16x16, the NVFP4 block on both axes) so that X and
-         * X^T share one scale per block; codesT is the transpose of codes. */
-        float tile[256];
-        uint64_t et[256];
-        uint8_t ct[256];
-        for (int64_t bi = 0; bi < M; bi += 16)
-            for (int64_t bj = 0; bj < K; bj += 16) {
+        /* [TI]: 2D blocks (the group size on both axes: 16x16 NVFP4, 32x32
+         * MXFP4) so that X and X^T share one scale per block; codesT is the
+         * transpose of codes. */
+        int T = g;
+        float *tile = (float *)malloc(sizeof(float) * 1024);
+        uint64_t *et = (uint64_t *)malloc(sizeof(uint64_t) * 1024);
+        uint8_t *ct = (uint8_t *)malloc(1024);
+        for (int64_t bi = 0; bi < M; bi += T)
+            for (int64_t bj = 0; bj < K; bj += T) {
                 float amax = 0.0f;
-                for (int r = 0; r < 16; ++r)
-                    for (int c = 0; c < 16; ++c) {
+                for (int r = 0; r < T; ++r)
+                    for (int c = 0; c < T; ++c) {
                         int64_t e = (bi + r) * K + bj + c;
-                        tile[r * 16 + c] = load_elem(x, xdt, e);
-                        et[r * 16 + c] = (uint64_t)e;
-                        amax = fmaxf(amax, fabsf(tile[r * 16 + c]));
+                        tile[r * T + c] = load_elem(x, xdt, e);
+                        et[r * T + c] = (uint64_t)e;
+                        amax = fmaxf(amax, fabsf(tile[r * T + c]));
                     }
-                uint8_t enc = nv_enc(amax, s_t, 6.0f);
-                quant_block(tile, et, 256, nv_seff(enc, s_t), rounding, seed, ct);
-                for (int r = 0; r < 16; ++r)
-                    for (int c = 0; c < 16; ++c) {
+                uint8_t enc;
+                float S;
+                if (fmt == OR_MXFP4) {
+                    int k = amax == 0.0f ? -127 : mx_exp(amax, rule);
+                    enc = amax == 0.0f ? 0 : (uint8_t)(k + 127);
+                    S = amax == 0.0f ? 0.0f : (float)ldexp(1.0, k);
+                } else {
+                    enc = nv_enc(amax, s_t, 6.0f, rule);
+                    S = nv_seff(enc, s_t);
+                }
+                quant_block(tile, et, T * T, S, rounding, seed, ct);
+                for (int r = 0; r < T; ++r)
+                    for (int c = 0; c < T; ++c) {
                         int64_t i = bi + r, j = bj + c;
-                        put_nibble(codes, i * K + j, ct[r * 16 + c]);
-                        if (codesT) put_nibble(codesT, j * M + i, ct[r * 16 + c]);
+                        put_nibble(codes, i * K + j, ct[r * T + c]);
+                        if (codesT) put_nibble(codesT, j * M + i, ct[r * T + c]);
                     }
-                for (int r = 0; r < 16; ++r) scales[(bi + r) * (K / 16) + bj / 16] = enc;
+                for (int r = 0; r < T; ++r) scales[(bi + r) * (K / T) + bj / T] = enc;
                 if (scalesT)
-                    for (int c = 0; c < 16; ++c) scalesT[(bj + c) * (M / 16) + bi / 16] = enc;
+                    for (int c = 0; c < T; ++c) scalesT[(bj + c) * (M / T) + bi / T] = enc;
             }
+        free(tile);
+        free(et);
+        free(ct);
         free(row);
         return OR_OK;
     }
 
     for (int64_t i = 0; i < M; ++i) {
         load_row(x, xdt, K, i, rotate, row);
-        quantize_row_1d(row, i, K, fmt, rounding, four6, seed, s_t, codes, scales);
+        quantize_row_1d(row, row0 + i, i, K, fmt, rounding, four6, rule, seed, s_t, codes, scales);
     }
 
     if (codesT) {
@@ -466,18 +584,11 @@ int or_quantize(const void *x, int xdt, int64_t M, int64_t K,
                 }
                 uint8_t sbyte;
                 if (fmt == OR_MXFP4) {
-                    if (amax == 0.0f) {
-                        sbyte = 0;
-                        memset(cg, 0, sizeof cg);
-                    } else {
-                        int k = or_scale_exp(amax, 6.0);
-                        sbyte = (uint8_t)(k + 127);
-                        quant_block(xg, eg, g, (float)ldexp(1.0, k), rounding, seed, cg);
-                    }
+                    or_mxfp4_group(xg, eg, rounding, four6, rule, seed, &sbyte, cg);
                 } else if (four6) {
-                    or_four6_pick(xg, s_t, &sbyte, cg);
+                    nv_four6(xg, s_t, rule, &sbyte, cg);
                 } else {
-                    sbyte = nv_enc(amax, s_t, 6.0f);
+                    sbyte = nv_enc(amax, s_t, 6.0f, rule);
                     quant_block(xg, eg, g, nv_seff(sbyte, s_t), rounding, seed, cg);
                 }
                 scalesT[j * (M / g) + i0 / g] = sbyte;
@@ -486,6 +597,17 @@ int or_quantize(const void *x, int xdt, int64_t M, int64_t K,
     }
     free(row);
     return OR_OK;
+}
+
+int or_quantize(const void *x, int xdt, int64_t M, int64_t K,
+                int fmt, int rounding, int rotate, int block2d, int four6,
+                uint64_t seed,
+                uint8_t *codes, uint8_t *scales,
+                uint8_t *codesT, uint8_t *scalesT,
+                float *tscale)
+{
+    return or_quantize_ex(x, xdt, M, K, fmt, rounding, rotate, block2d, four6, OR_RULE_DEFAULT, seed, 0,
+                          NULL, codes, scales, codesT, scalesT, tscale, NULL);
 }
 
 /* ========================================================================
@@ -590,6 +712,8 @@ static uint8_t get_nibble(const uint8_t *buf, int64_t idx)
 static double deq_elem(const uint8_t *codes, const uint8_t *scales, double s_t,
                        int64_t K, int fmt, int64_t i, int64_t j)
 {
+    if (fmt == OR_MXFP8)                             /* one E4M3 byte per element */
+        return (double)or_e4m3_value(codes[i * K + j]) * or_e8m0_value(scales[i * (K / 32) + j / 32]);
     int g = fmt == OR_MXFP4 ? 32 : 16;
     double val = or_e2m1_value(get_nibble(codes, i * K + j));
     uint8_t sb = scales[i * (K / g) + j / g];
@@ -648,10 +772,12 @@ uint16_t or_f64_to_bf16(double v)
 }
 
 /* ========================================================================
- * GEMM reference ([QN] §QuTLASS: MXFP4/NVFP4 inputs, FP32 accumulate):
+ * GEMM reference ([QN] §QuTLASS: MXFP4/NVFP4 inputs, FP32 accumulate; the
+ * FP8 backward of [QN]'s forward/backward split and [TI]'s MXFP8 operands):
  * Y[m][n] = sum_k deqA[m][k] * deqB[n][k], A M x K and B N x K (both
  * K-major), in binary64 over the dequantized operands.  For NVFP4 the sum
- * runs over code * dec(enc) and the tensor scales multiply the result.
+ * runs over code * dec(enc) and the tensor scales multiply the result;
+ * MXFP8 operands are E4M3 bytes under E8M0 scales per 32.
  * ====================================================================== */
 int or_gemm_sampled(const uint8_t *A_codes, const uint8_t *A_scales, const float *A_tscale,
                     const uint8_t *B_codes, const uint8_t *B_scales, const float *B_tscale,
@@ -660,8 +786,8 @@ int or_gemm_sampled(const uint8_t *A_codes, const uint8_t *A_scales, const float
                     double *out, double *absmag)
 {
     if (M < 0 || N < 0 || K < 0) return OR_ERR_SHAPE;
-    if (fmt != OR_MXFP4 && fmt != OR_NVFP4) return OR_ERR_ARG;
-    int g = fmt == OR_MXFP4 ? 32 : 16;
+    if (fmt != OR_MXFP4 && fmt != OR_NVFP4 && fmt != OR_MXFP8) return OR_ERR_ARG;
+    int g = fmt == OR_NVFP4 ? 16 : 32;
     if (K % g) return OR_ERR_SHAPE;
     if (fmt == OR_NVFP4 && (!A_tscale || !B_tscale)) return OR_ERR_ARG;
     double tA = fmt == OR_NVFP4 ? (double)*A_tscale : 1.0;

@@ -42,7 +42,8 @@
 extern "C" {
 #endif
 
-enum { OR_MXFP4 = 0, OR_NVFP4 = 1 };           /* group formats            */
+enum { OR_MXFP4 = 0, OR_NVFP4 = 1, OR_MXFP8 = 2 };   /* group formats (MXFP8: GEMM reference only) */
+enum { OR_RULE_DEFAULT = 0, OR_RULE_OCP_FLOOR = 1, OR_RULE_E4M3_UP = 2 };   /* scale rules */
 enum { OR_RNE = 0, OR_SR = 1 };                /* rounding                 */
 enum { OR_BF16 = 0, OR_F32 = 1 };              /* input / output dtypes    */
 enum { OR_GRAN_TENSOR = 0, OR_GRAN_ROW = 1, OR_GRAN_GROUP16 = 2, OR_GRAN_GROUP32 = 3 };
@@ -59,6 +60,8 @@ uint8_t or_e4m3_rne(float v);                     /* nearest, satfinite      */
 uint8_t or_e4m3_sr(float v, uint32_t r);          /* stochastic, satfinite   */
 double  or_e8m0_value(uint8_t b);                 /* 2^(b-127)               */
 int     or_scale_exp(float amax, double top);     /* least k: top*2^k>=amax  */
+int     or_scale_exp_floor(float amax, int emax); /* OCP: floor(log2 amax)-emax */
+uint8_t or_e4m3_up(float v);                      /* least E4M3 >= |v|, sat.  */
 
 /* ---- building blocks -------------------------------------------------- */
 void     or_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]);
@@ -74,9 +77,35 @@ int or_quantize(const void *x, int xdt, int64_t M, int64_t K,
                 uint8_t *codesT, uint8_t *scalesT,
                 float *tscale);
 
+/* The same with the scale-rule variants and a given tensor amax:
+ *   rule      OR_RULE_DEFAULT (MXFP4 truncation-free E8M0, NVFP4 E4M3 nearest),
+ *             OR_RULE_OCP_FLOOR (MXFP4: k = floor(log2 amax) - 2, may clip),
+ *             OR_RULE_E4M3_UP (NVFP4: block scale byte rounded up, no clipping);
+ *   four6     NVFP4 16-blocks, or MXFP4 32-groups (candidate 4 * 2^k4 >= amax);
+ *   block2d   16x16 NVFP4 or 32x32 MXFP4 tiles;
+ *   row0      logical index of x's first row (random words keyed on
+ *             (row0 + i) * K + j), so row slices can be quantized apart (1D);
+ *   amax_in   NVFP4: NULL = the tensor's own amax; else s_t = *amax_in / 2688;
+ *   amax_out  NVFP4: NULL, or receives the tensor's own (rotated) amax. */
+int or_quantize_ex(const void *x, int xdt, int64_t M, int64_t K,
+                   int fmt, int rounding, int rotate, int block2d, int four6, int rule,
+                   uint64_t seed, int64_t row0, const float *amax_in,
+                   uint8_t *codes, uint8_t *scales,
+                   uint8_t *codesT, uint8_t *scalesT,
+                   float *tscale, float *amax_out);
+
+/* max |x| over the tensor after the optional rotation (NVFP4's amax_t) */
+float or_tensor_amax(const void *x, int xdt, int64_t M, int64_t K, int rotate);
+
 /* four-over-six decision for one 16-block (returns 1 if the amax/4 candidate
  * is chosen); exposed for brute-force pins. */
 int or_four6_pick(const float *x16, float s_t, uint8_t *enc_out, uint8_t codes_out[16]);
+
+/* one MXFP4 group of 32 values x (logical indices e): scale byte and codes
+ * under `rule`, with the four-over-six choice when four6 (returns 1 when the
+ * 4 * 2^k4 candidate is kept); exposed for brute-force pins. */
+int or_mxfp4_group(const float *x, const uint64_t *e, int rounding, int four6, int rule,
+                   uint64_t seed, uint8_t *sbyte, uint8_t codes[32]);
 
 /* ---- MXFP8 E4M3 quantize ------------------------------------------------ */
 int or_quantize_mxfp8(const void *x, int xdt, int64_t M, int64_t K,

@@ -261,6 +261,44 @@ def test_worked_outlier_example_per_tensor_row_group():
     assert len(diff) and all(i == 17 and j // 32 == 300 // 32 for i, j in diff)
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_fp32_scale_is_amax_over_six_and_never_clips(dtype):
+    """[LB] "FP4" section: S = |W|max / 6, so the largest magnitude lands on
+    the top grid value 6 and nothing is clipped.  Pinned independently of the
+    oracle's arithmetic: numpy's maximum of |x| over the tensor, each row and
+    each group, divided by 6 in binary32, must equal the oracle's scale for
+    every granularity (a divisor of 4 or 8 fails here), the element holding
+    the maximum must decode to +-6, and every code must be the grid value
+    nearest to fl(x / S) (brute force over the 8 magnitudes)."""
+    rng = np.random.default_rng(77)
+    M, K = 24, 96
+    x = (rng.standard_normal((M, K)) * np.exp(rng.uniform(-3, 3, (M, 1)))).astype(np.float32)
+    x[3, 5] = 0.0
+    x[7] = 0.0                                            # an all-zero row: S = 0, +0 codes
+    if dtype == "bf16":
+        x = synth.f32_to_bf16_bits(x)
+    xf = _f32(x).astype(np.float32)
+    ax = np.abs(xf)
+    grans = {oracle.GRAN_TENSOR: ax.max().reshape(1), oracle.GRAN_ROW: ax.max(axis=1),
+             oracle.GRAN_GROUP16: ax.reshape(M, K // 16, 16).max(axis=2).ravel(),
+             oracle.GRAN_GROUP32: ax.reshape(M, K // 32, 32).max(axis=2).ravel()}
+    width = {oracle.GRAN_TENSOR: M * K, oracle.GRAN_ROW: K, oracle.GRAN_GROUP16: 16, oracle.GRAN_GROUP32: 32}
+    for gran, amax in grans.items():
+        q = oracle.quantize_fp32scale(x, gran)
+        want = (amax.astype(np.float32) / np.float32(6.0)).astype(np.float32)
+        assert np.array_equal(q["scales"].view(np.uint32), want.view(np.uint32)), gran
+        S = np.repeat(want.astype(np.float64), width[gran]).reshape(M, K)
+        nib = _nib(q["codes"], M, K)
+        S32 = S.astype(np.float32)                            # v = fl(x / S) in binary32 (reading c4)
+        v = np.divide(xf, S32, out=np.zeros_like(xf), where=S32 > 0).astype(np.float64)
+        dist = np.abs(np.abs(v)[..., None] - GRID)
+        ok = dist[np.arange(M)[:, None], np.arange(K)[None, :], nib & 7] <= dist.min(axis=-1) + 1e-12
+        assert ok.all(), gran
+        top = (ax == np.repeat(amax, width[gran]).reshape(M, K)) & (ax > 0)
+        assert ((nib[top] & 7) == 7).all(), gran          # the maximum decodes to +-6
+        assert not (nib[S == 0] & 7).any()
+
+
 def test_power_of_two_scale_costs_a_little_mse():
     """[LB] §3 table: a 2^k group scale costs 1.0-1.4x the MSE of an FP group scale."""
     tb = _tables()["scale_cost"]
@@ -391,11 +429,28 @@ def test_argument_validation():
     x = np.zeros((32, 128), np.float32)
     st = oracle.quantize_status
     assert st(x, oracle.MXFP4) == oracle.OK
-    assert st(x, oracle.MXFP4, four6=True) == oracle.ERR_UNSUPPORTED
+    assert st(x, oracle.MXFP4, four6=True) == oracle.OK              # MXFP4 four-over-six (32-groups)
     assert st(x, oracle.NVFP4, four6=True, rounding=oracle.SR) == oracle.ERR_UNSUPPORTED
-    assert st(x, oracle.MXFP4, block2d=True) == oracle.ERR_UNSUPPORTED
+    assert st(x, oracle.MXFP4, block2d=True) == oracle.OK            # 32 x 32 MXFP4 tiles
+    assert st(np.zeros((48, 128), np.float32), oracle.MXFP4, block2d=True) == oracle.ERR_SHAPE
+    assert st(x, oracle.MXFP4, block2d=True, four6=True) == oracle.ERR_UNSUPPORTED
     assert st(x, oracle.NVFP4, block2d=True, rotate=True) == oracle.ERR_UNSUPPORTED
     assert st(x, oracle.NVFP4, rotate=True, transposed=True) == oracle.ERR_UNSUPPORTED
     assert st(np.zeros((32, 48), np.float32), oracle.MXFP4) == oracle.ERR_SHAPE
     assert st(np.zeros((32, 96), np.float32), oracle.NVFP4, rotate=True) == oracle.ERR_SHAPE
     assert st(np.zeros((24, 64), np.float32), oracle.NVFP4, block2d=True) == oracle.ERR_SHAPE
+
+
+def test_argument_validation_of_the_extended_call():
+    x = np.zeros((32, 128), np.float32)
+    st = oracle.quantize_ex_status
+    assert st(x, oracle.MXFP4, rule=oracle.RULE_OCP_FLOOR) == oracle.OK
+    assert st(x, oracle.NVFP4, rule=oracle.RULE_E4M3_UP) == oracle.OK
+    assert st(x, oracle.NVFP4, rule=oracle.RULE_OCP_FLOOR) == oracle.ERR_UNSUPPORTED   # E8M0 rule only
+    assert st(x, oracle.MXFP4, rule=oracle.RULE_E4M3_UP) == oracle.ERR_UNSUPPORTED     # E4M3 rule only
+    assert st(x, oracle.MXFP4, rule=5) == oracle.ERR_ARG
+    assert st(x, oracle.MXFP4, amax_in=1.0) == oracle.ERR_UNSUPPORTED                  # tensor amax: NVFP4
+    assert st(x, oracle.NVFP4, amax_in=1.0) == oracle.OK
+    assert st(x, oracle.NVFP4, row0=3) == oracle.OK
+    assert st(x, oracle.NVFP4, row0=3, block2d=True) == oracle.ERR_UNSUPPORTED
+    assert st(x, oracle.NVFP4, row0=-1) == oracle.ERR_ARG
