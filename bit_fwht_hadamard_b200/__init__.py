@@ -23,13 +23,14 @@ MXFP4, NVFP4 = 0, 1
 RNE, SR = 0, 1
 BF16, F32 = 0, 1
 GRAN_TENSOR, GRAN_ROW, GRAN_GROUP16, GRAN_GROUP32 = 0, 1, 2, 3
+SCALE_DEFAULT, SCALE_OCP_FLOOR, SCALE_E4M3_UP = 0, 1, 2
 OK, ERR_ARG, ERR_SHAPE, ERR_UNSUPPORTED, ERR_ALIGN, ERR_CUDA, ERR_TIMEOUT = 0, -1, -2, -3, -4, -5, -6
 DEV_ERR_TIMEOUT = 1
 
 EXPORTS = [
-    "qfp4_quantize_workspace_bytes", "qfp4_quantize", "qfp4_quantize_mxfp8", "qfp4_quantize_fp32scale",
+    "qfp4_quantize_workspace_bytes", "qfp4_quantize", "qfp4_quantize_ex", "qfp4_quantize_mxfp8", "qfp4_quantize_fp32scale",
     "qfp4_dequantize", "qfp4_gemm_workspace_bytes", "qfp4_gemm_blockscaled", "qfp4_gemm_fused_rq_workspace_bytes",
-    "qfp4_gemm_fused_rq", "qfp4_gemm_blockscaled_noalloc",
+    "qfp4_gemm_fused_rq", "qfp4_gemm_fused_rq_workspace_layout", "qfp4_gemm_blockscaled_noalloc",
     "qfp4_status_string", "qfp4_last_device_error", "qfp4_selftest_wait_timeout", "qfp4_version",
     "qfp4_launch_count",
 ]
@@ -57,6 +58,9 @@ def lib():
         L.qfp4_quantize.restype = c_int
         L.qfp4_quantize.argtypes = [P, c_int, c_int64, c_int64, c_int, c_int, c_int, c_int, c_int, c_uint64,
                                     P, P, P, P, P, P, c_size_t, P]
+        L.qfp4_quantize_ex.restype = c_int
+        L.qfp4_quantize_ex.argtypes = [P, c_int, c_int64, c_int64, c_int, c_int, c_int, c_int, c_int, c_int,
+                                       c_uint64, P, P, P, P, P, P, P, P, c_size_t, P]
         L.qfp4_quantize_mxfp8.restype = c_int
         L.qfp4_quantize_mxfp8.argtypes = [P, c_int, c_int64, c_int64, c_int, c_uint64, P, P, P, P, P]
         L.qfp4_quantize_fp32scale.restype = c_int
@@ -75,6 +79,8 @@ def lib():
         L.qfp4_gemm_fused_rq.restype = c_int
         L.qfp4_gemm_fused_rq.argtypes = [P, c_int64, c_int64, c_int, c_int, c_int, P, P, P, c_int64, P, c_size_t,
                                          c_int, P, P]
+        L.qfp4_gemm_fused_rq_workspace_layout.restype = c_int
+        L.qfp4_gemm_fused_rq_workspace_layout.argtypes = [c_int64, c_int64, c_int64, c_int, P, P, P]
         L.qfp4_status_string.restype = c_char_p
         L.qfp4_status_string.argtypes = [c_int]
         L.qfp4_last_device_error.restype = c_int
@@ -102,6 +108,13 @@ def qfp4_quantize(x, xdt, M, K, fmt, rounding, rotate, block2d, four6, seed, cod
                   tscale, workspace, workspace_bytes, stream):
     return lib().qfp4_quantize(x, xdt, M, K, fmt, rounding, rotate, block2d, four6, seed & ((1 << 64) - 1), codes,
                                scales, codesT, scalesT, tscale, workspace, workspace_bytes, stream)
+
+
+def qfp4_quantize_ex(x, xdt, M, K, fmt, rounding, rotate, block2d, four6, rule, seed, amax_in, amax_out, codes,
+                     scales, codesT, scalesT, tscale, workspace, workspace_bytes, stream):
+    return lib().qfp4_quantize_ex(x, xdt, M, K, fmt, rounding, rotate, block2d, four6, rule, seed & ((1 << 64) - 1),
+                                  amax_in, amax_out, codes, scales, codesT, scalesT, tscale, workspace,
+                                  workspace_bytes, stream)
 
 
 def qfp4_quantize_mxfp8(x, xdt, M, K, rounding, seed, codes, scales, codesT, scalesT, stream):
@@ -143,6 +156,15 @@ def qfp4_gemm_fused_rq(A_bf16, M, K, rotate, four6, fmt, B_codes, B_scales, B_ts
                        workspace_bytes, out_dt, out, stream):
     return lib().qfp4_gemm_fused_rq(A_bf16, M, K, rotate, four6, fmt, B_codes, B_scales, B_tscale, N, workspace,
                                     workspace_bytes, out_dt, out, stream)
+
+
+def qfp4_gemm_fused_rq_workspace_layout(M, N, K, fmt):
+    """(codes, scales, tscale) byte offsets of A's quantized operand in the
+    fused call's workspace."""
+    offs = [ctypes.c_size_t() for _ in range(3)]
+    st = lib().qfp4_gemm_fused_rq_workspace_layout(M, N, K, fmt, *[ctypes.byref(o) for o in offs])
+    _check(st, "qfp4_gemm_fused_rq_workspace_layout")
+    return tuple(o.value for o in offs)
 
 
 def qfp4_status_string(status):
@@ -196,10 +218,12 @@ def _check(st, where):
 
 
 def quantize(x, fmt=MXFP4, rounding=RNE, rotate=False, block2d=False, four6=False, seed=0, transposed=False,
-             stream=None, out=None, workspace=None):
+             stream=None, out=None, workspace=None, rule=SCALE_DEFAULT, amax_in=None, amax_out=None):
     """Quantize a contiguous (M, K) bf16/fp32 CUDA tensor; returns a dict of
     uint8 codes (M, K/2), scales (M, K/g), optional codesT/scalesT, and the
-    float32 tscale (NVFP4).  ``out`` may supply preallocated buffers."""
+    float32 tscale (NVFP4).  ``out`` may supply preallocated buffers.
+    ``rule``, ``amax_in`` / ``amax_out`` (one-element float32 CUDA tensors)
+    are qfp4_quantize_ex's scale rule and tensor-amax options."""
     torch = _torch()
     assert x.is_cuda and x.is_contiguous() and x.dim() == 2
     M, K = x.shape
@@ -217,10 +241,10 @@ def quantize(x, fmt=MXFP4, rounding=RNE, rotate=False, block2d=False, four6=Fals
     wsb = qfp4_quantize_workspace_bytes(M, K, fmt, rotate, block2d)
     if workspace is None and wsb:
         workspace = torch.empty(wsb, dtype=torch.uint8, device=dev)
-    st = qfp4_quantize(_ptr(x), _xdt(x), M, K, fmt, rounding, int(rotate), int(block2d), int(four6), seed,
-                       _ptr(o["codes"]), _ptr(o["scales"]), _ptr(o.get("codesT")), _ptr(o.get("scalesT")),
-                       _ptr(o.get("tscale")), _ptr(workspace), wsb, _stream(stream))
-    _check(st, "qfp4_quantize")
+    st = qfp4_quantize_ex(_ptr(x), _xdt(x), M, K, fmt, rounding, int(rotate), int(block2d), int(four6), rule, seed,
+                          _ptr(amax_in), _ptr(amax_out), _ptr(o["codes"]), _ptr(o["scales"]), _ptr(o.get("codesT")),
+                          _ptr(o.get("scalesT")), _ptr(o.get("tscale")), _ptr(workspace), wsb, _stream(stream))
+    _check(st, "qfp4_quantize_ex")
     return o
 
 

@@ -10,10 +10,11 @@ int quantize_fp32scale(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4
                        float *scales, float *partials, cudaStream_t stream);
 int quantize_columns(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_fmt fmt, qfp4_round rounding,
                      int four6, uint64_t seed, uint8_t *codesT, uint8_t *scalesT, const float *partials,
-                     int n_partials, cudaStream_t stream);
-int quantize2d(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_round rounding, uint64_t seed,
-               uint8_t *codes, uint8_t *scales, uint8_t *codesT, uint8_t *scalesT, float *tscale, float *partials,
-               cudaStream_t stream);
+                     int n_partials, cudaStream_t stream, const QuantOpts &opt);
+int quantize2d(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_fmt fmt, qfp4_round rounding,
+               uint64_t seed, uint8_t *codes, uint8_t *scales, uint8_t *codesT, uint8_t *scalesT, float *tscale,
+               float *partials, cudaStream_t stream, const QuantOpts &opt);
+int tscale_from_amax(const float *amax_in, float *tscale, cudaStream_t stream);
 int quantize_mxfp8(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_round rounding, uint64_t seed,
                    uint8_t *codes, uint8_t *scales, uint8_t *codesT, uint8_t *scalesT, cudaStream_t stream);
 int gemm_blockscaled(const uint8_t *A_codes, const uint8_t *A_scales, const float *A_tscale, const uint8_t *B_codes,
@@ -24,6 +25,8 @@ int gemm_fused_rq(const void *A_bf16, int64_t M, int64_t K, int rotate, int four
                   const uint8_t *B_codes, const uint8_t *B_scales, const float *B_tscale, int64_t N, void *workspace,
                   qfp4_dtype out_dt, void *out, cudaStream_t stream);
 size_t gemm_fused_rq_workspace(int64_t M, int64_t N, int64_t K, qfp4_fmt fmt);
+void gemm_fused_rq_layout(int64_t M, int64_t N, int64_t K, qfp4_fmt fmt, size_t *codes, size_t *scales,
+                          size_t *tscale);
 }  // namespace qfp4
 
 using namespace qfp4;
@@ -36,48 +39,76 @@ extern "C" size_t qfp4_quantize_workspace_bytes(int64_t M, int64_t K, qfp4_fmt f
     return fmt == QFP4_NVFP4 ? sizeof(float) * kMaxPartials : 0;
 }
 
-extern "C" int qfp4_quantize(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_fmt fmt, qfp4_round rounding,
-                             int rotate, int block2d, int four6, uint64_t seed, uint8_t *codes, uint8_t *scales,
-                             uint8_t *codesT, uint8_t *scalesT, float *tscale, void *workspace,
-                             size_t workspace_bytes, qfp4_stream_t stream_)
+extern "C" int qfp4_quantize_ex(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_fmt fmt,
+                                qfp4_round rounding, int rotate, int block2d, int four6, qfp4_scale_rule rule,
+                                uint64_t seed, const float *amax_in, float *amax_out, uint8_t *codes,
+                                uint8_t *scales, uint8_t *codesT, uint8_t *scalesT, float *tscale, void *workspace,
+                                size_t workspace_bytes, qfp4_stream_t stream_)
 {
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     if (M < 0 || K < 0) return QFP4_ERR_SHAPE;
     if (fmt != QFP4_MXFP4 && fmt != QFP4_NVFP4) return QFP4_ERR_ARG;
     if (rounding != QFP4_RNE && rounding != QFP4_SR) return QFP4_ERR_ARG;
     if (xdt != QFP4_BF16 && xdt != QFP4_F32) return QFP4_ERR_ARG;
+    if (rule != QFP4_SCALE_DEFAULT && rule != QFP4_SCALE_OCP_FLOOR && rule != QFP4_SCALE_E4M3_UP) return QFP4_ERR_ARG;
     const int64_t n = M * K;
     if (n > 0 && (!x || !codes || !scales)) return QFP4_ERR_ARG;
     if ((codesT == nullptr) != (scalesT == nullptr)) return QFP4_ERR_ARG;
     if (fmt == QFP4_NVFP4 && !tscale) return QFP4_ERR_ARG;
     const int g = fmt == QFP4_MXFP4 ? 32 : 16;
-    if (four6 && (fmt != QFP4_NVFP4 || block2d || rounding != QFP4_RNE)) return QFP4_ERR_UNSUPPORTED;
-    if (block2d && (fmt != QFP4_NVFP4 || rotate)) return QFP4_ERR_UNSUPPORTED;
+    if (rule == QFP4_SCALE_OCP_FLOOR && fmt != QFP4_MXFP4) return QFP4_ERR_UNSUPPORTED;
+    if (rule == QFP4_SCALE_E4M3_UP && fmt != QFP4_NVFP4) return QFP4_ERR_UNSUPPORTED;
+    if ((amax_in || amax_out) && fmt != QFP4_NVFP4) return QFP4_ERR_UNSUPPORTED;
+    if (four6 && (block2d || rounding != QFP4_RNE)) return QFP4_ERR_UNSUPPORTED;
+    if (four6 && fmt == QFP4_MXFP4 && codesT) return QFP4_ERR_UNSUPPORTED;
+    if (block2d && rotate) return QFP4_ERR_UNSUPPORTED;
     if (!block2d && rotate && codesT) return QFP4_ERR_UNSUPPORTED;
     if (K % g) return QFP4_ERR_SHAPE;
     if (rotate && K % 128) return QFP4_ERR_SHAPE;
-    if (block2d && (M % 16 || K % 16)) return QFP4_ERR_SHAPE;
+    if (block2d && (M % g || K % g)) return QFP4_ERR_SHAPE;
     if (!block2d && codesT && M % g) return QFP4_ERR_SHAPE;
     if (!ok_align(x) || !ok_align(codes) || !ok_align(scales) || !ok_align(codesT) || !ok_align(scalesT))
         return QFP4_ERR_ALIGN;
-    if (fmt == QFP4_NVFP4 && (!workspace || workspace_bytes < sizeof(float) * kMaxPartials)) return QFP4_ERR_ARG;
-    if (fmt == QFP4_NVFP4 && !ok_align(workspace)) return QFP4_ERR_ALIGN;
+    const bool needs_ws = fmt == QFP4_NVFP4 && (!amax_in || amax_out);
+    if (needs_ws && (!workspace || workspace_bytes < sizeof(float) * kMaxPartials)) return QFP4_ERR_ARG;
+    if (needs_ws && !ok_align(workspace)) return QFP4_ERR_ALIGN;
     float *partials = static_cast<float *>(workspace);
+    QuantOpts opt;
+    opt.rule = rule;
+    opt.amax_in = amax_in;
+    opt.amax_out = amax_out;
 
     if (n == 0) {
-        if (fmt == QFP4_NVFP4 && cudaMemsetAsync(tscale, 0, sizeof(float), stream) != cudaSuccess)
-            return QFP4_ERR_CUDA;
+        if (fmt == QFP4_NVFP4) {
+            if (amax_in) {
+                const int st = tscale_from_amax(amax_in, tscale, stream);   // s_t = fl(amax / 2688)
+                if (st != QFP4_OK) return st;
+            } else if (cudaMemsetAsync(tscale, 0, sizeof(float), stream) != cudaSuccess) {
+                return QFP4_ERR_CUDA;
+            }
+            if (amax_out && cudaMemsetAsync(amax_out, 0, sizeof(float), stream) != cudaSuccess) return QFP4_ERR_CUDA;
+        }
         return QFP4_OK;
     }
     if (block2d)
-        return quantize2d(x, xdt, M, K, rounding, seed, codes, scales, codesT, scalesT, tscale, partials, stream);
+        return quantize2d(x, xdt, M, K, fmt, rounding, seed, codes, scales, codesT, scalesT, tscale, partials, stream,
+                          opt);
     int n_parts = 0;
     int st = quantize1d(x, xdt, n, fmt, rounding, rotate, four6, seed, codes, scales, tscale, partials, &n_parts,
-                        stream);
+                        stream, opt);
     if (st != QFP4_OK || !codesT) return st;
     // The NVFP4 amax pass above left its partial maxima in the workspace:
     // the column-wise quantization reuses them for the same s_t.
-    return quantize_columns(x, xdt, M, K, fmt, rounding, four6, seed, codesT, scalesT, partials, n_parts, stream);
+    return quantize_columns(x, xdt, M, K, fmt, rounding, four6, seed, codesT, scalesT, partials, n_parts, stream, opt);
+}
+
+extern "C" int qfp4_quantize(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_fmt fmt, qfp4_round rounding,
+                             int rotate, int block2d, int four6, uint64_t seed, uint8_t *codes, uint8_t *scales,
+                             uint8_t *codesT, uint8_t *scalesT, float *tscale, void *workspace,
+                             size_t workspace_bytes, qfp4_stream_t stream)
+{
+    return qfp4_quantize_ex(x, xdt, M, K, fmt, rounding, rotate, block2d, four6, QFP4_SCALE_DEFAULT, seed, nullptr,
+                            nullptr, codes, scales, codesT, scalesT, tscale, workspace, workspace_bytes, stream);
 }
 
 extern "C" int qfp4_quantize_mxfp8(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_round rounding,
@@ -168,6 +199,16 @@ extern "C" int qfp4_gemm_blockscaled(const uint8_t *A_codes, const uint8_t *A_sc
 extern "C" size_t qfp4_gemm_fused_rq_workspace_bytes(int64_t M, int64_t N, int64_t K, qfp4_fmt fmt)
 {
     return gemm_fused_rq_workspace(M, N, K, fmt);
+}
+
+extern "C" int qfp4_gemm_fused_rq_workspace_layout(int64_t M, int64_t N, int64_t K, qfp4_fmt fmt, size_t *codes_off,
+                                                   size_t *scales_off, size_t *tscale_off)
+{
+    if (fmt != QFP4_MXFP4 && fmt != QFP4_NVFP4) return QFP4_ERR_ARG;
+    if (!codes_off || !scales_off || !tscale_off) return QFP4_ERR_ARG;
+    if (M < 0 || N < 0 || K < 0) return QFP4_ERR_SHAPE;
+    gemm_fused_rq_layout(M, N, K, fmt, codes_off, scales_off, tscale_off);
+    return QFP4_OK;
 }
 
 extern "C" int qfp4_gemm_fused_rq(const void *A_bf16, int64_t M, int64_t K, int rotate, int four6, qfp4_fmt fmt,

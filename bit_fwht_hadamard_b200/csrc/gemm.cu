@@ -1049,6 +1049,15 @@ static FusedLayout fused_layout(int64_t M, int64_t N, int64_t K, qfp4_fmt fmt)
     return L;
 }
 
+void gemm_fused_rq_layout(int64_t M, int64_t N, int64_t K, qfp4_fmt fmt, size_t *codes, size_t *scales,
+                          size_t *tscale)
+{
+    const FusedLayout F = fused_layout(M, N, K, fmt);
+    *codes = F.codes;
+    *scales = F.scales;
+    *tscale = F.tscale;
+}
+
 size_t gemm_fused_rq_workspace(int64_t M, int64_t N, int64_t K, qfp4_fmt fmt)
 {
     if (M <= 0 || N <= 0 || K <= 0) return 0;

@@ -436,6 +436,33 @@ __device__ __forceinline__ int scale_exp(float amax, uint32_t top_frac, int top_
     return max(-127, min(127, k));
 }
 
+// The OCP microscaling exponent: k = floor(log2(amax)) - emax (emax = 2 for
+// E2M1), the largest k with 2^(k + emax) <= amax, clamped to [-127, 127];
+// amax / 2^k lies in [2^emax, 2^(emax+1)), so magnitudes above the format's
+// largest value clip.  amax == 0 gives -127.
+__device__ __forceinline__ int scale_exp_floor(float amax, int emax)
+{
+    const uint32_t u = __float_as_uint(amax) & 0x7FFFFFFFu;
+    if (u == 0) return -127;
+    const uint32_t E = u >> 23;
+    const int e = E == 0 ? (31 - __clz(u)) - 149 : static_cast<int>(E) - 127;
+    return max(-127, min(127, e - emax));
+}
+
+// Scale rules (qfp4_scale_rule): the E8M0 exponent of an MXFP4 group.
+__device__ __forceinline__ int mx_scale_exp(float amax, int rule)
+{
+    return rule == QFP4_SCALE_OCP_FLOOR ? scale_exp_floor(amax, 2) : scale_exp(amax, 0x400000u, 2);
+}
+
+// E4M3 byte of t >= 0 rounded up: the least finite E4M3 value >= t,
+// saturating at 448.  Non-negative E4M3 bytes 0x00 .. 0x7E increase with
+// their value, so one step up from the nearest byte when it lies below t.
+__device__ __forceinline__ uint32_t e4m3_up_byte(float t, uint32_t nearest)
+{
+    return (nearest < 0x7Eu && e4m3_value(nearest) < t) ? nearest + 1u : nearest;
+}
+
 // 2^k as binary32 for k in [-127, 127] (2^-127 is the subnormal 0x00400000).
 __device__ __forceinline__ float exp2i(int k)
 {

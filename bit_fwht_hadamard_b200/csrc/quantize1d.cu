@@ -89,11 +89,14 @@ __device__ __forceinline__ uint64_t div_rn_by2(uint64_t a, uint64_t y2, uint64_t
     return q | (a & 0x8000000080000000ull);
 }
 
-// fl(x_i / S) for 16 values held as 8 packed pairs, S > 0.  Outside
-// [2^-125, 2^125] (1/S not normal) the IEEE division.
-__device__ __forceinline__ void nv_quot16_pairs(const uint64_t *pp, float S, uint64_t *q)
+// fl(x_i / S) for 16 values held as 8 packed pairs, S > 0, amax = max |x_i|.
+// Outside S in [2^-125, 2^125] (1/S not normal), and when a quotient could
+// overflow (a block scale saturated under a caller-supplied tensor amax far
+// below the block's values), the IEEE division, whose infinities saturate
+// like any magnitude beyond 6.
+__device__ __forceinline__ void nv_quot16_pairs(const uint64_t *pp, float S, float amax, uint64_t *q)
 {
-    if (S >= 0x1p-125f && S <= 0x1p125f) {
+    if (S >= 0x1p-125f && S <= 0x1p125f && amax <= S * 0x1p100f) {
         const float y = __frcp_rn(S);
         const uint64_t y2 = f2pack(y, y), nS2 = f2pack(-S, -S);
 #pragma unroll
@@ -109,10 +112,10 @@ __device__ __forceinline__ void nv_quot16_pairs(const uint64_t *pp, float S, uin
 }
 
 // E2M1 round-to-nearest-even codes of fl(x_i / S): two words of nibbles.
-__device__ __forceinline__ void nv_codes16_pairs(const uint64_t *pp, float S, uint32_t *w2)
+__device__ __forceinline__ void nv_codes16_pairs(const uint64_t *pp, float S, float amax, uint32_t *w2)
 {
     uint64_t q[8];
-    nv_quot16_pairs(pp, S, q);
+    nv_quot16_pairs(pp, S, amax, q);
     w2[0] = e2m1x8_rne_pairs(q[0], q[1], q[2], q[3]);
     w2[1] = e2m1x8_rne_pairs(q[4], q[5], q[6], q[7]);
 }
@@ -121,10 +124,10 @@ __device__ __forceinline__ void nv_codes16_pairs(const uint64_t *pp, float S, ui
 // (2 words), and when `sse` is given the binary32 squared error of the
 // dequantized values, sum(fl(fl(fl(g_i S) - x_i)^2)) as a fixed tree
 // (i + 8 into i, then i + 4, i + 2, i + 1).
-__device__ __forceinline__ void nv_block_rne_pairs(const uint64_t *pp, float S, uint32_t *w2, float *sse)
+__device__ __forceinline__ void nv_block_rne_pairs(const uint64_t *pp, float S, float amax, uint32_t *w2, float *sse)
 {
     if (S == 0.0f) w2[0] = w2[1] = 0u;
-    else nv_codes16_pairs(pp, S, w2);
+    else nv_codes16_pairs(pp, S, amax, w2);
     if (sse) {
         // Scalar IEEE operations: the multiply feeding the subtraction must
         // stay two roundings (the packed forms gave occasional one-ulp
@@ -151,41 +154,52 @@ __device__ __forceinline__ void nv_block_rne_pairs(const uint64_t *pp, float S, 
 }
 
 // The same for 16 unpacked values.
-__device__ __forceinline__ void nv_block_rne(const float *x, float S, uint32_t *w2, float *sse)
+__device__ __forceinline__ void nv_block_rne(const float *x, float S, float amax, uint32_t *w2, float *sse)
 {
     uint64_t pp[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) pp[j] = f2pack(x[2 * j], x[2 * j + 1]);
-    nv_block_rne_pairs(pp, S, w2, sse);
+    nv_block_rne_pairs(pp, S, amax, w2, sse);
 }
 
 // NVFP4 block scale bytes enc = E4M3_RNE(fl(fl(amax / d) / s_t)), d = 6 or 4,
 // with the quotients from div_rn_by: fl(amax / 6) by y = fl(1/6), fl(amax / 4)
 // is exact, and fl(t / s_t) by fl(1/s_t), worked out once per thread.  The
 // fast path needs amax / d and 1/s_t normal; otherwise IEEE divisions.
+// rule: QFP4_SCALE_DEFAULT (E4M3 nearest) or QFP4_SCALE_E4M3_UP (the least
+// E4M3 value not below the quotient, so no element of the block clips).
+// A quotient of 448 or more (also +inf, from a caller-supplied tensor amax
+// far below the block's values) takes the largest byte, 0x7E.
 struct NvScale {
     float s_t, y_t;
     bool fast;
+    int rule;
 };
 
-__device__ __forceinline__ NvScale nv_scale_setup(float s_t)
+__device__ __forceinline__ NvScale nv_scale_setup(float s_t, int rule = QFP4_SCALE_DEFAULT)
 {
     NvScale z;
     z.s_t = s_t;
     z.fast = s_t >= 0x1p-120f && s_t <= 0x1p120f;
     z.y_t = z.fast ? __frcp_rn(s_t) : 0.0f;
+    z.rule = rule;
     return z;
 }
 
 template <bool D6>
 __device__ __forceinline__ uint32_t nv_scale_byte(float amax, const NvScale &z)
 {
+    float r;
     if (z.fast && amax >= 0x1p-120f) {
         const float t = D6 ? div_rn_by(amax, __uint_as_float(0x3E2AAAABu), -6.0f)   // fl(1/6)
                            : __fmul_rn(amax, 0.25f);
-        return e4m3_rne(div_rn_by(t, z.y_t, -z.s_t));
+        r = div_rn_by(t, z.y_t, -z.s_t);
+    } else {
+        r = __fdiv_rn(__fdiv_rn(amax, D6 ? 6.0f : 4.0f), z.s_t);
     }
-    return e4m3_rne(__fdiv_rn(__fdiv_rn(amax, D6 ? 6.0f : 4.0f), z.s_t));
+    if (!(r < 448.0f)) return 0x7Eu;              // saturated; a NaN from an overflowed chain too
+    const uint32_t enc = e4m3_rne(r);
+    return z.rule == QFP4_SCALE_E4M3_UP ? e4m3_up_byte(r, enc) : enc;
 }
 
 // Stochastic rounding of 16 (NVFP4) or 32 (MXFP4) values v (already divided
@@ -210,6 +224,56 @@ __device__ __forceinline__ void sr_group(const float *v, uint64_t e, uint64_t se
     }
 }
 
+// binary32 squared error of 32 values x under codes w (4 words) and scale
+// 2^k: sum(fl(fl(fl(g_i 2^k) - x_i)^2)) as a fixed tree (i + 16 into i, then
+// + 8, + 4, + 2, + 1); g_i 2^k is exact.
+__device__ __forceinline__ float mx_sse32(const float *x, const uint32_t *w, int k)
+{
+    const float sc = exp2i(k);
+    float e[32];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        uint64_t g4[4];
+        e2m1x8_values(w[t], g4);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float g0, g1;
+            f2unpack(g4[j], g0, g1);
+            const float d0 = __fsub_rn(__fmul_rn(g0, sc), x[8 * t + 2 * j]);
+            const float d1 = __fsub_rn(__fmul_rn(g1, sc), x[8 * t + 2 * j + 1]);
+            e[8 * t + 2 * j] = __fmul_rn(d0, d0);
+            e[8 * t + 2 * j + 1] = __fmul_rn(d1, d1);
+        }
+    }
+#pragma unroll
+    for (int h = 16; h >= 1; h >>= 1)
+#pragma unroll
+        for (int i = 0; i < h; ++i) e[i] = __fadd_rn(e[i], e[i + h]);
+    return e[0];
+}
+
+// Four-over-six on an MXFP4 group of 32 (RNE): the second candidate is the
+// least k4 with 4 * 2^k4 >= amax; it replaces the rule's exponent k (codes w)
+// only when its squared error is strictly lower.  Returns the kept exponent.
+__device__ __forceinline__ int mx_four6(const float *x, float amax, int k, uint32_t *w)
+{
+    const int k4 = scale_exp(amax, 0u, 2);
+    if (k4 == k) return k;
+    const float m4 = exp2i(-k4);
+    uint32_t w4[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        float q8[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) q8[u] = __fmul_rn(x[8 * t + u], m4);
+        w4[t] = e2m1x8_rne(q8);
+    }
+    if (!(mx_sse32(x, w4, k4) < mx_sse32(x, w, k))) return k;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) w[t] = w4[t];
+    return k4;
+}
+
 template <int FMT, bool SR, bool FOUR6>
 __device__ __forceinline__ void quant_unit(const float (&v)[64], uint64_t e0, const NvScale &nz, uint64_t seed,
                                            UnitOut &o)
@@ -226,8 +290,7 @@ __device__ __forceinline__ void quant_unit(const float (&v)[64], uint64_t e0, co
                 w[0] = w[1] = w[2] = w[3] = 0u;
                 continue;
             }
-            const int k = scale_exp(amax, 0x400000u, 2);
-            o.scales |= static_cast<uint32_t>(k + 127) << (8 * g);
+            int k = mx_scale_exp(amax, nz.rule);
             const float mul = exp2i(-k);             // x * 2^-k == x / 2^k exactly
             float q[32];
 #pragma unroll
@@ -238,6 +301,8 @@ __device__ __forceinline__ void quant_unit(const float (&v)[64], uint64_t e0, co
 #pragma unroll
                 for (int t = 0; t < 4; ++t) w[t] = e2m1x8_rne(q + 8 * t);
             }
+            if (FOUR6) k = mx_four6(v + 32 * g, amax, k, w);
+            o.scales |= static_cast<uint32_t>(k + 127) << (8 * g);
         }
     } else {
 #pragma unroll
@@ -262,8 +327,8 @@ __device__ __forceinline__ void quant_unit(const float (&v)[64], uint64_t e0, co
                     enc4 = nv_scale_byte<false>(amax, nz);
                     S4 = __fmul_rn(e4m3_value(enc4), nz.s_t);
                 }
-                nv_block_rne(x, S, w6, &sse6);
-                nv_block_rne(x, S4, w4, &sse4);
+                nv_block_rne(x, S, amax, w6, &sse6);
+                nv_block_rne(x, S4, amax, w4, &sse4);
                 const bool pick4 = sse4 < sse6;
                 w[0] = pick4 ? w4[0] : w6[0];
                 w[1] = pick4 ? w4[1] : w6[1];
@@ -275,14 +340,14 @@ __device__ __forceinline__ void quant_unit(const float (&v)[64], uint64_t e0, co
                     uint64_t pp[8], qq[8];
 #pragma unroll
                     for (int j = 0; j < 8; ++j) pp[j] = f2pack(x[2 * j], x[2 * j + 1]);
-                    nv_quot16_pairs(pp, S, qq);
+                    nv_quot16_pairs(pp, S, amax, qq);
                     float q[16];
 #pragma unroll
                     for (int j = 0; j < 8; ++j) f2unpack(qq[j], q[2 * j], q[2 * j + 1]);
                     sr_group<16>(q, e0 + 16 * b, seed, w);
                 }
             } else {
-                nv_block_rne(x, S, w, nullptr);
+                nv_block_rne(x, S, amax, w, nullptr);
             }
             o.scales |= enc << (8 * b);
         }
@@ -316,8 +381,11 @@ __device__ __forceinline__ float tensor_scale_from(const float *partials, int n_
     return __fdiv_rn(m, 2688.0f);
 }
 
+// s_t of a quantize pass: from the caller's tensor amax when given (uniform
+// over the grid), else from the partial maxima of the amax pass.
 __device__ __forceinline__ float tensor_scale(const QuantParams &p, float *red)
 {
+    if (p.amax_in) return __fdiv_rn(*p.amax_in, 2688.0f);
     return tensor_scale_from(p.partials, p.n_partials, red);
 }
 
@@ -443,7 +511,7 @@ template <int UP, int FMT, bool SR, bool FOUR6, bool RAW = false>
 __device__ __forceinline__ void quant_unit_packed(uint64_t (&p)[UP], uint64_t e0, const NvScale &nz, uint64_t seed,
                                                   UnitP<UP> &o)
 {
-    static_assert(!RAW || (FMT == QFP4_MXFP4 && !SR), "raw values only on the MXFP4 round-to-nearest path");
+    static_assert(!RAW || (FMT == QFP4_MXFP4 && !SR && !FOUR6), "raw values only on the plain MXFP4 round-to-nearest path");
     o.scales[0] = o.scales[1] = 0u;
     if (FMT == QFP4_MXFP4) {
 #pragma unroll
@@ -455,8 +523,7 @@ __device__ __forceinline__ void quant_unit_packed(uint64_t (&p)[UP], uint64_t e0
                 w[0] = w[1] = w[2] = w[3] = 0u;
                 continue;
             }
-            const int k = scale_exp(amax, 0x400000u, 2);
-            o.scales[0] |= static_cast<uint32_t>(k + 127) << (8 * g);
+            int k = mx_scale_exp(amax, nz.rule);
             if (RAW && k > 120) {
                 const uint64_t c2 = f2pack(inv_sqrt128(), inv_sqrt128());
 #pragma unroll
@@ -464,6 +531,11 @@ __device__ __forceinline__ void quant_unit_packed(uint64_t (&p)[UP], uint64_t e0
             }
             const float mk = (RAW && k <= 120) ? __fmul_rn(inv_sqrt128(), exp2i(-k)) : exp2i(-k);
             const uint64_t m2 = f2pack(mk, mk);      // x * 2^-k == x / 2^k exactly
+            float xs[FOUR6 ? 32 : 1];                 // the group's values, for four-over-six
+            if (FOUR6) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) f2unpack(pg[j], xs[2 * j], xs[2 * j + 1]);
+            }
 #pragma unroll
             for (int j = 0; j < 16; ++j) pg[j] = f2mul(pg[j], m2);
             if (SR) {
@@ -475,6 +547,8 @@ __device__ __forceinline__ void quant_unit_packed(uint64_t (&p)[UP], uint64_t e0
 #pragma unroll
                 for (int t = 0; t < 4; ++t) w[t] = e2m1x8_rne_pairs(pg[4 * t], pg[4 * t + 1], pg[4 * t + 2], pg[4 * t + 3]);
             }
+            if (FOUR6) k = mx_four6(xs, amax, k, w);
+            o.scales[0] |= static_cast<uint32_t>(k + 127) << (8 * g);
         }
     } else {
 #pragma unroll
@@ -497,8 +571,8 @@ __device__ __forceinline__ void quant_unit_packed(uint64_t (&p)[UP], uint64_t e0
                     enc4 = nv_scale_byte<false>(amax, nz);
                     S4 = __fmul_rn(e4m3_value(enc4), nz.s_t);
                 }
-                nv_block_rne_pairs(p + 8 * b, S, w6, &sse6);
-                nv_block_rne_pairs(p + 8 * b, S4, w4, &sse4);
+                nv_block_rne_pairs(p + 8 * b, S, amax, w6, &sse6);
+                nv_block_rne_pairs(p + 8 * b, S4, amax, w4, &sse4);
                 const bool pick4 = sse4 < sse6;
                 w[0] = pick4 ? w4[0] : w6[0];
                 w[1] = pick4 ? w4[1] : w6[1];
@@ -508,14 +582,14 @@ __device__ __forceinline__ void quant_unit_packed(uint64_t (&p)[UP], uint64_t e0
                     w[0] = w[1] = 0u;
                 } else {
                     uint64_t qq[8];
-                    nv_quot16_pairs(p + 8 * b, S, qq);
+                    nv_quot16_pairs(p + 8 * b, S, amax, qq);
                     float q[16];
 #pragma unroll
                     for (int j = 0; j < 8; ++j) f2unpack(qq[j], q[2 * j], q[2 * j + 1]);
                     sr_group<16>(q, e0 + 16 * b, seed, w);
                 }
             } else {
-                nv_block_rne_pairs(p + 8 * b, S, w, nullptr);
+                nv_block_rne_pairs(p + 8 * b, S, amax, w, nullptr);
             }
             o.scales[b >> 2] |= enc << (8 * (b & 3));
         }
@@ -636,7 +710,10 @@ __global__ void __launch_bounds__(32 * WARPS, 1) k_quant1d_tma(const __grid_cons
         s_t = tensor_scale(p, red);
         if (p.write_tscale && blockIdx.x == 0 && threadIdx.x == 0) *p.tscale_out = s_t;
     }
-    const NvScale nz = nv_scale_setup(s_t);
+    const NvScale nz = nv_scale_setup(s_t, p.rule);
+    // a quantize pass under a caller-supplied amax can still report this
+    // tensor's own amax: partial maxima of the (rotated) values it reads
+    const bool own_max = MODE == MODE_AMAX || p.partials_out != nullptr;
 
     auto issue = [&](int64_t t, int s) {
         mbar_arrive_expect_tx(&bars[s], STAGE_BYTES);
@@ -688,11 +765,11 @@ __global__ void __launch_bounds__(32 * WARPS, 1) k_quant1d_tma(const __grid_cons
 
         const int64_t row0 = t * TILE_ROWS + ROWS_PER_LANE * lane;   // first 64-element row of the unit
         const int64_t n_valid = imin<int64_t>(2 * UP, (rows - row0) * 64);
-        constexpr bool RAW = ROT && MODE == MODE_QUANT && FMT == QFP4_MXFP4 && !SR;
+        constexpr bool RAW = ROT && MODE == MODE_QUANT && FMT == QFP4_MXFP4 && !SR && !FOUR6;
         if (ROT) fwht_packed<UP, !RAW>(v, (lane & 1) != 0);
-        if (MODE == MODE_AMAX) {
+        if (MODE == MODE_AMAX || (FMT == QFP4_NVFP4 && own_max))
             tmax = fmaxf(tmax, absmax_pairs<UP>(v));   // rows past the end were zero-filled by TMA
-        } else if (n_valid > 0) {
+        if (MODE == MODE_QUANT && n_valid > 0) {
             const uint64_t e0 = p.e_base + static_cast<uint64_t>(row0) * 64u;
             if constexpr (FMT == FMT_MXFP8) {
                 uint32_t cw[UP / 2], sc;
@@ -706,7 +783,7 @@ __global__ void __launch_bounds__(32 * WARPS, 1) k_quant1d_tma(const __grid_cons
         }
     }
     if (gave_up && lane == 0) settle_ns(kSettleNs);   // loads of this warp's ring may still be landing
-    if (MODE == MODE_AMAX) {
+    if (MODE == MODE_AMAX || (FMT == QFP4_NVFP4 && own_max)) {
         tmax = block_max(tmax, red);
         if (threadIdx.x == 0) p.partials_out[blockIdx.x] = tmax;
     }
@@ -735,7 +812,8 @@ __global__ void __launch_bounds__(128) k_quant1d_direct(const T *__restrict__ x,
         s_t = tensor_scale(p, red);
         if (p.write_tscale && blockIdx.x == 0 && threadIdx.x == 0) *p.tscale_out = s_t;
     }
-    const NvScale nz = nv_scale_setup(s_t);
+    const NvScale nz = nv_scale_setup(s_t, p.rule);
+    const bool own_max = MODE == MODE_AMAX || p.partials_out != nullptr;
     const int64_t units = (p.n + 63) / 64;
     float tmax = 0.0f;
     for (int64_t u0 = static_cast<int64_t>(blockIdx.x) * blockDim.x; u0 < units;
@@ -776,17 +854,18 @@ __global__ void __launch_bounds__(128) k_quant1d_direct(const T *__restrict__ x,
             }
         }
         if (ROT) fwht128_pair(v, (threadIdx.x & 1) != 0);   // n % 128 == 0: pairs are whole
-        if (MODE == MODE_AMAX) {
+        if (MODE == MODE_AMAX || (FMT == QFP4_NVFP4 && own_max)) {
 #pragma unroll
             for (int i = 0; i < 64; ++i) tmax = fmaxf(tmax, fabsf(v[i]));
-        } else if (n_valid > 0) {
+        }
+        if (MODE == MODE_QUANT && n_valid > 0) {
             const uint64_t e0 = p.e_base + static_cast<uint64_t>(off);
             UnitOut o;
             quant_unit<FMT, SR, FOUR6>(v, e0, nz, p.seed, o);
             store_unit<G>(o, p, e0, n_valid);
         }
     }
-    if (MODE == MODE_AMAX) {
+    if (MODE == MODE_AMAX || (FMT == QFP4_NVFP4 && own_max)) {
         tmax = block_max(tmax, red);
         if (threadIdx.x == 0) p.partials_out[blockIdx.x] = tmax;
     }
@@ -903,9 +982,52 @@ int amax_partials(const void *x, qfp4_dtype xdt, int64_t n, float *partials, int
     return run_pass<MODE_AMAX, QFP4_NVFP4, false, false, false>(x, xdt, n, p, stream, n_parts);
 }
 
+// amax_out = max of n partial maxima (one block)
+__global__ void __launch_bounds__(256) k_partials_max(const float *partials, int n, float *amax_out)
+{
+    __shared__ float red[32];
+    pdl_wait();
+    pdl_trigger();
+    float m = 0.0f;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) m = fmaxf(m, partials[i]);
+    m = block_max(m, red);
+    if (threadIdx.x == 0) *amax_out = m;
+}
+
+int partials_max(const float *partials, int n, float *amax_out, cudaStream_t stream)
+{
+    if (launch_pdl(k_partials_max, dim3(1), dim3(256), 0, stream, partials, n, amax_out) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return QFP4_ERR_CUDA;
+    }
+    QFP4_LAUNCH_CHECK();
+    return QFP4_OK;
+}
+
+__global__ void k_tscale_from_amax(const float *amax_in, float *tscale)
+{
+    pdl_wait();
+    pdl_trigger();
+    if (threadIdx.x == 0) *tscale = __fdiv_rn(*amax_in, 2688.0f);
+}
+
+int tscale_from_amax(const float *amax_in, float *tscale, cudaStream_t stream)
+{
+    if (launch_pdl(k_tscale_from_amax, dim3(1), dim3(32), 0, stream, amax_in, tscale) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return QFP4_ERR_CUDA;
+    }
+    QFP4_LAUNCH_CHECK();
+    return QFP4_OK;
+}
+
+// NVFP4: with no caller amax, an amax pass (partial maxima into `partials`)
+// then the quantize pass; with a caller amax, the quantize pass alone, which
+// also writes its own partial maxima when the tensor's amax is asked for.
 template <int FMT, bool ROT, bool SR, bool FOUR6>
 static int quantize1d_t(const void *x, qfp4_dtype xdt, int64_t n, uint64_t seed, uint8_t *codes, uint8_t *scales,
-                        float *tscale, float *partials, int *n_parts_out, cudaStream_t stream)
+                        float *tscale, float *partials, int *n_parts_out, const QuantOpts &opt,
+                        cudaStream_t stream)
 {
     QuantParams p{};
     p.n = n;
@@ -915,8 +1037,9 @@ static int quantize1d_t(const void *x, qfp4_dtype xdt, int64_t n, uint64_t seed,
     p.seed = seed;
     p.tscale_out = tscale;
     p.write_tscale = true;
+    p.rule = opt.rule;
     int n_parts = 0;
-    if (FMT == QFP4_NVFP4) {
+    if (FMT == QFP4_NVFP4 && !opt.amax_in) {
         p.partials_out = partials;
         int st = run_pass<MODE_AMAX, FMT, ROT, false, false>(x, xdt, n, p, stream, &n_parts);
         if (st != QFP4_OK) return st;
@@ -924,29 +1047,35 @@ static int quantize1d_t(const void *x, qfp4_dtype xdt, int64_t n, uint64_t seed,
         p.partials = partials;
         p.n_partials = n_parts;
     }
+    if (FMT == QFP4_NVFP4 && opt.amax_in) {
+        p.amax_in = opt.amax_in;
+        p.partials_out = opt.amax_out ? partials : nullptr;
+    }
+    int quant_parts = 0;
+    int st = run_pass<MODE_QUANT, FMT, ROT, SR, FOUR6>(x, xdt, n, p, stream, &quant_parts);
+    if (st != QFP4_OK) return st;
+    if (opt.amax_in && opt.amax_out) n_parts = quant_parts;
     if (n_parts_out) *n_parts_out = n_parts;
-    return run_pass<MODE_QUANT, FMT, ROT, SR, FOUR6>(x, xdt, n, p, stream, nullptr);
+    if (FMT == QFP4_NVFP4 && opt.amax_out) return partials_max(partials, n_parts, opt.amax_out, stream);
+    return QFP4_OK;
 }
 
 int quantize1d(const void *x, qfp4_dtype xdt, int64_t n, qfp4_fmt fmt, qfp4_round rounding, int rotate, int four6,
                uint64_t seed, uint8_t *codes, uint8_t *scales, float *tscale, float *partials, int *n_parts_out,
-               cudaStream_t stream)
+               cudaStream_t stream, const QuantOpts &opt)
 {
     const bool sr = rounding == QFP4_SR;
+#define QFP4_Q1(F, R, S, F6) \
+    quantize1d_t<F, R, S, F6>(x, xdt, n, seed, codes, scales, tscale, partials, n_parts_out, opt, stream)
     if (fmt == QFP4_MXFP4) {
-        if (rotate) return sr ? quantize1d_t<QFP4_MXFP4, true, true, false>(x, xdt, n, seed, codes, scales, tscale, partials, n_parts_out, stream)
-                              : quantize1d_t<QFP4_MXFP4, true, false, false>(x, xdt, n, seed, codes, scales, tscale, partials, n_parts_out, stream);
-        return sr ? quantize1d_t<QFP4_MXFP4, false, true, false>(x, xdt, n, seed, codes, scales, tscale, partials, n_parts_out, stream)
-                  : quantize1d_t<QFP4_MXFP4, false, false, false>(x, xdt, n, seed, codes, scales, tscale, partials, n_parts_out, stream);
+        if (four6) return rotate ? QFP4_Q1(QFP4_MXFP4, true, false, true) : QFP4_Q1(QFP4_MXFP4, false, false, true);
+        if (rotate) return sr ? QFP4_Q1(QFP4_MXFP4, true, true, false) : QFP4_Q1(QFP4_MXFP4, true, false, false);
+        return sr ? QFP4_Q1(QFP4_MXFP4, false, true, false) : QFP4_Q1(QFP4_MXFP4, false, false, false);
     }
-    if (four6) {
-        if (rotate) return quantize1d_t<QFP4_NVFP4, true, false, true>(x, xdt, n, seed, codes, scales, tscale, partials, n_parts_out, stream);
-        return quantize1d_t<QFP4_NVFP4, false, false, true>(x, xdt, n, seed, codes, scales, tscale, partials, n_parts_out, stream);
-    }
-    if (rotate) return sr ? quantize1d_t<QFP4_NVFP4, true, true, false>(x, xdt, n, seed, codes, scales, tscale, partials, n_parts_out, stream)
-                          : quantize1d_t<QFP4_NVFP4, true, false, false>(x, xdt, n, seed, codes, scales, tscale, partials, n_parts_out, stream);
-    return sr ? quantize1d_t<QFP4_NVFP4, false, true, false>(x, xdt, n, seed, codes, scales, tscale, partials, n_parts_out, stream)
-              : quantize1d_t<QFP4_NVFP4, false, false, false>(x, xdt, n, seed, codes, scales, tscale, partials, n_parts_out, stream);
+    if (four6) return rotate ? QFP4_Q1(QFP4_NVFP4, true, false, true) : QFP4_Q1(QFP4_NVFP4, false, false, true);
+    if (rotate) return sr ? QFP4_Q1(QFP4_NVFP4, true, true, false) : QFP4_Q1(QFP4_NVFP4, true, false, false);
+    return sr ? QFP4_Q1(QFP4_NVFP4, false, true, false) : QFP4_Q1(QFP4_NVFP4, false, false, false);
+#undef QFP4_Q1
 }
 
 }  // namespace qfp4

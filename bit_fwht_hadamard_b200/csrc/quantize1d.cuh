@@ -24,11 +24,25 @@ struct QuantParams {
     float *partials_out;       // amax pass: where this launch writes its partials
     float *tscale_out;         // NVFP4: s_t output
     bool write_tscale;         // this launch's block 0 writes *tscale_out
+    int rule;                  // qfp4_scale_rule
+    const float *amax_in;      // NVFP4 quantize pass: caller-supplied tensor amax (device), or NULL
+};
+
+// Options beyond the defaults: the scale rule, and for NVFP4 a caller-supplied
+// tensor amax (device pointer; the tensor scale is fl(amax / 2688)) and where
+// to write this tensor's own (rotated) amax.
+struct QuantOpts {
+    int rule = QFP4_SCALE_DEFAULT;
+    const float *amax_in = nullptr;
+    float *amax_out = nullptr;
 };
 
 int quantize1d(const void *x, qfp4_dtype xdt, int64_t n, qfp4_fmt fmt, qfp4_round rounding, int rotate, int four6,
                uint64_t seed, uint8_t *codes, uint8_t *scales, float *tscale, float *partials, int *n_parts_out,
-               cudaStream_t stream);
+               cudaStream_t stream, const QuantOpts &opt = QuantOpts{});
+
+// *amax_out = max(partials[0 .. n)) (one block, dependent launch).
+int partials_max(const float *partials, int n, float *amax_out, cudaStream_t stream);
 
 // MXFP8 row-wise over a bf16 stream of n elements (n % 64 == 0) through the
 // TMA kernel.

@@ -29,11 +29,21 @@ namespace qfp4 {
 struct Q2DParams {
     int64_t M, K;
     uint8_t *codes, *scales, *codesT, *scalesT;
-    const float *partials;
+    const float *partials;       // NVFP4: partial maxima of the amax pass
     int n_partials;
     float *tscale_out;
     uint64_t seed;
+    int rule;                    // qfp4_scale_rule
+    const float *amax_in;        // NVFP4: caller-supplied tensor amax (device), or NULL
 };
+
+// NVFP4 tensor scale s_t = amax_t / (6 * 448): amax_t from the caller or
+// from the partial maxima of the amax pass (uniform over the block).
+__device__ __forceinline__ float q2d_tensor_scale(const Q2DParams &p, float *red)
+{
+    if (p.amax_in) return __fdiv_rn(*p.amax_in, 2688.0f);
+    return tensor_scale_from(p.partials, p.n_partials, red);
+}
 
 // 16 consecutive elements as raw words (bf16: 32 bytes, binary32: 64 bytes),
 // so that the next task's loads can be in flight during this task's work.
@@ -112,9 +122,9 @@ template <bool SR, typename T>
 __global__ void __launch_bounds__(256) k_quant2d(const T *__restrict__ x, Q2DParams p)
 {
     __shared__ float red[32];
-    const float s_t = tensor_scale_from(p.partials, p.n_partials, red);
+    const float s_t = q2d_tensor_scale(p, red);
     if (p.tscale_out && blockIdx.x == 0 && threadIdx.x == 0) *p.tscale_out = s_t;
-    const NvScale nz = nv_scale_setup(s_t);
+    const NvScale nz = nv_scale_setup(s_t, p.rule);
 
     const int lane = threadIdx.x & 31, half = lane >> 4, r = lane & 15;
     const int64_t tiles_k = p.K / 16, pairs = (tiles_k + 1) / 2;
@@ -154,13 +164,13 @@ __global__ void __launch_bounds__(256) k_quant2d(const T *__restrict__ x, Q2DPar
                 uint64_t pp[8], qq[8];
 #pragma unroll
                 for (int t = 0; t < 8; ++t) pp[t] = f2pack(v[2 * t], v[2 * t + 1]);
-                nv_quot16_pairs(pp, S, qq);
+                nv_quot16_pairs(pp, S, amax, qq);
                 float q[16];
 #pragma unroll
                 for (int t = 0; t < 8; ++t) f2unpack(qq[t], q[2 * t], q[2 * t + 1]);
                 sr_group<16>(q, static_cast<uint64_t>(i * p.K + j0), p.seed, w);
             } else {
-                nv_block_rne(v, S, w, nullptr);
+                nv_block_rne(v, S, amax, w, nullptr);
             }
         }
         if (valid) {
@@ -179,14 +189,97 @@ __global__ void __launch_bounds__(256) k_quant2d(const T *__restrict__ x, Q2DPar
     }
 }
 
+// Transpose a 32 x 32 nibble matrix held as one 128-bit row per lane (4
+// words, nibble j of lane r = element (r, j) in word j / 8); afterwards
+// nibble j of lane r is element (j, r).  Block swaps of 16 and 8 nibbles move
+// whole words, those of 4, 2 and 1 nibbles masked parts of each word.
+__device__ __forceinline__ void transpose32x32_nibbles(uint32_t (&w)[4], int r)
+{
+    {   // 16: words {0,1} of the upper lane <-> words {2,3} of the lower lane
+        const bool up = (r & 16) != 0;
+        const uint32_t a = __shfl_xor_sync(0xFFFFFFFFu, up ? w[0] : w[2], 16);
+        const uint32_t b = __shfl_xor_sync(0xFFFFFFFFu, up ? w[1] : w[3], 16);
+        if (up) { w[0] = a; w[1] = b; } else { w[2] = a; w[3] = b; }
+    }
+    {   // 8: word 1 / 3 of the lower lane <-> word 0 / 2 of the upper lane
+        const bool up = (r & 8) != 0;
+        const uint32_t a = __shfl_xor_sync(0xFFFFFFFFu, up ? w[0] : w[1], 8);
+        const uint32_t b = __shfl_xor_sync(0xFFFFFFFFu, up ? w[2] : w[3], 8);
+        if (up) { w[0] = a; w[2] = b; } else { w[1] = a; w[3] = b; }
+    }
+#pragma unroll
+    for (int s = 4; s >= 1; s >>= 1) {
+        const uint32_t m = s == 4 ? 0xFFFF0000u : s == 2 ? 0xFF00FF00u : 0xF0F0F0F0u;   // nibbles with (j & s) != 0
+        const bool up = (r & s) != 0;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const uint32_t o = __shfl_xor_sync(0xFFFFFFFFu, w[k], s);
+            w[k] = up ? ((w[k] & m) | ((o & m) >> (4 * s))) : ((w[k] & ~m) | ((o & ~m) << (4 * s)));
+        }
+    }
+}
+
+// ---------------------------------------------------------------- 2D MXFP4 (32 x 32 tiles)
+// A warp takes one 32 x 32 tile: lane r loads row r (32 elements), the tile
+// amax is a 32-lane reduction, the E8M0 exponent follows the scale rule, each
+// lane rounds its row once (RNE or Philox SR keyed on X's index) and stores
+// its 16 code bytes; the nibble transpose then gives each lane one column of
+// the tile, the codes of X^T.
+template <bool SR, typename T>
+__global__ void __launch_bounds__(256) k_quant2d_mx(const T *__restrict__ x, Q2DParams p)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t tiles_k = p.K / 32, tasks = (p.M / 32) * tiles_k;
+    const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    for (int64_t task = warp0; task < tasks; task += nwarps) {
+        const int64_t bi = (task / tiles_k) * 32, bj = (task % tiles_k) * 32;
+        const int64_t i = bi + lane;
+        float v[32];
+        Raw16<T> r0, r1;
+        raw_load16(x, i * p.K + bj, true, r0);
+        raw_load16(x, i * p.K + bj + 16, true, r1);
+        raw_to_f32(r0, v);
+        raw_to_f32(r1, v + 16);
+        float amax = 0.0f;
+#pragma unroll
+        for (int t = 0; t < 32; ++t) amax = fmaxf(amax, fabsf(v[t]));
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+        uint32_t w[4] = {0u, 0u, 0u, 0u}, sbyte = 0u;
+        if (amax != 0.0f) {
+            const int k = mx_scale_exp(amax, p.rule);
+            sbyte = static_cast<uint32_t>(k + 127);
+            const float mul = exp2i(-k);
+            float q[32];
+#pragma unroll
+            for (int t = 0; t < 32; ++t) q[t] = __fmul_rn(v[t], mul);
+            if (SR) {
+                sr_group<32>(q, static_cast<uint64_t>(i * p.K + bj), p.seed, w);
+            } else {
+#pragma unroll
+                for (int t = 0; t < 4; ++t) w[t] = e2m1x8_rne(q + 8 * t);
+            }
+        }
+        *reinterpret_cast<uint4 *>(p.codes + (i * p.K + bj) / 2) = make_uint4(w[0], w[1], w[2], w[3]);
+        p.scales[i * tiles_k + bj / 32] = static_cast<uint8_t>(sbyte);
+        if (p.codesT) {
+            transpose32x32_nibbles(w, lane);
+            const int64_t jr = bj + lane;                     // column of X = row of X^T
+            *reinterpret_cast<uint4 *>(p.codesT + (jr * p.M + bi) / 2) = make_uint4(w[0], w[1], w[2], w[3]);
+            p.scalesT[jr * (p.M / 32) + bi / 32] = static_cast<uint8_t>(sbyte);
+        }
+    }
+}
+
 // ---------------------------------------------------------------- 1D column-wise (X^T baseline)
 template <int FMT, bool SR, bool FOUR6, typename T>
 __global__ void __launch_bounds__(256) k_quant_cols(const T *__restrict__ x, Q2DParams p)
 {
     __shared__ float red[32];
     float s_t = 0.0f;
-    if (FMT == QFP4_NVFP4) s_t = tensor_scale_from(p.partials, p.n_partials, red);
-    const NvScale nz = nv_scale_setup(s_t);
+    if (FMT == QFP4_NVFP4) s_t = q2d_tensor_scale(p, red);
+    const NvScale nz = nv_scale_setup(s_t, p.rule);
     constexpr int G = FMT == QFP4_MXFP4 ? 32 : 16;
     const int lane = threadIdx.x & 31;
     const int64_t col_blocks = (p.K + 31) / 32, row_blocks = (p.M + 31) / 32;
@@ -213,7 +306,7 @@ __global__ void __launch_bounds__(256) k_quant_cols(const T *__restrict__ x, Q2D
             float S = 0.0f, mul = 0.0f;
             if (FMT == QFP4_MXFP4) {
                 if (amax != 0.0f) {
-                    const int k = scale_exp(amax, 0x400000u, 2);
+                    const int k = mx_scale_exp(amax, p.rule);
                     sbyte = static_cast<uint32_t>(k + 127);
                     S = exp2i(k);
                     mul = exp2i(-k);
@@ -229,8 +322,8 @@ __global__ void __launch_bounds__(256) k_quant_cols(const T *__restrict__ x, Q2D
                     enc4 = nv_scale_byte<false>(amax, nz);
                     S4 = __fmul_rn(e4m3_value(enc4), s_t);
                 }
-                nv_block_rne(xg, S, w6, &sse6);
-                nv_block_rne(xg, S4, w4, &sse4);
+                nv_block_rne(xg, S, amax, w6, &sse6);
+                nv_block_rne(xg, S4, amax, w4, &sse4);
                 const bool pick4 = sse4 < sse6;
                 wg[0] = pick4 ? w4[0] : w6[0];
                 wg[1] = pick4 ? w4[1] : w6[1];
@@ -239,7 +332,7 @@ __global__ void __launch_bounds__(256) k_quant_cols(const T *__restrict__ x, Q2D
 #pragma unroll
                 for (int t = 0; t < G / 8; ++t) wg[t] = 0u;
             } else if (FMT == QFP4_NVFP4 && !SR) {
-                nv_block_rne(xg, S, wg, nullptr);
+                nv_block_rne(xg, S, amax, wg, nullptr);
             } else {
                 float q[G];
                 if (FMT == QFP4_MXFP4) {
@@ -249,7 +342,7 @@ __global__ void __launch_bounds__(256) k_quant_cols(const T *__restrict__ x, Q2D
                     uint64_t pp[G / 2], qq[G / 2];
 #pragma unroll
                     for (int t = 0; t < G / 2; ++t) pp[t] = f2pack(xg[2 * t], xg[2 * t + 1]);
-                    nv_quot16_pairs(pp, S, qq);
+                    nv_quot16_pairs(pp, S, amax, qq);
 #pragma unroll
                     for (int t = 0; t < G / 2; ++t) f2unpack(qq[t], q[2 * t], q[2 * t + 1]);
                 }
@@ -371,8 +464,8 @@ __global__ void __launch_bounds__(256) k_cols4(const uint16_t *__restrict__ x, Q
     constexpr int G = NV ? 16 : 32, NG = 32 / G;
     __shared__ float red[32];
     float s_t = 0.0f;
-    if (NV) s_t = tensor_scale_from(p.partials, p.n_partials, red);
-    const NvScale nz = nv_scale_setup(s_t);
+    if (NV) s_t = q2d_tensor_scale(p, red);
+    const NvScale nz = nv_scale_setup(s_t, p.rule);
     const int lane = threadIdx.x & 31;
     const int64_t col_blocks = (p.K + 127) / 128, row_blocks = (p.M + 31) / 32;
     const int64_t tasks = row_blocks * col_blocks;
@@ -396,7 +489,7 @@ __global__ void __launch_bounds__(256) k_cols4(const uint16_t *__restrict__ x, Q
         auto val = [&](int r, int c) -> float { return (c & 1) ? bf16hi(raw[r][c >> 1]) : bf16lo(raw[r][c >> 1]); };
 
         // scales per (group, column)
-        float S[NG][4], Y[NG][4], mul[4];
+        float S[NG][4], Y[NG][4], A[NG][4], mul[4];
         bool fast[NG][4];
         uint32_t sb[NG][4], w[4][MX8 ? 8 : 4];
 #pragma unroll
@@ -410,6 +503,7 @@ __global__ void __launch_bounds__(256) k_cols4(const uint16_t *__restrict__ x, Q
                 float amax = 0.0f;
 #pragma unroll
                 for (int r = 0; r < G; ++r) amax = fmaxf(amax, fabsf(val(G * g + r, c)));
+                A[g][c] = amax;
                 sb[g][c] = 0u;
                 S[g][c] = 0.0f;
                 Y[g][c] = 0.0f;
@@ -417,7 +511,7 @@ __global__ void __launch_bounds__(256) k_cols4(const uint16_t *__restrict__ x, Q
                 if (!NV) {
                     mul[c] = 0.0f;
                     if (amax != 0.0f) {
-                        const int k = MX8 ? scale_exp(amax, 0x600000u, 8) : scale_exp(amax, 0x400000u, 2);
+                        const int k = MX8 ? scale_exp(amax, 0x600000u, 8) : mx_scale_exp(amax, p.rule);
                         sb[g][c] = static_cast<uint32_t>(k + 127);
                         S[g][c] = 1.0f;                      // marks a nonzero group
                         mul[c] = exp2i(-k);
@@ -433,8 +527,8 @@ __global__ void __launch_bounds__(256) k_cols4(const uint16_t *__restrict__ x, Q
                         const float S4 = __fmul_rn(e4m3_value(enc4), s_t);
                         uint32_t w6[2], w4[2];
                         float sse6, sse4;
-                        nv_block_rne(xg, Sv, w6, &sse6);
-                        nv_block_rne(xg, S4, w4, &sse4);
+                        nv_block_rne(xg, Sv, amax, w6, &sse6);
+                        nv_block_rne(xg, S4, amax, w4, &sse4);
                         const bool pick4 = sse4 < sse6;
                         w[c][2 * g] = pick4 ? w4[0] : w6[0];
                         w[c][2 * g + 1] = pick4 ? w4[1] : w6[1];
@@ -442,7 +536,7 @@ __global__ void __launch_bounds__(256) k_cols4(const uint16_t *__restrict__ x, Q
                     }
                     sb[g][c] = enc;
                     S[g][c] = Sv;
-                    fast[g][c] = Sv >= 0x1p-125f && Sv <= 0x1p125f;
+                    fast[g][c] = Sv >= 0x1p-125f && Sv <= 0x1p125f && amax <= Sv * 0x1p100f;
                     Y[g][c] = fast[g][c] ? __frcp_rn(Sv) : 0.0f;
                 }
             }
@@ -475,7 +569,7 @@ __global__ void __launch_bounds__(256) k_cols4(const uint16_t *__restrict__ x, Q
                         float xg[16];
 #pragma unroll
                         for (int r = 0; r < 16; ++r) xg[r] = val(16 * g + r, c);
-                        nv_block_rne(xg, S[g][c], &w[c][2 * g], nullptr);
+                        nv_block_rne(xg, S[g][c], A[g][c], &w[c][2 * g], nullptr);
                     } else if (MX8) {
 #pragma unroll
                         for (int t = 0; t < 8; ++t)
@@ -545,16 +639,35 @@ static void launch_tiles(int64_t warp_tasks, const void *x, const Q2DParams &p, 
     Kern<<<grid_for_warps<Kern>(warp_tasks), 256, 0, stream>>>(static_cast<const T *>(x), p);
 }
 
-int quantize2d(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_round rounding, uint64_t seed,
-               uint8_t *codes, uint8_t *scales, uint8_t *codesT, uint8_t *scalesT, float *tscale, float *partials,
-               cudaStream_t stream)
+// 2D blocks: NVFP4 16 x 16 (after the amax pass, unless the caller gives
+// the tensor amax and does not ask for it back) or MXFP4 32 x 32 tiles.
+int quantize2d(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_fmt fmt, qfp4_round rounding,
+               uint64_t seed, uint8_t *codes, uint8_t *scales, uint8_t *codesT, uint8_t *scalesT, float *tscale,
+               float *partials, cudaStream_t stream, const QuantOpts &opt)
 {
-    int n_parts = 0;
-    int st = amax_partials(x, xdt, M * K, partials, &n_parts, stream);
-    if (st != QFP4_OK) return st;
-    Q2DParams p{M, K, codes, scales, codesT, scalesT, partials, n_parts, tscale, seed};
-    const int64_t tasks = (M / 16) * ((K / 16 + 1) / 2);
     const bool sr = rounding == QFP4_SR;
+    Q2DParams p{M, K, codes, scales, codesT, scalesT, partials, 0, tscale, seed, opt.rule, opt.amax_in};
+    if (fmt == QFP4_MXFP4) {
+        const int64_t tasks = (M / 32) * (K / 32);
+        if (xdt == QFP4_BF16) {
+            if (sr) launch_tiles<k_quant2d_mx<true, uint16_t>, uint16_t>(tasks, x, p, stream);
+            else launch_tiles<k_quant2d_mx<false, uint16_t>, uint16_t>(tasks, x, p, stream);
+        } else {
+            if (sr) launch_tiles<k_quant2d_mx<true, float>, float>(tasks, x, p, stream);
+            else launch_tiles<k_quant2d_mx<false, float>, float>(tasks, x, p, stream);
+        }
+        QFP4_LAUNCH_CHECK();
+        return QFP4_OK;
+    }
+    if (!opt.amax_in || opt.amax_out) {
+        int st = amax_partials(x, xdt, M * K, partials, &p.n_partials, stream);
+        if (st != QFP4_OK) return st;
+        if (opt.amax_out) {
+            st = partials_max(partials, p.n_partials, opt.amax_out, stream);
+            if (st != QFP4_OK) return st;
+        }
+    }
+    const int64_t tasks = (M / 16) * ((K / 16 + 1) / 2);
     if (xdt == QFP4_BF16) {
         if (sr) launch_tiles<k_quant2d<true, uint16_t>, uint16_t>(tasks, x, p, stream);
         else launch_tiles<k_quant2d<false, uint16_t>, uint16_t>(tasks, x, p, stream);
@@ -580,9 +693,9 @@ static int launch_cols(const void *x, qfp4_dtype xdt, const Q2DParams &p, cudaSt
 
 int quantize_columns(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_fmt fmt, qfp4_round rounding, int four6,
                      uint64_t seed, uint8_t *codesT, uint8_t *scalesT, const float *partials, int n_partials,
-                     cudaStream_t stream)
+                     cudaStream_t stream, const QuantOpts &opt)
 {
-    Q2DParams p{M, K, nullptr, nullptr, codesT, scalesT, partials, n_partials, nullptr, seed};
+    Q2DParams p{M, K, nullptr, nullptr, codesT, scalesT, partials, n_partials, nullptr, seed, opt.rule, opt.amax_in};
     const bool sr = rounding == QFP4_SR;
     if (fmt == QFP4_MXFP4)
         return sr ? launch_cols<QFP4_MXFP4, true, false>(x, xdt, p, stream)
@@ -595,7 +708,7 @@ int quantize_columns(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_f
 int quantize_mxfp8(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_round rounding, uint64_t seed,
                    uint8_t *codes, uint8_t *scales, uint8_t *codesT, uint8_t *scalesT, cudaStream_t stream)
 {
-    Q2DParams p{M, K, codes, scales, codesT, scalesT, nullptr, 0, nullptr, seed};
+    Q2DParams p{M, K, codes, scales, codesT, scalesT, nullptr, 0, nullptr, seed, QFP4_SCALE_DEFAULT, nullptr};
     const int64_t tasks = ((M + 31) / 32) * (K / 32);
     const bool sr = rounding == QFP4_SR, cols = codesT != nullptr;
     if (xdt == QFP4_BF16 && (M * K) % 64 == 0) {

@@ -54,6 +54,12 @@ typedef enum { QFP4_BF16 = 0, QFP4_F32 = 1 } qfp4_dtype;
 typedef enum {
     QFP4_GRAN_TENSOR = 0, QFP4_GRAN_ROW = 1, QFP4_GRAN_GROUP16 = 2, QFP4_GRAN_GROUP32 = 3
 } qfp4_gran;
+/* Scale rules of qfp4_quantize_ex (see there). */
+typedef enum {
+    QFP4_SCALE_DEFAULT = 0,     /* MXFP4: truncation-free E8M0; NVFP4: E4M3 block scale to nearest */
+    QFP4_SCALE_OCP_FLOOR = 1,   /* MXFP4 only: E8M0 k = floor(log2 amax) - 2 (the OCP rule; may clip) */
+    QFP4_SCALE_E4M3_UP = 2      /* NVFP4 only: E4M3 block scale rounded up (no element clips) */
+} qfp4_scale_rule;
 
 enum {
     QFP4_OK = 0,
@@ -80,7 +86,7 @@ enum {
  *       s_t = amax_t / (6*448) in binary32 over the whole (rotated) tensor;
  *       per 16-block enc = E4M3_RNE_satfinite((amax_b / 6) / s_t) and the
  *       effective scale S = e4m3(enc) * s_t (binary32).
- *   (3) four6 != 0 (NVFP4, RNE, 1D only): a second candidate scale from
+ *   (3) four6 != 0 (RNE, 1D only; MXFP4: see qfp4_quantize_ex): a second candidate scale from
  *       amax_b / 4; each block keeps the candidate whose binary32 squared
  *       error sum(deq - x)^2 (summed as pairs i,i+8; +4; +2; +1) is lower,
  *       ties keeping amax/6.
@@ -91,11 +97,11 @@ enum {
  *       w is word (e mod 4) of Philox4x32-10 keyed (seed low 32, seed high
  *       32) at counter (e/4 low 32, e/4 high 32, 0, 0).  The code's sign
  *       bit is the sign of v.
- *   (5) block2d != 0 (NVFP4 only, no rotation, no four6): 16x16 tiles share
- *       one scale (amax over the tile), so X and X^T use the same scales.
- *       scales[i][j/16] and scalesT[j][i/16] both hold tile (i/16, j/16);
- *       codesT (K x M/2) is exactly the transpose of codes.  Needs M % 16
- *       == 0 and K % 16 == 0.
+ *   (5) block2d != 0 (no rotation, no four6): T x T tiles share one scale
+ *       (amax over the tile), so X and X^T use the same scales; T = 16 for
+ *       NVFP4, 32 for MXFP4.  scales[i][j/T] and scalesT[j][i/T] both hold
+ *       tile (i/T, j/T); codesT (K x M/2) is exactly the transpose of codes.
+ *       Needs M % T == 0 and K % T == 0.
  *   In 1D mode a non-NULL codesT/scalesT asks for an independent
  *   quantization of every column (groups of g along M; K x M/2 codes,
  *   K x M/g scales), the baseline [TI] contrasts with 2D blocks; needs
@@ -112,9 +118,9 @@ enum {
  *                tensor maxima; contents on entry do not matter).  MXFP4:
  *                may be NULL.
  * Errors: QFP4_ERR_SHAPE for K % g != 0, K % 128 != 0 with rotate, M or K
- *   not a multiple of 16 with block2d, M % g != 0 with a 1D codesT;
- *   QFP4_ERR_UNSUPPORTED for four6 with MXFP4, SR or block2d, block2d with
- *   MXFP4 or rotate, rotate with a 1D codesT.
+ *   not a multiple of the tile with block2d, M % g != 0 with a 1D codesT;
+ *   QFP4_ERR_UNSUPPORTED for four6 with SR or block2d (or MXFP4 with a 1D
+ *   codesT), block2d with rotate, rotate with a 1D codesT.
  * ---------------------------------------------------------------------- */
 size_t qfp4_quantize_workspace_bytes(int64_t M, int64_t K, qfp4_fmt fmt, int rotate, int block2d);
 
@@ -126,6 +132,53 @@ int qfp4_quantize(const void *x, qfp4_dtype xdt, int64_t M, int64_t K,
                   float *tscale,
                   void *workspace, size_t workspace_bytes,
                   qfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * qfp4_quantize_ex -- qfp4_quantize with the scale-rule variants, the 2D and
+ * four-over-six options on MXFP4, and a caller-supplied tensor amax.
+ * qfp4_quantize(...) is qfp4_quantize_ex(..., QFP4_SCALE_DEFAULT, seed,
+ * NULL, NULL, ...).
+ *   rule   QFP4_SCALE_DEFAULT, or the ablations the pages imply ([LB] §3:
+ *          what a power-of-two scale costs; [TI]: truncation-free scaling):
+ *          QFP4_SCALE_OCP_FLOOR (MXFP4): k = floor(log2 amax) - 2, the
+ *            largest k with 2^(k+2) <= amax, so amax / 2^k is in [4, 8) and
+ *            magnitudes above 6 * 2^k saturate to 6;
+ *          QFP4_SCALE_E4M3_UP (NVFP4): enc = the least E4M3 value >=
+ *            (amax_b / d) / s_t (saturating at 448), so S >= amax_b / d.
+ *   four6  NVFP4 as in qfp4_quantize; MXFP4 (RNE, 1D rows only): the
+ *          second candidate exponent is the least k4 with 4 * 2^k4 >= amax,
+ *          kept only when the group's binary32 squared error (summed as
+ *          pairs i, i+16; +8; +4; +2; +1) is strictly lower ([46]).  Under
+ *          the default rule it never is (the 2^(k+1) grid is a subset below
+ *          amax); under the OCP floor rule it trades clipping for range.
+ *   block2d  NVFP4 16 x 16 tiles, or MXFP4 32 x 32 tiles (one E8M0 scale per
+ *          tile, the scale rule applied to the tile amax); needs M and K
+ *          multiples of the tile size.
+ *   amax_in  NVFP4: NULL (the call measures the tensor's amax: an extra read
+ *          of X), or a DEVICE pointer to a finite amax_t >= 0 from elsewhere
+ *          -- a previous step's, a moving average of several ([QN] open
+ *          questions: EMA / delayed activation scales), or a calibrated clip
+ *          (qfp4_kl_calibrate).  s_t = fl(*amax_in / 2688); the quantize
+ *          then reads X once, and blocks whose values exceed the implied
+ *          range saturate (E4M3 byte 0x7E, codes +-6).  MXFP4: must be NULL.
+ *   amax_out NVFP4: NULL, or a DEVICE float that receives this tensor's own
+ *          amax (after rotation), e.g. for the next step's amax_in.
+ *          MXFP4: must be NULL.
+ *   workspace NVFP4: needed (qfp4_quantize_workspace_bytes) unless amax_in
+ *          is given and amax_out is NULL.
+ * Errors: as qfp4_quantize, plus QFP4_ERR_ARG for an unknown rule,
+ *   QFP4_ERR_UNSUPPORTED for a rule of the other format, amax_in / amax_out
+ *   with MXFP4, MXFP4 four6 with a 1D codesT.
+ * ---------------------------------------------------------------------- */
+int qfp4_quantize_ex(const void *x, qfp4_dtype xdt, int64_t M, int64_t K,
+                     qfp4_fmt fmt, qfp4_round rounding, int rotate, int block2d, int four6,
+                     qfp4_scale_rule rule, uint64_t seed,
+                     const float *amax_in, float *amax_out,
+                     uint8_t *codes, uint8_t *scales,
+                     uint8_t *codesT, uint8_t *scalesT,
+                     float *tscale,
+                     void *workspace, size_t workspace_bytes,
+                     qfp4_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * qfp4_quantize_mxfp8 -- MXFP8 variant ([TI]: MXFP8 for the sensitive Q/K
@@ -232,6 +285,16 @@ int qfp4_gemm_fused_rq(const void *A_bf16, int64_t M, int64_t K, int rotate, int
                        const uint8_t *B_codes, const uint8_t *B_scales, const float *B_tscale, int64_t N,
                        void *workspace, size_t workspace_bytes,
                        qfp4_dtype out_dt, void *out, qfp4_stream_t stream);
+
+/* Where qfp4_gemm_fused_rq leaves A's quantized operand in its workspace
+ * once the call's work is done: codes (M*K/2 bytes, as qfp4_quantize writes
+ * them) at byte *codes_off, row-major scales (M*(K/g) bytes) at
+ * *scales_off, and for NVFP4 the tensor scale (one float) at *tscale_off;
+ * each offset is a multiple of 256.  The three out-pointers are host
+ * memory.  Returns QFP4_ERR_ARG for a bad fmt or a NULL out-pointer,
+ * QFP4_ERR_SHAPE for a negative dimension. */
+int qfp4_gemm_fused_rq_workspace_layout(int64_t M, int64_t N, int64_t K, qfp4_fmt fmt, size_t *codes_off,
+                                        size_t *scales_off, size_t *tscale_off);
 
 /* Human-readable text of a status code (static storage). */
 const char *qfp4_status_string(int status);

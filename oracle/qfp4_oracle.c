@@ -411,6 +411,7 @@ static int check_quantize_args(const void *x, int xdt, int64_t M, int64_t K, int
     if (rule == OR_RULE_E4M3_UP && fmt != OR_NVFP4) return OR_ERR_UNSUPPORTED;
     if ((amax_in || amax_out) && fmt != OR_NVFP4) return OR_ERR_UNSUPPORTED;
     if (four6 && (block2d || rounding != OR_RNE)) return OR_ERR_UNSUPPORTED;
+    if (four6 && fmt == OR_MXFP4 && codesT) return OR_ERR_UNSUPPORTED;
     if (block2d && rotate) return OR_ERR_UNSUPPORTED;
     if (!block2d && rotate && codesT) return OR_ERR_UNSUPPORTED;
     if (row0 && (block2d || codesT)) return OR_ERR_UNSUPPORTED;

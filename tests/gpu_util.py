@@ -129,7 +129,8 @@ def _fmt_g(fmt):
     return 32 if fmt == q.MXFP4 else 16
 
 
-def quantize(x, fmt, rounding=0, rotate=False, block2d=False, four6=False, seed=0, transposed=False):
+def quantize(x, fmt, rounding=0, rotate=False, block2d=False, four6=False, seed=0, transposed=False, rule=0,
+             amax_in=None, amax_out=None):
     """q.quantize with every output in a guarded buffer."""
     import bit_fwht_hadamard_b200 as q
     M, K = x.shape
@@ -141,7 +142,7 @@ def quantize(x, fmt, rounding=0, rotate=False, block2d=False, four6=False, seed=
     if fmt == q.NVFP4:
         o["tscale"] = guarded((1,), torch.float32)
     return q.quantize(x, fmt, rounding, rotate=rotate, block2d=block2d, four6=four6, seed=seed,
-                      transposed=transposed, out=o)
+                      transposed=transposed, out=o, rule=rule, amax_in=amax_in, amax_out=amax_out)
 
 
 def quantize_mxfp8(x, rounding=0, seed=0, transposed=False):

@@ -37,8 +37,8 @@ def test_argument_errors_return_before_any_launch():
     fake = 1 << 20                      # never dereferenced: validation fails first
     st = q.qfp4_quantize(fake, q.BF16, 4, 48, q.MXFP4, q.RNE, 0, 0, 0, 0, fake, fake, None, None, None, None, 0, None)
     assert st == q.ERR_SHAPE
-    st = q.qfp4_quantize(fake, q.BF16, 4, 64, q.MXFP4, q.RNE, 0, 0, 1, 0, fake, fake, None, None, None, None, 0, None)
-    assert st == q.ERR_UNSUPPORTED
+    st = q.qfp4_quantize(fake, q.BF16, 4, 64, q.MXFP4, q.SR, 0, 0, 1, 0, fake, fake, None, None, None, None, 0, None)
+    assert st == q.ERR_UNSUPPORTED                          # four-over-six is round-to-nearest only
     st = q.qfp4_quantize(fake + 2, q.BF16, 4, 64, q.MXFP4, q.RNE, 0, 0, 0, 0, fake, fake, None, None, None, None, 0,
                          None)
     assert st == q.ERR_ALIGN
@@ -61,8 +61,9 @@ def test_more_argument_errors_follow_the_header():
     # four-over-six only with NVFP4, 1D, round-to-nearest
     assert Q(f, q.BF16, 16, 64, q.NVFP4, q.SR, 0, 0, 1, 0, f, f, None, None, f, f, 4096, None) == q.ERR_UNSUPPORTED
     assert Q(f, q.BF16, 16, 64, q.NVFP4, q.RNE, 0, 1, 1, 0, f, f, None, None, f, f, 4096, None) == q.ERR_UNSUPPORTED
-    # 2D blocks only with NVFP4 and without rotation
-    assert Q(f, q.BF16, 16, 128, q.MXFP4, q.RNE, 0, 1, 0, 0, f, f, None, None, None, None, 0, None) == q.ERR_UNSUPPORTED
+    # 2D blocks without rotation; MXFP4 tiles are 32 x 32
+    assert Q(f, q.BF16, 16, 128, q.MXFP4, q.RNE, 0, 1, 0, 0, f, f, None, None, None, None, 0, None) == q.ERR_SHAPE
+    assert Q(f, q.BF16, 32, 128, q.MXFP4, q.RNE, 1, 1, 0, 0, f, f, None, None, None, None, 0, None) == q.ERR_UNSUPPORTED
     assert Q(f, q.BF16, 16, 128, q.NVFP4, q.RNE, 1, 1, 0, 0, f, f, None, None, f, f, 4096, None) == q.ERR_UNSUPPORTED
     # 1D column-wise output not with rotation; codesT and scalesT together
     assert Q(f, q.BF16, 32, 128, q.MXFP4, q.RNE, 1, 0, 0, 0, f, f, f, f, None, None, 0, None) == q.ERR_UNSUPPORTED
@@ -90,3 +91,23 @@ def test_more_argument_errors_follow_the_header():
 def test_selftest_wait_limit_is_checked_on_the_host():
     assert q.qfp4_selftest_wait_timeout(0, None) == q.ERR_ARG
     assert q.qfp4_selftest_wait_timeout(1_000_001, None) == q.ERR_ARG
+
+
+def test_quantize_ex_argument_errors():
+    """qfp4_quantize_ex's own rejections, decided on the host."""
+    f = 1 << 20
+    X = q.qfp4_quantize_ex
+
+    def call(fmt, rule=q.SCALE_DEFAULT, rounding=q.RNE, four6=0, block2d=0, amax_in=None, amax_out=None,
+             M=32, K=128, T=False, ws=None, wsb=0):
+        return X(f, q.BF16, M, K, fmt, rounding, 0, block2d, four6, rule, 0, amax_in, amax_out, f, f,
+                 f if T else None, f if T else None, f, ws, wsb, None)
+
+    assert call(q.MXFP4, rule=3) == q.ERR_ARG
+    assert call(q.NVFP4, rule=q.SCALE_OCP_FLOOR, ws=f, wsb=4096) == q.ERR_UNSUPPORTED
+    assert call(q.MXFP4, rule=q.SCALE_E4M3_UP) == q.ERR_UNSUPPORTED
+    assert call(q.MXFP4, amax_in=f) == q.ERR_UNSUPPORTED
+    assert call(q.MXFP4, amax_out=f) == q.ERR_UNSUPPORTED
+    assert call(q.MXFP4, four6=1, T=True) == q.ERR_UNSUPPORTED          # MXFP4 four-over-six: rows only
+    assert call(q.NVFP4, amax_out=f) == q.ERR_ARG                        # own amax needs the workspace
+    assert call(q.MXFP4, block2d=1, M=48) == q.ERR_SHAPE
