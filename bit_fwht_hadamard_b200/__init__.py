@@ -19,7 +19,7 @@ from ctypes import c_int, c_int64, c_size_t, c_uint64, c_void_p, c_char_p
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libqfp4.so")
 
-MXFP4, NVFP4 = 0, 1
+MXFP4, NVFP4, MXFP8 = 0, 1, 2
 RNE, SR = 0, 1
 BF16, F32 = 0, 1
 GRAN_TENSOR, GRAN_ROW, GRAN_GROUP16, GRAN_GROUP32 = 0, 1, 2, 3
@@ -31,6 +31,8 @@ EXPORTS = [
     "qfp4_quantize_workspace_bytes", "qfp4_quantize", "qfp4_quantize_ex", "qfp4_quantize_mxfp8", "qfp4_quantize_fp32scale",
     "qfp4_dequantize", "qfp4_gemm_workspace_bytes", "qfp4_gemm_blockscaled", "qfp4_gemm_fused_rq_workspace_bytes",
     "qfp4_gemm_fused_rq", "qfp4_gemm_fused_rq_workspace_layout", "qfp4_gemm_blockscaled_noalloc",
+    "qfp4_linear_forward_workspace_bytes", "qfp4_linear_forward", "qfp4_linear_backward_workspace_bytes",
+    "qfp4_linear_backward", "qfp4_kl_calibrate_workspace_bytes", "qfp4_kl_calibrate",
     "qfp4_status_string", "qfp4_last_device_error", "qfp4_selftest_wait_timeout", "qfp4_version",
     "qfp4_launch_count",
 ]
@@ -81,6 +83,19 @@ def lib():
                                          c_int, P, P]
         L.qfp4_gemm_fused_rq_workspace_layout.restype = c_int
         L.qfp4_gemm_fused_rq_workspace_layout.argtypes = [c_int64, c_int64, c_int64, c_int, P, P, P]
+        L.qfp4_linear_forward_workspace_bytes.restype = c_size_t
+        L.qfp4_linear_forward_workspace_bytes.argtypes = [c_int64, c_int64, c_int64, c_int]
+        L.qfp4_linear_forward.restype = c_int
+        L.qfp4_linear_forward.argtypes = [P, P, c_int64, c_int64, c_int64, c_int, c_int, c_int, P, P, c_size_t, P]
+        L.qfp4_linear_backward_workspace_bytes.restype = c_size_t
+        L.qfp4_linear_backward_workspace_bytes.argtypes = [c_int64, c_int64, c_int64, c_int]
+        L.qfp4_linear_backward.restype = c_int
+        L.qfp4_linear_backward.argtypes = [P, P, P, c_int64, c_int64, c_int64, c_int, c_uint64, c_int, P, P, P,
+                                           c_size_t, P]
+        L.qfp4_kl_calibrate_workspace_bytes.restype = c_size_t
+        L.qfp4_kl_calibrate_workspace_bytes.argtypes = [c_int, c_int, c_int]
+        L.qfp4_kl_calibrate.restype = c_int
+        L.qfp4_kl_calibrate.argtypes = [P, c_int, c_int64, c_int, c_int, c_int, P, P, P, P, P, c_size_t, P]
         L.qfp4_status_string.restype = c_char_p
         L.qfp4_status_string.argtypes = [c_int]
         L.qfp4_last_device_error.restype = c_int
@@ -165,6 +180,33 @@ def qfp4_gemm_fused_rq_workspace_layout(M, N, K, fmt):
     st = lib().qfp4_gemm_fused_rq_workspace_layout(M, N, K, fmt, *[ctypes.byref(o) for o in offs])
     _check(st, "qfp4_gemm_fused_rq_workspace_layout")
     return tuple(o.value for o in offs)
+
+
+def qfp4_linear_forward_workspace_bytes(M, N, K, fmt):
+    return lib().qfp4_linear_forward_workspace_bytes(M, N, K, fmt)
+
+
+def qfp4_linear_forward(X, W, M, N, K, fmt, four6, out_dt, Y, workspace, workspace_bytes, stream):
+    return lib().qfp4_linear_forward(X, W, M, N, K, fmt, four6, out_dt, Y, workspace, workspace_bytes, stream)
+
+
+def qfp4_linear_backward_workspace_bytes(M, N, K, fmt):
+    return lib().qfp4_linear_backward_workspace_bytes(M, N, K, fmt)
+
+
+def qfp4_linear_backward(G, X, W, M, N, K, fmt, seed, out_dt, dX, dW, workspace, workspace_bytes, stream):
+    return lib().qfp4_linear_backward(G, X, W, M, N, K, fmt, seed & ((1 << 64) - 1), out_dt, dX, dW, workspace,
+                                      workspace_bytes, stream)
+
+
+def qfp4_kl_calibrate_workspace_bytes(bins, levels, grid):
+    return lib().qfp4_kl_calibrate_workspace_bytes(bins, levels, grid)
+
+
+def qfp4_kl_calibrate(x, xdt, n, bins, levels, grid, clip_out, best_bins_out, kl_out, hist_out, workspace,
+                      workspace_bytes, stream):
+    return lib().qfp4_kl_calibrate(x, xdt, n, bins, levels, grid, clip_out, best_bins_out, kl_out, hist_out,
+                                   workspace, workspace_bytes, stream)
 
 
 def qfp4_status_string(status):
@@ -326,3 +368,62 @@ def gemm_fused_rq(A_bf16, B, N, fmt=NVFP4, rotate=True, four6=False, out_dtype=N
                             _ptr(out), _stream(stream))
     _check(st, "qfp4_gemm_fused_rq")
     return out
+
+
+def linear_forward(X, W, fmt=NVFP4, four6=False, out_dtype=None, out=None, workspace=None, stream=None):
+    """Y = X W^T through rotated FP4 operands (qfp4_linear_forward); X (M, K)
+    and W (N, K) bf16 CUDA tensors."""
+    torch = _torch()
+    M, K = X.shape
+    N = W.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float32 if out_dtype is None else out_dtype, device=X.device)
+    wsb = qfp4_linear_forward_workspace_bytes(M, N, K, fmt)
+    if workspace is None:
+        workspace = torch.empty(max(wsb, 16), dtype=torch.uint8, device=X.device)
+    st = qfp4_linear_forward(_ptr(X), _ptr(W), M, N, K, fmt, int(four6), F32 if out.dtype == torch.float32 else BF16,
+                             _ptr(out), _ptr(workspace), wsb, _stream(stream))
+    _check(st, "qfp4_linear_forward")
+    return out
+
+
+def linear_backward(G, X, W, fmt=NVFP4, seed=0, out_dtype=None, want_dx=True, want_dw=True, out=None,
+                    workspace=None, stream=None):
+    """(dX, dW) = (G W, G^T X) through quantized operands
+    (qfp4_linear_backward); G (M, N), X (M, K), W (N, K) bf16 CUDA tensors."""
+    torch = _torch()
+    M, N = G.shape
+    K = X.shape[1] if X is not None else W.shape[1]
+    dt = torch.float32 if out_dtype is None else out_dtype
+    o = dict(out) if out is not None else {}
+    if want_dx and "dX" not in o:
+        o["dX"] = torch.empty((M, K), dtype=dt, device=G.device)
+    if want_dw and "dW" not in o:
+        o["dW"] = torch.empty((N, K), dtype=dt, device=G.device)
+    wsb = qfp4_linear_backward_workspace_bytes(M, N, K, fmt)
+    if workspace is None:
+        workspace = torch.empty(max(wsb, 16), dtype=torch.uint8, device=G.device)
+    st = qfp4_linear_backward(_ptr(G), _ptr(X), _ptr(W), M, N, K, fmt, seed, F32 if dt == torch.float32 else BF16,
+                              _ptr(o.get("dX")), _ptr(o.get("dW")), _ptr(workspace), wsb, _stream(stream))
+    _check(st, "qfp4_linear_backward")
+    return o.get("dX"), o.get("dW")
+
+
+def kl_calibrate(x, bins=2048, levels=8, grid=0, stream=None, out=None):
+    """KL-divergence clip point of a CUDA tensor (qfp4_kl_calibrate); returns
+    dict(clip (1,) float32, best (1,) int32, kl (bins - first + 1,) float64,
+    hist (bins,) int64 holding the uint64 counts)."""
+    torch = _torch()
+    dev = x.device
+    first = 8 if grid else levels
+    o = dict(out) if out is not None else {
+        "clip": torch.empty(1, dtype=torch.float32, device=dev), "best": torch.empty(1, dtype=torch.int32, device=dev),
+        "kl": torch.empty(bins - first + 1, dtype=torch.float64, device=dev),
+        "hist": torch.empty(bins, dtype=torch.int64, device=dev)}
+    wsb = qfp4_kl_calibrate_workspace_bytes(bins, levels, grid)
+    ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
+    st = qfp4_kl_calibrate(_ptr(x), _xdt(x), x.numel(), bins, levels, grid, _ptr(o["clip"]), _ptr(o["best"]),
+                           _ptr(o["kl"]), _ptr(o["hist"]), _ptr(ws), wsb, _stream(stream))
+    _check(st, "qfp4_kl_calibrate")
+    return o
+

@@ -179,7 +179,7 @@ extern "C" int qfp4_gemm_blockscaled(const uint8_t *A_codes, const uint8_t *A_sc
                                      int64_t M, int64_t N, int64_t K, qfp4_fmt fmt, qfp4_dtype out_dt, void *out,
                                      void *workspace, size_t workspace_bytes, qfp4_stream_t stream)
 {
-    if (fmt != QFP4_MXFP4 && fmt != QFP4_NVFP4) return QFP4_ERR_ARG;
+    if (fmt != QFP4_MXFP4 && fmt != QFP4_NVFP4 && fmt != QFP4_MXFP8) return QFP4_ERR_ARG;
     if (out_dt != QFP4_BF16 && out_dt != QFP4_F32) return QFP4_ERR_ARG;
     int st = gemm_shape_check(M, N, K, out_dt);
     if (st != QFP4_OK) return st;

@@ -24,8 +24,12 @@
 
 namespace qfp4 {
 
-constexpr int GM_BM = 128, GM_BN = 256, GM_BK = 256;      // tile (elements)
-constexpr int GM_BKB = GM_BK / 2;                         // bytes of one row per stage
+constexpr int GM_BM = 128, GM_BN = 256;                  // tile rows / columns
+constexpr int GM_BKB = 128;                               // bytes of one operand row per stage
+// Element format of the GEMM besides QFP4_MXFP4 / QFP4_NVFP4: MXFP8 (E4M3
+// bytes under E8M0 scales per 32) is QFP4_MXFP8.
+// k-tile length in elements: 128 bytes of a row hold 256 FP4 or 128 FP8 values.
+__host__ __device__ constexpr int gm_bk(int fmt) { return fmt == QFP4_MXFP8 ? 128 : 256; }
 constexpr int GM_STAGES = 4;
 constexpr int GM_A_BYTES = GM_BM * GM_BKB;                // 16 KiB
 constexpr int GM_B_BYTES = GM_BN * GM_BKB;                // 32 KiB
@@ -40,7 +44,7 @@ constexpr uint32_t GM_SF_COL = 256;                       // scale factors after
 constexpr int GM_GROUP_M = 8;                             // tile raster: 8 m-blocks per band
 
 // chunks of 4 scale groups per stage and 128-row block
-__host__ __device__ constexpr int gm_cps(int fmt) { return fmt == QFP4_NVFP4 ? 4 : 2; }
+__host__ __device__ constexpr int gm_cps(int fmt) { return fmt == QFP4_NVFP4 ? 4 : fmt == QFP4_MXFP4 ? 2 : 1; }
 
 struct GemmParams {
     int M, N, K;
@@ -87,7 +91,13 @@ template <int FMT>
 __device__ __forceinline__ void umma_blockscaled(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa,
                                                  uint32_t sfb, uint32_t accumulate)
 {
-    if (FMT == QFP4_NVFP4)
+    if (FMT == QFP4_MXFP8)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+            "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+            : "memory");
+    else if (FMT == QFP4_NVFP4)
         asm volatile(
             "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
             "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
@@ -169,12 +179,14 @@ __device__ __forceinline__ uint64_t desc_sf_chunk(const void *p)
            (static_cast<uint64_t>(1) << 46);
 }
 
-// Instruction descriptor of the block-scaled MMA: E2M1 A and B, K-major,
-// N >> 3 at bit 17, scale format (0 = UE4M3, 1 = UE8M0) at bit 23,
+// Instruction descriptor of the block-scaled MMA: A and B types at bits 7
+// and 10 (E2M1 = 1 for kind::mxf4 / mxf4nvf4; E4M3 = 0 for kind::mxf8f6f4),
+// K-major, N >> 3 at bit 17, scale format (0 = UE4M3, 1 = UE8M0) at bit 23,
 // M >> 4 at bit 24, scale-factor byte selectors at bits 4 (B) and 29 (A).
 __host__ __device__ constexpr uint32_t idesc_blockscaled(int fmt, int M, int N, uint32_t sf_id)
 {
-    return (sf_id << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+    const uint32_t ty = fmt == QFP4_MXFP8 ? 0u : 1u;
+    return (sf_id << 4) | (ty << 7) | (ty << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
            ((fmt == QFP4_NVFP4 ? 0u : 1u) << 23) | (static_cast<uint32_t>(M >> 4) << 24) | (sf_id << 29);
 }
 
@@ -344,12 +356,18 @@ __global__ void __launch_bounds__(GM_THREADS, 1)
                     const uint64_t adesc = desc_k_sw128(stage_a(s));
                     const uint64_t bdesc = desc_k_sw128(stage_b(s));
 #pragma unroll
-                    for (int k = 0; k < GM_BK / 64; ++k) {
+                    for (int k = 0; k < 4; ++k) {       // four MMAs of 64 (FP4) or 32 (FP8) elements
                         uint32_t sfa, sfb, id;
                         if (FMT == QFP4_NVFP4) {
                             sfa = sfa_col + 4 * k;
                             sfb = sfb_col + 8 * k;
                             id = idesc_blockscaled(FMT, GM_BM, GM_BN, 0);
+                        } else if (FMT == QFP4_MXFP8) {
+                            // one chunk per k-tile; MMA k takes byte k (its one block-32 scale)
+                            const uint32_t sel = static_cast<uint32_t>(k);
+                            sfa = sfa_col | (sel << 30);
+                            sfb = sfb_col | (sel << 30);
+                            id = idesc_blockscaled(FMT, GM_BM, GM_BN, sel);
                         } else {
                             const uint32_t sel = 2u * (k & 1);
                             sfa = (sfa_col + 4 * (k >> 1)) | (sel << 30);
@@ -495,17 +513,17 @@ __device__ __forceinline__ void cluster_sync()
 {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-// Arrive on a barrier of the leader CTA, given by its shared::cluster address.
-// The leader's own threads arrive with the default release at CTA scope.  The
-// partner's arrivals cross CTAs, so they release at cluster scope: that orders
-// the partner's completed tensor-memory accesses (tcgen05.wait + fence) before
-// the leader's acquire in the memory model, not only in practice.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr, bool remote)
+// Arrive on a barrier of the leader CTA, given by its shared::cluster address
+// (the partner's arrivals cross CTAs).  Default semantics, release at CTA
+// scope: what an arrival publishes is tensor-memory state whose accesses
+// tcgen05.wait::st / wait::ld already completed in the arriving thread before
+// the arrive issues, and the pair's tcgen05.fence::before / after_thread_sync
+// bracket the hand-off; no generic-memory data crosses CTAs through these
+// barriers.  The cluster-scope release puts a cluster-wide fence in every
+// arrival: it took the 8192 x 11008 x 4096 GEMM from 199 us to 361 us.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
 {
-    if (remote)
-        asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-    else
-        asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 __device__ __forceinline__ void tma_load_2d_cg2(void *smem_dst, const CUtensorMap *map, uint32_t leader_bar, int c0, int c1)
 {
@@ -541,7 +559,13 @@ template <int FMT>
 __device__ __forceinline__ void umma_blockscaled_cg2(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa,
                                                      uint32_t sfb, uint32_t accumulate)
 {
-    if (FMT == QFP4_NVFP4)
+    if (FMT == QFP4_MXFP8)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+            "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+            : "memory");
+    else if (FMT == QFP4_NVFP4)
         asm volatile(
             "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
             "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
@@ -680,17 +704,17 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
         if (leader && lane == 0) {
             int it = 0, ti = 0;
             for (int t = cluster; t < ntiles && !abort_flag; t += nclusters, ++ti) {
-                if (!mbar_wait_cluster(&acc_empty, (ti & 1) ^ 1u)) { abort_flag = 1; break; }
+                if (!mbar_wait(&acc_empty, (ti & 1) ^ 1u)) { abort_flag = 1; break; }
                 tc_fence_after();
                 for (int kt = 0; kt < p.KT; ++kt, ++it) {
                     const int s = it % G2_STAGES, b = it % NBUF;
                     if (!mbar_wait(&full[s], (it / G2_STAGES) & 1u)) { abort_flag = 1; break; }
-                    if (!mbar_wait_cluster(&sf_full[b], (it / NBUF) & 1u)) { abort_flag = 1; break; }
+                    if (!mbar_wait(&sf_full[b], (it / NBUF) & 1u)) { abort_flag = 1; break; }
                     tc_fence_after();
                     const uint64_t adesc = desc_k_sw128(stage_a(s));
                     const uint64_t bdesc = desc_k_sw128(stage_b(s));
 #pragma unroll
-                    for (int k = 0; k < GM_BK / 64; ++k) {
+                    for (int k = 0; k < 4; ++k) {       // four MMAs of 64 (FP4) or 32 (FP8) elements
                         umma_blockscaled_cg2<FMT>(tmem, adesc + 2 * k, bdesc + 2 * k,
                                                   idesc_blockscaled(FMT, G2_BM, G2_BN, 0), buf_a(b) + 4 * k,
                                                   buf_b(b) + 8 * k, (kt | k) != 0);
@@ -766,29 +790,36 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
                 fence_proxy_async();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sfs_empty[s]);
-                // one TMEM word per MMA k (K = 64): NVFP4 uses a whole raw word,
-                // MXFP4 the half of one (its two block-32 scales, in bytes 0-1)
-                auto mma_word = [&](uint32_t raw4, uint32_t raw2, int k) -> uint32_t {
-                    return FMT == QFP4_NVFP4 ? raw4 : (raw2 >> (16 * (k & 1))) & 0xFFFFu;
+                // one TMEM word per MMA k: NVFP4 (K = 64) uses a whole raw word,
+                // MXFP4 (K = 64) the half of one (its two block-32 scales, in
+                // bytes 0-1), MXFP8 (K = 32) one byte (its one block-32 scale)
+                auto mma_word = [&](const uint32_t *raw, int k) -> uint32_t {
+                    if constexpr (FMT == QFP4_NVFP4) return raw[k];
+                    else if constexpr (FMT == QFP4_MXFP4) return (raw[k >> 1] >> (16 * (k & 1))) & 0xFFFFu;
+                    else return (raw[0] >> (8 * k)) & 0xFFu;
                 };
                 uint32_t av[16], bv[32];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    const uint32_t wa = mma_word(ra[k % CPS], ra[k >> 1], k);
+                    const uint32_t wa = mma_word(ra, k);
 #pragma unroll
                     for (int c = 0; c < 4; ++c) av[4 * k + c] = wa;
 #pragma unroll
                     for (int h = 0; h < 2; ++h)
 #pragma unroll
-                        for (int mm = 0; mm < 4; ++mm)
-                            bv[8 * k + 4 * h + mm] = mma_word(rb[h][k % CPS][mm], rb[h][k >> 1][mm], k);
+                        for (int mm = 0; mm < 4; ++mm) {
+                            uint32_t col[CPS];
+#pragma unroll
+                            for (int w = 0; w < CPS; ++w) col[w] = rb[h][w][mm];
+                            bv[8 * k + 4 * h + mm] = mma_word(col, k);
+                        }
                 }
                 tmem_st_x16(buf_a(b) + lane_base, av);
                 tmem_st_x32(buf_b(b) + lane_base, bv);
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&sf_full[b]), 0), !leader);
+                if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&sf_full[b]), 0));
             }
         }
         // the leader's last releases of the scale buffers are multicast into
@@ -822,7 +853,7 @@ __global__ void __launch_bounds__(G2_THREADS, 1)
             // next tile's MMAs overlap these stores
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(acc_empty_leader, !leader);
+            if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
 
             const int col0 = nb * G2_BN + 128 * h + 2 * (lane & 3);
             const int row_base = mb * G2_BM + 128 * static_cast<int>(rank);
@@ -868,7 +899,7 @@ static GemmLayout gemm_layout(int64_t M, int64_t N, int64_t K, qfp4_fmt fmt)
     GemmLayout L;
     L.MB = static_cast<int>((M + GM_BM - 1) / GM_BM);
     L.NT = static_cast<int>((N + GM_BN - 1) / GM_BN);
-    L.KT = static_cast<int>((K + GM_BK - 1) / GM_BK);
+    L.KT = static_cast<int>((K + gm_bk(fmt) - 1) / gm_bk(fmt));
     L.NC = L.KT * gm_cps(fmt);
     L.sfa_bytes = static_cast<size_t>(L.MB) * L.NC * 512;
     L.sfb_bytes = static_cast<size_t>(2 * L.NT) * L.NC * 512;
@@ -886,7 +917,7 @@ size_t gemm_workspace(int64_t M, int64_t N, int64_t K, qfp4_fmt fmt)
 int rearrange_scales(const uint8_t *a_scales, int64_t M, int n_blocks_a, uint8_t *sfa, const uint8_t *b_scales,
                      int64_t N, int n_blocks_b, uint8_t *sfb, int64_t K, qfp4_fmt fmt, int NC, cudaStream_t stream)
 {
-    const int g = fmt == QFP4_MXFP4 ? 32 : 16;
+    const int g = fmt == QFP4_NVFP4 ? 16 : 32;
     const SfJob ja{a_scales, static_cast<int>(M), n_blocks_a, sfa};
     const SfJob jb{b_scales, static_cast<int>(N), n_blocks_b, sfb};
     const dim3 grid((NC + SF_CHUNKS_PER_BLOCK - 1) / SF_CHUNKS_PER_BLOCK, n_blocks_a + n_blocks_b);
@@ -949,17 +980,18 @@ int gemm_core(const uint8_t *A_codes, const uint8_t *sfa, const float *A_tscale,
     const GemmLayout L = gemm_layout(M, N, K, fmt);
     const bool pair = M > GM_BM;
     CUtensorMap ta, tb;
+    const uint64_t row_bytes = static_cast<uint64_t>(fmt == QFP4_MXFP8 ? K : K / 2);
     {
-        const uint64_t dims[2] = {static_cast<uint64_t>(K / 2), static_cast<uint64_t>(M)};
-        const uint64_t strides[1] = {static_cast<uint64_t>(K / 2)};
+        const uint64_t dims[2] = {row_bytes, static_cast<uint64_t>(M)};
+        const uint64_t strides[1] = {row_bytes};
         const uint32_t box[2] = {GM_BKB, GM_BM};
         int st = encode_tensor_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(A_codes), dims,
                                    strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
         if (st != QFP4_OK) return st;
     }
     {
-        const uint64_t dims[2] = {static_cast<uint64_t>(K / 2), static_cast<uint64_t>(N)};
-        const uint64_t strides[1] = {static_cast<uint64_t>(K / 2)};
+        const uint64_t dims[2] = {row_bytes, static_cast<uint64_t>(N)};
+        const uint64_t strides[1] = {row_bytes};
         const uint32_t box[2] = {GM_BKB, static_cast<uint32_t>(pair ? 128 : GM_BN)};
         int st = encode_tensor_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(B_codes), dims,
                                    strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -1001,6 +1033,9 @@ int gemm_core(const uint8_t *A_codes, const uint8_t *sfa, const float *A_tscale,
         }
         const int ntiles = static_cast<int>(((M + G2_BM - 1) / G2_BM) * ((N + G2_BN - 1) / G2_BN));
         const int grid = 2 * imin<int>(ntiles, num_sms() / 2);
+        if (fmt == QFP4_MXFP8)
+            return out_dt == QFP4_F32 ? launch_gemm2<QFP4_MXFP8, QFP4_F32>(ta, tb, tsa, tsb, p, grid, stream)
+                                      : launch_gemm2<QFP4_MXFP8, QFP4_BF16>(ta, tb, tsa, tsb, p, grid, stream);
         if (fmt == QFP4_NVFP4)
             return out_dt == QFP4_F32 ? launch_gemm2<QFP4_NVFP4, QFP4_F32>(ta, tb, tsa, tsb, p, grid, stream)
                                       : launch_gemm2<QFP4_NVFP4, QFP4_BF16>(ta, tb, tsa, tsb, p, grid, stream);
@@ -1008,6 +1043,9 @@ int gemm_core(const uint8_t *A_codes, const uint8_t *sfa, const float *A_tscale,
                                   : launch_gemm2<QFP4_MXFP4, QFP4_BF16>(ta, tb, tsa, tsb, p, grid, stream);
     }
     const int grid = static_cast<int>(imin<int64_t>(static_cast<int64_t>(L.MB) * L.NT, num_sms()));
+    if (fmt == QFP4_MXFP8)
+        return out_dt == QFP4_F32 ? launch_gemm<QFP4_MXFP8, QFP4_F32>(ta, tb, p, grid, stream)
+                                  : launch_gemm<QFP4_MXFP8, QFP4_BF16>(ta, tb, p, grid, stream);
     if (fmt == QFP4_NVFP4)
         return out_dt == QFP4_F32 ? launch_gemm<QFP4_NVFP4, QFP4_F32>(ta, tb, p, grid, stream)
                                   : launch_gemm<QFP4_NVFP4, QFP4_BF16>(ta, tb, p, grid, stream);

@@ -61,7 +61,7 @@ extern "C" int qfp4_gemm_blockscaled_noalloc(const uint8_t *A_codes, const uint8
     // The checks qfp4_gemm_blockscaled makes first (enums, then shape rules
     // including M, N, K < 2^30), so the scratch size below cannot overflow and
     // an invalid call gets the same status from both entry points.
-    if (fmt != QFP4_MXFP4 && fmt != QFP4_NVFP4) return QFP4_ERR_ARG;
+    if (fmt != QFP4_MXFP4 && fmt != QFP4_NVFP4 && fmt != QFP4_MXFP8) return QFP4_ERR_ARG;
     if (out_dt != QFP4_BF16 && out_dt != QFP4_F32) return QFP4_ERR_ARG;
     const int shape = gemm_shape_check(M, N, K, out_dt);
     if (shape != QFP4_OK) return shape;

@@ -7,3 +7,5 @@
 #include "gemm.cu"
 #include "api.cu"
 #include "gemm_noalloc.cu"
+#include "linear.cu"
+#include "calib.cu"

@@ -102,32 +102,15 @@ __device__ __forceinline__ void settle_ns(uint64_t ns)
 }
 constexpr uint64_t kSettleNs = 100000ull;
 
-// The same poll with acquire at cluster scope, for a barrier that threads of
-// the partner CTA arrive on with release at cluster scope.
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
 // Bounded wait: true when the phase completed, false (error recorded) when
 // limit_ns of wall time (or kSpinLimit polls) ran out.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
-template <bool CLUSTER = false>
 __device__ __forceinline__ bool mbar_wait_for(uint64_t *bar, uint32_t parity, uint64_t limit_ns)
 {
-    auto poll = [&] { return CLUSTER ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
-    if (poll()) return true;
+    if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     for (uint32_t i = 0; i < kSpinLimit; ++i) {
-        if (poll()) return true;
+        if (mbar_try_wait(bar, parity)) return true;
         if ((i & 255u) == 255u && global_ns() - t0 > limit_ns) break;
     }
     record_error(DEV_ERR_TIMEOUT);
@@ -135,11 +118,7 @@ __device__ __forceinline__ bool mbar_wait_for(uint64_t *bar, uint32_t parity, ui
 }
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
 {
-    return mbar_wait_for<false>(bar, parity, kWaitLimitNs);
-}
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity)
-{
-    return mbar_wait_for<true>(bar, parity, kWaitLimitNs);
+    return mbar_wait_for(bar, parity, kWaitLimitNs);
 }
 
 // ------------------------------------------------------------------ dependent launches

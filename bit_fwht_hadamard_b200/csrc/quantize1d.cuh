@@ -8,7 +8,7 @@ enum { MODE_AMAX = 0, MODE_QUANT = 1 };
 
 // Element format of the 1D kernels besides QFP4_MXFP4 / QFP4_NVFP4: MXFP8
 // (E4M3 elements, E8M0 scale per 32), row-wise.
-constexpr int FMT_MXFP8 = 2;
+constexpr int FMT_MXFP8 = QFP4_MXFP8;
 
 // Upper bound on the number of partial tensor maxima a pass writes.
 constexpr int kMaxPartials = 1024;

@@ -739,4 +739,24 @@ int quantize_mxfp8(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_rou
     return QFP4_OK;
 }
 
+// MXFP8 column-wise output alone (groups of 32 along M, K x M codes): the
+// transposed operands of the FP8 backward GEMMs.  Needs M % 32 == 0.
+int quantize_mxfp8_columns(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_round rounding, uint64_t seed,
+                           uint8_t *codesT, uint8_t *scalesT, cudaStream_t stream)
+{
+    Q2DParams p{M, K, nullptr, nullptr, codesT, scalesT, nullptr, 0, nullptr, seed, QFP4_SCALE_DEFAULT, nullptr};
+    const bool sr = rounding == QFP4_SR;
+    if (xdt == QFP4_BF16) {
+        const int64_t tasks4 = ((M + 31) / 32) * ((K + 127) / 128);
+        if (sr) launch_tiles<k_cols4<FMT_MXFP8, true, false>, uint16_t>(tasks4, x, p, stream);
+        else launch_tiles<k_cols4<FMT_MXFP8, false, false>, uint16_t>(tasks4, x, p, stream);
+    } else {
+        const int64_t tasks = ((M + 31) / 32) * (K / 32);
+        if (sr) launch_tiles<k_mxfp8<true, false, true, float>, float>(tasks, x, p, stream);
+        else launch_tiles<k_mxfp8<false, false, true, float>, float>(tasks, x, p, stream);
+    }
+    QFP4_LAUNCH_CHECK();
+    return QFP4_OK;
+}
+
 }  // namespace qfp4

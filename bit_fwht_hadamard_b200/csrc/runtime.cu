@@ -85,7 +85,7 @@ __global__ void k_wait_timeout(uint64_t limit_ns)
     if (threadIdx.x != 0) return;
     qfp4::mbar_init(&bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    (void)qfp4::mbar_wait_for<false>(&bar, 0, limit_ns);
+    (void)qfp4::mbar_wait_for(&bar, 0, limit_ns);
 }
 
 extern "C" int qfp4_selftest_wait_timeout(int64_t limit_us, qfp4_stream_t stream)

@@ -48,7 +48,12 @@ extern "C" {
 
 typedef struct CUstream_st *qfp4_stream_t;   /* == cudaStream_t */
 
-typedef enum { QFP4_MXFP4 = 0, QFP4_NVFP4 = 1 } qfp4_fmt;
+typedef enum {
+    QFP4_MXFP4 = 0,             /* E2M1 elements, E8M0 scale per 32                          */
+    QFP4_NVFP4 = 1,             /* E2M1 elements, E4M3 scale per 16, fp32 tensor scale       */
+    QFP4_MXFP8 = 2              /* E4M3 elements (one byte each), E8M0 scale per 32, as
+                                   qfp4_quantize_mxfp8 writes them: GEMM operands only       */
+} qfp4_fmt;
 typedef enum { QFP4_RNE = 0, QFP4_SR = 1 } qfp4_round;
 typedef enum { QFP4_BF16 = 0, QFP4_F32 = 1 } qfp4_dtype;
 typedef enum {
@@ -224,12 +229,15 @@ int qfp4_dequantize(const uint8_t *codes, const uint8_t *scales, const float *ts
 /* ------------------------------------------------------------------------
  * qfp4_gemm_blockscaled -- Y = deq(A) * deq(B)^T ([QN] §QuTLASS: MXFP4 /
  * NVFP4 operands, FP32 accumulation; [LB] §FP4: Blackwell FP4 tensor
- * cores).  A is M x K and B is N x K, both K-major (codes + scales exactly
- * as qfp4_quantize writes them); for NVFP4 the tensor scales multiply the
- * accumulated sum: Y = acc * (s_tA * s_tB) (A_tscale, B_tscale device
- * pointers; ignored for MXFP4).  out: M x N row-major, binary32 or bf16
- * (round to nearest even).  Runs on 5th-generation tensor cores (tcgen05
- * block-scaled MMA, fp32 accumulators in tensor memory).
+ * cores; [QN] forward/backward split and [TI]: MXFP8 operands for the FP8
+ * backward and the Q/K projections).  A is M x K and B is N x K, both
+ * K-major (codes + scales exactly as qfp4_quantize writes them, or for
+ * fmt = QFP4_MXFP8 as qfp4_quantize_mxfp8 writes them); for NVFP4 the
+ * tensor scales multiply the accumulated sum: Y = acc * (s_tA * s_tB)
+ * (A_tscale, B_tscale device pointers; ignored for MXFP4 and MXFP8).  out:
+ * M x N row-major, binary32 or bf16 (round to nearest even).  Runs on
+ * 5th-generation tensor cores (tcgen05 block-scaled MMA: kind::mxf4,
+ * kind::mxf4nvf4 or kind::mxf8f6f4; fp32 accumulators in tensor memory).
  * workspace: device scratch of at least qfp4_gemm_workspace_bytes(M, N, K,
  *   fmt) bytes; it receives the scales rearranged for the tensor cores
  *   (contents on entry do not matter, the call overwrites them).
@@ -295,6 +303,81 @@ int qfp4_gemm_fused_rq(const void *A_bf16, int64_t M, int64_t K, int rotate, int
  * QFP4_ERR_SHAPE for a negative dimension. */
 int qfp4_gemm_fused_rq_workspace_layout(int64_t M, int64_t N, int64_t K, qfp4_fmt fmt, size_t *codes_off,
                                         size_t *scales_off, size_t *tscale_off);
+
+/* ------------------------------------------------------------------------
+ * qfp4_linear_forward -- the forward of a Quartet-style linear layer,
+ * Y = X W^T computed as Q(X H) Q(W H)^T ([QN] Hadamard rotation: y = xW^T =
+ * (xH)(WH)^T with H orthogonal, so the rotation cancels; FP4 forward).
+ *   X  M x K bf16 activations, W  N x K bf16 weights (out x in features),
+ *      both row-major device memory, rotated along K in 128-blocks and
+ *      quantized (fmt = QFP4_MXFP4 or QFP4_NVFP4, RNE, four6 for NVFP4) as
+ *      qfp4_quantize does; Y  M x N, out_dt binary32 or bf16.
+ *   workspace: qfp4_linear_forward_workspace_bytes(M, N, K, fmt) bytes of
+ *      device scratch (the quantized operands and the GEMM's scale chunks).
+ * Needs K % 128 == 0, N % 4 (binary32 out) or N % 8 (bf16 out).  Errors as
+ * qfp4_quantize and qfp4_gemm_blockscaled.
+ * ---------------------------------------------------------------------- */
+size_t qfp4_linear_forward_workspace_bytes(int64_t M, int64_t N, int64_t K, qfp4_fmt fmt);
+
+int qfp4_linear_forward(const void *X, const void *W, int64_t M, int64_t N, int64_t K, qfp4_fmt fmt, int four6,
+                        qfp4_dtype out_dt, void *Y, void *workspace, size_t workspace_bytes, qfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * qfp4_linear_backward -- the backward of the same layer from the output
+ * gradient G: dX = G W (M x K) and dW = G^T X (N x K), with the gradient
+ * stochastically rounded (Philox keyed on seed and G's element index) and
+ * each operand quantized once for both of its uses ([QN] forward/backward
+ * split: FP4 or FP8 backward; [TI] transposition-invariant 2D blocks, MXFP8
+ * operands):
+ *   fmt = QFP4_NVFP4: G, W and X in 2D 16 x 16 NVFP4 blocks (G by SR, W and X
+ *     by RNE), each pass emitting the operand and its transpose;
+ *   fmt = QFP4_MXFP8: G as MXFP8 rows (groups along N) and columns (along M)
+ *     by SR, W and X as MXFP8 columns by RNE.
+ *   dX = GEMM(A = G, B = W^T) and dW = GEMM(A = G^T, B = X^T) on the
+ *   block-scaled tensor cores.
+ *   G  M x N, X  M x K, W  N x K bf16; dX  M x K and dW  N x K out_dt; either
+ *   output may be NULL to skip it (X or W is then not read).
+ *   workspace: qfp4_linear_backward_workspace_bytes(M, N, K, fmt) bytes.
+ * Needs M % 32 == 0, N % 32 == 0, K % 16 (NVFP4) or K % 32 (MXFP8) == 0.
+ * ---------------------------------------------------------------------- */
+size_t qfp4_linear_backward_workspace_bytes(int64_t M, int64_t N, int64_t K, qfp4_fmt fmt);
+
+int qfp4_linear_backward(const void *G, const void *X, const void *W, int64_t M, int64_t N, int64_t K,
+                         qfp4_fmt fmt, uint64_t seed, qfp4_dtype out_dt, void *dX, void *dW,
+                         void *workspace, size_t workspace_bytes, qfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * qfp4_kl_calibrate -- KL-divergence clip point of an activation tensor
+ * ([LB] §5, the TensorRT method): for each candidate clip T, P = the
+ * histogram of |x| cut at T with the tail counted in the last kept bin, Q =
+ * the kept histogram quantized to the levels and spread back over P's
+ * nonzero bins; the T with the least D_KL(P || Q) is the clip point.
+ *   x         n elements (bf16 or binary32), device memory.
+ *   bins      histogram bins over [0, amax] (8 .. 8192); bin of |x| =
+ *             min(bins-1, trunc(fl(|x| * fl(bins / amax)))).
+ *   grid      0: `levels` uniform levels (2 .. bins; a bin b of the i kept
+ *             ones is in level floor(b / floor(i / levels)), the last level
+ *             taking the remainder), candidates i = levels .. bins;
+ *             1: the E2M1 magnitudes scaled so T maps to 6 (a bin goes to the
+ *             magnitude nearest its centre, ties to the even code; `levels`
+ *             is ignored), candidates i = 8 .. bins.
+ *   KL in binary64 (p, q normalised; a bin with P > 0 and Q = 0 rejects the
+ *   candidate); the least KL wins, the smallest i on a tie; all rejected
+ *   keeps every bin.  T = fl(i * fl(amax / bins)).
+ *   clip_out       device float, receives T (for example as the amax_in of
+ *                  qfp4_quantize_ex, or S = T / 6 for a per-tensor scale).
+ *   best_bins_out  device int (or NULL): the winning i.
+ *   kl_out         device double[bins - first + 1] (or NULL): every KL.
+ *   hist_out       device uint64[bins] (or NULL): the histogram.
+ *   workspace      qfp4_kl_calibrate_workspace_bytes(bins, levels, grid).
+ * Errors: QFP4_ERR_ARG for bins, levels or grid out of range, a NULL x
+ * (n > 0) or clip_out, a short workspace.
+ * ---------------------------------------------------------------------- */
+size_t qfp4_kl_calibrate_workspace_bytes(int bins, int levels, int grid);
+
+int qfp4_kl_calibrate(const void *x, qfp4_dtype xdt, int64_t n, int bins, int levels, int grid,
+                      float *clip_out, int *best_bins_out, double *kl_out, uint64_t *hist_out,
+                      void *workspace, size_t workspace_bytes, qfp4_stream_t stream);
 
 /* Human-readable text of a status code (static storage). */
 const char *qfp4_status_string(int status);

@@ -88,6 +88,14 @@ def lib():
         L.or_tensor_amax.argtypes = [c_void_p, c_int, c_int64, c_int64, c_int]
         L.or_mxfp4_group.restype = c_int
         L.or_mxfp4_group.argtypes = [c_void_p, c_void_p, c_int, c_int, c_int, c_uint64, c_void_p, c_void_p]
+        L.or_abs_histogram.restype = c_int
+        L.or_abs_histogram.argtypes = [c_void_p, c_int, c_int64, c_int, c_float, c_void_p]
+        L.or_e2m1_level_of_bin.restype = c_int
+        L.or_e2m1_level_of_bin.argtypes = [c_int64, c_int64]
+        L.or_kl_calibrate.restype = c_int
+        L.or_kl_calibrate.argtypes = [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p]
+        L.or_kl_threshold.restype = c_float
+        L.or_kl_threshold.argtypes = [c_float, c_int, c_int]
         L.or_four6_pick.restype = c_int
         L.or_four6_pick.argtypes = [c_void_p, c_float, c_void_p, c_void_p]
         L.or_quantize_mxfp8.restype = c_int
@@ -371,3 +379,31 @@ def f64_to_bf16_array(v: np.ndarray) -> np.ndarray:
     L = lib()
     flat = np.asarray(v, np.float64).ravel()
     return np.array([L.or_f64_to_bf16(float(t)) for t in flat], np.uint16).reshape(np.shape(v))
+
+
+# ---------------------------------------------------------------- KL calibration
+def abs_histogram(x: np.ndarray, bins: int, amax: float) -> np.ndarray:
+    x = np.ascontiguousarray(x)
+    h = np.zeros(bins, np.uint64)
+    _check(lib().or_abs_histogram(_p(x), _xdt(x), x.size, bins, amax, _p(h)))
+    return h
+
+
+def e2m1_level_of_bin(b: int, i: int) -> int:
+    return lib().or_e2m1_level_of_bin(b, i)
+
+
+def kl_calibrate(hist: np.ndarray, levels: int = 8, grid: int = 0):
+    """(best i, kl array over candidates first .. bins)."""
+    hist = np.ascontiguousarray(hist, np.uint64)
+    bins = hist.size
+    first = 8 if grid else levels
+    kl = np.zeros(bins - first + 1, np.float64)
+    best = np.zeros(1, np.int32)
+    _check(lib().or_kl_calibrate(_p(hist), bins, levels, grid, _p(kl), _p(best)))
+    return int(best[0]), kl
+
+
+def kl_threshold(amax: float, bins: int, i: int) -> float:
+    return float(np.float32(lib().or_kl_threshold(amax, bins, i)))
+

@@ -808,3 +808,124 @@ int or_gemm_sampled(const uint8_t *A_codes, const uint8_t *A_scales, const float
     }
     return OR_OK;
 }
+
+/* ========================================================================
+ * KL-divergence clip calibration ([LB] §5, the TensorRT method the page
+ * describes): for each candidate clip point T, P = the histogram of |x|
+ * cut at T with everything beyond T counted in the last kept bin, and Q =
+ * the kept histogram quantized to the quantizer's levels and spread back
+ * over P's bins; the T with the least D_KL(P || Q) loses the least
+ * information.  Readings (the page gives the idea, not the arithmetic):
+ *   - histogram: `bins` bins over [0, amax] of the tensor; bin of |x| =
+ *     min(bins - 1, trunc(fl(|x| * fl(bins / amax)))) in binary32;
+ *   - candidates: i = first .. bins kept bins, T_i = fl(i * fl(amax / bins));
+ *     first = levels (uniform) or 8 (E2M1);
+ *   - levels: grid 0 = `levels` uniform levels, kept bin b in level
+ *     floor(b / floor(i / levels)), the last level taking the remainder;
+ *     grid 1 = the 8 E2M1 magnitudes {0,.5,1,1.5,2,3,4,6} scaled so that T
+ *     maps to 6: bin b goes to the nearest magnitude of its centre,
+ *     6 (b + 1/2) / i, ties to the even mantissa (decided exactly);
+ *   - Q: each level's kept mass divided evenly among its bins where P != 0;
+ *   - KL = sum over P > 0 of p log(p / q) with p, q normalised, binary64,
+ *     bins in ascending order; a bin with P > 0 and Q = 0 makes the
+ *     candidate's KL +infinity (rejected);
+ *   - the least KL wins, the smallest i on a tie.
+ * ====================================================================== */
+int or_abs_histogram(const void *x, int xdt, int64_t n, int bins, float amax, uint64_t *hist)
+{
+    if (n < 0 || bins < 1 || !(amax >= 0.0f)) return OR_ERR_ARG;
+    memset(hist, 0, sizeof(uint64_t) * (size_t)bins);
+    if (amax == 0.0f) {                            /* all zeros: everything in bin 0 */
+        hist[0] = (uint64_t)n;
+        return OR_OK;
+    }
+    float inv = (float)bins / amax;
+    for (int64_t e = 0; e < n; ++e) {
+        float t = fabsf(load_elem(x, xdt, e)) * inv;
+        int64_t b = (int64_t)t;                    /* truncation toward zero */
+        if (b > bins - 1) b = bins - 1;
+        hist[b] += 1;
+    }
+    return OR_OK;
+}
+
+/* E2M1 magnitude index (0..7) nearest to 6 (2b + 1) / (2i), ties to the even
+ * mantissa: compared as integers against the midpoints m = 0.25, 0.75, 1.25,
+ * 1.75, 2.5, 3.5, 5 (scaled by 8: 2, 6, 10, 14, 20, 28, 40): v < m iff
+ * 24 (2b + 1) < 8 m i. */
+int or_e2m1_level_of_bin(int64_t b, int64_t i)
+{
+    static const int64_t mid8[7] = {2, 6, 10, 14, 20, 28, 40};
+    int64_t num = 24 * (2 * b + 1);                /* 8 * 6 (2b + 1) / 2, over i */
+    int level = 0;
+    for (int t = 0; t < 7; ++t) {
+        int64_t rhs = mid8[t] * i;
+        if (num > rhs) level = t + 1;
+        else if (num == rhs) { level = ((t + 1) & 1) ? t : t + 1; break; }   /* tie: even code */
+        else break;
+    }
+    return level;
+}
+
+static double kl_for_candidate(const uint64_t *hist, int bins, int i, int levels, int grid, int *level_of, double *qmass,
+                               int64_t *nz)
+{
+    int L = grid ? 8 : levels;
+    int per = grid ? 0 : i / levels;
+    for (int l = 0; l < L; ++l) { qmass[l] = 0.0; nz[l] = 0; }
+    uint64_t outliers = 0;
+    for (int b = i; b < bins; ++b) outliers += hist[b];
+    double total_p = 0.0;
+    for (int b = 0; b < i; ++b) {
+        int l = grid ? or_e2m1_level_of_bin(b, i) : (b / per < levels ? b / per : levels - 1);
+        level_of[b] = l;
+        qmass[l] += (double)hist[b];
+        double pb = (double)hist[b] + (b == i - 1 ? (double)outliers : 0.0);
+        if (pb != 0.0) nz[l] += 1;
+        total_p += pb;
+    }
+    double total_q = 0.0;
+    for (int l = 0; l < L; ++l) total_q += qmass[l];
+    if (total_p == 0.0) return 0.0;
+    if (total_q == 0.0) return INFINITY;
+    double kl = 0.0;
+    for (int b = 0; b < i; ++b) {
+        double pb = (double)hist[b] + (b == i - 1 ? (double)outliers : 0.0);
+        if (pb == 0.0) continue;
+        int l = level_of[b];
+        double qb = nz[l] ? qmass[l] / (double)nz[l] : 0.0;
+        if (qb == 0.0) return INFINITY;
+        double p = pb / total_p, q = qb / total_q;
+        kl += p * log(p / q);
+    }
+    return kl;
+}
+
+int or_kl_calibrate(const uint64_t *hist, int bins, int levels, int grid, double *kl, int *best_i)
+{
+    if (bins < 8 || (grid != 0 && grid != 1)) return OR_ERR_ARG;
+    if (!grid && (levels < 2 || levels > bins)) return OR_ERR_ARG;
+    int first = grid ? 8 : levels;
+    int *level_of = (int *)malloc(sizeof(int) * (size_t)bins);
+    double qmass[4096 + 8];
+    int64_t nz[4096 + 8];
+    if (!level_of || (!grid && levels > 4096)) { free(level_of); return OR_ERR_ARG; }
+    int best = bins;
+    double best_kl = INFINITY;
+    for (int i = first; i <= bins; ++i) {
+        double d = kl_for_candidate(hist, bins, i, levels, grid, level_of, qmass, nz);
+        if (kl) kl[i - first] = d;
+        if (d < best_kl) { best_kl = d; best = i; }
+    }
+    free(level_of);
+    *best_i = best;
+    return OR_OK;
+}
+
+/* the clip point of candidate i: T = fl(i * fl(amax / bins)) */
+float or_kl_threshold(float amax, int bins, int i)
+{
+    float w = amax / (float)bins;
+    return (float)i * w;
+}
+

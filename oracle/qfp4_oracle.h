@@ -135,6 +135,17 @@ int or_gemm_sampled(const uint8_t *A_codes, const uint8_t *A_scales, const float
                     const int64_t *rows, const int64_t *cols, int64_t n_out,
                     double *out, double *absmag);
 
+/* ---- KL-divergence clip calibration ([LB] §5) ------------------------- */
+/* histogram of |x| over [0, amax] in `bins` bins (see the .c for the bin rule) */
+int or_abs_histogram(const void *x, int xdt, int64_t n, int bins, float amax, uint64_t *hist);
+/* E2M1 magnitude index nearest to bin b's centre when i kept bins map to [0, 6] */
+int or_e2m1_level_of_bin(int64_t b, int64_t i);
+/* KL for every candidate i = first .. bins (kl[i - first], may be NULL) and
+ * the winning i; grid 0: `levels` uniform levels (first = levels), grid 1:
+ * the E2M1 magnitudes (first = 8). */
+int or_kl_calibrate(const uint64_t *hist, int bins, int levels, int grid, double *kl, int *best_i);
+float or_kl_threshold(float amax, int bins, int i);
+
 #ifdef __cplusplus
 }
 #endif

@@ -179,3 +179,17 @@ def cfg5_A(M: int, K: int, seed: int = 1005) -> np.ndarray:
 
 def cfg5_B(N: int, K: int, seed: int = 1005) -> np.ndarray:
     return gaussian_bf16(N, K, seed, 1.0, 40)
+
+
+def relu_activation(M: int, K: int, seed: int = 1006) -> np.ndarray:
+    """bf16 ReLU-like activation: max(0, z1 + 0.3 * t3), z1 ~ N(0,1) and t3 a
+    Student-t(3) draw (z2 / sqrt(chi2_3 / 3)), so most mass sits near zero and
+    a thin tail reaches far out (the activation shape of the low-bit blog's
+    KL clipping section)."""
+    n = M * K
+    z = normal(n, seed, 0)
+    zz = normal(n, seed, 1)
+    c = normal(3 * n, seed, 2).reshape(3, n)
+    t3 = zz / np.sqrt((c * c).sum(0) / 3.0)
+    return to_bf16(np.maximum(0.0, z + 0.3 * t3), (M, K))
+

@@ -111,3 +111,15 @@ def test_quantize_ex_argument_errors():
     assert call(q.MXFP4, four6=1, T=True) == q.ERR_UNSUPPORTED          # MXFP4 four-over-six: rows only
     assert call(q.NVFP4, amax_out=f) == q.ERR_ARG                        # own amax needs the workspace
     assert call(q.MXFP4, block2d=1, M=48) == q.ERR_SHAPE
+
+
+def test_kl_calibrate_argument_errors():
+    f = 1 << 20
+    C = q.qfp4_kl_calibrate
+    assert C(f, q.BF16, 64, 4, 2, 0, f, None, None, None, f, 1 << 20, None) == q.ERR_ARG        # bins < 8
+    assert C(f, q.BF16, 64, 9000, 8, 0, f, None, None, None, f, 1 << 20, None) == q.ERR_ARG     # bins > 8192
+    assert C(f, q.BF16, 64, 64, 65, 0, f, None, None, None, f, 1 << 20, None) == q.ERR_ARG      # levels > bins
+    assert C(f, q.BF16, 64, 64, 8, 2, f, None, None, None, f, 1 << 20, None) == q.ERR_ARG       # grid
+    assert C(f, q.BF16, 64, 64, 8, 0, None, None, None, None, f, 1 << 20, None) == q.ERR_ARG    # no clip output
+    assert C(f, q.BF16, 64, 64, 8, 0, f, None, None, None, f, 16, None) == q.ERR_ARG            # short workspace
+    assert q.qfp4_kl_calibrate_workspace_bytes(2048, 8, 0) > 2048 * 8

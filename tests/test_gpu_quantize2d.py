@@ -9,7 +9,7 @@ import torch
 import bit_fwht_hadamard_b200 as q
 import oracle
 import synth
-import gpu_util as G
+import gpu_util as GU
 from gpu_util import (blocks_to_rows, blocks_to_tiles, encode_input, host, mismatch_report, nvfp4_boundary_blocks,
                       to_dev)
 
@@ -30,7 +30,7 @@ def _cmp(got, ref, keys=("codes", "scales", "codesT", "scalesT", "tscale")):
 @pytest.mark.parametrize("transposed", [False, True], ids=["x", "x+xT"])
 def test_2d_matches_oracle(M, K, rounding, transposed):
     x = synth.cfg4_G(M, K, seed=M + K)
-    got = G.quantize(to_dev(x), q.NVFP4, rounding, block2d=True, seed=1004, transposed=transposed)
+    got = GU.quantize(to_dev(x), q.NVFP4, rounding, block2d=True, seed=1004, transposed=transposed)
     ref = oracle.quantize(x, oracle.NVFP4, rounding, block2d=True, seed=1004, transposed=transposed)
     _cmp(got, ref)
     if transposed:                                   # X^T codes are exactly the transpose of X's
@@ -46,7 +46,7 @@ def test_2d_matches_oracle(M, K, rounding, transposed):
 def test_2d_float32_input():
     x = synth.bf16_bits_to_f32(synth.cfg4_G(64, 96, seed=5))
     for rounding in (q.RNE, q.SR):
-        _cmp(G.quantize(to_dev(x), q.NVFP4, rounding, block2d=True, seed=3, transposed=True),
+        _cmp(GU.quantize(to_dev(x), q.NVFP4, rounding, block2d=True, seed=3, transposed=True),
              oracle.quantize(x, oracle.NVFP4, rounding, block2d=True, seed=3, transposed=True))
 
 
@@ -54,7 +54,7 @@ def test_2d_full_size_gradient_sr():
     """G bf16 8192 x 4096 ~ N(0, 1e-3^2) with 0.1% entries x100: 2D 16x16 NVFP4 + Philox SR (seed 1004),
     G and G^T operands from one pass."""
     g = synth.cfg4_G()
-    got = G.quantize(to_dev(g), q.NVFP4, q.SR, block2d=True, seed=1004, transposed=True)
+    got = GU.quantize(to_dev(g), q.NVFP4, q.SR, block2d=True, seed=1004, transposed=True)
     ref = oracle.quantize(g, oracle.NVFP4, oracle.SR, block2d=True, seed=1004, transposed=True)
     _cmp(got, ref)
 
@@ -66,7 +66,7 @@ def test_2d_rounding_boundaries(kind):
     midpoints: X and X^T codes and scales bit-exact."""
     x = encode_input(blocks_to_tiles(nvfp4_boundary_blocks(kind)), kind)
     for transposed in (False, True):
-        got = G.quantize(to_dev(x), q.NVFP4, q.RNE, block2d=True, transposed=transposed)
+        got = GU.quantize(to_dev(x), q.NVFP4, q.RNE, block2d=True, transposed=transposed)
         ref = oracle.quantize(x, oracle.NVFP4, oracle.RNE, block2d=True, transposed=transposed)
         _cmp(got, ref)
 
@@ -81,7 +81,7 @@ def test_1d_columnwise_matches_oracle(M, K, fmt, mode):
         pytest.skip("shape / option not valid for this format")
     x = synth.cfg2_X(M, K, seed=M * 7 + K)
     rounding = q.SR if mode == "sr" else q.RNE
-    got = G.quantize(to_dev(x), fmt[0], rounding, four6=(mode == "four6"), seed=99, transposed=True)
+    got = GU.quantize(to_dev(x), fmt[0], rounding, four6=(mode == "four6"), seed=99, transposed=True)
     ref = oracle.quantize(x, fmt[1], rounding, four6=(mode == "four6"), seed=99, transposed=True)
     _cmp(got, ref)
 
@@ -95,7 +95,7 @@ def test_columnwise_rounding_boundaries(kind, four6):
     padded = np.zeros((R, rows.shape[1]))
     padded[:rows.shape[0]] = rows
     x = encode_input(np.ascontiguousarray(padded.T), kind)        # (128, R), blocks along M
-    got = G.quantize(to_dev(x), q.NVFP4, q.RNE, four6=four6, transposed=True)
+    got = GU.quantize(to_dev(x), q.NVFP4, q.RNE, four6=four6, transposed=True)
     ref = oracle.quantize(x, oracle.NVFP4, oracle.RNE, four6=four6, transposed=True)
     _cmp(got, ref)
 
@@ -108,7 +108,7 @@ def test_mxfp8_matches_oracle(M, K, rounding, transposed):
     if transposed and M % 32:
         pytest.skip("column output needs M % 32 == 0")
     x = synth.cfg4_G(M, K, seed=M + 3 * K)
-    got = G.quantize_mxfp8(to_dev(x), rounding, seed=1004, transposed=transposed)
+    got = GU.quantize_mxfp8(to_dev(x), rounding, seed=1004, transposed=transposed)
     ref = oracle.quantize_mxfp8(x, rounding, seed=1004, transposed=transposed)
     _cmp(got, ref)
 
@@ -116,7 +116,7 @@ def test_mxfp8_matches_oracle(M, K, rounding, transposed):
 def test_mxfp8_full_size_gradient():
     g = synth.cfg4_G()
     for rounding in (q.RNE, q.SR):
-        got = G.quantize_mxfp8(to_dev(g), rounding, seed=1004, transposed=True)
+        got = GU.quantize_mxfp8(to_dev(g), rounding, seed=1004, transposed=True)
         ref = oracle.quantize_mxfp8(g, rounding, seed=1004, transposed=True)
         _cmp(got, ref)
 
@@ -133,9 +133,9 @@ def test_backward_gemms_on_2d_operands():
     qg = oracle.quantize(G, oracle.NVFP4, oracle.SR, block2d=True, seed=1004, transposed=True)
     qw = oracle.quantize(W, oracle.NVFP4, oracle.RNE, block2d=True, transposed=True)
     qx = oracle.quantize(X, oracle.NVFP4, oracle.RNE, block2d=True, transposed=True)
-    dg = G.quantize(to_dev(G), q.NVFP4, q.SR, block2d=True, seed=1004, transposed=True)
-    dw = G.quantize(to_dev(W), q.NVFP4, q.RNE, block2d=True, transposed=True)
-    dx = G.quantize(to_dev(X), q.NVFP4, q.RNE, block2d=True, transposed=True)
+    dg = GU.quantize(to_dev(G), q.NVFP4, q.SR, block2d=True, seed=1004, transposed=True)
+    dw = GU.quantize(to_dev(W), q.NVFP4, q.RNE, block2d=True, transposed=True)
+    dx = GU.quantize(to_dev(X), q.NVFP4, q.RNE, block2d=True, transposed=True)
     for got, ref in ((dg, qg), (dw, qw), (dx, qx)):
         _cmp(got, ref)
 
@@ -149,7 +149,7 @@ def test_backward_gemms_on_2d_operands():
 
     for (A, B, rA, rB, M, N, K) in ((op(dg, False), op(dw, True), rop(qg, False), rop(qw, True), T, I, O),
                                     (op(dg, True), op(dx, True), rop(qg, True), rop(qx, True), O, I, T)):
-        y = host(G.gemm(A, B, M, N, K, q.NVFP4))
+        y = host(GU.gemm(A, B, M, N, K, q.NVFP4))
         r, c = np.meshgrid(np.arange(M), np.arange(N), indexing="ij")
         ref, mag = oracle.gemm_sampled(rA, rB, M, N, K, oracle.NVFP4, r.ravel(), c.ravel())
         err = np.abs(y[r.ravel(), c.ravel()] - ref)
