@@ -10,8 +10,12 @@ with Philox stochastic rounding (seed 7).  value = algorithmic bytes moved
 Also reported: the roofline of the dominant kernel (live CUDA-event
 durations, measured HBM peak), the block-scaled FP4 GEMM of the NVFP4
 forward linear (8192 x 11008 x 4096) in TFLOP/s against the dense FP4 peak,
-the end-to-end figure through host buffers, SM clocks sampled during the
-timed region, and the CPU oracle on the host cores.
+the largest configuration's calls (`largest_config`: the 2^30-element
+quantize, FWHT + MXFP4 and NVFP4 under a given amax, and the fused rotate +
+quantize + GEMM at 16384 x 14336 x 4096), the end-to-end figure through host
+buffers, SM clocks sampled during the timed region, and the CPU oracle on
+the host cores (single-threaded and row-partitioned over every core, plus
+the binary64 oracle GEMM on a sub-problem, extrapolated by flops).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 Under torchrun (N > 1) every rank runs the same per-GPU workload (weak
@@ -53,6 +57,7 @@ def parse():
     ap.add_argument("--impl", default="libqfp4", choices=["libqfp4", "reference"])
     ap.add_argument("--no-gemm", action="store_true", help="skip the GEMM sub-measurement")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--no-cfg5", action="store_true", help="skip the largest-configuration sub-measurements")
     ap.add_argument("--profile-case", choices=["quant", "gemm", "quant-nvfp4", "backward"], default=None,
                     help="run a few untimed calls of one kernel family (for ncu captures) and exit")
     ap.add_argument("--rows", nargs="?", const="", default=None, metavar="FILTER",
@@ -155,29 +160,32 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ reference arm (CPU oracle)
 def run_reference(args, rank, world):
+    """The oracle as it stands on the machine's host cores: each step is the
+    default step (FWHT + MXFP4, RNE then SR seed 7) on a bounded sample of X,
+    rows 0..1023, row-partitioned over every core."""
     if rank != 0:
         return
     import oracle
     import synth
-    rows = 512                                           # bounded sample: 512 of the 4096 rows per step
+    rows = 1024
     x = synth.cfg2_X()[:rows].copy()
     n = rows * K2
+    cores = os.cpu_count() or 1
     for _ in range(args.warmup):
-        oracle.quantize(x, oracle.MXFP4, oracle.RNE, rotate=True)
-        oracle.quantize(x, oracle.MXFP4, oracle.SR, rotate=True, seed=7)
+        _oracle_step_parallel(oracle, x, cores)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle.quantize(x, oracle.MXFP4, oracle.RNE, rotate=True)
-        oracle.quantize(x, oracle.MXFP4, oracle.SR, rotate=True, seed=7)
+        _oracle_step_parallel(oracle, x, cores)
     dt = (time.perf_counter() - t0) / max(args.steps, 1)
     gbs = 2 * n * BYTES_PER_ELEM_MXFP4 / dt / 1e9
-    sample = f"rows 0..{rows - 1} of X (4096 x 4096 bf16), RNE + SR per step, single-threaded C oracle"
+    sample = (f"rows 0..{rows - 1} of X (4096 x 4096 bf16), RNE + SR per step, the C oracle row-partitioned over "
+              f"{cores} threads")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": workload_config(),
-        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }))
 
@@ -190,16 +198,62 @@ def workload_config():
 
 
 # ------------------------------------------------------------------ CPU baseline (oracle on the host)
+def _oracle_step_parallel(oracle, x, threads):
+    """The default step (FWHT + MXFP4, RNE then SR seed 7) by the oracle on
+    row slices in `threads` threads (its ctypes calls release the GIL); each
+    slice passes its first row so the random words stay keyed on the whole
+    tensor's element index, which reassembles the single-threaded result."""
+    from concurrent.futures import ThreadPoolExecutor
+    M = x.shape[0]
+    step = -(-M // (4 * threads))
+    slices = [(a, min(M, a + step)) for a in range(0, M, step)]
+    out = []
+    with ThreadPoolExecutor(threads) as ex:
+        for rounding, seed in ((oracle.RNE, 0), (oracle.SR, 7)):
+            parts = list(ex.map(lambda s: oracle.quantize_ex(x[s[0]:s[1]], oracle.MXFP4, rounding, rotate=True,
+                                                             seed=seed, row0=s[0]), slices))
+            out.append({k: np.concatenate([p[k] for p in parts]) for k in ("codes", "scales")})
+    return out
+
+
 def cpu_baseline():
+    """The oracle on the host cores: one full default step single-threaded,
+    the same step row-partitioned over every core (checked identical), and
+    the binary64 oracle GEMM on a 128 x 128 x 4096 sub-problem, extrapolated
+    by flops to the 8192 x 11008 x 4096 GEMM."""
     import oracle
     import synth
     x = synth.cfg2_X()
+    nproc = os.cpu_count() or 1
+    step_bytes = 2 * x.size * BYTES_PER_ELEM_MXFP4
     t0 = time.perf_counter()
-    oracle.quantize(x, oracle.MXFP4, oracle.RNE, rotate=True)
-    oracle.quantize(x, oracle.MXFP4, oracle.SR, rotate=True, seed=7)
-    dt = time.perf_counter() - t0
-    return {"value": 2 * x.size * BYTES_PER_ELEM_MXFP4 / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": "one full step (X 4096x4096, RNE + SR), single-threaded C oracle", "seconds": dt}
+    single = [oracle.quantize(x, oracle.MXFP4, oracle.RNE, rotate=True),
+              oracle.quantize(x, oracle.MXFP4, oracle.SR, rotate=True, seed=7)]
+    dt1 = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    par = _oracle_step_parallel(oracle, x, nproc)
+    dtn = time.perf_counter() - t0
+    identical = all(np.array_equal(a[k], b[k]) for a, b in zip(single, par) for k in ("codes", "scales"))
+    # oracle GEMM: binary64 sum over dequantized NVFP4 operands, every output of a small sub-problem
+    m = n = 128
+    K = GEMM_SHAPE[2]
+    A = oracle.quantize(synth.cfg3_X(m, K), oracle.NVFP4, four6=True)
+    B = oracle.quantize(synth.cfg3_W(n, K), oracle.NVFP4, four6=True)
+    r, c = np.meshgrid(np.arange(m), np.arange(n), indexing="ij")
+    t0 = time.perf_counter()
+    oracle.gemm_sampled(A, B, m, n, K, oracle.NVFP4, r.ravel(), c.ravel())
+    dtg = time.perf_counter() - t0
+    gflops = 2.0 * m * n * K / dtg / 1e9
+    Mg, Ng, Kg = GEMM_SHAPE
+    return {"value": step_bytes / dtn / 1e9, "unit": "GB/s", "cores": nproc, "kind": "oracle",
+            "sample": f"one full step (X 4096x4096, FWHT-128 + MXFP4, RNE + SR) row-partitioned over {nproc} "
+                      f"threads, output identical to the single-threaded run: {identical}",
+            "seconds": dtn, "identical_to_single_thread": identical, "nproc": nproc,
+            "single_thread": {"value": step_bytes / dt1 / 1e9, "unit": "GB/s", "cores": 1, "seconds": dt1},
+            "gemm": {"value": gflops, "unit": "GFLOP/s", "cores": 1, "kind": "oracle",
+                     "sample": f"binary64 oracle GEMM, every output of {m}x{n}x{K} (NVFP4 four-over-six operands)",
+                     "seconds": dtg, "extrapolated_ms_for": f"{Mg}x{Ng}x{Kg}",
+                     "extrapolated_ms": 2.0 * Mg * Ng * Kg / (gflops * 1e9) * 1e3, "label": "extrapolated"}}
 
 
 def max_over_ranks(x, dist, device):
@@ -374,6 +428,9 @@ def run_gpu(args, rank, world):
     gemm = None
     if not args.no_gemm:
         gemm = bench_gemm(q, synth, dev, stream, bf16_peak, peak_src, max(3, min(args.steps, 20)))
+    cfg5 = None
+    if not args.no_cfg5:
+        cfg5 = bench_cfg5(q, synth, dev, stream, hbm_peak, bf16_peak, peak_src, max(3, min(args.steps, 10)))
 
     result = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -384,6 +441,8 @@ def run_gpu(args, rank, world):
     }
     if gemm is not None:
         result["gemm"] = gemm
+    if cfg5 is not None:
+        result["largest_config"] = cfg5
     if rank == 0 and world == 1 and not args.no_cpu:
         result["cpu_baseline"] = cpu_baseline()
     if dist is not None:
@@ -420,6 +479,69 @@ def bench_gemm(q, synth, dev, stream, bf16_peak, peak_src, iters):
                          "frac": tflops / peak, "traffic": ncu_traffic("gemm_nvfp4_f32"),
                          "kernel": "gemm_nvfp4_f32 (scale-chunk prepass + 2-CTA tcgen05 main loop)",
                          "peak_source": f"{peak_src} bf16_tflops x {FP4_PER_BF16} (nominal FP4:BF16 dense ratio)"}}
+
+
+def bench_cfg5(q, synth, dev, stream, hbm_peak, bf16_peak, peak_src, iters):
+    """The largest configuration's two headline calls, each timed with CUDA
+    events around every call on the launching stream: the standalone quantize
+    of 2^30 bf16 elements (262144 x 4096; inputs far larger than L2) -- FWHT-128
+    + MXFP4 RNE, and NVFP4 RNE under a caller-supplied tensor amax (one read) --
+    and the fused rotate + quantize + GEMM at 16384 x 14336 x 4096."""
+    import torch
+    out = {}
+    bf = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)   # noqa: E731
+    base = bf(synth.cfg5_A(16384, 4096))
+    x = base.repeat(16, 1)                                  # 2^30 elements, 2 GiB
+    M, K = x.shape
+    n = M * K
+
+    def timed(call):
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+        for a, b in evs:
+            a.record(stream)
+            call()
+            b.record(stream)
+        torch.cuda.synchronize()
+        return statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+    o = q.quantize(x, q.MXFP4, q.RNE, rotate=True)
+    ms = timed(lambda: q.quantize(x, q.MXFP4, q.RNE, rotate=True, out=o))
+    nbytes = n * BYTES_PER_ELEM_MXFP4
+    out["quantize_2^30_fwht_mxfp4_rne"] = {
+        "workload": f"2^30 bf16 elements ({M}x{K}, N(0,1), 0.5% channels x30): FWHT-128 + MXFP4 RNE",
+        "ms_per_call": ms, "roofline": {"bound": "hbm", "achieved": nbytes / (ms * 1e-3) / 1e9, "peak": hbm_peak,
+                                        "unit": "GB/s", "frac": nbytes / (ms * 1e-3) / 1e9 / hbm_peak,
+                                        "algorithmic_bytes_per_launch": nbytes, "traffic": None,
+                                        "peak_source": f"{peak_src} hbm_gbs"}}
+    amax = torch.tensor([float(x.abs().max())], dtype=torch.float32, device=dev)
+    o = q.quantize(x, q.NVFP4, q.RNE, amax_in=amax)
+    ms = timed(lambda: q.quantize(x, q.NVFP4, q.RNE, amax_in=amax, out=o))
+    nbytes = n * (2 + 0.5 + 1 / 16)
+    out["quantize_2^30_nvfp4_rne_given_amax"] = {
+        "workload": f"2^30 bf16 elements ({M}x{K}): NVFP4 RNE with a caller-supplied tensor amax (one read of X)",
+        "ms_per_call": ms, "roofline": {"bound": "hbm", "achieved": nbytes / (ms * 1e-3) / 1e9, "peak": hbm_peak,
+                                        "unit": "GB/s", "frac": nbytes / (ms * 1e-3) / 1e9 / hbm_peak,
+                                        "algorithmic_bytes_per_launch": nbytes, "traffic": None,
+                                        "peak_source": f"{peak_src} hbm_gbs"}}
+    del x, o
+    M, N, K = 16384, 14336, 4096
+    a5 = base
+    B5 = q.quantize(bf(synth.cfg5_B(N, K)), q.NVFP4, q.RNE, rotate=True)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(q.qfp4_gemm_fused_rq_workspace_bytes(M, N, K, q.NVFP4), dtype=torch.uint8, device=dev)
+    ms = timed(lambda: q.gemm_fused_rq(a5, B5, N, fmt=q.NVFP4, rotate=True, out=y, workspace=ws))
+    tf = 2.0 * M * N * K / (ms * 1e-3) / 1e12
+    peak = bf16_peak * FP4_PER_BF16
+    out["fused_rotate_quantize_gemm_16384x14336x4096"] = {
+        "workload": "A bf16 16384x4096 (0.5% channels x30) rotated + NVFP4-quantized inside the call, "
+                    "B 14336x4096 pre-rotated NVFP4, bf16 out",
+        "ms_per_call": ms, "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
+                                        "frac": tf / peak, "flops_per_launch": 2.0 * M * N * K, "traffic": None,
+                                        "peak_source": f"{peak_src} bf16_tflops x {FP4_PER_BF16}"}}
+    return out
 
 
 def run_profile_case(case):

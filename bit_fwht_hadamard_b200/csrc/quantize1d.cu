@@ -226,23 +226,20 @@ __device__ __forceinline__ void sr_group(const float *v, uint64_t e, uint64_t se
 
 // binary32 squared error of 32 values x under codes w (4 words) and scale
 // 2^k: sum(fl(fl(fl(g_i 2^k) - x_i)^2)) as a fixed tree (i + 16 into i, then
-// + 8, + 4, + 2, + 1); g_i 2^k is exact.
+// + 8, + 4, + 2, + 1); g_i 2^k is exact.  The code values come from the E2M1
+// bit fields (e2m1_value), not from the hardware nibble-pair conversion: on
+// B200 that conversion, fed words just produced by cvt.rn.satfinite.e2m1x2
+// in the same function, returned zeros for bytes 2-3 of the word.
 __device__ __forceinline__ float mx_sse32(const float *x, const uint32_t *w, int k)
 {
     const float sc = exp2i(k);
     float e[32];
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
-        uint64_t g4[4];
-        e2m1x8_values(w[t], g4);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            float g0, g1;
-            f2unpack(g4[j], g0, g1);
-            const float d0 = __fsub_rn(__fmul_rn(g0, sc), x[8 * t + 2 * j]);
-            const float d1 = __fsub_rn(__fmul_rn(g1, sc), x[8 * t + 2 * j + 1]);
-            e[8 * t + 2 * j] = __fmul_rn(d0, d0);
-            e[8 * t + 2 * j + 1] = __fmul_rn(d1, d1);
+        for (int u = 0; u < 8; ++u) {
+            const float d = __fsub_rn(__fmul_rn(e2m1_value((w[t] >> (4 * u)) & 0xFu), sc), x[8 * t + u]);
+            e[8 * t + u] = __fmul_rn(d, d);
         }
     }
 #pragma unroll
@@ -825,22 +822,30 @@ __global__ void __launch_bounds__(128) k_quant1d_direct(const T *__restrict__ x,
 #pragma unroll
         for (int i = 0; i < 64; ++i) v[i] = 0.0f;
         if (n_valid > 0) {
+            // whole 16-byte vectors where they lie inside the range, single
+            // elements for a last partial vector (the amax pass of an
+            // arbitrary-length input reaches one; the quantize passes, whose
+            // lengths are multiples of the group, do not)
             if (sizeof(T) == 4) {
                 const float4 *src = reinterpret_cast<const float4 *>(x + off);
 #pragma unroll
-                for (int c = 0; c < 16; ++c)
-                    if (4 * c < n_valid) {
+                for (int c = 0; c < 16; ++c) {
+                    if (4 * c + 4 <= n_valid) {
                         const float4 f = src[c];
                         v[4 * c] = f.x;
                         v[4 * c + 1] = f.y;
                         v[4 * c + 2] = f.z;
                         v[4 * c + 3] = f.w;
+                    } else if (4 * c < n_valid) {
+                        for (int t = 0; t < 4; ++t)
+                            if (4 * c + t < n_valid) v[4 * c + t] = reinterpret_cast<const float *>(x + off)[4 * c + t];
                     }
+                }
             } else {
                 const uint4 *src = reinterpret_cast<const uint4 *>(x + off);
 #pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    if (8 * c < n_valid) {
+                for (int c = 0; c < 8; ++c) {
+                    if (8 * c + 8 <= n_valid) {
                         const uint4 w = src[c];
                         v[8 * c] = bf16lo(w.x);
                         v[8 * c + 1] = bf16hi(w.x);
@@ -850,7 +855,13 @@ __global__ void __launch_bounds__(128) k_quant1d_direct(const T *__restrict__ x,
                         v[8 * c + 5] = bf16hi(w.z);
                         v[8 * c + 6] = bf16lo(w.w);
                         v[8 * c + 7] = bf16hi(w.w);
+                    } else if (8 * c < n_valid) {
+                        const uint16_t *h = reinterpret_cast<const uint16_t *>(x + off);
+                        for (int t = 0; t < 8; ++t)
+                            if (8 * c + t < n_valid)
+                                v[8 * c + t] = __uint_as_float(static_cast<uint32_t>(h[8 * c + t]) << 16);
                     }
+                }
             }
         }
         if (ROT) fwht128_pair(v, (threadIdx.x & 1) != 0);   // n % 128 == 0: pairs are whole
