@@ -151,3 +151,50 @@ def test_gemm_argument_errors():
         G.gemm(A, A, 128, 130, 256, q.MXFP4)                      # N % 4
     assert e.value.status == q.ERR_SHAPE
     assert q.qfp4_last_device_error() == 0
+
+
+# shapes of the in-kernel quantization (M > 128, K % 64 == 0): ragged M, a K
+# tail short of the 256-element k-tile, several 128-row blocks of A
+FUSED_SHAPES = [(300, 264, 640), (256, 512, 1024), (1000, 768, 384), (129, 256, 2048)]
+
+
+@pytest.mark.parametrize("M,N,K", FUSED_SHAPES)
+@pytest.mark.parametrize("fmt", FMTS, ids=["mxfp4", "nvfp4"])
+@pytest.mark.parametrize("rotate", [True, False], ids=["rot", "plain"])
+def test_fused_in_kernel_quantization(M, N, K, fmt, rotate):
+    """A quantized by the GEMM kernel's own quantizer warps: its codes, scales
+    and tensor scale left in the workspace equal the oracle's bit for bit, and
+    every output is within the bound of the binary64 reference."""
+    if rotate and K % 128:
+        pytest.skip()
+    a = synth.cfg5_A(M, K, seed=M + 7 * K)
+    b = synth.cfg5_B(N, K, seed=N + 5 * K)
+    B = oracle.quantize(b, fmt[1], rotate=rotate)
+    A = oracle.quantize(a, fmt[1], rotate=rotate)
+    wsb = q.qfp4_gemm_fused_rq_workspace_bytes(M, N, K, fmt[0])
+    ws = G.guarded((wsb,), torch.uint8)
+    y = G.guarded((M, N), torch.float32)
+    q.gemm_fused_rq(to_dev(a), _upload(B), N, fmt=fmt[0], rotate=rotate, out=y, workspace=ws)
+    co, so, to = q.qfp4_gemm_fused_rq_workspace_layout(M, N, K, fmt[0])
+    g = 32 if fmt[1] == oracle.MXFP4 else 16
+    w = host(ws)
+    assert np.array_equal(w[co:co + M * K // 2], A["codes"].ravel())
+    assert np.array_equal(w[so:so + M * K // g], A["scales"].ravel())
+    if fmt[1] == oracle.NVFP4:
+        assert w[to:to + 4].view(np.float32)[0] == A["tscale"][0]
+    rows, cols = _all_pairs(M, N)
+    _check(host(y), A, B, M, N, K, fmt[1], rows, cols)
+    assert q.qfp4_last_device_error() == 0
+
+
+def test_fused_in_kernel_quantization_is_repeatable():
+    """Quantizer warps and GEMM roles overlap differently from call to call;
+    the output must not depend on it."""
+    M, N, K = 2048, 4096, 4096
+    a = to_dev(synth.cfg5_A(M, K, seed=3))
+    B = q.quantize(to_dev(synth.cfg5_B(N, K, seed=4)), q.NVFP4, rotate=True)
+    ys = [q.gemm_fused_rq(a, B, N, fmt=q.NVFP4, rotate=True, out_dtype=torch.bfloat16) for _ in range(4)]
+    torch.cuda.synchronize()
+    for y in ys[1:]:
+        assert int((y.view(torch.int16) != ys[0].view(torch.int16)).sum()) == 0
+    assert q.qfp4_last_device_error() == 0
