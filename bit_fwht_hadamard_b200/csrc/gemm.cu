@@ -650,8 +650,10 @@ __device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int *p)
     return v;
 }
 
-// Wait (bounded) until `want` rows of a 128-row block of A are quantized,
-// then order the TMA (async-proxy) reads of them after the acquire.
+// Wait (bounded) until `want` (> 0) rows of a 128-row block of A are
+// quantized, then order the TMA (async-proxy) reads of them after the
+// acquire.  A block past the end of A (the partner half of the last tile
+// pair) has no rows and is not waited on.
 __device__ __forceinline__ bool wait_rows_ready(const unsigned int *ready, unsigned int want)
 {
     if (ld_acquire_gpu(ready) < want) {
@@ -824,7 +826,8 @@ __global__ void __launch_bounds__(g2_threads(FUSED), 1)
                 int mb, nb;
                 tile_coords(t, tiles_m, tiles_n, mb, nb);
                 const int rb_a = 2 * mb + static_cast<int>(rank);   // this CTA's 128-row block of A
-                if (FUSED && !wait_rows_ready(p.fq.ready + rb_a, rows_in_block(rb_a, p.M))) { abort_flag = 1; break; }
+                if (FUSED && rows_in_block(rb_a, p.M) &&
+                    !wait_rows_ready(p.fq.ready + rb_a, rows_in_block(rb_a, p.M))) { abort_flag = 1; break; }
                 for (int kt = 0; kt < p.KT; ++kt, ++it) {
                     const int s = it % G2_STAGES;
                     const uint32_t ph = (it / G2_STAGES) & 1u;
@@ -881,7 +884,8 @@ __global__ void __launch_bounds__(g2_threads(FUSED), 1)
                 int mb, nb;
                 tile_coords(t, tiles_m, tiles_n, mb, nb);
                 const int rb_a = 2 * mb + static_cast<int>(rank);
-                if (FUSED && !wait_rows_ready(p.fq.ready + rb_a, rows_in_block(rb_a, p.M))) { abort_flag = 1; break; }
+                if (FUSED && rows_in_block(rb_a, p.M) &&
+                    !wait_rows_ready(p.fq.ready + rb_a, rows_in_block(rb_a, p.M))) { abort_flag = 1; break; }
                 for (int kt = 0; kt < p.KT; ++kt, ++it) {
                     const int s = it % G2_SF_SLOTS;
                     if (!mbar_wait(&sfs_empty[s], ((it / G2_SF_SLOTS) & 1u) ^ 1u)) { abort_flag = 1; break; }
