@@ -30,7 +30,7 @@ DEV_ERR_TIMEOUT = 1
 EXPORTS = [
     "qfp4_quantize_workspace_bytes", "qfp4_quantize", "qfp4_quantize_ex", "qfp4_quantize_mxfp8", "qfp4_quantize_fp32scale",
     "qfp4_dequantize", "qfp4_gemm_workspace_bytes", "qfp4_gemm_blockscaled", "qfp4_gemm_fused_rq_workspace_bytes",
-    "qfp4_gemm_fused_rq", "qfp4_gemm_fused_rq_workspace_layout", "qfp4_gemm_blockscaled_noalloc",
+    "qfp4_gemm_fused_rq", "qfp4_gemm_fused_rq_ex", "qfp4_gemm_fused_rq_workspace_layout", "qfp4_gemm_blockscaled_noalloc",
     "qfp4_linear_forward_workspace_bytes", "qfp4_linear_forward", "qfp4_linear_backward_workspace_bytes",
     "qfp4_linear_backward", "qfp4_kl_calibrate_workspace_bytes", "qfp4_kl_calibrate",
     "qfp4_status_string", "qfp4_last_device_error", "qfp4_selftest_wait_timeout", "qfp4_version",
@@ -81,6 +81,9 @@ def lib():
         L.qfp4_gemm_fused_rq.restype = c_int
         L.qfp4_gemm_fused_rq.argtypes = [P, c_int64, c_int64, c_int, c_int, c_int, P, P, P, c_int64, P, c_size_t,
                                          c_int, P, P]
+        L.qfp4_gemm_fused_rq_ex.restype = c_int
+        L.qfp4_gemm_fused_rq_ex.argtypes = [P, c_int64, c_int64, c_int, c_int, c_int, P, P, P, P, P, c_int64, P,
+                                            c_size_t, c_int, P, P]
         L.qfp4_gemm_fused_rq_workspace_layout.restype = c_int
         L.qfp4_gemm_fused_rq_workspace_layout.argtypes = [c_int64, c_int64, c_int64, c_int, P, P, P]
         L.qfp4_linear_forward_workspace_bytes.restype = c_size_t
@@ -171,6 +174,12 @@ def qfp4_gemm_fused_rq(A_bf16, M, K, rotate, four6, fmt, B_codes, B_scales, B_ts
                        workspace_bytes, out_dt, out, stream):
     return lib().qfp4_gemm_fused_rq(A_bf16, M, K, rotate, four6, fmt, B_codes, B_scales, B_tscale, N, workspace,
                                     workspace_bytes, out_dt, out, stream)
+
+
+def qfp4_gemm_fused_rq_ex(A_bf16, M, K, rotate, four6, fmt, A_amax_in, A_amax_out, B_codes, B_scales, B_tscale, N,
+                          workspace, workspace_bytes, out_dt, out, stream):
+    return lib().qfp4_gemm_fused_rq_ex(A_bf16, M, K, rotate, four6, fmt, A_amax_in, A_amax_out, B_codes, B_scales,
+                                       B_tscale, N, workspace, workspace_bytes, out_dt, out, stream)
 
 
 def qfp4_gemm_fused_rq_workspace_layout(M, N, K, fmt):
@@ -353,8 +362,10 @@ def gemm(A, B, M, N, K, fmt, out_dtype=None, out=None, workspace=None, stream=No
 
 
 def gemm_fused_rq(A_bf16, B, N, fmt=NVFP4, rotate=True, four6=False, out_dtype=None, out=None, workspace=None,
-                  stream=None):
-    """Y = Q(rot(A)) deq(B)^T with A bf16 (M, K) quantized inside the call."""
+                  stream=None, A_amax_in=None, A_amax_out=None):
+    """Y = Q(rot(A)) deq(B)^T with A bf16 (M, K) quantized inside the call;
+    A_amax_in / A_amax_out: NVFP4 tensor amax of A supplied / reported
+    (one-element float32 CUDA tensors)."""
     torch = _torch()
     M, K = A_bf16.shape
     out_dtype = torch.float32 if out_dtype is None else out_dtype
@@ -363,10 +374,10 @@ def gemm_fused_rq(A_bf16, B, N, fmt=NVFP4, rotate=True, four6=False, out_dtype=N
     wsb = qfp4_gemm_fused_rq_workspace_bytes(M, N, K, fmt)
     if workspace is None:
         workspace = torch.empty(max(wsb, 16), dtype=torch.uint8, device=A_bf16.device)
-    st = qfp4_gemm_fused_rq(_ptr(A_bf16), M, K, int(rotate), int(four6), fmt, _ptr(B["codes"]), _ptr(B["scales"]),
-                            _ptr(B.get("tscale")), N, _ptr(workspace), wsb, F32 if out.dtype == torch.float32 else BF16,
-                            _ptr(out), _stream(stream))
-    _check(st, "qfp4_gemm_fused_rq")
+    st = qfp4_gemm_fused_rq_ex(_ptr(A_bf16), M, K, int(rotate), int(four6), fmt, _ptr(A_amax_in), _ptr(A_amax_out),
+                               _ptr(B["codes"]), _ptr(B["scales"]), _ptr(B.get("tscale")), N, _ptr(workspace), wsb,
+                               F32 if out.dtype == torch.float32 else BF16, _ptr(out), _stream(stream))
+    _check(st, "qfp4_gemm_fused_rq_ex")
     return out
 
 

@@ -23,7 +23,7 @@ int gemm_blockscaled(const uint8_t *A_codes, const uint8_t *A_scales, const floa
 size_t gemm_workspace(int64_t M, int64_t N, int64_t K, qfp4_fmt fmt);
 int gemm_fused_rq(const void *A_bf16, int64_t M, int64_t K, int rotate, int four6, qfp4_fmt fmt,
                   const uint8_t *B_codes, const uint8_t *B_scales, const float *B_tscale, int64_t N, void *workspace,
-                  qfp4_dtype out_dt, void *out, cudaStream_t stream);
+                  qfp4_dtype out_dt, void *out, cudaStream_t stream, const float *amax_in, float *amax_out);
 size_t gemm_fused_rq_workspace(int64_t M, int64_t N, int64_t K, qfp4_fmt fmt);
 void gemm_fused_rq_layout(int64_t M, int64_t N, int64_t K, qfp4_fmt fmt, size_t *codes, size_t *scales,
                           size_t *tscale);
@@ -211,10 +211,10 @@ extern "C" int qfp4_gemm_fused_rq_workspace_layout(int64_t M, int64_t N, int64_t
     return QFP4_OK;
 }
 
-extern "C" int qfp4_gemm_fused_rq(const void *A_bf16, int64_t M, int64_t K, int rotate, int four6, qfp4_fmt fmt,
-                                  const uint8_t *B_codes, const uint8_t *B_scales, const float *B_tscale, int64_t N,
-                                  void *workspace, size_t workspace_bytes, qfp4_dtype out_dt, void *out,
-                                  qfp4_stream_t stream)
+extern "C" int qfp4_gemm_fused_rq_ex(const void *A_bf16, int64_t M, int64_t K, int rotate, int four6, qfp4_fmt fmt,
+                                     const float *A_amax_in, float *A_amax_out, const uint8_t *B_codes,
+                                     const uint8_t *B_scales, const float *B_tscale, int64_t N, void *workspace,
+                                     size_t workspace_bytes, qfp4_dtype out_dt, void *out, qfp4_stream_t stream)
 {
     if (fmt != QFP4_MXFP4 && fmt != QFP4_NVFP4) return QFP4_ERR_ARG;
     if (out_dt != QFP4_BF16 && out_dt != QFP4_F32) return QFP4_ERR_ARG;
@@ -223,13 +223,27 @@ extern "C" int qfp4_gemm_fused_rq(const void *A_bf16, int64_t M, int64_t K, int 
     if (M * N > 0 && (!A_bf16 || !B_codes || !B_scales || !out)) return QFP4_ERR_ARG;
     if (fmt == QFP4_NVFP4 && M * N > 0 && !B_tscale) return QFP4_ERR_ARG;
     if (four6 && fmt != QFP4_NVFP4) return QFP4_ERR_UNSUPPORTED;
+    if ((A_amax_in || A_amax_out) && fmt != QFP4_NVFP4) return QFP4_ERR_UNSUPPORTED;
     if (rotate && K % 128) return QFP4_ERR_SHAPE;
     if (!ok_align(A_bf16) || !ok_align(B_codes) || !ok_align(B_scales) || !ok_align(out) || !ok_align(workspace))
         return QFP4_ERR_ALIGN;
-    if (M * N == 0) return QFP4_OK;
-    if (K == 0) return cudaMemsetAsync(out, 0, M * N * (out_dt == QFP4_F32 ? 4 : 2),
-                                       reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? QFP4_OK : QFP4_ERR_CUDA;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (M * N == 0 || K == 0) {
+        if (A_amax_out && cudaMemsetAsync(A_amax_out, 0, sizeof(float), s) != cudaSuccess) return QFP4_ERR_CUDA;
+        if (M * N == 0) return QFP4_OK;
+        return cudaMemsetAsync(out, 0, M * N * (out_dt == QFP4_F32 ? 4 : 2), s) == cudaSuccess ? QFP4_OK
+                                                                                               : QFP4_ERR_CUDA;
+    }
     if (!workspace || workspace_bytes < gemm_fused_rq_workspace(M, N, K, fmt)) return QFP4_ERR_ARG;
-    return gemm_fused_rq(A_bf16, M, K, rotate, four6, fmt, B_codes, B_scales, B_tscale, N, workspace, out_dt, out,
-                         reinterpret_cast<cudaStream_t>(stream));
+    return gemm_fused_rq(A_bf16, M, K, rotate, four6, fmt, B_codes, B_scales, B_tscale, N, workspace, out_dt, out, s,
+                         A_amax_in, A_amax_out);
+}
+
+extern "C" int qfp4_gemm_fused_rq(const void *A_bf16, int64_t M, int64_t K, int rotate, int four6, qfp4_fmt fmt,
+                                  const uint8_t *B_codes, const uint8_t *B_scales, const float *B_tscale, int64_t N,
+                                  void *workspace, size_t workspace_bytes, qfp4_dtype out_dt, void *out,
+                                  qfp4_stream_t stream)
+{
+    return qfp4_gemm_fused_rq_ex(A_bf16, M, K, rotate, four6, fmt, nullptr, nullptr, B_codes, B_scales, B_tscale, N,
+                                 workspace, workspace_bytes, out_dt, out, stream);
 }

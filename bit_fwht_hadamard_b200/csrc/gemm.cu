@@ -56,6 +56,8 @@ struct FusedQuant {
     float *tscale;              // out: NVFP4 s_t
     const float *partials;      // NVFP4: partial maxima of the amax pass
     int n_partials;
+    const float *amax_in;       // NVFP4: caller-supplied tensor amax of A (then no amax pass), or NULL
+    float *amax_out;            // NVFP4: receives A's own (rotated) amax, or NULL (zeroed by the host)
     unsigned int *ready;        // per 128-row block of A: rows quantized so far
 };
 
@@ -643,6 +645,12 @@ __device__ __forceinline__ void fence_proxy_async_global()
     asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
+// pull `bytes` (a multiple of 16, 16-byte aligned) of global memory into L2
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int *p)
 {
     unsigned int v;
@@ -670,6 +678,18 @@ __device__ __forceinline__ bool wait_rows_ready(const unsigned int *ready, unsig
     return true;
 }
 
+// NVFP4 s_t of A in the fused kernel (every lane of a warp gets it): from the
+// caller's amax, or the maximum of the amax pass's partial maxima.
+__device__ __forceinline__ float fused_tscale(const FusedQuant &fq, int lane)
+{
+    if (fq.amax_in) return __fdiv_rn(*fq.amax_in, 2688.0f);
+    float m = 0.0f;
+    for (int i = lane; i < fq.n_partials; i += 32) m = fmaxf(m, fq.partials[i]);
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    return __fdiv_rn(m, 2688.0f);
+}
+
 // Rows of A quantized by the fused kernel's quantizer warps: warp g of G
 // takes rows g, g + G, ... (ascending, so the 128-row blocks the tile raster
 // needs first are ready first).  A lane holds 64 consecutive elements of a
@@ -686,17 +706,22 @@ __device__ __forceinline__ void fused_quantize_rows(const GemmParams &p, int qwa
     constexpr bool RAW = ROT && FMT == QFP4_MXFP4;     // normalisation folded into the 2^-k multiply
     float s_t = 0.0f;
     if (FMT == QFP4_NVFP4) {
-        float m = 0.0f;
-        for (int i = lane; i < p.fq.n_partials; i += 32) m = fmaxf(m, p.fq.partials[i]);
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-        s_t = __fdiv_rn(m, 2688.0f);
+        s_t = fused_tscale(p.fq, lane);
         if (qwarp == 0 && lane == 0) *p.fq.tscale = s_t;
     }
     const NvScale nz = nv_scale_setup(s_t);
     const int units = p.K / 64;
     const int64_t K = p.K;
+    // the rows this warp takes next are pulled into L2 two rows ahead, so the
+    // row loads below meet L2 rather than HBM latency
+    auto prefetch_row = [&](int rp) {
+        if (lane == 0 && rp < p.M) bulk_prefetch_l2(p.fq.A + static_cast<int64_t>(rp) * K, static_cast<uint32_t>(2 * K));
+    };
+    prefetch_row(qwarp);
+    prefetch_row(qwarp + nqwarps);
+    float own_max = 0.0f;                        // this warp's |x| maximum (after rotation), when asked for
     for (int r = qwarp; r < p.M && !*abort_flag; r += nqwarps) {
+        prefetch_row(r + 2 * nqwarps);
         const uint16_t *row = p.fq.A + static_cast<int64_t>(r) * K;
         const int64_t rb = r >> 7, rr = r & 127;
         for (int c0 = 0; c0 < units; c0 += 32) {
@@ -718,6 +743,7 @@ __device__ __forceinline__ void fused_quantize_rows(const GemmParams &p, int qwa
                 for (int c = 0; c < 32; ++c) v[c] = 0ull;
             }
             if (ROT) fwht_packed<32, !RAW>(v, (lane & 1) != 0);
+            if (p.fq.amax_out) own_max = fmaxf(own_max, absmax_pairs<32>(v));   // NVFP4 (not RAW): normalised values
             UnitP<32> o;
             quant_unit_packed<32, FMT, false, false, RAW>(v, 0, nz, 0, o);
             if (active) {
@@ -740,6 +766,12 @@ __device__ __forceinline__ void fused_quantize_rows(const GemmParams &p, int qwa
         __threadfence();
         __syncwarp();
         if (lane == 0) atomicAdd(&p.fq.ready[rb], 1u);
+    }
+    if (p.fq.amax_out) {
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) own_max = fmaxf(own_max, __shfl_xor_sync(0xFFFFFFFFu, own_max, o));
+        // non-negative binary32 values order like their bit patterns; the host zeroed *amax_out
+        if (lane == 0) atomicMax(reinterpret_cast<unsigned int *>(p.fq.amax_out), __float_as_uint(own_max));
     }
 }
 
@@ -1001,12 +1033,8 @@ __global__ void __launch_bounds__(g2_threads(FUSED), 1)
         float alpha = 1.0f;
         if (FMT == QFP4_NVFP4) {
             float tA;
-            if constexpr (FUSED) {                        // A's s_t from the amax pass, as the quantizer warps form it
-                float m = 0.0f;
-                for (int i = lane; i < p.fq.n_partials; i += 32) m = fmaxf(m, p.fq.partials[i]);
-#pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-                tA = __fdiv_rn(m, 2688.0f);
+            if constexpr (FUSED) {
+                tA = fused_tscale(p.fq, lane);              // A's s_t, as the quantizer warps form it
             } else {
                 tA = *p.tA;
             }
@@ -1351,7 +1379,7 @@ size_t gemm_fused_rq_workspace(int64_t M, int64_t N, int64_t K, qfp4_fmt fmt)
 // either way.
 int gemm_fused_rq(const void *A_bf16, int64_t M, int64_t K, int rotate, int four6, qfp4_fmt fmt,
                   const uint8_t *B_codes, const uint8_t *B_scales, const float *B_tscale, int64_t N, void *workspace,
-                  qfp4_dtype out_dt, void *out, cudaStream_t stream)
+                  qfp4_dtype out_dt, void *out, cudaStream_t stream, const float *amax_in, float *amax_out)
 {
     const FusedLayout F = fused_layout(M, N, K, fmt);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -1371,10 +1399,20 @@ int gemm_fused_rq(const void *A_bf16, int64_t M, int64_t K, int rotate, int four
         fa.fq.tscale = a_tscale;
         fa.fq.partials = partials;
         fa.fq.n_partials = 0;
+        fa.fq.amax_in = amax_in;
+        fa.fq.amax_out = nullptr;
         fa.fq.ready = reinterpret_cast<unsigned int *>(ws + F.ready);
-        if (fmt == QFP4_NVFP4) {
+        if (fmt == QFP4_NVFP4 && !amax_in) {
             st = amax_pass_bf16(A_bf16, M * K, rotate != 0, partials, &fa.fq.n_partials, stream);
             if (st != QFP4_OK) return st;
+            if (amax_out) {
+                st = partials_max(partials, fa.fq.n_partials, amax_out, stream);
+                if (st != QFP4_OK) return st;
+            }
+        } else if (fmt == QFP4_NVFP4 && amax_out) {
+            // the quantizer warps raise it with atomic maxima of their rows
+            if (cudaMemsetAsync(amax_out, 0, sizeof(float), stream) != cudaSuccess) return QFP4_ERR_CUDA;
+            fa.fq.amax_out = amax_out;
         }
         if (cudaMemsetAsync(fa.fq.ready, 0, sizeof(unsigned int) * ((M + 127) / 128), stream) != cudaSuccess)
             return QFP4_ERR_CUDA;
@@ -1384,8 +1422,11 @@ int gemm_fused_rq(const void *A_bf16, int64_t M, int64_t K, int rotate, int four
         if (st != QFP4_OK) return st;
         return gemm_core(a_codes, sfa, a_tscale, B_codes, sfb, B_tscale, M, N, K, fmt, out_dt, out, stream, &fa);
     }
+    QuantOpts opt;
+    opt.amax_in = amax_in;
+    opt.amax_out = amax_out;
     st = quantize1d(A_bf16, QFP4_BF16, M * K, fmt, QFP4_RNE, rotate, four6, 0, a_codes, a_scales, a_tscale, partials,
-                    nullptr, stream);
+                    nullptr, stream, opt);
     if (st != QFP4_OK) return st;
     st = rearrange_scales(a_scales, M, L.MB, sfa, B_scales, N, 2 * L.NT, sfb, K, fmt, L.NC, stream);
     if (st != QFP4_OK) return st;

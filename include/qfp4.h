@@ -281,8 +281,12 @@ int qfp4_gemm_blockscaled_noalloc(const uint8_t *A_codes, const uint8_t *A_scale
  * qfp4_quantize) inside the call, then multiplied by the pre-quantized B
  * ([QN] §QuTLASS: fused rotation and online quantization before the GEMM;
  * B is expected to be rotated the same way offline, so that
- * (xH)(WH)^T = xW^T).  A is quantized once into the workspace (not once
- * per output tile), then consumed by the tensor-core kernel.
+ * (xH)(WH)^T = xW^T).  A is quantized once, not once per output tile: for
+ * M > 128, K % 64 == 0 and four6 == 0 by quantizer warps inside the
+ * tensor-core kernel itself, overlapped with the MMAs of the rows already
+ * quantized; otherwise by the 1D quantize kernel before the GEMM.  NVFP4
+ * first measures A's tensor amax (an extra read of A; see
+ * qfp4_gemm_fused_rq_ex to supply it).
  * workspace: at least qfp4_gemm_fused_rq_workspace_bytes(M, N, K, fmt)
  * bytes of device scratch.  Same shape rules as qfp4_gemm_blockscaled,
  * plus K % 128 == 0 with rotate.
@@ -293,6 +297,17 @@ int qfp4_gemm_fused_rq(const void *A_bf16, int64_t M, int64_t K, int rotate, int
                        const uint8_t *B_codes, const uint8_t *B_scales, const float *B_tscale, int64_t N,
                        void *workspace, size_t workspace_bytes,
                        qfp4_dtype out_dt, void *out, qfp4_stream_t stream);
+
+/* qfp4_gemm_fused_rq with NVFP4's tensor amax of A supplied and / or
+ * reported, as in qfp4_quantize_ex: A_amax_in (device float, or NULL) gives
+ * s_t = fl(*A_amax_in / 2688) and removes the extra read of A; A_amax_out
+ * (device float, or NULL) receives A's own amax after rotation.  MXFP4: both
+ * must be NULL (QFP4_ERR_UNSUPPORTED). */
+int qfp4_gemm_fused_rq_ex(const void *A_bf16, int64_t M, int64_t K, int rotate, int four6, qfp4_fmt fmt,
+                          const float *A_amax_in, float *A_amax_out,
+                          const uint8_t *B_codes, const uint8_t *B_scales, const float *B_tscale, int64_t N,
+                          void *workspace, size_t workspace_bytes,
+                          qfp4_dtype out_dt, void *out, qfp4_stream_t stream);
 
 /* Where qfp4_gemm_fused_rq leaves A's quantized operand in its workspace
  * once the call's work is done: codes (M*K/2 bytes, as qfp4_quantize writes

@@ -173,7 +173,8 @@ def gemm(A, B, M, N, K, fmt, out_dtype=None):
     return q.gemm(A, B, M, N, K, fmt, out=guarded((M, N), out_dtype or torch.float32))
 
 
-def gemm_fused_rq(A_bf16, B, N, fmt, rotate=True, four6=False, out_dtype=None):
+def gemm_fused_rq(A_bf16, B, N, fmt, rotate=True, four6=False, out_dtype=None, A_amax_in=None, A_amax_out=None):
     import bit_fwht_hadamard_b200 as q
     return q.gemm_fused_rq(A_bf16, B, N, fmt=fmt, rotate=rotate, four6=four6,
-                           out=guarded((A_bf16.shape[0], N), out_dtype or torch.float32))
+                           out=guarded((A_bf16.shape[0], N), out_dtype or torch.float32), A_amax_in=A_amax_in,
+                           A_amax_out=A_amax_out)

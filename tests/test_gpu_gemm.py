@@ -198,3 +198,32 @@ def test_fused_in_kernel_quantization_is_repeatable():
     for y in ys[1:]:
         assert int((y.view(torch.int16) != ys[0].view(torch.int16)).sum()) == 0
     assert q.qfp4_last_device_error() == 0
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 264, 640), (1000, 768, 384), (100, 256, 512)])
+@pytest.mark.parametrize("scale", [1.0, 0.5])
+def test_fused_with_given_and_reported_amax(M, N, K, scale):
+    """NVFP4 fused call under a supplied tensor amax of A (the own amax, or a
+    stale one x0.5 that saturates the top blocks): A's operand and the
+    outputs follow the oracle under the same amax, and the amax the call
+    reports is A's own (rotated) amax bit for bit.  M = 100 takes the
+    quantize-then-GEMM path."""
+    a = synth.cfg5_A(M, K, seed=M + K)
+    B = oracle.quantize(synth.cfg5_B(N, K, seed=N), oracle.NVFP4, rotate=True)
+    own = oracle.tensor_amax(a, rotate=True)
+    amax = float(np.float32(own * scale))
+    A = oracle.quantize_ex(a, oracle.NVFP4, rotate=True, amax_in=amax)
+    got_amax = G.guarded((1,), torch.float32)
+    wsb = q.qfp4_gemm_fused_rq_workspace_bytes(M, N, K, q.NVFP4)
+    ws = G.guarded((wsb,), torch.uint8)
+    y = G.guarded((M, N), torch.float32)
+    q.gemm_fused_rq(to_dev(a), _upload(B), N, fmt=q.NVFP4, rotate=True, out=y, workspace=ws,
+                    A_amax_in=torch.tensor([amax], dtype=torch.float32, device="cuda"), A_amax_out=got_amax)
+    co, so, to = q.qfp4_gemm_fused_rq_workspace_layout(M, N, K, q.NVFP4)
+    w = host(ws)
+    assert np.array_equal(w[co:co + M * K // 2], A["codes"].ravel())
+    assert np.array_equal(w[so:so + M * K // 16], A["scales"].ravel())
+    assert w[to:to + 4].view(np.float32)[0] == A["tscale"][0]
+    assert host(got_amax)[0] == np.float32(own)
+    rows, cols = _all_pairs(M, N)
+    _check(host(y), A, B, M, N, K, oracle.NVFP4, rows, cols)
