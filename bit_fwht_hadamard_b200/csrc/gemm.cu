@@ -507,9 +507,11 @@ __global__ void __launch_bounds__(GM_THREADS, 1)
 // No TMA multicast.
 constexpr int G2_BM = 256, G2_BN = 256;                   // cluster tile
 // warp roles by warpgroup: 0 operand producer, 1 MMA issuer, 2 scale producer
-// (3 idle); 4..7 scale warps; 8..15 epilogue.  setmaxnreg moves registers from the first two
-// warpgroups to the epilogue: 128 x 48 + 128 x 80 + 256 x 184 = 63488 of the
-// 512 x 128 = 65536 the block is launched with.
+// (3 idle); 4..7 scale warps; 8..15 epilogue; in the fused kernel 16..19
+// quantizer warps.  setmaxnreg moves registers from the first two warpgroups
+// to the others: 128 x 48 + 128 x 80 + 256 x 184 = 63488 of the 512 x 128 =
+// 65536 the plain kernel is launched with; 128 x 40 + 128 x 80 + 256 x 112 +
+// 128 x 120 = 59392 of the 640 x 96 = 61440 of the fused kernel.
 constexpr int G2_SF_WARPS = 4;
 constexpr int G2_THREADS = 512;
 constexpr int G2_SF_WARP0 = 4, G2_EPI_WARP0 = 8;
@@ -711,61 +713,76 @@ __device__ __forceinline__ void fused_quantize_rows(const GemmParams &p, int qwa
     }
     const NvScale nz = nv_scale_setup(s_t);
     const int units = p.K / 64;
+    const int cpr = (units + 31) / 32;           // 2048-element chunks per row
     const int64_t K = p.K;
-    // the rows this warp takes next are pulled into L2 two rows ahead, so the
-    // row loads below meet L2 rather than HBM latency
+    // This warp's work is the sequence of (row, chunk) items of its rows.
+    // The loads of the next item are issued before the current one is
+    // worked on, so their latency overlaps the arithmetic; the rows two
+    // ahead are also pulled into L2.
     auto prefetch_row = [&](int rp) {
         if (lane == 0 && rp < p.M) bulk_prefetch_l2(p.fq.A + static_cast<int64_t>(rp) * K, static_cast<uint32_t>(2 * K));
+    };
+    auto load_item = [&](int r, int c, uint4 (&raw)[8]) {
+        const int u = 32 * c + lane;
+        if (r < p.M && u < units) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(p.fq.A + static_cast<int64_t>(r) * K + u * 64);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) raw[i] = src[i];
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) raw[i] = make_uint4(0u, 0u, 0u, 0u);
+        }
     };
     prefetch_row(qwarp);
     prefetch_row(qwarp + nqwarps);
     float own_max = 0.0f;                        // this warp's |x| maximum (after rotation), when asked for
-    for (int r = qwarp; r < p.M && !*abort_flag; r += nqwarps) {
-        prefetch_row(r + 2 * nqwarps);
-        const uint16_t *row = p.fq.A + static_cast<int64_t>(r) * K;
-        const int64_t rb = r >> 7, rr = r & 127;
-        for (int c0 = 0; c0 < units; c0 += 32) {
-            const int u = c0 + lane;
-            const bool active = u < units;               // pairs of lanes are active together (units is even with ROT)
-            uint64_t v[32];
-            if (active) {
-                const uint4 *src = reinterpret_cast<const uint4 *>(row + static_cast<int64_t>(u) * 64);
+    int r = qwarp, c = 0;
+    uint4 cur[8];
+    load_item(r, c, cur);
+    while (r < p.M && !*abort_flag) {
+        const int rn = c + 1 < cpr ? r : r + nqwarps, cn = c + 1 < cpr ? c + 1 : 0;
+        if (c == 0) prefetch_row(r + 2 * nqwarps);
+        uint4 nxt[8];
+        load_item(rn, cn, nxt);
+        const int u = 32 * c + lane;
+        const bool active = u < units;           // pairs of lanes are active together (units is even with ROT)
+        uint64_t v[32];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint4 w = src[c];
-                    v[4 * c + 0] = bf16x2_to_f2(w.x);
-                    v[4 * c + 1] = bf16x2_to_f2(w.y);
-                    v[4 * c + 2] = bf16x2_to_f2(w.z);
-                    v[4 * c + 3] = bf16x2_to_f2(w.w);
-                }
+        for (int i = 0; i < 8; ++i) {
+            v[4 * i + 0] = bf16x2_to_f2(cur[i].x);
+            v[4 * i + 1] = bf16x2_to_f2(cur[i].y);
+            v[4 * i + 2] = bf16x2_to_f2(cur[i].z);
+            v[4 * i + 3] = bf16x2_to_f2(cur[i].w);
+        }
+        if (ROT) fwht_packed<32, !RAW>(v, (lane & 1) != 0);
+        if (p.fq.amax_out) own_max = fmaxf(own_max, absmax_pairs<32>(v));   // NVFP4 (not RAW): normalised values
+        UnitP<32> o;
+        quant_unit_packed<32, FMT, false, false, RAW>(v, 0, nz, 0, o);
+        if (active) {
+            const int64_t rb = r >> 7, rr = r & 127;
+            uint4 *cd = reinterpret_cast<uint4 *>(p.fq.codes + (static_cast<int64_t>(r) * K + u * 64) / 2);
+            cd[0] = make_uint4(o.codes[0], o.codes[1], o.codes[2], o.codes[3]);
+            cd[1] = make_uint4(o.codes[4], o.codes[5], o.codes[6], o.codes[7]);
+            uint8_t *chunk = p.fq.chunks + (rb * p.NC) * 512 + (rr & 31) * 16 + (rr >> 5) * 4;
+            if (FMT == QFP4_NVFP4) {
+                *reinterpret_cast<uint32_t *>(p.fq.scales + static_cast<int64_t>(r) * (K / 16) + u * 4) = o.scales[0];
+                *reinterpret_cast<uint32_t *>(chunk + static_cast<int64_t>(u) * 512) = o.scales[0];
             } else {
-#pragma unroll
-                for (int c = 0; c < 32; ++c) v[c] = 0ull;
-            }
-            if (ROT) fwht_packed<32, !RAW>(v, (lane & 1) != 0);
-            if (p.fq.amax_out) own_max = fmaxf(own_max, absmax_pairs<32>(v));   // NVFP4 (not RAW): normalised values
-            UnitP<32> o;
-            quant_unit_packed<32, FMT, false, false, RAW>(v, 0, nz, 0, o);
-            if (active) {
-                uint4 *cd = reinterpret_cast<uint4 *>(p.fq.codes + (static_cast<int64_t>(r) * K + u * 64) / 2);
-                cd[0] = make_uint4(o.codes[0], o.codes[1], o.codes[2], o.codes[3]);
-                cd[1] = make_uint4(o.codes[4], o.codes[5], o.codes[6], o.codes[7]);
-                uint8_t *chunk = p.fq.chunks + (rb * p.NC) * 512 + (rr & 31) * 16 + (rr >> 5) * 4;
-                if (FMT == QFP4_NVFP4) {
-                    *reinterpret_cast<uint32_t *>(p.fq.scales + static_cast<int64_t>(r) * (K / 16) + u * 4) =
-                        o.scales[0];
-                    *reinterpret_cast<uint32_t *>(chunk + static_cast<int64_t>(u) * 512) = o.scales[0];
-                } else {
-                    const uint16_t sc = static_cast<uint16_t>(o.scales[0]);
-                    *reinterpret_cast<uint16_t *>(p.fq.scales + static_cast<int64_t>(r) * (K / 32) + u * 2) = sc;
-                    *reinterpret_cast<uint16_t *>(chunk + static_cast<int64_t>(u >> 1) * 512 + (u & 1) * 2) = sc;
-                }
+                const uint16_t sc = static_cast<uint16_t>(o.scales[0]);
+                *reinterpret_cast<uint16_t *>(p.fq.scales + static_cast<int64_t>(r) * (K / 32) + u * 2) = sc;
+                *reinterpret_cast<uint16_t *>(chunk + static_cast<int64_t>(u >> 1) * 512 + (u & 1) * 2) = sc;
             }
         }
-        fence_proxy_async_global();
-        __threadfence();
-        __syncwarp();
-        if (lane == 0) atomicAdd(&p.fq.ready[rb], 1u);
+        if (c == cpr - 1) {                      // row r complete: publish it
+            fence_proxy_async_global();
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) atomicAdd(&p.fq.ready[r >> 7], 1u);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) cur[i] = nxt[i];
+        r = rn;
+        c = cn;
     }
     if (p.fq.amax_out) {
 #pragma unroll
@@ -1010,7 +1027,7 @@ __global__ void __launch_bounds__(g2_threads(FUSED), 1)
     }
     if constexpr (FUSED) {
         if (warp >= G2_Q_WARP0) {
-            asm volatile("setmaxnreg.inc.sync.aligned.u32 112;");
+            asm volatile("setmaxnreg.inc.sync.aligned.u32 120;");
             // ------------------------------------------------ quantizer warps (fused kernel, both CTAs)
             fused_quantize_rows<FMT, ROT>(p, static_cast<int>(blockIdx.x) * G2_Q_WARPS + (warp - G2_Q_WARP0),
                                           static_cast<int>(gridDim.x) * G2_Q_WARPS, lane, &abort_flag);
@@ -1022,7 +1039,7 @@ __global__ void __launch_bounds__(g2_threads(FUSED), 1)
         // The fused kernel's epilogue warps hold half as many registers: they
         // read the accumulator in two 64-column chunks (hand-back after the
         // second read), the plain kernel's in one of 128 columns.
-        if constexpr (FUSED) asm volatile("setmaxnreg.inc.sync.aligned.u32 120;");
+        if constexpr (FUSED) asm volatile("setmaxnreg.inc.sync.aligned.u32 112;");
         else asm volatile("setmaxnreg.inc.sync.aligned.u32 184;");
         // ------------------------------------------------ epilogue (both CTAs: own 128 rows)
         constexpr int CH = FUSED ? 2 : 1;                 // column chunks per tile
