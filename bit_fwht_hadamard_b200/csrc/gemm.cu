@@ -46,31 +46,15 @@ constexpr int GM_GROUP_M = 8;                             // tile raster: 8 m-bl
 // chunks of 4 scale groups per stage and 128-row block
 __host__ __device__ constexpr int gm_cps(int fmt) { return fmt == QFP4_NVFP4 ? 4 : fmt == QFP4_MXFP4 ? 2 : 1; }
 
-// The fused rotate + quantize + GEMM: A given in bf16, quantized inside the
-// GEMM kernel by its quantizer warps into the workspace.
-struct FusedQuant {
-    const uint16_t *A;          // bf16 M x K, row-major
-    uint8_t *codes;             // out: M x K/2 codes
-    uint8_t *scales;            // out: row-major M x K/g scales
-    uint8_t *chunks;            // out: A's scale chunks (the GEMM's sfa)
-    float *tscale;              // out: NVFP4 s_t
-    const float *partials;      // NVFP4: partial maxima of the amax pass
-    int n_partials;
-    const float *amax_in;       // NVFP4: caller-supplied tensor amax of A (then no amax pass), or NULL
-    float *amax_out;            // NVFP4: receives A's own (rotated) amax, or NULL (zeroed by the host)
-    unsigned int *ready;        // per 128-row block of A: rows quantized so far
-};
-
 struct GemmParams {
     int M, N, K;
-    int KT;                 // k tiles (256 FP4 or 128 FP8 elements)
+    int KT;                 // k tiles of 256
     int tiles_m, tiles_n;
     int NC;                 // scale chunks per 128-row block (KT * cps)
     const uint8_t *sfa;     // rearranged scales (workspace)
     const uint8_t *sfb;
     const float *tA, *tB;   // NVFP4 tensor scales
     void *out;
-    FusedQuant fq;          // fused kernel only
 };
 
 // ------------------------------------------------------------------ PTX: tcgen05
@@ -156,18 +140,6 @@ __device__ __forceinline__ void tmem_ld16x256b_x16(uint32_t taddr, uint32_t *r)
           "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]),
           "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]),
           "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
-        : "r"(taddr));
-}
-// the same shape with 8 repetitions: 64 consecutive columns, 32 registers
-__device__ __forceinline__ void tmem_ld16x256b_x8(uint32_t taddr, uint32_t *r)
-{
-    asm volatile(
-        "tcgen05.ld.sync.aligned.16x256b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
-        "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
-          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
-          "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
@@ -507,17 +479,12 @@ __global__ void __launch_bounds__(GM_THREADS, 1)
 // No TMA multicast.
 constexpr int G2_BM = 256, G2_BN = 256;                   // cluster tile
 // warp roles by warpgroup: 0 operand producer, 1 MMA issuer, 2 scale producer
-// (3 idle); 4..7 scale warps; 8..15 epilogue; in the fused kernel 16..19
-// quantizer warps.  setmaxnreg moves registers from the first two warpgroups
-// to the others: 128 x 48 + 128 x 80 + 256 x 184 = 63488 of the 512 x 128 =
-// 65536 the plain kernel is launched with; 128 x 40 + 128 x 80 + 256 x 112 +
-// 128 x 120 = 59392 of the 640 x 96 = 61440 of the fused kernel.
+// (3 idle); 4..7 scale warps; 8..15 epilogue.  setmaxnreg moves registers from the first two
+// warpgroups to the epilogue: 128 x 48 + 128 x 80 + 256 x 184 = 63488 of the
+// 512 x 128 = 65536 the block is launched with.
 constexpr int G2_SF_WARPS = 4;
 constexpr int G2_THREADS = 512;
 constexpr int G2_SF_WARP0 = 4, G2_EPI_WARP0 = 8;
-// The fused kernel adds a fifth warpgroup (warps 16..19) of quantizer warps.
-constexpr int G2_Q_WARP0 = 16, G2_Q_WARPS = 4;
-__host__ __device__ constexpr int g2_threads(bool fused) { return fused ? G2_THREADS + 32 * G2_Q_WARPS : G2_THREADS; }
 constexpr int G2_A_BYTES = 128 * GM_BKB;                  // this CTA's A rows
 constexpr int G2_B_BYTES = 128 * GM_BKB;                  // this CTA's half of B
 constexpr int G2_STAGE_BYTES = G2_A_BYTES + G2_B_BYTES;
@@ -641,166 +608,8 @@ __device__ __forceinline__ void g2_exit(uint32_t tmem, bool dealloc)
     if (dealloc) tmem_dealloc_cg2(tmem, GM_TMEM_COLS);
 }
 
-// ------------------------------------------------------------------ fused quantizer
-__device__ __forceinline__ void fence_proxy_async_global()
-{
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
-// pull `bytes` (a multiple of 16, 16-byte aligned) of global memory into L2
-__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes)
-{
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-
-__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int *p)
-{
-    unsigned int v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// Wait (bounded) until `want` (> 0) rows of a 128-row block of A are
-// quantized, then order the TMA (async-proxy) reads of them after the
-// acquire.  A block past the end of A (the partner half of the last tile
-// pair) has no rows and is not waited on.
-__device__ __forceinline__ bool wait_rows_ready(const unsigned int *ready, unsigned int want)
-{
-    if (ld_acquire_gpu(ready) < want) {
-        const uint64_t t0 = global_ns();
-        for (uint32_t i = 0;; ++i) {
-            if (ld_acquire_gpu(ready) >= want) break;
-            if (i >= kSpinLimit || ((i & 255u) == 255u && global_ns() - t0 > kWaitLimitNs)) {
-                record_error(DEV_ERR_TIMEOUT);
-                return false;
-            }
-        }
-    }
-    fence_proxy_async_global();
-    return true;
-}
-
-// NVFP4 s_t of A in the fused kernel (every lane of a warp gets it): from the
-// caller's amax, or the maximum of the amax pass's partial maxima.
-__device__ __forceinline__ float fused_tscale(const FusedQuant &fq, int lane)
-{
-    if (fq.amax_in) return __fdiv_rn(*fq.amax_in, 2688.0f);
-    float m = 0.0f;
-    for (int i = lane; i < fq.n_partials; i += 32) m = fmaxf(m, fq.partials[i]);
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    return __fdiv_rn(m, 2688.0f);
-}
-
-// Rows of A quantized by the fused kernel's quantizer warps: warp g of G
-// takes rows g, g + G, ... (ascending, so the 128-row blocks the tile raster
-// needs first are ready first).  A lane holds 64 consecutive elements of a
-// row (lanes 2i, 2i+1 one 128-element rotation block), exactly as in the
-// 1D quantize kernel: FWHT-128 (rotate), then the group scales and RNE
-// codes.  It writes its 32 code bytes, its row-major scale bytes and its
-// word (NVFP4) or half word (MXFP4) of the scale chunk the GEMM reads; after
-// the whole row, the block's counter is raised (release at GPU scope after a
-// proxy fence, since the GEMM reads these bytes with TMA).
-template <int FMT, bool ROT>
-__device__ __forceinline__ void fused_quantize_rows(const GemmParams &p, int qwarp, int nqwarps, int lane,
-                                                    volatile int *abort_flag)
-{
-    constexpr bool RAW = ROT && FMT == QFP4_MXFP4;     // normalisation folded into the 2^-k multiply
-    float s_t = 0.0f;
-    if (FMT == QFP4_NVFP4) {
-        s_t = fused_tscale(p.fq, lane);
-        if (qwarp == 0 && lane == 0) *p.fq.tscale = s_t;
-    }
-    const NvScale nz = nv_scale_setup(s_t);
-    const int units = p.K / 64;
-    const int cpr = (units + 31) / 32;           // 2048-element chunks per row
-    const int64_t K = p.K;
-    // This warp's work is the sequence of (row, chunk) items of its rows.
-    // The loads of the next item are issued before the current one is
-    // worked on, so their latency overlaps the arithmetic; the rows two
-    // ahead are also pulled into L2.
-    auto prefetch_row = [&](int rp) {
-        if (lane == 0 && rp < p.M) bulk_prefetch_l2(p.fq.A + static_cast<int64_t>(rp) * K, static_cast<uint32_t>(2 * K));
-    };
-    auto load_item = [&](int r, int c, uint4 (&raw)[8]) {
-        const int u = 32 * c + lane;
-        if (r < p.M && u < units) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(p.fq.A + static_cast<int64_t>(r) * K + u * 64);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) raw[i] = src[i];
-        } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) raw[i] = make_uint4(0u, 0u, 0u, 0u);
-        }
-    };
-    prefetch_row(qwarp);
-    prefetch_row(qwarp + nqwarps);
-    float own_max = 0.0f;                        // this warp's |x| maximum (after rotation), when asked for
-    int r = qwarp, c = 0;
-    uint4 cur[8];
-    load_item(r, c, cur);
-    while (r < p.M && !*abort_flag) {
-        const int rn = c + 1 < cpr ? r : r + nqwarps, cn = c + 1 < cpr ? c + 1 : 0;
-        if (c == 0) prefetch_row(r + 2 * nqwarps);
-        uint4 nxt[8];
-        load_item(rn, cn, nxt);
-        const int u = 32 * c + lane;
-        const bool active = u < units;           // pairs of lanes are active together (units is even with ROT)
-        uint64_t v[32];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            v[4 * i + 0] = bf16x2_to_f2(cur[i].x);
-            v[4 * i + 1] = bf16x2_to_f2(cur[i].y);
-            v[4 * i + 2] = bf16x2_to_f2(cur[i].z);
-            v[4 * i + 3] = bf16x2_to_f2(cur[i].w);
-        }
-        if (ROT) fwht_packed<32, !RAW>(v, (lane & 1) != 0);
-        if (p.fq.amax_out) own_max = fmaxf(own_max, absmax_pairs<32>(v));   // NVFP4 (not RAW): normalised values
-        UnitP<32> o;
-        quant_unit_packed<32, FMT, false, false, RAW>(v, 0, nz, 0, o);
-        if (active) {
-            const int64_t rb = r >> 7, rr = r & 127;
-            uint4 *cd = reinterpret_cast<uint4 *>(p.fq.codes + (static_cast<int64_t>(r) * K + u * 64) / 2);
-            cd[0] = make_uint4(o.codes[0], o.codes[1], o.codes[2], o.codes[3]);
-            cd[1] = make_uint4(o.codes[4], o.codes[5], o.codes[6], o.codes[7]);
-            uint8_t *chunk = p.fq.chunks + (rb * p.NC) * 512 + (rr & 31) * 16 + (rr >> 5) * 4;
-            if (FMT == QFP4_NVFP4) {
-                *reinterpret_cast<uint32_t *>(p.fq.scales + static_cast<int64_t>(r) * (K / 16) + u * 4) = o.scales[0];
-                *reinterpret_cast<uint32_t *>(chunk + static_cast<int64_t>(u) * 512) = o.scales[0];
-            } else {
-                const uint16_t sc = static_cast<uint16_t>(o.scales[0]);
-                *reinterpret_cast<uint16_t *>(p.fq.scales + static_cast<int64_t>(r) * (K / 32) + u * 2) = sc;
-                *reinterpret_cast<uint16_t *>(chunk + static_cast<int64_t>(u >> 1) * 512 + (u & 1) * 2) = sc;
-            }
-        }
-        if (c == cpr - 1) {                      // row r complete: publish it
-            fence_proxy_async_global();
-            __threadfence();
-            __syncwarp();
-            if (lane == 0) atomicAdd(&p.fq.ready[r >> 7], 1u);
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) cur[i] = nxt[i];
-        r = rn;
-        c = cn;
-    }
-    if (p.fq.amax_out) {
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) own_max = fmaxf(own_max, __shfl_xor_sync(0xFFFFFFFFu, own_max, o));
-        // non-negative binary32 values order like their bit patterns; the host zeroed *amax_out
-        if (lane == 0) atomicMax(reinterpret_cast<unsigned int *>(p.fq.amax_out), __float_as_uint(own_max));
-    }
-}
-
-// rows of 128-row block rb of A (0 past the end)
-__device__ __forceinline__ unsigned int rows_in_block(int rb, int M)
-{
-    const int r = M - rb * 128;
-    return r <= 0 ? 0u : static_cast<unsigned int>(r < 128 ? r : 128);
-}
-
-template <int FMT, int OUT, bool FUSED = false, bool ROT = false>
-__global__ void __launch_bounds__(g2_threads(FUSED), 1)
+template <int FMT, int OUT>
+__global__ void __launch_bounds__(G2_THREADS, 1)
     k_gemm_bs2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB, GemmParams p)
 {
@@ -864,8 +673,7 @@ __global__ void __launch_bounds__(g2_threads(FUSED), 1)
     // Each role ends with its own copy of the exit sequence, so that the
     // register-count regions set by setmaxnreg never merge again.
     if (warp < G2_SF_WARP0) {
-        if constexpr (FUSED) asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
-        else asm volatile("setmaxnreg.dec.sync.aligned.u32 48;");
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 48;");
         if (warp == 0) {
         // ------------------------------------------------ producer (both CTAs)
         if (lane == 0) {
@@ -875,8 +683,6 @@ __global__ void __launch_bounds__(g2_threads(FUSED), 1)
                 int mb, nb;
                 tile_coords(t, tiles_m, tiles_n, mb, nb);
                 const int rb_a = 2 * mb + static_cast<int>(rank);   // this CTA's 128-row block of A
-                if (FUSED && rows_in_block(rb_a, p.M) &&
-                    !wait_rows_ready(p.fq.ready + rb_a, rows_in_block(rb_a, p.M))) { abort_flag = 1; break; }
                 for (int kt = 0; kt < p.KT; ++kt, ++it) {
                     const int s = it % G2_STAGES;
                     const uint32_t ph = (it / G2_STAGES) & 1u;
@@ -933,8 +739,6 @@ __global__ void __launch_bounds__(g2_threads(FUSED), 1)
                 int mb, nb;
                 tile_coords(t, tiles_m, tiles_n, mb, nb);
                 const int rb_a = 2 * mb + static_cast<int>(rank);
-                if (FUSED && rows_in_block(rb_a, p.M) &&
-                    !wait_rows_ready(p.fq.ready + rb_a, rows_in_block(rb_a, p.M))) { abort_flag = 1; break; }
                 for (int kt = 0; kt < p.KT; ++kt, ++it) {
                     const int s = it % G2_SF_SLOTS;
                     if (!mbar_wait(&sfs_empty[s], ((it / G2_SF_SLOTS) & 1u) ^ 1u)) { abort_flag = 1; break; }
@@ -1025,93 +829,60 @@ __global__ void __launch_bounds__(g2_threads(FUSED), 1)
         g2_exit(tmem, false);
         return;
     }
-    if constexpr (FUSED) {
-        if (warp >= G2_Q_WARP0) {
-            asm volatile("setmaxnreg.inc.sync.aligned.u32 120;");
-            // ------------------------------------------------ quantizer warps (fused kernel, both CTAs)
-            fused_quantize_rows<FMT, ROT>(p, static_cast<int>(blockIdx.x) * G2_Q_WARPS + (warp - G2_Q_WARP0),
-                                          static_cast<int>(gridDim.x) * G2_Q_WARPS, lane, &abort_flag);
-            g2_exit(tmem, false);
-            return;
-        }
-    }
     {
-        // The fused kernel's epilogue warps hold half as many registers: they
-        // read the accumulator in two 64-column chunks (hand-back after the
-        // second read), the plain kernel's in one of 128 columns.
-        if constexpr (FUSED) asm volatile("setmaxnreg.inc.sync.aligned.u32 112;");
-        else asm volatile("setmaxnreg.inc.sync.aligned.u32 184;");
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 184;");
         // ------------------------------------------------ epilogue (both CTAs: own 128 rows)
-        constexpr int CH = FUSED ? 2 : 1;                 // column chunks per tile
-        constexpr int RPH = 64 / CH;                      // registers per 16-lane half per chunk
         const int q = warp & 3;
         const int h = (warp - G2_EPI_WARP0) >> 2;
         const uint32_t acc_empty_leader = mapa_shared(smem_u32(&acc_empty), 0);
         float alpha = 1.0f;
-        if (FMT == QFP4_NVFP4) {
-            float tA;
-            if constexpr (FUSED) {
-                tA = fused_tscale(p.fq, lane);              // A's s_t, as the quantizer warps form it
-            } else {
-                tA = *p.tA;
-            }
-            alpha = __fmul_rn(tA, *p.tB);
-        }
+        if (FMT == QFP4_NVFP4) alpha = __fmul_rn(*p.tA, *p.tB);
         int ti = 0;
         for (int t = cluster; t < ntiles && !abort_flag; t += nclusters, ++ti) {
             int mb, nb;
             tile_coords(t, tiles_m, tiles_n, mb, nb);
             if (!warp_wait(&acc_full, ti & 1)) { abort_flag = 1; break; }
             tc_fence_after();
+            uint32_t r[128];
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+                tmem_ld16x256b_x16(tmem + (static_cast<uint32_t>(32 * q + 16 * hh) << 16) + 128 * h, r + 64 * hh);
+            tmem_ld_wait();
+            reg_fence<128>(r);
+            // the accumulator is in registers: hand it back at once, so the
+            // next tile's MMAs overlap these stores
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+
+            const int col0 = nb * G2_BN + 128 * h + 2 * (lane & 3);
             const int row_base = mb * G2_BM + 128 * static_cast<int>(rank);
 #pragma unroll
-            for (int ch = 0; ch < CH; ++ch) {
-                uint32_t r[2 * RPH];
+            for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const uint32_t addr = tmem + (static_cast<uint32_t>(32 * q + 16 * hh) << 16) + 128 * h + 64 * ch;
-                    if constexpr (CH == 1) tmem_ld16x256b_x16(addr, r + RPH * hh);
-                    else tmem_ld16x256b_x8(addr, r + RPH * hh);
-                }
-                tmem_ld_wait();
-                reg_fence<2 * RPH>(r);
-                if (ch == CH - 1) {
-                    // the whole accumulator is in registers: hand it back at
-                    // once, so the next tile's MMAs overlap these stores
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
-                }
-                // r[RPH hh + 4j + {0,1}]: row 32q + 16hh + lane/4, columns 8j + 2(lane%4) + {0,1}
-                // of the chunk; r[RPH hh + 4j + {2,3}]: the row 8 below
-                const int col0 = nb * G2_BN + 128 * h + 64 * ch + 2 * (lane & 3);
+                for (int e = 0; e < 2; ++e) {
+                    const int row = row_base + 32 * q + 16 * hh + 8 * e + (lane >> 2);
+                    if (row >= p.M) continue;
+                    if (OUT == QFP4_F32) {
+                        float *o = static_cast<float *>(p.out) + static_cast<int64_t>(row) * p.N + col0;
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh)
+                        for (int j = 0; j < 16; ++j)
+                            if (col0 + 8 * j < p.N)
+                                *reinterpret_cast<float2 *>(o + 8 * j) =
+                                    make_float2(__fmul_rn(__uint_as_float(r[64 * hh + 4 * j + 2 * e]), alpha),
+                                                __fmul_rn(__uint_as_float(r[64 * hh + 4 * j + 2 * e + 1]), alpha));
+                    } else {
+                        uint16_t *o = static_cast<uint16_t *>(p.out) + static_cast<int64_t>(row) * p.N + col0;
 #pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int row = row_base + 32 * q + 16 * hh + 8 * e + (lane >> 2);
-                        if (row >= p.M) continue;
-                        if (OUT == QFP4_F32) {
-                            float *o = static_cast<float *>(p.out) + static_cast<int64_t>(row) * p.N + col0;
-#pragma unroll
-                            for (int j = 0; j < RPH / 4; ++j)
-                                if (col0 + 8 * j < p.N)
-                                    *reinterpret_cast<float2 *>(o + 8 * j) =
-                                        make_float2(__fmul_rn(__uint_as_float(r[RPH * hh + 4 * j + 2 * e]), alpha),
-                                                    __fmul_rn(__uint_as_float(r[RPH * hh + 4 * j + 2 * e + 1]), alpha));
-                        } else {
-                            uint16_t *o = static_cast<uint16_t *>(p.out) + static_cast<int64_t>(row) * p.N + col0;
-#pragma unroll
-                            for (int j = 0; j < RPH / 4; ++j)
-                                if (col0 + 8 * j < p.N) {
-                                    const __nv_bfloat162 b2 = __floats2bfloat162_rn(
-                                        __fmul_rn(__uint_as_float(r[RPH * hh + 4 * j + 2 * e]), alpha),
-                                        __fmul_rn(__uint_as_float(r[RPH * hh + 4 * j + 2 * e + 1]), alpha));
-                                    *reinterpret_cast<__nv_bfloat162 *>(o + 8 * j) = b2;
-                                }
-                        }
+                        for (int j = 0; j < 16; ++j)
+                            if (col0 + 8 * j < p.N) {
+                                const __nv_bfloat162 b2 =
+                                    __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[64 * hh + 4 * j + 2 * e]), alpha),
+                                                          __fmul_rn(__uint_as_float(r[64 * hh + 4 * j + 2 * e + 1]), alpha));
+                                *reinterpret_cast<__nv_bfloat162 *>(o + 8 * j) = b2;
+                            }
                     }
-            }
+                }
         }
     }
     g2_exit(tmem, false);
@@ -1171,56 +942,15 @@ static int launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const GemmP
     return QFP4_OK;
 }
 
-// Clusters of the 2-CTA kernel that can be resident at once on this device
-// (the fused kernel's producers wait on rows that quantizer warps of other
-// CTAs write, so its whole grid must be resident).  Cached per device.
-template <auto Kern>
-static int max_resident_clusters(int threads, int smem)
-{
-    constexpr int kMaxDevices = 64;
-    static std::atomic<int> cache[kMaxDevices];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) {
-        (void)cudaGetLastError();
-        return 0;
-    }
-    if (dev >= 0 && dev < kMaxDevices && cache[dev].load() > 0) return cache[dev].load();
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2, 1, 1);
-    cfg.blockDim = dim3(threads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, Kern, &cfg) != cudaSuccess) {
-        (void)cudaGetLastError();
-        return 0;
-    }
-    if (dev >= 0 && dev < kMaxDevices && n > 0) cache[dev].store(n);
-    return n;
-}
-
-template <int FMT, int OUT, bool FUSED = false, bool ROT = false>
+template <int FMT, int OUT>
 static int launch_gemm2(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tsa, const CUtensorMap &tsb,
-                        const GemmParams &p, int ntiles, cudaStream_t s)
+                        const GemmParams &p, int grid, cudaStream_t s)
 {
-    auto kern = k_gemm_bs2<FMT, OUT, FUSED, ROT>;
-    constexpr int threads = g2_threads(FUSED);
-    if (ensure_dyn_smem<k_gemm_bs2<FMT, OUT, FUSED, ROT>>(G2_SMEM) != QFP4_OK) return QFP4_ERR_CUDA;
-    int clusters = imin<int>(ntiles, num_sms() / 2);
-    if (FUSED) {
-        const int resident = max_resident_clusters<k_gemm_bs2<FMT, OUT, FUSED, ROT>>(threads, G2_SMEM);
-        if (resident < 1) return QFP4_ERR_CUDA;
-        clusters = imin(clusters, resident);
-    }
+    auto kern = k_gemm_bs2<FMT, OUT>;
+    if (ensure_dyn_smem<k_gemm_bs2<FMT, OUT>>(G2_SMEM) != QFP4_OK) return QFP4_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * clusters, 1, 1);
-    cfg.blockDim = dim3(threads, 1, 1);
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(G2_THREADS, 1, 1);
     cfg.dynamicSmemBytes = G2_SMEM;
     cfg.stream = s;
     cudaLaunchAttribute attr[2];
@@ -1243,15 +973,9 @@ static int launch_gemm2(const CUtensorMap &ta, const CUtensorMap &tb, const CUte
 // Main kernel on already rearranged scales (sfa / sfb in the chunk layout).
 // Problems taller than one 128-row block run on CTA pairs (256 x 256 tiles),
 // the rest on single CTAs (128 x 256 tiles).
-// What the fused kernel needs besides the plain GEMM's arguments.
-struct FusedArgs {
-    FusedQuant fq;
-    bool rotate;
-};
-
 int gemm_core(const uint8_t *A_codes, const uint8_t *sfa, const float *A_tscale, const uint8_t *B_codes,
               const uint8_t *sfb, const float *B_tscale, int64_t M, int64_t N, int64_t K, qfp4_fmt fmt,
-              qfp4_dtype out_dt, void *out, cudaStream_t stream, const FusedArgs *fused = nullptr)
+              qfp4_dtype out_dt, void *out, cudaStream_t stream)
 {
     const GemmLayout L = gemm_layout(M, N, K, fmt);
     const bool pair = M > GM_BM;
@@ -1286,7 +1010,6 @@ int gemm_core(const uint8_t *A_codes, const uint8_t *sfa, const float *A_tscale,
     p.tA = A_tscale;
     p.tB = B_tscale;
     p.out = out;
-    p.fq = fused ? fused->fq : FusedQuant{};
     if (pair) {
         // scale chunks viewed as rows of 128 B (4 rows per 512-byte chunk)
         const int cps = gm_cps(fmt);
@@ -1309,23 +1032,15 @@ int gemm_core(const uint8_t *A_codes, const uint8_t *sfa, const float *A_tscale,
             if (st != QFP4_OK) return st;
         }
         const int ntiles = static_cast<int>(((M + G2_BM - 1) / G2_BM) * ((N + G2_BN - 1) / G2_BN));
-        if (fused) {
-            // A is quantized inside the kernel (rotate: FWHT-128 first)
-#define QFP4_F(F, O) (fused->rotate ? launch_gemm2<F, O, true, true>(ta, tb, tsa, tsb, p, ntiles, stream) \
-                                    : launch_gemm2<F, O, true, false>(ta, tb, tsa, tsb, p, ntiles, stream))
-            if (fmt == QFP4_NVFP4) return out_dt == QFP4_F32 ? QFP4_F(QFP4_NVFP4, QFP4_F32) : QFP4_F(QFP4_NVFP4, QFP4_BF16);
-            if (fmt == QFP4_MXFP4) return out_dt == QFP4_F32 ? QFP4_F(QFP4_MXFP4, QFP4_F32) : QFP4_F(QFP4_MXFP4, QFP4_BF16);
-#undef QFP4_F
-            return QFP4_ERR_UNSUPPORTED;
-        }
+        const int grid = 2 * imin<int>(ntiles, num_sms() / 2);
         if (fmt == QFP4_MXFP8)
-            return out_dt == QFP4_F32 ? launch_gemm2<QFP4_MXFP8, QFP4_F32>(ta, tb, tsa, tsb, p, ntiles, stream)
-                                      : launch_gemm2<QFP4_MXFP8, QFP4_BF16>(ta, tb, tsa, tsb, p, ntiles, stream);
+            return out_dt == QFP4_F32 ? launch_gemm2<QFP4_MXFP8, QFP4_F32>(ta, tb, tsa, tsb, p, grid, stream)
+                                      : launch_gemm2<QFP4_MXFP8, QFP4_BF16>(ta, tb, tsa, tsb, p, grid, stream);
         if (fmt == QFP4_NVFP4)
-            return out_dt == QFP4_F32 ? launch_gemm2<QFP4_NVFP4, QFP4_F32>(ta, tb, tsa, tsb, p, ntiles, stream)
-                                      : launch_gemm2<QFP4_NVFP4, QFP4_BF16>(ta, tb, tsa, tsb, p, ntiles, stream);
-        return out_dt == QFP4_F32 ? launch_gemm2<QFP4_MXFP4, QFP4_F32>(ta, tb, tsa, tsb, p, ntiles, stream)
-                                  : launch_gemm2<QFP4_MXFP4, QFP4_BF16>(ta, tb, tsa, tsb, p, ntiles, stream);
+            return out_dt == QFP4_F32 ? launch_gemm2<QFP4_NVFP4, QFP4_F32>(ta, tb, tsa, tsb, p, grid, stream)
+                                      : launch_gemm2<QFP4_NVFP4, QFP4_BF16>(ta, tb, tsa, tsb, p, grid, stream);
+        return out_dt == QFP4_F32 ? launch_gemm2<QFP4_MXFP4, QFP4_F32>(ta, tb, tsa, tsb, p, grid, stream)
+                                  : launch_gemm2<QFP4_MXFP4, QFP4_BF16>(ta, tb, tsa, tsb, p, grid, stream);
     }
     const int grid = static_cast<int>(imin<int64_t>(static_cast<int64_t>(L.MB) * L.NT, num_sms()));
     if (fmt == QFP4_MXFP8)
@@ -1354,7 +1069,7 @@ int gemm_blockscaled(const uint8_t *A_codes, const uint8_t *A_scales, const floa
 // Workspace: quantized A (codes M*K/2, row-major scales M*K/g), its tensor
 // scale, the partial maxima of the amax pass, then the scale chunks of A and B.
 struct FusedLayout {
-    size_t codes, scales, tscale, partials, chunks, ready, total;
+    size_t codes, scales, tscale, partials, chunks, total;
 };
 
 static size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -1368,8 +1083,7 @@ static FusedLayout fused_layout(int64_t M, int64_t N, int64_t K, qfp4_fmt fmt)
     L.tscale = L.scales + align256(static_cast<size_t>(M) * K / g);
     L.partials = L.tscale + 256;
     L.chunks = L.partials + align256(sizeof(float) * kMaxPartials);
-    L.ready = L.chunks + align256(gemm_workspace(M, N, K, fmt));
-    L.total = L.ready + align256(sizeof(unsigned int) * ((M + 127) / 128));
+    L.total = L.chunks + align256(gemm_workspace(M, N, K, fmt));
     return L;
 }
 
@@ -1388,12 +1102,10 @@ size_t gemm_fused_rq_workspace(int64_t M, int64_t N, int64_t K, qfp4_fmt fmt)
     return fused_layout(M, N, K, fmt).total;
 }
 
-// A is quantized inside the GEMM kernel (rows overlapped with the MMAs of
-// rows already quantized) when the CTA-pair kernel runs (M > 128), K is a
-// multiple of 64 and four-over-six is off; otherwise A is quantized by the
-// 1D quantize kernel first and the plain GEMM follows.  NVFP4 needs the
-// tensor amax of the rotated A before any block scale: that pass runs first
-// either way.
+// A is rotated and quantized once by the 1D quantize kernel into the
+// workspace, then the scale prepass and the CTA-pair GEMM run; the kernels
+// follow each other through dependent launches.  NVFP4 measures A's tensor
+// amax first unless the caller supplies it (one read of A instead of two).
 int gemm_fused_rq(const void *A_bf16, int64_t M, int64_t K, int rotate, int four6, qfp4_fmt fmt,
                   const uint8_t *B_codes, const uint8_t *B_scales, const float *B_tscale, int64_t N, void *workspace,
                   qfp4_dtype out_dt, void *out, cudaStream_t stream, const float *amax_in, float *amax_out)
@@ -1403,48 +1115,14 @@ int gemm_fused_rq(const void *A_bf16, int64_t M, int64_t K, int rotate, int four
     uint8_t *a_codes = ws + F.codes, *a_scales = ws + F.scales;
     float *a_tscale = reinterpret_cast<float *>(ws + F.tscale);
     float *partials = reinterpret_cast<float *>(ws + F.partials);
-    const GemmLayout L = gemm_layout(M, N, K, fmt);
-    uint8_t *sfa = ws + F.chunks, *sfb = sfa + L.sfa_bytes;
-    int st;
-    if (M > GM_BM && K % 64 == 0 && !four6) {
-        FusedArgs fa;
-        fa.rotate = rotate != 0;
-        fa.fq.A = static_cast<const uint16_t *>(A_bf16);
-        fa.fq.codes = a_codes;
-        fa.fq.scales = a_scales;
-        fa.fq.chunks = sfa;
-        fa.fq.tscale = a_tscale;
-        fa.fq.partials = partials;
-        fa.fq.n_partials = 0;
-        fa.fq.amax_in = amax_in;
-        fa.fq.amax_out = nullptr;
-        fa.fq.ready = reinterpret_cast<unsigned int *>(ws + F.ready);
-        if (fmt == QFP4_NVFP4 && !amax_in) {
-            st = amax_pass_bf16(A_bf16, M * K, rotate != 0, partials, &fa.fq.n_partials, stream);
-            if (st != QFP4_OK) return st;
-            if (amax_out) {
-                st = partials_max(partials, fa.fq.n_partials, amax_out, stream);
-                if (st != QFP4_OK) return st;
-            }
-        } else if (fmt == QFP4_NVFP4 && amax_out) {
-            // the quantizer warps raise it with atomic maxima of their rows
-            if (cudaMemsetAsync(amax_out, 0, sizeof(float), stream) != cudaSuccess) return QFP4_ERR_CUDA;
-            fa.fq.amax_out = amax_out;
-        }
-        if (cudaMemsetAsync(fa.fq.ready, 0, sizeof(unsigned int) * ((M + 127) / 128), stream) != cudaSuccess)
-            return QFP4_ERR_CUDA;
-        // scale chunks past K (a K tail short of the 256-element k-tile) are read as scales of zero codes
-        if (K % gm_bk(fmt) && cudaMemsetAsync(sfa, 0, L.sfa_bytes, stream) != cudaSuccess) return QFP4_ERR_CUDA;
-        st = rearrange_scales(nullptr, 0, 0, nullptr, B_scales, N, 2 * L.NT, sfb, K, fmt, L.NC, stream);
-        if (st != QFP4_OK) return st;
-        return gemm_core(a_codes, sfa, a_tscale, B_codes, sfb, B_tscale, M, N, K, fmt, out_dt, out, stream, &fa);
-    }
     QuantOpts opt;
     opt.amax_in = amax_in;
     opt.amax_out = amax_out;
-    st = quantize1d(A_bf16, QFP4_BF16, M * K, fmt, QFP4_RNE, rotate, four6, 0, a_codes, a_scales, a_tscale, partials,
-                    nullptr, stream, opt);
+    int st = quantize1d(A_bf16, QFP4_BF16, M * K, fmt, QFP4_RNE, rotate, four6, 0, a_codes, a_scales, a_tscale,
+                        partials, nullptr, stream, opt);
     if (st != QFP4_OK) return st;
+    const GemmLayout L = gemm_layout(M, N, K, fmt);
+    uint8_t *sfa = ws + F.chunks, *sfb = sfa + L.sfa_bytes;
     st = rearrange_scales(a_scales, M, L.MB, sfa, B_scales, N, 2 * L.NT, sfb, K, fmt, L.NC, stream);
     if (st != QFP4_OK) return st;
     return gemm_core(a_codes, sfa, a_tscale, B_codes, sfb, B_tscale, M, N, K, fmt, out_dt, out, stream);

@@ -985,15 +985,6 @@ int mxfp8_rows(const void *x, int64_t n, bool sr, uint64_t seed, uint8_t *codes,
               : launch_tma<MODE_QUANT, FMT_MXFP8, false, false, false>(tm, q, grid, stream);
 }
 
-int amax_pass_bf16(const void *x, int64_t n, bool rotate, float *partials, int *n_parts, cudaStream_t stream)
-{
-    QuantParams p{};
-    p.n = n;
-    p.partials_out = partials;
-    return rotate ? run_pass<MODE_AMAX, QFP4_NVFP4, true, false, false>(x, QFP4_BF16, n, p, stream, n_parts)
-                  : run_pass<MODE_AMAX, QFP4_NVFP4, false, false, false>(x, QFP4_BF16, n, p, stream, n_parts);
-}
-
 int amax_partials(const void *x, qfp4_dtype xdt, int64_t n, float *partials, int *n_parts, cudaStream_t stream)
 {
     QuantParams p{};

@@ -51,7 +51,4 @@ int mxfp8_rows(const void *x, int64_t n, bool sr, uint64_t seed, uint8_t *codes,
 
 int amax_partials(const void *x, qfp4_dtype xdt, int64_t n, float *partials, int *n_parts, cudaStream_t stream);
 
-// Partial maxima of |x| over a bf16 stream, after the FWHT-128 when rotate.
-int amax_pass_bf16(const void *x, int64_t n, bool rotate, float *partials, int *n_parts, cudaStream_t stream);
-
 }  // namespace qfp4

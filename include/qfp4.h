@@ -281,10 +281,9 @@ int qfp4_gemm_blockscaled_noalloc(const uint8_t *A_codes, const uint8_t *A_scale
  * qfp4_quantize) inside the call, then multiplied by the pre-quantized B
  * ([QN] §QuTLASS: fused rotation and online quantization before the GEMM;
  * B is expected to be rotated the same way offline, so that
- * (xH)(WH)^T = xW^T).  A is quantized once, not once per output tile: for
- * M > 128, K % 64 == 0 and four6 == 0 by quantizer warps inside the
- * tensor-core kernel itself, overlapped with the MMAs of the rows already
- * quantized; otherwise by the 1D quantize kernel before the GEMM.  NVFP4
+ * (xH)(WH)^T = xW^T).  A is quantized once (not once per output tile) into
+ * the workspace by the 1D quantize kernel, then consumed by the tensor-core
+ * kernel; the launches follow each other as dependent launches.  NVFP4
  * first measures A's tensor amax (an extra read of A; see
  * qfp4_gemm_fused_rq_ex to supply it).
  * workspace: at least qfp4_gemm_fused_rq_workspace_bytes(M, N, K, fmt)

@@ -153,18 +153,18 @@ def test_gemm_argument_errors():
     assert q.qfp4_last_device_error() == 0
 
 
-# shapes of the in-kernel quantization (M > 128, K % 64 == 0): ragged M, a K
-# tail short of the 256-element k-tile, several 128-row blocks of A
+# fused-call shapes on the CTA-pair kernel: ragged M, a K tail short of the
+# 256-element k-tile, several 128-row blocks of A
 FUSED_SHAPES = [(300, 264, 640), (256, 512, 1024), (1000, 768, 384), (129, 256, 2048)]
 
 
 @pytest.mark.parametrize("M,N,K", FUSED_SHAPES)
 @pytest.mark.parametrize("fmt", FMTS, ids=["mxfp4", "nvfp4"])
 @pytest.mark.parametrize("rotate", [True, False], ids=["rot", "plain"])
-def test_fused_in_kernel_quantization(M, N, K, fmt, rotate):
-    """A quantized by the GEMM kernel's own quantizer warps: its codes, scales
-    and tensor scale left in the workspace equal the oracle's bit for bit, and
-    every output is within the bound of the binary64 reference."""
+def test_fused_call_shapes(M, N, K, fmt, rotate):
+    """A's codes, scales and tensor scale left in the workspace equal the
+    oracle's bit for bit, and every output is within the bound of the
+    binary64 reference."""
     if rotate and K % 128:
         pytest.skip()
     a = synth.cfg5_A(M, K, seed=M + 7 * K)
@@ -187,9 +187,9 @@ def test_fused_in_kernel_quantization(M, N, K, fmt, rotate):
     assert q.qfp4_last_device_error() == 0
 
 
-def test_fused_in_kernel_quantization_is_repeatable():
-    """Quantizer warps and GEMM roles overlap differently from call to call;
-    the output must not depend on it."""
+def test_fused_call_is_repeatable():
+    """Kernels of the call overlap through dependent launches differently from
+    call to call; the output must not depend on it."""
     M, N, K = 2048, 4096, 4096
     a = to_dev(synth.cfg5_A(M, K, seed=3))
     B = q.quantize(to_dev(synth.cfg5_B(N, K, seed=4)), q.NVFP4, rotate=True)
@@ -206,8 +206,8 @@ def test_fused_with_given_and_reported_amax(M, N, K, scale):
     """NVFP4 fused call under a supplied tensor amax of A (the own amax, or a
     stale one x0.5 that saturates the top blocks): A's operand and the
     outputs follow the oracle under the same amax, and the amax the call
-    reports is A's own (rotated) amax bit for bit.  M = 100 takes the
-    quantize-then-GEMM path."""
+    reports is A's own (rotated) amax bit for bit (M = 100 runs on the
+    single-CTA GEMM kernel)."""
     a = synth.cfg5_A(M, K, seed=M + K)
     B = oracle.quantize(synth.cfg5_B(N, K, seed=N), oracle.NVFP4, rotate=True)
     own = oracle.tensor_amax(a, rotate=True)
