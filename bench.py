@@ -532,15 +532,20 @@ def bench_cfg5(q, synth, dev, stream, hbm_peak, bf16_peak, peak_src, iters):
     B5 = q.quantize(bf(synth.cfg5_B(N, K)), q.NVFP4, q.RNE, rotate=True)
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     ws = torch.empty(q.qfp4_gemm_fused_rq_workspace_bytes(M, N, K, q.NVFP4), dtype=torch.uint8, device=dev)
-    ms = timed(lambda: q.gemm_fused_rq(a5, B5, N, fmt=q.NVFP4, rotate=True, out=y, workspace=ws))
-    tf = 2.0 * M * N * K / (ms * 1e-3) / 1e12
     peak = bf16_peak * FP4_PER_BF16
-    out["fused_rotate_quantize_gemm_16384x14336x4096"] = {
-        "workload": "A bf16 16384x4096 (0.5% channels x30) rotated + NVFP4-quantized inside the call, "
-                    "B 14336x4096 pre-rotated NVFP4, bf16 out",
-        "ms_per_call": ms, "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
-                                        "frac": tf / peak, "flops_per_launch": 2.0 * M * N * K, "traffic": None,
-                                        "peak_source": f"{peak_src} bf16_tflops x {FP4_PER_BF16}"}}
+    a_amax = torch.empty(1, dtype=torch.float32, device=dev)
+    q.gemm_fused_rq(a5, B5, N, fmt=q.NVFP4, rotate=True, out=y, workspace=ws, A_amax_out=a_amax)
+    for key, given, what in (("fused_rotate_quantize_gemm_16384x14336x4096", None, "A's own tensor amax (two reads of A)"),
+                             ("fused_rotate_quantize_gemm_16384x14336x4096_given_amax", a_amax,
+                              "a supplied tensor amax of A (one read of A)")):
+        ms = timed(lambda: q.gemm_fused_rq(a5, B5, N, fmt=q.NVFP4, rotate=True, out=y, workspace=ws, A_amax_in=given))
+        tf = 2.0 * M * N * K / (ms * 1e-3) / 1e12
+        out[key] = {
+            "workload": "A bf16 16384x4096 (0.5% channels x30) rotated + NVFP4-quantized inside the call under "
+                        f"{what}, B 14336x4096 pre-rotated NVFP4, bf16 out",
+            "ms_per_call": ms, "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
+                                            "frac": tf / peak, "flops_per_launch": 2.0 * M * N * K, "traffic": None,
+                                            "peak_source": f"{peak_src} bf16_tflops x {FP4_PER_BF16}"}}
     return out
 
 
@@ -629,7 +634,7 @@ def run_rows(only=""):
         if st != q.OK:
             bad.append(st)
 
-    def emit(row, workload, ms, nbytes=None, flops=None, **extra):
+    def emit(row, workload, ms, nbytes=None, flops=None, peak_ratio=FP4_PER_BF16, **extra):
         d = {"row": row, "workload": workload, "ms_per_call": ms}
         if nbytes is not None:
             a = nbytes / (ms * 1e-3) / 1e9
@@ -637,8 +642,9 @@ def run_rows(only=""):
                      frac=a / hbm_peak, peak_source=f"{peak_src} hbm_gbs")
         else:
             a = flops / (ms * 1e-3) / 1e12
-            d.update(bound="tensor", flops=flops, achieved=a, unit="TFLOP/s", peak=fp4_peak, frac=a / fp4_peak,
-                     peak_source=f"{peak_src} bf16_tflops x {FP4_PER_BF16}")
+            pk = bf16_peak * peak_ratio
+            d.update(bound="tensor", flops=flops, achieved=a, unit="TFLOP/s", peak=pk, frac=a / pk,
+                     peak_source=f"{peak_src} bf16_tflops x {peak_ratio} (nominal dense ratio to bf16)")
         d.update(extra)
         print(json.dumps(d), flush=True)
 
@@ -646,18 +652,22 @@ def run_rows(only=""):
         return max(1, -(-(512 << 20) // nbytes))            # > 4x L2 between two calls on the same set
 
     def fp4_row(row, workload, x, fmt, rounding, bpe, rotate=False, block2d=False, four6=False, transposed=False,
-                seed=0):
+                seed=0, rule=q.SCALE_DEFAULT, amax_in=False):
         M, K = x.shape
         ns = n_sets(x.numel() * 2)
         xs = [x] + [x.clone() for _ in range(ns - 1)]
         outs = [q.quantize(x, fmt, rounding, rotate=rotate, block2d=block2d, four6=four6, seed=seed,
-                           transposed=transposed) for _ in range(ns)]
+                           transposed=transposed, rule=rule) for _ in range(ns)]
         wsb = q.qfp4_quantize_workspace_bytes(M, K, fmt, rotate, block2d)
         ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
-        av = [(xs[b].data_ptr(), q.BF16, M, K, fmt, rounding, int(rotate), int(block2d), int(four6), seed,
-               o["codes"].data_ptr(), o["scales"].data_ptr(), q._ptr(o.get("codesT")), q._ptr(o.get("scalesT")),
-               q._ptr(o.get("tscale")), ws.data_ptr(), wsb, sh) for b, o in enumerate(outs)]
-        ms = time_calls(torch, stream, lambda i: ok(L.qfp4_quantize(*av[i % ns])))
+        amax = None
+        if amax_in:                                     # the tensor's own amax, as a previous step would supply it
+            amax = torch.empty(1, dtype=torch.float32, device=dev)
+            q.quantize(x, fmt, rounding, rotate=rotate, amax_out=amax)
+        av = [(xs[b].data_ptr(), q.BF16, M, K, fmt, rounding, int(rotate), int(block2d), int(four6), rule, seed,
+               q._ptr(amax), None, o["codes"].data_ptr(), o["scales"].data_ptr(), q._ptr(o.get("codesT")),
+               q._ptr(o.get("scalesT")), q._ptr(o.get("tscale")), ws.data_ptr(), wsb, sh) for b, o in enumerate(outs)]
+        ms = time_calls(torch, stream, lambda i: ok(L.qfp4_quantize_ex(*av[i % ns])))
         emit(row, workload, ms, nbytes=bpe * M * K, bytes_per_element=bpe, input_sets=ns)
 
     def mxfp8_row(row, workload, x, rounding, transposed, seed=0):
@@ -684,7 +694,7 @@ def run_rows(only=""):
         ms = time_calls(torch, stream, lambda i: ok(L.qfp4_dequantize(*av[i % ns])))
         emit(row, workload, ms, nbytes=bpe * M * K, bytes_per_element=bpe, input_sets=ns)
 
-    def gemm_row(row, workload, A, B, M, N, K, fmt, out_dtype):
+    def gemm_row(row, workload, A, B, M, N, K, fmt, out_dtype, peak_ratio=FP4_PER_BF16):
         out = torch.empty((M, N), dtype=out_dtype, device=dev)
         wsb = q.qfp4_gemm_workspace_bytes(M, N, K, fmt)
         ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
@@ -693,7 +703,7 @@ def run_rows(only=""):
               B["scales"].data_ptr(), q._ptr(B.get("tscale")), M, N, K, fmt, odt, out.data_ptr(), ws.data_ptr(), wsb,
               sh)
         ms = time_calls(torch, stream, lambda i: ok(L.qfp4_gemm_blockscaled(*av)))
-        emit(row, workload, ms, flops=2.0 * M * N * K)
+        emit(row, workload, ms, flops=2.0 * M * N * K, peak_ratio=peak_ratio)
 
     def fused_row(row, workload, A_bf16, B, N, fmt, out_dtype):
         M, K = A_bf16.shape
@@ -705,6 +715,12 @@ def run_rows(only=""):
               q._ptr(B.get("tscale")), N, ws.data_ptr(), wsb, odt, out.data_ptr(), sh)
         ms = time_calls(torch, stream, lambda i: ok(L.qfp4_gemm_fused_rq(*av)))
         emit(row, workload, ms, flops=2.0 * M * N * K)
+        amax = torch.empty(1, dtype=torch.float32, device=dev)
+        q.quantize(A_bf16, fmt, q.RNE, rotate=True, amax_out=amax)
+        av2 = (A_bf16.data_ptr(), M, K, 1, 0, fmt, amax.data_ptr(), None, B["codes"].data_ptr(), B["scales"].data_ptr(),
+               q._ptr(B.get("tscale")), N, ws.data_ptr(), wsb, odt, out.data_ptr(), sh)
+        ms = time_calls(torch, stream, lambda i: ok(L.qfp4_gemm_fused_rq_ex(*av2)))
+        emit(row, workload.replace("NVFP4 RNE of A", "NVFP4 RNE of A (supplied amax)"), ms, flops=2.0 * M * N * K)
 
     F32, BF = torch.float32, torch.bfloat16
     with ClockSampler(0) as clk:
@@ -728,6 +744,14 @@ def run_rows(only=""):
             if want("nvfp4"):
                 fp4_row("nvfp4", "X bf16 8192x4096 Student-t(3)*0.5: NVFP4 RNE", x3, q.NVFP4, q.RNE, nv)
                 fp4_row("nvfp4", "X bf16 8192x4096 Student-t(3)*0.5: NVFP4 Philox SR", x3, q.NVFP4, q.SR, nv, seed=7)
+                fp4_row("nvfp4", "X bf16 8192x4096: NVFP4 RNE, supplied tensor amax (one read)", x3, q.NVFP4, q.RNE,
+                        nv, amax_in=True)
+                fp4_row("nvfp4", "X bf16 8192x4096: FWHT-128 + NVFP4 RNE", x3, q.NVFP4, q.RNE, nv, rotate=True)
+                fp4_row("nvfp4", "X bf16 8192x4096: FWHT-128 + NVFP4 RNE, supplied tensor amax", x3, q.NVFP4, q.RNE,
+                        nv, rotate=True, amax_in=True)
+            if want("scale rules"):
+                fp4_row("scale rules", "X bf16 8192x4096: NVFP4 RNE, E4M3 block scale rounded up", x3, q.NVFP4, q.RNE,
+                        nv, rule=q.SCALE_E4M3_UP)
             if want("dequantize"):
                 dequant_row("dequantize", "NVFP4 codes of X 8192x4096 -> bf16", x3, q.NVFP4, BF)
                 dequant_row("dequantize", "NVFP4 codes of X 8192x4096 -> fp32", x3, q.NVFP4, F32)
@@ -735,6 +759,13 @@ def run_rows(only=""):
         # Quartet-style backward: 2D blocks, MXFP8, column-wise 1D, backward GEMMs
         if want("2d blocks", "column-wise", "mxfp8", "gemm"):
             g4 = bf16(synth.cfg4_G())
+            if want("scale rules"):
+                fp4_row("scale rules", "G bf16 8192x4096: MXFP4 RNE, OCP floor E8M0 exponent", g4, q.MXFP4, q.RNE,
+                        2 + 0.5 + 1 / 32, rule=q.SCALE_OCP_FLOOR)
+                fp4_row("scale rules", "G bf16 8192x4096: MXFP4 four-over-six under the OCP floor rule", g4, q.MXFP4,
+                        q.RNE, 2 + 0.5 + 1 / 32, four6=True, rule=q.SCALE_OCP_FLOOR)
+                fp4_row("scale rules", "G bf16 8192x4096: 2D 32x32 MXFP4 RNE, G and G^T", g4, q.MXFP4, q.RNE,
+                        2 + 2 * (0.5 + 1 / 32), block2d=True, transposed=True)
             if want("2d blocks"):
                 fp4_row("2d blocks", "G bf16 8192x4096 (N(0,1e-6), 0.1% x100): 2D 16x16 NVFP4 Philox SR, G and G^T", g4,
                         q.NVFP4, q.SR, 2 + 2 * (0.5 + 1 / 16), block2d=True, transposed=True, seed=11)
@@ -760,7 +791,15 @@ def run_rows(only=""):
                 gemm_row("gemm", "dX = G W: NVFP4 8192x4096x4096, fp32 out", G2, T(W2), 8192, 4096, 4096, q.NVFP4, F32)
                 gemm_row("gemm", "dW = G^T X: NVFP4 4096x4096x8192, fp32 out", T(G2), T(X2), 4096, 4096, 8192, q.NVFP4,
                          F32)
-                del G2, W2, X2, x4, w4
+                # the FP8 backward: MXFP8 block-scaled GEMMs on kind::mxf8f6f4
+                G8 = q.quantize_mxfp8(g4, q.SR, seed=11, transposed=True)
+                W8 = q.quantize_mxfp8(w4, q.RNE, transposed=True)
+                X8 = q.quantize_mxfp8(x4, q.RNE, transposed=True)
+                gemm_row("gemm", "dX = G W: MXFP8 8192x4096x4096, fp32 out", G8, T(W8), 8192, 4096, 4096, q.MXFP8,
+                         F32, peak_ratio=2.0)
+                gemm_row("gemm", "dW = G^T X: MXFP8 4096x4096x8192, fp32 out", T(G8), T(X8), 4096, 4096, 8192, q.MXFP8,
+                         F32, peak_ratio=2.0)
+                del G2, W2, X2, G8, W8, X8, x4, w4
             del g4
         # 7B-class linear shapes: the GEMM alone and the fused rotate + quantize + GEMM
         if want("gemm", "fused rotate + quantize + gemm"):
@@ -776,6 +815,48 @@ def run_rows(only=""):
                               f"fused FWHT-128 + NVFP4 RNE of A bf16 + GEMM {M}x{N}x{K}, bf16 out", a5, B5, N, q.NVFP4,
                               BF)
                 del a5, B5, A5
+        # the Quartet-style linear layer: forward on the forward-linear shapes, backward on the gradient shapes
+        if want("linear"):
+            x3, w3 = bf16(synth.cfg3_X()), bf16(synth.cfg3_W())
+            M, K = x3.shape
+            N = w3.shape[0]
+            y = torch.empty((M, N), dtype=BF, device=dev)
+            wsb = q.qfp4_linear_forward_workspace_bytes(M, N, K, q.NVFP4)
+            ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+            av = (x3.data_ptr(), w3.data_ptr(), M, N, K, q.NVFP4, 0, q.BF16, y.data_ptr(), ws.data_ptr(), wsb, sh)
+            ms = time_calls(torch, stream, lambda i: ok(L.qfp4_linear_forward(*av)))
+            emit("linear", f"forward Y = Q(XH) Q(WH)^T: X {M}x{K}, W {N}x{K} bf16, NVFP4, bf16 out", ms,
+                 flops=2.0 * M * N * K)
+            del x3, w3, y, ws
+            g4, x4, w4 = bf16(synth.cfg4_G()), bf16(synth.cfg4_X()), bf16(synth.cfg4_W())
+            M, N = g4.shape
+            K = x4.shape[1]
+            dX = torch.empty((M, K), dtype=F32, device=dev)
+            dW = torch.empty((N, K), dtype=F32, device=dev)
+            for fmt, name, ratio in ((q.NVFP4, "2D NVFP4 (G stochastic)", FP4_PER_BF16),
+                                     (q.MXFP8, "MXFP8 (G stochastic)", 2.0)):
+                wsb = q.qfp4_linear_backward_workspace_bytes(M, N, K, fmt)
+                ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+                av = (g4.data_ptr(), x4.data_ptr(), w4.data_ptr(), M, N, K, fmt, 11, q.F32, dX.data_ptr(),
+                      dW.data_ptr(), ws.data_ptr(), wsb, sh)
+                ms = time_calls(torch, stream, lambda i: ok(L.qfp4_linear_backward(*av)))
+                emit("linear", f"backward dX = G W, dW = G^T X: G {M}x{N}, X {M}x{K}, W {N}x{K}, {name}, fp32 out",
+                     ms, flops=2 * 2.0 * M * N * K, peak_ratio=ratio)
+                del ws
+            del g4, x4, w4, dX, dW
+        if want("kl calibration"):
+            xr = bf16(synth.relu_activation(8192, 4096))
+            out = {"clip": torch.empty(1, dtype=F32, device=dev), "best": torch.empty(1, dtype=torch.int32, device=dev),
+                   "kl": torch.empty(2048 - 8 + 1, dtype=torch.float64, device=dev),
+                   "hist": torch.empty(2048, dtype=torch.int64, device=dev)}
+            wsb = q.qfp4_kl_calibrate_workspace_bytes(2048, 8, 1)
+            ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+            av = (xr.data_ptr(), q.BF16, xr.numel(), 2048, 8, 1, out["clip"].data_ptr(), out["best"].data_ptr(),
+                  out["kl"].data_ptr(), out["hist"].data_ptr(), ws.data_ptr(), wsb, sh)
+            ms = time_calls(torch, stream, lambda i: ok(L.qfp4_kl_calibrate(*av)))
+            emit("kl calibration", "ReLU-like activation bf16 8192x4096: |x| histogram (2048 bins) + KL over every "
+                 "candidate clip (E2M1 levels)", ms, nbytes=2 * 2.0 * xr.numel())
+            del xr
         # standalone quantize bandwidth over 2^20 .. 2^30 bf16 elements (K = 4096):
         # rows of the 16384 x 4096 outlier-channel input, repeated past 2^26 elements
         if want("quantize sweep"):
@@ -784,6 +865,8 @@ def run_rows(only=""):
                 M = (1 << e) // 4096
                 x = base[:M].clone() if M <= 16384 else base.repeat(M // 16384, 1)
                 fp4_row("quantize sweep", f"2^{e} bf16 elements ({M}x4096): NVFP4 RNE", x, q.NVFP4, q.RNE, nv)
+                fp4_row("quantize sweep", f"2^{e} bf16 elements ({M}x4096): NVFP4 RNE, supplied tensor amax", x,
+                        q.NVFP4, q.RNE, nv, amax_in=True)
                 fp4_row("quantize sweep", f"2^{e} bf16 elements ({M}x4096): FWHT-128 + MXFP4 RNE", x, q.MXFP4, q.RNE,
                         2 + 0.5 + 1 / 32, rotate=True)
                 del x
