@@ -787,7 +787,7 @@ def run_rows(only=""):
                 G2 = q.quantize(g4, q.NVFP4, q.SR, block2d=True, transposed=True, seed=11)
                 W2 = q.quantize(w4, q.NVFP4, q.RNE, block2d=True, transposed=True)
                 X2 = q.quantize(x4, q.NVFP4, q.RNE, block2d=True, transposed=True)
-                T = lambda o: {"codes": o["codesT"], "scales": o["scalesT"], "tscale": o["tscale"]}   # noqa: E731
+                T = lambda o: {"codes": o["codesT"], "scales": o["scalesT"], **({"tscale": o["tscale"]} if "tscale" in o else {})}   # noqa: E731,E501
                 gemm_row("gemm", "dX = G W: NVFP4 8192x4096x4096, fp32 out", G2, T(W2), 8192, 4096, 4096, q.NVFP4, F32)
                 gemm_row("gemm", "dW = G^T X: NVFP4 4096x4096x8192, fp32 out", T(G2), T(X2), 4096, 4096, 8192, q.NVFP4,
                          F32)

@@ -118,6 +118,14 @@ __device__ __forceinline__ uint64_t transpose16x16_nibbles(uint64_t w, int r)
 }
 
 // ---------------------------------------------------------------- 2D NVFP4
+// A warp task is 64 rows x 32 columns: four 16-row bands of two 16 x 16
+// tiles.  Lane (h, r) = (lane / 16, lane % 16) holds row r of tile (b, h) for
+// each band b (16 values; 32 contiguous bytes of bf16).  After rounding, the
+// nibble transpose of each band gives lane (h, r) column r of tile (b, h):
+// 16 consecutive elements of X^T row j = 16 tc + r, so the four bands are 32
+// contiguous bytes of that row (one full sector, two 16-byte stores) and its
+// four scale bytes are contiguous in scalesT (one 4-byte store).  The four
+// bands' shuffles are independent, which hides their latency.
 template <bool SR, typename T>
 __global__ void __launch_bounds__(256) k_quant2d(const T *__restrict__ x, Q2DParams p)
 {
@@ -127,63 +135,94 @@ __global__ void __launch_bounds__(256) k_quant2d(const T *__restrict__ x, Q2DPar
     const NvScale nz = nv_scale_setup(s_t, p.rule);
 
     const int lane = threadIdx.x & 31, half = lane >> 4, r = lane & 15;
-    const int64_t tiles_k = p.K / 16, pairs = (tiles_k + 1) / 2;
-    const int64_t tasks = (p.M / 16) * pairs;
+    const int64_t tiles_k = p.K / 16, bands = p.M / 16;
+    const int64_t pairs = (tiles_k + 1) / 2, quads = (bands + 3) / 4;
+    const int64_t tasks = quads * pairs;
     const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-    // this lane's row of a task: row band*16 + r, columns tc*16 .. +15
-    auto fetch = [&](int64_t task, Raw16<T> &dst) {
-        const int64_t band = task / pairs, tc = (task % pairs) * 2 + half;
-        raw_load16(x, (band * 16 + r) * p.K + tc * 16, tc < tiles_k, dst);
-    };
-    Raw16<T> cur;
-    if (warp0 < tasks) fetch(warp0, cur);
     for (int64_t task = warp0; task < tasks; task += nwarps) {
-        Raw16<T> nxt{};
-        if (task + nwarps < tasks) fetch(task + nwarps, nxt);      // in flight during this task
-        const int64_t band = task / pairs, tc = (task % pairs) * 2 + half;
-        const bool valid = tc < tiles_k;
-        const int64_t i = band * 16 + r, j0 = tc * 16;
-        float v[16];
-        raw_to_f32(cur, v);
-        cur = nxt;
-        float amax = 0.0f;
+        const int64_t bq = task / pairs, tc = (task % pairs) * 2 + half;
+        const bool colv = tc < tiles_k;
+        const int64_t j0 = tc * 16;
+        Raw16<T> raw[4];
+        bool bv[4];
 #pragma unroll
-        for (int t = 0; t < 16; ++t) amax = fmaxf(amax, fabsf(v[t]));
-#pragma unroll
-        for (int o = 8; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-        uint32_t enc = 0u;
-        float S = 0.0f;
-        if (s_t != 0.0f) {
-            enc = nv_scale_byte<true>(amax, nz);
-            S = __fmul_rn(e4m3_value(enc), s_t);
+        for (int b = 0; b < 4; ++b) {
+            const int64_t band = bq * 4 + b;
+            bv[b] = band < bands;
+            raw_load16(x, (band * 16 + r) * p.K + j0, colv && bv[b], raw[b]);
         }
-        uint32_t w[2] = {0u, 0u};
-        if (S != 0.0f) {
-            if (SR) {
-                uint64_t pp[8], qq[8];
+        uint32_t w[4][2], enc[4];
 #pragma unroll
-                for (int t = 0; t < 8; ++t) pp[t] = f2pack(v[2 * t], v[2 * t + 1]);
-                nv_quot16_pairs(pp, S, amax, qq);
-                float q[16];
+        for (int b = 0; b < 4; ++b) {
+            float v[16];
+            raw_to_f32(raw[b], v);
+            float amax = 0.0f;
 #pragma unroll
-                for (int t = 0; t < 8; ++t) f2unpack(qq[t], q[2 * t], q[2 * t + 1]);
-                sr_group<16>(q, static_cast<uint64_t>(i * p.K + j0), p.seed, w);
-            } else {
-                nv_block_rne(v, S, amax, w, nullptr);
+            for (int t = 0; t < 16; ++t) amax = fmaxf(amax, fabsf(v[t]));
+#pragma unroll
+            for (int o = 8; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+            enc[b] = 0u;
+            float S = 0.0f;
+            if (s_t != 0.0f) {
+                enc[b] = nv_scale_byte<true>(amax, nz);
+                S = __fmul_rn(e4m3_value(enc[b]), s_t);
+            }
+            w[b][0] = w[b][1] = 0u;
+            if (S != 0.0f) {
+                if (SR) {
+                    uint64_t pp[8], qq[8];
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) pp[t] = f2pack(v[2 * t], v[2 * t + 1]);
+                    nv_quot16_pairs(pp, S, amax, qq);
+                    float q[16];
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) f2unpack(qq[t], q[2 * t], q[2 * t + 1]);
+                    const int64_t i = (bq * 4 + b) * 16 + r;
+                    sr_group<16>(q, static_cast<uint64_t>(i * p.K + j0), p.seed, w[b]);
+                } else {
+                    nv_block_rne(v, S, amax, w[b], nullptr);
+                }
             }
         }
-        if (valid) {
-            *reinterpret_cast<uint2 *>(p.codes + (i * p.K + j0) / 2) = make_uint2(w[0], w[1]);
-            p.scales[i * tiles_k + tc] = static_cast<uint8_t>(enc);
+        // row-wise outputs: 8 code bytes and one scale byte per band
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            if (colv && bv[b]) {
+                const int64_t i = (bq * 4 + b) * 16 + r;
+                *reinterpret_cast<uint2 *>(p.codes + (i * p.K + j0) / 2) = make_uint2(w[b][0], w[b][1]);
+                p.scales[i * tiles_k + tc] = static_cast<uint8_t>(enc[b]);
+            }
         }
         if (p.codesT) {
-            const uint64_t t = transpose16x16_nibbles((static_cast<uint64_t>(w[1]) << 32) | w[0], r);
-            if (valid) {
-                const int64_t jr = j0 + r;                  // column of X = row of X^T
-                *reinterpret_cast<uint2 *>(p.codesT + (jr * p.M + band * 16) / 2) =
-                    make_uint2(static_cast<uint32_t>(t), static_cast<uint32_t>(t >> 32));
-                p.scalesT[jr * (p.M / 16) + band] = static_cast<uint8_t>(enc);
+            uint64_t tw[4];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) tw[b] = transpose16x16_nibbles((static_cast<uint64_t>(w[b][1]) << 32) | w[b][0], r);
+            if (colv) {
+                const int64_t jr = j0 + r;                       // column of X = row of X^T
+                const int64_t base = jr * p.M + bq * 64;         // X^T element index of band 0
+                const bool full = bv[3];                         // all four bands inside M
+                if (full && (p.M % 32) == 0) {                   // 32 contiguous bytes, 16-byte aligned
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.codesT + base / 2);
+                    dst[0] = make_uint4(static_cast<uint32_t>(tw[0]), static_cast<uint32_t>(tw[0] >> 32),
+                                        static_cast<uint32_t>(tw[1]), static_cast<uint32_t>(tw[1] >> 32));
+                    dst[1] = make_uint4(static_cast<uint32_t>(tw[2]), static_cast<uint32_t>(tw[2] >> 32),
+                                        static_cast<uint32_t>(tw[3]), static_cast<uint32_t>(tw[3] >> 32));
+                } else {
+#pragma unroll
+                    for (int b = 0; b < 4; ++b)
+                        if (bv[b])
+                            *reinterpret_cast<uint2 *>(p.codesT + (base + 16 * b) / 2) =
+                                make_uint2(static_cast<uint32_t>(tw[b]), static_cast<uint32_t>(tw[b] >> 32));
+                }
+                uint8_t *sdst = p.scalesT + jr * bands + bq * 4;
+                if (full && (bands % 4) == 0) {
+                    *reinterpret_cast<uint32_t *>(sdst) = enc[0] | (enc[1] << 8) | (enc[2] << 16) | (enc[3] << 24);
+                } else {
+#pragma unroll
+                    for (int b = 0; b < 4; ++b)
+                        if (bv[b]) sdst[b] = static_cast<uint8_t>(enc[b]);
+                }
             }
         }
     }
@@ -667,7 +706,7 @@ int quantize2d(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_fmt fmt
             if (st != QFP4_OK) return st;
         }
     }
-    const int64_t tasks = (M / 16) * ((K / 16 + 1) / 2);
+    const int64_t tasks = ((M / 16 + 3) / 4) * ((K / 16 + 1) / 2);     // 64 x 32 warp tasks
     if (xdt == QFP4_BF16) {
         if (sr) launch_tiles<k_quant2d<true, uint16_t>, uint16_t>(tasks, x, p, stream);
         else launch_tiles<k_quant2d<false, uint16_t>, uint16_t>(tasks, x, p, stream);
