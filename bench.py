@@ -102,10 +102,11 @@ def csrc_hash(files=None):
     return h.hexdigest()[:12]
 
 
-def ncu_traffic(key):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the kernel's current sources (else None)."""
-    p = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+def _ncu_figure(key, fname):
+    """A per-launch figure from a committed ncu summary file (`key value
+    source-hash ...` lines), if it was taken on the kernel's current sources
+    (else None)."""
+    p = os.path.join(ROOT, "profiles", fname)
     if not os.path.exists(p) or key not in KERNEL_SOURCES:
         return None
     cur = csrc_hash(KERNEL_SOURCES[key])
@@ -115,6 +116,32 @@ def ncu_traffic(key):
             if len(t) >= 3 and not line.startswith("#") and t[0] == key and t[2] == cur:
                 return float(t[1])
     return None
+
+
+def ncu_traffic(key):
+    """DRAM bytes (read + write) per launch of the kernel, from ncu."""
+    return _ncu_figure(key, "ncu_traffic.txt")
+
+
+def ncu_warp_insts(key):
+    """Warp instructions executed per launch of the kernel, from ncu."""
+    return _ncu_figure(key, "ncu_issue.txt")
+
+
+def issue_roofline(key, ms, n_elem, sms, sm_mhz):
+    """Instruction-issue roofline of a kernel: its warp instructions per
+    launch (ncu) over its event-timed duration, against one warp
+    instruction per cycle on each of the 4 schedulers of every SM at the
+    SM clock seen during the run."""
+    w = ncu_warp_insts(key)
+    if w is None or not ms or not sm_mhz:
+        return None
+    peak = sms * 4 * sm_mhz * 1e6 / 1e9                   # G warp instructions / s
+    achieved = w / (ms * 1e-3) / 1e9
+    return {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "G warp-inst/s", "frac": achieved / peak,
+            "warp_inst_per_launch": w, "thread_inst_per_element": 32.0 * w / n_elem,
+            "issue_bound_ms": w / (peak * 1e9) * 1e3,
+            "peak_source": f"{sms} SMs x 4 schedulers x 1 warp instruction/cycle x {sm_mhz:.0f} MHz (median SM clock)"}
 
 
 # ------------------------------------------------------------------ clocks
@@ -432,11 +459,15 @@ def run_gpu(args, rank, world):
     if not args.no_cfg5:
         cfg5 = bench_cfg5(q, synth, dev, stream, hbm_peak, bf16_peak, peak_src, max(3, min(args.steps, 10)))
 
+    clocks = clk.summary()
+    # the dominant kernel is issue-bound: its instruction roofline beside the HBM one
+    roofline["issue"] = issue_roofline(dom_name, dom_ms, n, torch.cuda.get_device_properties(dev).multi_processor_count,
+                                       clocks.get("sm_mhz") or clocks.get("sm_max_mhz"))
     result = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": workload_config(),
-        "roofline": roofline, "e2e": e2e, "gpu_launches": int(n_launch), "clocks": clk.summary(),
+        "roofline": roofline, "e2e": e2e, "gpu_launches": int(n_launch), "clocks": clocks,
         "frac_of_hbm_peak": value / world / hbm_peak,
     }
     if gemm is not None:
