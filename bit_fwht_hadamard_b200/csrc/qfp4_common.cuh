@@ -332,6 +332,41 @@ __device__ __forceinline__ float e2m1_sr_grid(float v, uint32_t w)
     return __uint_as_float(__float_as_uint(r) | (__float_as_uint(v) & 0x80000000u));   // sign kept, also on zero
 }
 
+// add.rz on a packed binary32 pair.
+__device__ __forceinline__ uint64_t f2add_rz(uint64_t a, uint64_t b)
+{
+    uint64_t r;
+    asm("add.rz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+// e2m1_sr_grid on two values held as a packed binary32 pair (the even
+// element low) with random words w0 / w1, the pair's arithmetic on the
+// f32x2 pipe.  The grid spacing's exponent is clamped below only: |v| >= 8
+// keeps its own binade (spacing >= 4), so its grid value is >= 8, and grid
+// values above 6 are left for the saturating conversion that follows (all
+// are finite).  Same codes as e2m1_sr on each value.
+__device__ __forceinline__ uint64_t e2m1_sr_grid2(uint64_t vv, uint32_t w0, uint32_t w1)
+{
+    float v0, v1;
+    f2unpack(vv, v0, v1);
+    const uint32_t b0 = __float_as_uint(v0) & 0x7FFFFFFFu, b1 = __float_as_uint(v1) & 0x7FFFFFFFu;
+    const uint32_t m0 = imax(b0 >> 23, 127u), m1 = imax(b1 >> 23, 127u);
+    const uint64_t inv = f2pack(__uint_as_float((279u - m0) << 23), __uint_as_float((279u - m1) << 23));
+    const uint64_t sp = f2pack(__uint_as_float((m0 - 25u) << 23), __uint_as_float((m1 - 25u) << 23));
+    const uint64_t C = f2pack(211106232532992.0f, 211106232532992.0f);   // 1.5 * 2^47
+    const uint64_t q24 = f2mul(f2pack(__uint_as_float(b0), __uint_as_float(b1)), inv);
+    const uint64_t fl24 = f2sub(f2add_rz(q24, C), C);
+    float f0, f1;
+    f2unpack(f2sub(q24, fl24), f0, f1);
+    const uint64_t up = f2pack(static_cast<float>(w0 >> 8) < f0 ? 16777216.0f : 0.0f,
+                               static_cast<float>(w1 >> 8) < f1 ? 16777216.0f : 0.0f);
+    float r0, r1;
+    f2unpack(f2mul(f2add(fl24, up), sp), r0, r1);
+    return f2pack(__uint_as_float(__float_as_uint(r0) | (__float_as_uint(v0) & 0x80000000u)),
+                  __uint_as_float(__float_as_uint(r1) | (__float_as_uint(v1) & 0x80000000u)));
+}
+
 // The same rule as a 4-bit code.
 __device__ __forceinline__ uint32_t e2m1_sr(float v, uint32_t w)
 {

@@ -224,6 +224,23 @@ __device__ __forceinline__ void sr_group(const float *v, uint64_t e, uint64_t se
     }
 }
 
+// sr_group on values held as G / 2 packed pairs (e2m1_sr_grid2).
+template <int G>
+__device__ __forceinline__ void sr_group_pairs(const uint64_t *pp, uint64_t e, uint64_t seed, uint32_t *words)
+{
+#pragma unroll
+    for (int w = 0; w < G / 8; ++w) {
+        float r[8];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint4 rw = sr_words4(seed, (e >> 2) + 2 * w + h);
+            f2unpack(e2m1_sr_grid2(pp[4 * w + 2 * h], rw.x, rw.y), r[4 * h + 0], r[4 * h + 1]);
+            f2unpack(e2m1_sr_grid2(pp[4 * w + 2 * h + 1], rw.z, rw.w), r[4 * h + 2], r[4 * h + 3]);
+        }
+        words[w] = e2m1x8_rne(r);
+    }
+}
+
 // binary32 squared error of 32 values x under codes w (4 words) and scale
 // 2^k: sum(fl(fl(fl(g_i 2^k) - x_i)^2)) as a fixed tree (i + 16 into i, then
 // + 8, + 4, + 2, + 1); g_i 2^k is exact.  The code values come from the E2M1
@@ -536,10 +553,7 @@ __device__ __forceinline__ void quant_unit_packed(uint64_t (&p)[UP], uint64_t e0
 #pragma unroll
             for (int j = 0; j < 16; ++j) pg[j] = f2mul(pg[j], m2);
             if (SR) {
-                float q[32];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) f2unpack(pg[j], q[2 * j], q[2 * j + 1]);
-                sr_group<32>(q, e0 + 32 * g, seed, w);
+                sr_group_pairs<32>(pg, e0 + 32 * g, seed, w);
             } else {
 #pragma unroll
                 for (int t = 0; t < 4; ++t) w[t] = e2m1x8_rne_pairs(pg[4 * t], pg[4 * t + 1], pg[4 * t + 2], pg[4 * t + 3]);
@@ -580,10 +594,7 @@ __device__ __forceinline__ void quant_unit_packed(uint64_t (&p)[UP], uint64_t e0
                 } else {
                     uint64_t qq[8];
                     nv_quot16_pairs(p + 8 * b, S, amax, qq);
-                    float q[16];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) f2unpack(qq[j], q[2 * j], q[2 * j + 1]);
-                    sr_group<16>(q, e0 + 16 * b, seed, w);
+                    sr_group_pairs<16>(qq, e0 + 16 * b, seed, w);
                 }
             } else {
                 nv_block_rne_pairs(p + 8 * b, S, amax, w, nullptr);

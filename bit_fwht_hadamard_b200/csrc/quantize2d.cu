@@ -96,25 +96,43 @@ __device__ __forceinline__ float ld1(const T *x, int64_t i)
     return __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const uint16_t *>(x)[i]) << 16);
 }
 
-// Transpose a 16 x 16 nibble matrix held as one 64-bit row per lane of a
-// 16-lane group (nibble j of lane r = element (r, j)); afterwards nibble j of
-// lane r is element (j, r).  Shuffle partners stay inside the group.
-__device__ __forceinline__ uint64_t transpose16x16_nibbles(uint64_t w, int r)
+// Transpose a 16 x 16 nibble matrix held as one row per lane of a 16-lane
+// group (lo = nibbles 0-7, hi = nibbles 8-15; nibble j of lane r = element
+// (r, j)); afterwards nibble j of lane r is element (j, r).  Four block-swap
+// stages with the partner lane r ^ s: for s = 8 the swapped halves are whole
+// words, for s = 4 and 2 byte pairs and bytes (one byte permute packs what a
+// lane sends, two put what it receives in place), for s = 1 the odd or even
+// nibbles of every byte.  One shuffle a stage; shuffle partners stay inside
+// the group.
+__device__ __forceinline__ void transpose16x16_nibbles(uint32_t &lo, uint32_t &hi, int r)
 {
-#pragma unroll
-    for (int s = 8; s >= 1; s >>= 1) {
-        // nibble positions j with (j & s) != 0
-        const uint64_t m = s == 8 ? 0xFFFFFFFF00000000ull
-                         : s == 4 ? 0xFFFF0000FFFF0000ull
-                         : s == 2 ? 0xFF00FF00FF00FF00ull
-                                  : 0xF0F0F0F0F0F0F0F0ull;
-        const uint32_t lo = __shfl_xor_sync(0xFFFFFFFFu, static_cast<uint32_t>(w), s);
-        const uint32_t hi = __shfl_xor_sync(0xFFFFFFFFu, static_cast<uint32_t>(w >> 32), s);
-        const uint64_t o = (static_cast<uint64_t>(hi) << 32) | lo;
-        if ((r & s) == 0) w = (w & ~m) | ((o & ~m) << (4 * s));
-        else w = (w & m) | ((o & m) >> (4 * s));
+    {   // s = 8: the lower lane's hi <-> the upper lane's lo
+        const bool up = (r & 8) != 0;
+        const uint32_t got = __shfl_xor_sync(0xFFFFFFFFu, up ? lo : hi, 8);
+        if (up) lo = got;
+        else hi = got;
     }
-    return w;
+    {   // s = 4: bytes 2-3 of each word (lower lane) <-> bytes 0-1 (upper lane)
+        const bool up = (r & 4) != 0;
+        const uint32_t got = __shfl_xor_sync(0xFFFFFFFFu, __byte_perm(lo, hi, up ? 0x5410u : 0x7632u), 4);
+        lo = __byte_perm(lo, got, up ? 0x3254u : 0x5410u);
+        hi = __byte_perm(hi, got, up ? 0x3276u : 0x7610u);
+    }
+    {   // s = 2: bytes 1 and 3 (lower lane) <-> bytes 0 and 2 (upper lane)
+        const bool up = (r & 2) != 0;
+        const uint32_t got = __shfl_xor_sync(0xFFFFFFFFu, __byte_perm(lo, hi, up ? 0x6420u : 0x7531u), 2);
+        lo = __byte_perm(lo, got, up ? 0x3514u : 0x5240u);
+        hi = __byte_perm(hi, got, up ? 0x3716u : 0x7260u);
+    }
+    {   // s = 1: odd nibbles (lower lane) <-> even nibbles (upper lane); the
+        // sent word holds lo's share in its low nibbles and hi's in its high ones
+        const bool up = (r & 1) != 0;
+        const uint32_t M = 0x0F0F0F0Fu, km = up ? ~M : M;
+        const uint32_t send = ((lo >> (up ? 0 : 4)) & M) | ((hi << (up ? 4 : 0)) & ~M);
+        const uint32_t got = __shfl_xor_sync(0xFFFFFFFFu, send, 1);
+        lo = (lo & km) | ((got << (up ? 0 : 4)) & ~km);
+        hi = (hi & km) | ((got >> (up ? 4 : 0)) & ~km);
+    }
 }
 
 // ---------------------------------------------------------------- 2D NVFP4
@@ -141,7 +159,9 @@ __global__ void __launch_bounds__(256) k_quant2d(const T *__restrict__ x, Q2DPar
     const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
     for (int64_t task = warp0; task < tasks; task += nwarps) {
-        const int64_t bq = task / pairs, tc = (task % pairs) * 2 + half;
+        // tasks < 2^31 (checked on the host): 32-bit index arithmetic
+        const uint32_t t32 = static_cast<uint32_t>(task), bq32 = t32 / static_cast<uint32_t>(pairs);
+        const int64_t bq = bq32, tc = static_cast<int64_t>(t32 - bq32 * static_cast<uint32_t>(pairs)) * 2 + half;
         const bool colv = tc < tiles_k;
         const int64_t j0 = tc * 16;
         Raw16<T> raw[4];
@@ -175,11 +195,8 @@ __global__ void __launch_bounds__(256) k_quant2d(const T *__restrict__ x, Q2DPar
 #pragma unroll
                     for (int t = 0; t < 8; ++t) pp[t] = f2pack(v[2 * t], v[2 * t + 1]);
                     nv_quot16_pairs(pp, S, amax, qq);
-                    float q[16];
-#pragma unroll
-                    for (int t = 0; t < 8; ++t) f2unpack(qq[t], q[2 * t], q[2 * t + 1]);
                     const int64_t i = (bq * 4 + b) * 16 + r;
-                    sr_group<16>(q, static_cast<uint64_t>(i * p.K + j0), p.seed, w[b]);
+                    sr_group_pairs<16>(qq, static_cast<uint64_t>(i * p.K + j0), p.seed, w[b]);
                 } else {
                     nv_block_rne(v, S, amax, w[b], nullptr);
                 }
@@ -197,7 +214,11 @@ __global__ void __launch_bounds__(256) k_quant2d(const T *__restrict__ x, Q2DPar
         if (p.codesT) {
             uint64_t tw[4];
 #pragma unroll
-            for (int b = 0; b < 4; ++b) tw[b] = transpose16x16_nibbles((static_cast<uint64_t>(w[b][1]) << 32) | w[b][0], r);
+            for (int b = 0; b < 4; ++b) {
+                uint32_t lo = w[b][0], hi = w[b][1];
+                transpose16x16_nibbles(lo, hi, r);
+                tw[b] = (static_cast<uint64_t>(hi) << 32) | lo;
+            }
             if (colv) {
                 const int64_t jr = j0 + r;                       // column of X = row of X^T
                 const int64_t base = jr * p.M + bq * 64;         // X^T element index of band 0
@@ -698,6 +719,8 @@ int quantize2d(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_fmt fmt
         QFP4_LAUNCH_CHECK();
         return QFP4_OK;
     }
+    const int64_t tasks = ((M / 16 + 3) / 4) * ((K / 16 + 1) / 2);     // 64 x 32 warp tasks
+    if (tasks >= (int64_t(1) << 31)) return QFP4_ERR_SHAPE;            // the kernel indexes tasks in 32 bits
     if (!opt.amax_in || opt.amax_out) {
         int st = amax_partials(x, xdt, M * K, partials, &p.n_partials, stream);
         if (st != QFP4_OK) return st;
@@ -706,7 +729,6 @@ int quantize2d(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_fmt fmt
             if (st != QFP4_OK) return st;
         }
     }
-    const int64_t tasks = ((M / 16 + 3) / 4) * ((K / 16 + 1) / 2);     // 64 x 32 warp tasks
     if (xdt == QFP4_BF16) {
         if (sr) launch_tiles<k_quant2d<true, uint16_t>, uint16_t>(tasks, x, p, stream);
         else launch_tiles<k_quant2d<false, uint16_t>, uint16_t>(tasks, x, p, stream);
