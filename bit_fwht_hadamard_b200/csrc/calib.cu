@@ -4,13 +4,14 @@
 // the kept histogram quantized to the levels and spread back over P's bins;
 // the T with the least D_KL(P || Q) loses the least information).
 //
-// Three launches after the tensor-amax pass: a histogram of |x| over [0,
-// amax] privatized in shared memory; one thread per candidate computing its
-// KL (the level of a bin never decreases with the bin, so a level's bins are
-// one contiguous run: a first walk over the run gathers its kept mass and
-// the count of P's nonzero bins, a second adds the run's terms, bins in
-// ascending order); one block taking the least KL (smallest candidate on a
-// tie) and writing the clip point T = fl(i * fl(amax / bins)).
+// Four launches after the tensor-amax pass: a histogram of |x| over [0,
+// amax] privatized in shared memory; prefix sums of the histogram and of its
+// nonzero bins; one warp per candidate computing its KL (the level of a bin
+// never decreases with the bin, so a level's bins are one contiguous run
+// whose kept mass and nonzero count are two prefix lookups; the lanes form
+// the terms of 32 bins at a time and one lane adds them in ascending bin
+// order); one block taking the least KL (smallest candidate on a tie) and
+// writing the clip point T = fl(i * fl(amax / bins)).
 #include <math_constants.h>
 
 #include "qfp4_common.cuh"
@@ -98,51 +99,136 @@ __device__ __forceinline__ int kl_level(int b, int i, int levels, int grid)
     return l < levels ? l : levels - 1;
 }
 
-// KL of candidate i = first + thread index; +inf when Q is zero where P is not.
-__global__ void __launch_bounds__(128) k_kl(const unsigned long long *__restrict__ hist, int bins, int levels, int grid,
-                                            double *kl)
+// Prefix sums of the histogram and of its count of nonzero bins, so that a
+// level's kept mass and nonzero count are two lookups: ph[b] = sum of
+// hist[0 .. b), pnz[b] = number of nonzero bins in [0, b), b = 0 .. bins.
+// One block of 1024 threads, each summing 8 consecutive bins (bins <= 8192).
+__global__ void __launch_bounds__(1024) k_hist_prefix(const unsigned long long *__restrict__ hist, int bins,
+                                                      unsigned long long *ph, int *pnz)
 {
+    __shared__ unsigned long long sh[1024];
+    __shared__ int sn[1024];
     pdl_wait();
     pdl_trigger();
+    const int t = threadIdx.x, b0 = 8 * t;
+    unsigned long long h = 0ull;
+    int c = 0;
+    for (int b = b0; b < b0 + 8 && b < bins; ++b) {
+        h += hist[b];
+        c += hist[b] != 0ull;
+    }
+    sh[t] = h;
+    sn[t] = c;
+    __syncthreads();
+    for (int off = 1; off < 1024; off <<= 1) {          // inclusive scan of the per-thread sums
+        const unsigned long long hv = t >= off ? sh[t - off] : 0ull;
+        const int cv = t >= off ? sn[t - off] : 0;
+        __syncthreads();
+        sh[t] += hv;
+        sn[t] += cv;
+        __syncthreads();
+    }
+    unsigned long long run = t ? sh[t - 1] : 0ull;        // exclusive prefix of this thread's first bin
+    int runc = t ? sn[t - 1] : 0;
+    for (int b = b0; b < b0 + 8 && b < bins; ++b) {
+        ph[b] = run;
+        pnz[b] = runc;
+        run += hist[b];
+        runc += hist[b] != 0ull;
+    }
+    if (t == 1023) {                                      // the totals
+        ph[bins] = sh[1023];
+        pnz[bins] = sn[1023];
+    }
+}
+
+// KL of candidate i, one warp per candidate; +inf when Q is zero where P is
+// not.  The level runs of candidate i are contiguous: uniform levels from
+// per = floor(i / levels), the E2M1 ones from the smallest bin of each level
+// (a binary search on e2m1_level_of_bin, which is monotone in the bin), so a
+// level's kept mass and nonzero count come from the prefix sums (the last
+// kept bin also holds the tail beyond i, which can make it nonzero).  The
+// lanes compute the terms p log(p / q) of 32 consecutive bins; lane 0 adds
+// them in ascending bin order, the order of the plain loop.
+__global__ void __launch_bounds__(256) k_kl(const unsigned long long *__restrict__ hist,
+                                            const unsigned long long *__restrict__ ph, const int *__restrict__ pnz,
+                                            int bins, int levels, int grid, double *kl)
+{
+    __shared__ double terms[8][32];
+    pdl_wait();
+    pdl_trigger();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int first = grid ? 8 : levels;
-    const int i = first + static_cast<int>(blockIdx.x * blockDim.x + threadIdx.x);
-    if (i > bins) return;
-    unsigned long long outliers = 0ull, kept = 0ull;
-    for (int b = i; b < bins; ++b) outliers += hist[b];
-    for (int b = 0; b < i; ++b) kept += hist[b];
+    const int i = first + static_cast<int>(blockIdx.x) * 8 + warp;
+    if (i > bins) return;                                 // the whole warp
+    const unsigned long long kept = ph[i], outliers = ph[bins] - ph[i];
     const double total_p = static_cast<double>(kept + outliers), total_q = static_cast<double>(kept);
+    // E2M1 run starts: start[l] = smallest bin of level >= l (start[0] = 0, start[8] = i)
+    int bound = i;
+    if (grid && lane < 7) {                               // lane t: smallest b with level(b) >= t + 1
+        int lo = 0, hi = i;
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (e2m1_level_of_bin(mid, i) >= lane + 1) hi = mid;
+            else lo = mid + 1;
+        }
+        bound = lo;
+    }
+    int start[9];
+    start[0] = 0;
+#pragma unroll
+    for (int t = 0; t < 7; ++t) start[t + 1] = __shfl_sync(0xFFFFFFFFu, bound, t);
+    start[8] = i;
+    const int per = grid ? 1 : i / levels;
     double d = 0.0;
     if (total_p != 0.0) {
         if (total_q == 0.0) {
             d = CUDART_INF;
         } else {
-            int b0 = 0;
-            while (b0 < i && d != CUDART_INF) {
-                const int l = kl_level(b0, i, levels, grid);
-                int b1 = b0 + 1;
-                while (b1 < i && kl_level(b1, i, levels, grid) == l) ++b1;
-                unsigned long long mass = 0ull;
-                long long nz = 0;
-                for (int b = b0; b < b1; ++b) {
-                    mass += hist[b];
-                    nz += (hist[b] + (b == i - 1 ? outliers : 0ull)) != 0ull;
-                }
-                const double qb = nz ? static_cast<double>(mass) / static_cast<double>(nz) : 0.0;
-                for (int b = b0; b < b1; ++b) {
-                    const double pb = static_cast<double>(hist[b] + (b == i - 1 ? outliers : 0ull));
-                    if (pb == 0.0) continue;
-                    if (qb == 0.0) {
-                        d = CUDART_INF;
-                        break;
+            for (int c0 = 0; c0 < i; c0 += 32) {
+                const int b = c0 + lane;
+                double term = 0.0;
+                if (b < i) {
+                    const unsigned long long pb_u = hist[b] + (b == i - 1 ? outliers : 0ull);
+                    if (pb_u != 0ull) {
+                        int b0, b1;
+                        if (grid) {
+                            const int l = e2m1_level_of_bin(b, i);
+                            b0 = 0;
+                            b1 = i;
+#pragma unroll
+                            for (int t = 0; t < 8; ++t)
+                                if (t == l) {
+                                    b0 = start[t];
+                                    b1 = start[t + 1];
+                                }
+                        } else {
+                            const int l = imin(b / per, levels - 1);
+                            b0 = l * per;
+                            b1 = l == levels - 1 ? i : b0 + per;
+                        }
+                        const unsigned long long mass = ph[b1] - ph[b0];
+                        long long nz = pnz[b1] - pnz[b0];
+                        if (b1 == i && hist[i - 1] == 0ull && outliers != 0ull) ++nz;   // the tail makes bin i - 1 nonzero
+                        const double qb = nz ? static_cast<double>(mass) / static_cast<double>(nz) : 0.0;
+                        if (qb == 0.0) {
+                            term = CUDART_INF;
+                        } else {
+                            const double pp = static_cast<double>(pb_u) / total_p, qq = qb / total_q;
+                            term = pp * log(pp / qq);
+                        }
                     }
-                    const double p = pb / total_p, q = qb / total_q;
-                    d += p * log(p / q);
                 }
-                b0 = b1;
+                terms[warp][lane] = term;
+                __syncwarp();
+                if (lane == 0)
+#pragma unroll 8
+                    for (int k = 0; k < 32; ++k) d += terms[warp][k];
+                __syncwarp();
             }
         }
     }
-    kl[i - first] = d;
+    if (lane == 0) kl[i - first] = d;
 }
 
 // least KL (smallest candidate on a tie) -> clip point and winning candidate
@@ -183,7 +269,7 @@ __global__ void __launch_bounds__(256) k_kl_pick(const double *kl, int count, in
 }
 
 struct KlLayout {
-    size_t partials, amax, hist, kl, total;
+    size_t partials, amax, hist, kl, ph, pnz, total;
 };
 
 static KlLayout kl_layout(int bins, int levels, int grid)
@@ -195,7 +281,9 @@ static KlLayout kl_layout(int bins, int levels, int grid)
     L.amax = a256(sizeof(float) * kMaxPartials);
     L.hist = L.amax + 256;
     L.kl = L.hist + a256(sizeof(unsigned long long) * bins);
-    L.total = L.kl + a256(sizeof(double) * (bins - first + 1));
+    L.ph = L.kl + a256(sizeof(double) * (bins - first + 1));
+    L.pnz = L.ph + a256(sizeof(unsigned long long) * (bins + 1));
+    L.total = L.pnz + a256(sizeof(int) * (bins + 1));
     return L;
 }
 
@@ -273,8 +361,14 @@ extern "C" int qfp4_kl_calibrate(const void *x, qfp4_dtype xdt, int64_t n, int b
                                                     static_cast<const float *>(amax), hist);
         if (st != QFP4_OK) return st;
     }
-    st = launch_simple<k_kl>(dim3((count + 127) / 128), dim3(128), 0, stream,
-                             static_cast<const unsigned long long *>(hist), bins, levels, grid, kl);
+    auto *ph = reinterpret_cast<unsigned long long *>(ws + L.ph);
+    int *pnz = reinterpret_cast<int *>(ws + L.pnz);
+    st = launch_simple<k_hist_prefix>(dim3(1), dim3(1024), 0, stream, static_cast<const unsigned long long *>(hist),
+                                      bins, ph, pnz);
+    if (st != QFP4_OK) return st;
+    st = launch_simple<k_kl>(dim3((count + 7) / 8), dim3(256), 0, stream, static_cast<const unsigned long long *>(hist),
+                             static_cast<const unsigned long long *>(ph), static_cast<const int *>(pnz), bins, levels,
+                             grid, kl);
     if (st != QFP4_OK) return st;
     return launch_simple<k_kl_pick>(dim3(1), dim3(256), 0, stream, static_cast<const double *>(kl), count, first, bins,
                                     static_cast<const float *>(amax), clip_out, best_bins_out);

@@ -158,20 +158,32 @@ __global__ void __launch_bounds__(256) k_quant2d(const T *__restrict__ x, Q2DPar
     const int64_t tasks = quads * pairs;
     const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-    for (int64_t task = warp0; task < tasks; task += nwarps) {
-        // tasks < 2^31 (checked on the host): 32-bit index arithmetic
+    // task -> (band quad, tile column); tasks < 2^31 (checked on the host),
+    // so the division runs in 32 bits
+    auto task_pos = [&](int64_t task, int64_t &bq, int64_t &tc) {
         const uint32_t t32 = static_cast<uint32_t>(task), bq32 = t32 / static_cast<uint32_t>(pairs);
-        const int64_t bq = bq32, tc = static_cast<int64_t>(t32 - bq32 * static_cast<uint32_t>(pairs)) * 2 + half;
+        bq = bq32;
+        tc = static_cast<int64_t>(t32 - bq32 * static_cast<uint32_t>(pairs)) * 2 + half;
+    };
+    auto load_task = [&](int64_t task, Raw16<T> (&rw)[4]) {
+        int64_t bq, tc;
+        task_pos(task, bq, tc);
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const int64_t band = bq * 4 + b;
+            raw_load16(x, (band * 16 + r) * p.K + tc * 16, tc < tiles_k && band < bands, rw[b]);
+        }
+    };
+    for (int64_t task = warp0; task < tasks; task += nwarps) {
+        int64_t bq, tc;
+        task_pos(task, bq, tc);
         const bool colv = tc < tiles_k;
         const int64_t j0 = tc * 16;
         Raw16<T> raw[4];
         bool bv[4];
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            const int64_t band = bq * 4 + b;
-            bv[b] = band < bands;
-            raw_load16(x, (band * 16 + r) * p.K + j0, colv && bv[b], raw[b]);
-        }
+        for (int b = 0; b < 4; ++b) bv[b] = bq * 4 + b < bands;
+        load_task(task, raw);
         uint32_t w[4][2], enc[4];
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
@@ -502,14 +514,8 @@ __global__ void __launch_bounds__(256) k_mxfp8(const T *__restrict__ x, Q2DParam
 }
 
 // ---------------------------------------------------------------- column-wise outputs, 4 columns a lane
-// bf16 input: a warp covers 32 rows x 128 columns, lane l the 4 adjacent
-// columns jb = j0 + 4 l .. jb + 3, loaded as one 8-byte word per row (256
-// bytes per warp instruction).  The 32 rows stay as raw bf16 pairs (64
-// registers).  Per column: the group maxima, the scales, then the codes of
-// X^T row jb + c (E2M1 nibbles, or E4M3 bytes for FMT_MXFP8).  Stochastic
-// rounding runs row by row: the 4 columns of a row are one Philox counter
-// ((i0 + r) K + jb) / 4, so each call serves four elements.  Groups along M:
-// 32 (MXFP4, MXFP8) or 16 (NVFP4, where the last row block may have 16 rows).
+// fl(x / S) for one value: division-free when the block is on the fast path
+// (y = fl(1/S)), else the IEEE division; the sign of x is kept, also on zero.
 __device__ __forceinline__ float nv_quot1(float x, float S, float y, bool fast)
 {
     if (!fast) return __fdiv_rn(x, S);
@@ -517,7 +523,14 @@ __device__ __forceinline__ float nv_quot1(float x, float S, float y, bool fast)
     return __uint_as_float(__float_as_uint(q) | (__float_as_uint(x) & 0x80000000u));   // sign of x, also on zero
 }
 
-template <int FMT, bool SR, bool FOUR6>
+// Round-to-nearest column-wise outputs from bf16 input (stochastic rounding
+// has k_cols_sr): a warp covers 32 rows x 128 columns, lane l the 4 adjacent
+// columns jb = j0 + 4 l .. jb + 3, loaded as one 8-byte word per row (256
+// bytes per warp instruction).  The 32 rows stay as raw bf16 pairs (64
+// registers).  Per column: the group maxima, the scales, then the codes of
+// X^T row jb + c (E2M1 nibbles, or E4M3 bytes for FMT_MXFP8).  Groups along M:
+// 32 (MXFP4, MXFP8) or 16 (NVFP4, where the last row block may have 16 rows).
+template <int FMT, bool FOUR6>
 __global__ void __launch_bounds__(256) k_cols4(const uint16_t *__restrict__ x, Q2DParams p)
 {
     constexpr bool MX8 = FMT == FMT_MXFP8, NV = FMT == QFP4_NVFP4;
@@ -602,24 +615,7 @@ __global__ void __launch_bounds__(256) k_cols4(const uint16_t *__restrict__ x, Q
             }
 
         // codes
-        if (SR) {
-#pragma unroll
-            for (int r = 0; r < 32; ++r) {
-                if (r < rows) {
-                    const uint4 rw = sr_words4(p.seed, static_cast<uint64_t>((i0 + r) * p.K + jb) >> 2);
-                    const uint32_t wd[4] = {rw.x, rw.y, rw.z, rw.w};
-                    const int g = r / G;
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        if (S[g][c] == 0.0f) continue;       // zero group (or S = 0): code 0
-                        const float v = val(r, c);
-                        const float q = NV ? nv_quot1(v, S[g][c], Y[g][c], fast[g][c]) : __fmul_rn(v, mul[c]);
-                        if (MX8) w[c][r >> 2] |= e4m3_sr(q, wd[c]) << (8 * (r & 3));
-                        else w[c][r >> 3] |= e2m1_sr(q, wd[c]) << (4 * (r & 7));
-                    }
-                }
-            }
-        } else if (!FOUR6) {
+        if (!FOUR6) {
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
 #pragma unroll
@@ -740,13 +736,177 @@ int quantize2d(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_fmt fmt
     return QFP4_OK;
 }
 
-// bf16: the 4-columns-a-lane kernel (32 x 128 tasks); binary32: one column a lane.
+// Stochastic rounding of the column-wise outputs from bf16 input.  A warp
+// covers 32 rows x 64 columns; lanes 2p and 2p + 1 share the 4 adjacent
+// columns jb = j0 + 4p .. jb + 3, lane q = lane & 1 taking columns jb + 2q
+// and jb + 2q + 1, read as one 4-byte word per row (128 bytes per warp
+// instruction, 32 registers for the tile, so two blocks fit an SM where the
+// 4-columns-a-lane kernel fits one).  The Philox counter of a row's 4
+// columns is ((i0 + r) K + jb) / 4: in step k the lower lane of a pair draws
+// row k and the upper lane row 16 + k, each keeps the two words of its own
+// columns and sends the other two to its partner, so each call still serves
+// four elements.  The decision runs on the lane's two columns as a packed
+// pair.  All-zero groups (and NVFP4 blocks whose scale is 0) get +0 codes.
+// Groups along M: 32 (MXFP4, MXFP8) or 16 (NVFP4, whose last row block may
+// have 16 rows).  No lane leaves the loop early: the shuffles need the whole
+// warp, so lanes past K load zeros and store nothing.
+template <int FMT>
+__global__ void __launch_bounds__(256) k_cols_sr(const uint16_t *__restrict__ x, Q2DParams p)
+{
+    constexpr bool MX8 = FMT == FMT_MXFP8, NV = FMT == QFP4_NVFP4;
+    constexpr int G = NV ? 16 : 32, NG = 32 / G, CW = MX8 ? 8 : 4;   // code words per column
+    __shared__ float red[32];
+    float s_t = 0.0f;
+    if (NV) s_t = q2d_tensor_scale(p, red);
+    const NvScale nz = nv_scale_setup(s_t, p.rule);
+    const int lane = threadIdx.x & 31, q = lane & 1;
+    const int64_t col_blocks = (p.K + 63) / 64, row_blocks = (p.M + 31) / 32;
+    const int64_t tasks = row_blocks * col_blocks;
+    const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    for (int64_t task = warp0; task < tasks; task += nwarps) {
+        const int64_t i0 = (task / col_blocks) * 32, jb = (task % col_blocks) * 64 + 4 * (lane >> 1);
+        const int rows = static_cast<int>(imin<int64_t>(32, p.M - i0));   // 32, or 16 (NVFP4, M % 32 == 16)
+        const bool colv = jb < p.K;                 // K % 4 == 0: a pair's columns are all in or all out
+        const int64_t j = jb + 2 * q;               // this lane's first column
+        uint32_t raw[32];
+#pragma unroll
+        for (int r = 0; r < 32; ++r)
+            raw[r] = (colv && r < rows) ? *reinterpret_cast<const uint32_t *>(x + (i0 + r) * p.K + j) : 0u;
+
+        // per group and column: the scale byte, the divisor (or multiplier)
+        uint64_t mul2[NG], y2[NG], nS2[NG];
+        bool fast2[NG], zero[NG][2];
+        float Sg[NG][2], Yg[NG][2];
+        uint32_t sb[NG][2];
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+            uint32_t m = 0u;                        // |bf16| maxima of both columns as 16-bit integers
+#pragma unroll
+            for (int r = 0; r < G; ++r) {
+                uint32_t t;
+                asm("max.u16x2 %0, %1, %2;" : "=r"(t) : "r"(m), "r"(raw[G * g + r] & 0x7FFF7FFFu));
+                m = t;
+            }
+            const float amax[2] = {bf16lo(m), bf16hi(m)};
+            float mulc[2] = {0.0f, 0.0f};
+            bool fast[2] = {false, false};
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                sb[g][c] = 0u;
+                Sg[g][c] = 0.0f;
+                Yg[g][c] = 0.0f;
+                if (!NV) {
+                    zero[g][c] = amax[c] == 0.0f;
+                    if (!zero[g][c]) {
+                        const int k = MX8 ? scale_exp(amax[c], 0x600000u, 8) : mx_scale_exp(amax[c], p.rule);
+                        sb[g][c] = static_cast<uint32_t>(k + 127);
+                        mulc[c] = exp2i(-k);
+                    }
+                } else {
+                    if (s_t != 0.0f) {
+                        sb[g][c] = nv_scale_byte<true>(amax[c], nz);
+                        Sg[g][c] = __fmul_rn(e4m3_value(sb[g][c]), s_t);
+                    }
+                    zero[g][c] = Sg[g][c] == 0.0f;
+                    fast[c] = Sg[g][c] >= 0x1p-125f && Sg[g][c] <= 0x1p125f && amax[c] <= Sg[g][c] * 0x1p100f;
+                    Yg[g][c] = fast[c] ? __frcp_rn(Sg[g][c]) : 0.0f;
+                }
+            }
+            mul2[g] = f2pack(mulc[0], mulc[1]);
+            y2[g] = f2pack(Yg[g][0], Yg[g][1]);
+            nS2[g] = f2pack(-Sg[g][0], -Sg[g][1]);
+            fast2[g] = fast[0] && fast[1];
+        }
+
+        uint32_t code[2][CW];
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int t = 0; t < CW; ++t) code[c][t] = 0u;
+        // one element pair (row r, the lane's two columns) under words w0, w1
+        auto round_pair = [&](int r, uint32_t w0, uint32_t w1) {
+            const int g = r / G;
+            const uint64_t v = f2pack(bf16lo(raw[r]), bf16hi(raw[r]));
+            uint64_t qv;
+            if (!NV) {
+                qv = f2mul(v, mul2[g]);
+            } else if (fast2[g]) {
+                qv = div_rn_by2(v, y2[g], nS2[g]);
+            } else {
+                qv = f2pack(nv_quot1(bf16lo(raw[r]), Sg[g][0], Yg[g][0], Yg[g][0] != 0.0f),
+                            nv_quot1(bf16hi(raw[r]), Sg[g][1], Yg[g][1], Yg[g][1] != 0.0f));
+            }
+            if (MX8) {
+                float q0, q1;
+                f2unpack(qv, q0, q1);
+                code[0][r >> 2] |= e4m3_sr(q0, w0) << (8 * (r & 3));
+                code[1][r >> 2] |= e4m3_sr(q1, w1) << (8 * (r & 3));
+            } else {
+                float g0, g1;
+                f2unpack(e2m1_sr_grid2(qv, w0, w1), g0, g1);
+                uint32_t b;                         // low nibble: column 0, high nibble: column 1
+                asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
+                    : "=r"(b) : "f"(g1), "f"(g0));
+                code[0][r >> 3] |= (b & 0xFu) << (4 * (r & 7));
+                code[1][r >> 3] |= ((b >> 4) & 0xFu) << (4 * (r & 7));
+            }
+        };
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const int rr = k + 16 * q;               // the row this lane draws
+            const uint4 wd = sr_words4(p.seed, static_cast<uint64_t>((i0 + rr) * p.K + jb) >> 2);
+            const uint32_t own0 = q ? wd.z : wd.x, own1 = q ? wd.w : wd.y;
+            const uint32_t got0 = __shfl_xor_sync(0xFFFFFFFFu, q ? wd.x : wd.z, 1);
+            const uint32_t got1 = __shfl_xor_sync(0xFFFFFFFFu, q ? wd.y : wd.w, 1);
+            round_pair(k, q ? got0 : own0, q ? got1 : own1);                  // row k
+            if (16 + k < rows) round_pair(16 + k, q ? own0 : got0, q ? own1 : got1);   // row 16 + k
+        }
+#pragma unroll
+        for (int g = 0; g < NG; ++g)
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+                if (zero[g][c])
+#pragma unroll
+                    for (int t = g * CW / NG; t < (g + 1) * CW / NG; ++t) code[c][t] = 0u;
+
+        // stores: X^T rows j, j + 1; elements i0 .. i0 + rows - 1
+        if (colv) {
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                const int64_t jr = j + c;
+                if (MX8) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.codesT + jr * p.M + i0);
+                    dst[0] = make_uint4(code[c][0], code[c][1], code[c][2], code[c][3]);
+                    dst[1] = make_uint4(code[c][4], code[c][5], code[c][6], code[c][7]);
+                    p.scalesT[jr * (p.M / 32) + i0 / 32] = static_cast<uint8_t>(sb[0][c]);
+                } else {
+                    uint2 *dst = reinterpret_cast<uint2 *>(p.codesT + (jr * p.M + i0) / 2);
+                    dst[0] = make_uint2(code[c][0], code[c][1]);
+                    if (rows == 32) dst[1] = make_uint2(code[c][2], code[c][3]);
+                    if (G == 32) {
+                        p.scalesT[jr * (p.M / 32) + i0 / 32] = static_cast<uint8_t>(sb[0][c]);
+                    } else {
+                        p.scalesT[jr * (p.M / 16) + i0 / 16] = static_cast<uint8_t>(sb[0][c]);
+                        if (rows == 32) p.scalesT[jr * (p.M / 16) + i0 / 16 + 1] = static_cast<uint8_t>(sb[NG - 1][c]);
+                    }
+                }
+            }
+        }
+    }
+}
+
+// bf16: the lane-pair kernel for stochastic rounding (32 x 64 tasks), else the
+// 4-columns-a-lane kernel (32 x 128 tasks); binary32: one column a lane.
 template <int FMT, bool SR, bool FOUR6>
 static int launch_cols(const void *x, qfp4_dtype xdt, const Q2DParams &p, cudaStream_t stream)
 {
-    if (xdt == QFP4_BF16)
-        launch_tiles<k_cols4<FMT, SR, FOUR6>, uint16_t>(((p.M + 31) / 32) * ((p.K + 127) / 128), x, p, stream);
-    else
+    if (xdt == QFP4_BF16) {
+        if constexpr (SR)
+            launch_tiles<k_cols_sr<FMT>, uint16_t>(((p.M + 31) / 32) * ((p.K + 63) / 64), x, p, stream);
+        else
+            launch_tiles<k_cols4<FMT, FOUR6>, uint16_t>(((p.M + 31) / 32) * ((p.K + 127) / 128), x, p, stream);
+    } else
         launch_tiles<k_quant_cols<FMT, SR, FOUR6, float>, float>(((p.M + 31) / 32) * ((p.K + 31) / 32), x, p, stream);
     QFP4_LAUNCH_CHECK();
     return QFP4_OK;
@@ -777,9 +937,8 @@ int quantize_mxfp8(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, qfp4_rou
         // (if asked for) by the tile kernel without its row part
         int st = mxfp8_rows(x, M * K, sr, seed, codes, scales, stream);
         if (st != QFP4_OK || !cols) return st;
-        const int64_t tasks4 = ((M + 31) / 32) * ((K + 127) / 128);
-        if (sr) launch_tiles<k_cols4<FMT_MXFP8, true, false>, uint16_t>(tasks4, x, p, stream);
-        else launch_tiles<k_cols4<FMT_MXFP8, false, false>, uint16_t>(tasks4, x, p, stream);
+        if (sr) launch_tiles<k_cols_sr<FMT_MXFP8>, uint16_t>(((M + 31) / 32) * ((K + 63) / 64), x, p, stream);
+        else launch_tiles<k_cols4<FMT_MXFP8, false>, uint16_t>(((M + 31) / 32) * ((K + 127) / 128), x, p, stream);
         QFP4_LAUNCH_CHECK();
         return QFP4_OK;
     }
@@ -808,9 +967,8 @@ int quantize_mxfp8_columns(const void *x, qfp4_dtype xdt, int64_t M, int64_t K, 
     Q2DParams p{M, K, nullptr, nullptr, codesT, scalesT, nullptr, 0, nullptr, seed, QFP4_SCALE_DEFAULT, nullptr};
     const bool sr = rounding == QFP4_SR;
     if (xdt == QFP4_BF16) {
-        const int64_t tasks4 = ((M + 31) / 32) * ((K + 127) / 128);
-        if (sr) launch_tiles<k_cols4<FMT_MXFP8, true, false>, uint16_t>(tasks4, x, p, stream);
-        else launch_tiles<k_cols4<FMT_MXFP8, false, false>, uint16_t>(tasks4, x, p, stream);
+        if (sr) launch_tiles<k_cols_sr<FMT_MXFP8>, uint16_t>(((M + 31) / 32) * ((K + 63) / 64), x, p, stream);
+        else launch_tiles<k_cols4<FMT_MXFP8, false>, uint16_t>(((M + 31) / 32) * ((K + 127) / 128), x, p, stream);
     } else {
         const int64_t tasks = ((M + 31) / 32) * (K / 32);
         if (sr) launch_tiles<k_mxfp8<true, false, true, float>, float>(tasks, x, p, stream);
