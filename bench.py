@@ -245,9 +245,10 @@ def _oracle_step_parallel(oracle, x, threads):
 
 def cpu_baseline():
     """The oracle on the host cores: one full default step single-threaded,
-    the same step row-partitioned over every core (checked identical), and
-    the binary64 oracle GEMM on a 128 x 128 x 4096 sub-problem, extrapolated
-    by flops to the 8192 x 11008 x 4096 GEMM."""
+    the same step row-partitioned over every core (checked identical), the
+    single-threaded oracle on the full config-3 and config-4 quantize inputs,
+    and the binary64 oracle GEMM on a 128 x 128 x 4096 sub-problem,
+    extrapolated by flops to the 8192 x 11008 x 4096 GEMM."""
     import oracle
     import synth
     x = synth.cfg2_X()
@@ -272,11 +273,27 @@ def cpu_baseline():
     dtg = time.perf_counter() - t0
     gflops = 2.0 * m * n * K / dtg / 1e9
     Mg, Ng, Kg = GEMM_SHAPE
+    # single-threaded oracle on the full tensors of the other quantize configs
+    configs = {}
+    for name, fn, bpe in (
+            ("cfg3 X 8192x4096 NVFP4 four-over-six RNE",
+             lambda: oracle.quantize(synth.cfg3_X(), oracle.NVFP4, four6=True), 2.5625),
+            ("cfg3 W 11008x4096 NVFP4 four-over-six RNE",
+             lambda: oracle.quantize(synth.cfg3_W(), oracle.NVFP4, four6=True), 2.5625),
+            ("cfg4 G 8192x4096 2D 16x16 NVFP4 SR (seed 1004), G and G^T",
+             lambda: oracle.quantize(synth.cfg4_G(), oracle.NVFP4, oracle.SR, block2d=True, seed=1004,
+                                     transposed=True), 3.125)):
+        elems = {"cfg3 X": 8192 * 4096, "cfg3 W": 11008 * 4096, "cfg4 G": 8192 * 4096}[name[:6]]
+        t0 = time.perf_counter()
+        fn()
+        dt = time.perf_counter() - t0
+        configs[name] = {"seconds": dt, "elements_per_s": elems / dt, "GB/s": elems * bpe / dt / 1e9, "cores": 1}
     return {"value": step_bytes / dtn / 1e9, "unit": "GB/s", "cores": nproc, "kind": "oracle",
             "sample": f"one full step (X 4096x4096, FWHT-128 + MXFP4, RNE + SR) row-partitioned over {nproc} "
                       f"threads, output identical to the single-threaded run: {identical}",
             "seconds": dtn, "identical_to_single_thread": identical, "nproc": nproc,
             "single_thread": {"value": step_bytes / dt1 / 1e9, "unit": "GB/s", "cores": 1, "seconds": dt1},
+            "single_thread_configs": configs,
             "gemm": {"value": gflops, "unit": "GFLOP/s", "cores": 1, "kind": "oracle",
                      "sample": f"binary64 oracle GEMM, every output of {m}x{n}x{K} (NVFP4 four-over-six operands)",
                      "seconds": dtg, "extrapolated_ms_for": f"{Mg}x{Ng}x{Kg}",
@@ -451,6 +468,24 @@ def run_gpu(args, rank, world):
     e2e = {"value": world * step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
+    # ---- the same step with one input/output set, which stays in L2 (42.5 MB
+    # of a 126 MB L2): the L2-warm figure beside the flushed one
+    torch.cuda.synchronize()
+    w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for i in range(3):
+        step(0)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda._sleep(int(2e9 * min(0.5, 40e-6 * args.steps + 2e-3)))
+    w0.record(stream)
+    for i in range(args.steps):
+        step(0)
+    w1.record(stream)
+    torch.cuda.synchronize()
+    warm_ms = max_over_ranks(w0.elapsed_time(w1), dist, dev) / args.steps
+    l2_warm = {"value": world * step_bytes / (warm_ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": warm_ms,
+               "note": "one input/output set, L2-resident between steps"}
+
     # ---- GEMM of the NVFP4 forward linear (tensor-core roofline)
     gemm = None
     if not args.no_gemm:
@@ -467,7 +502,7 @@ def run_gpu(args, rank, world):
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": workload_config(),
-        "roofline": roofline, "e2e": e2e, "gpu_launches": int(n_launch), "clocks": clocks,
+        "roofline": roofline, "e2e": e2e, "l2_warm": l2_warm, "gpu_launches": int(n_launch), "clocks": clocks,
         "frac_of_hbm_peak": value / world / hbm_peak,
     }
     if gemm is not None:
