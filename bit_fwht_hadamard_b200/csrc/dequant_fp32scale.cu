@@ -5,87 +5,70 @@
 
 namespace qfp4 {
 
-// binary64 -> bfloat16, round to nearest even: 8 significant bits with the
-// binary32 exponent range (subnormal quantum 2^-133).
-__device__ __forceinline__ uint16_t f64_to_bf16_rn(double v)
-{
-    const double a = fabs(v);
-    uint32_t u = 0;
-    if (a != 0.0) {
-        const int e = ilogb(a);
-        const int qe = max(e - 7, -133);
-        const double r = ldexp(rint(ldexp(a, -qe)), qe);    // exact scalings, one rounding
-        u = __float_as_uint(static_cast<float>(r));         // r fits bfloat16, so binary32
-    }
-    return static_cast<uint16_t>((u >> 16) | (signbit(v) ? 0x8000u : 0u));
-}
-
-// bfloat16 bits of the exact product m * s, given p = fl(m * s) (binary32)
-// and its exact error e = m * s - p (one FMA).  Rounding p to bfloat16 by
-// ties-to-even gives the rounding of m * s except when p is itself a
-// bfloat16 midpoint, where the sign of e says on which side m * s lies.
-// Needs |p| >= 2^-100 (the error of the product is then representable) or
-// m * s exactly zero.
-__device__ __forceinline__ uint32_t bf16_from_split(float p, float e)
-{
-    const uint32_t u = __float_as_uint(p);
-    if ((u & 0xFFFFu) == 0x8000u && e != 0.0f) {
-        const bool away = (e > 0.0f) == (p > 0.0f);      // m * s beyond the midpoint in magnitude
-        return (away ? u + 0x8000u : u - 0x8000u) >> 16;
-    }
-    return (u + 0x7FFFu + ((u >> 16) & 1u)) >> 16;
-}
-
 // 2^(b - 128) for a byte b, as binary32 (2^-128 and 2^-127 are subnormal).
 __device__ __forceinline__ float exp2_b128(uint32_t b)
 {
     return __uint_as_float(b >= 2u ? (b - 1u) << 23 : 0x00200000u << b);
 }
 
-// One 16-element chunk (one NVFP4 block, half an MXFP4 group) from its code
-// word pair w and scale byte sb.  Every output is the exact value
-// g * scale (* s_t) rounded once:
+// E2M1 codes of four elements (16 bits, element t in bits 4t .. 4t + 3) as
+// two bfloat16 pairs (exact: bfloat16 holds every E2M1 value).  The high and
+// low bytes of the eight magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6 (bf16 0x0000,
+// 0x3F00, 0x3F80, 0x3FC0, 0x4000, 0x4040, 0x4080, 0x40C0) are two byte-permute
+// tables indexed by the 3-bit magnitudes, two more permutes interleave them,
+// and the sign bits go to bits 15 and 31.
+__device__ __forceinline__ void e2m1x4_to_bf16x2(uint32_t w16, uint32_t &p01, uint32_t &p23)
+{
+    const uint32_t sel = w16 & 0x7777u;
+    const uint32_t hi = __byte_perm(0x3F3F3F00u, 0x40404040u, sel);
+    const uint32_t lo = __byte_perm(0xC0800000u, 0xC0804000u, sel);
+    p01 = __byte_perm(lo, hi, 0x5140u) | ((w16 << 12) & 0x8000u) | ((w16 << 24) & 0x80000000u);
+    p23 = __byte_perm(lo, hi, 0x7362u) | ((w16 << 4) & 0x8000u) | ((w16 << 16) & 0x80000000u);
+}
+
+// Four consecutive elements e0 .. e0 + 3 from their two code bytes w16 and
+// their scale byte sb.  Every output is the exact value g * scale (* s_t)
+// rounded once:
 // - MXFP4: g * 2^(b-127) = (2 g) * 2^(b-128) has at most two significant bits
 //   and an exponent >= -129, so it is exact in binary32 and in bfloat16.
 // - NVFP4: m = g * dec(enc) is exact (at most 6 significant bits, inside the
 //   normal range), and fl(m * s_t) is the one rounding (binary32 out); for
-//   bfloat16 out the rounding uses the split above, or binary64 for products
-//   below 2^-100 or beyond the binary32 range.
+//   bfloat16 out the product is formed exactly in binary64 and converted
+//   once (cvt.rn.bf16.f64: one rounding, which the tests check on products
+//   placed on and next to bfloat16 midpoints).
 // A scale byte that encodes NaN (E8M0 0xFF, E4M3 0x7F / 0xFF) gives NaN.
 template <int FMT, int OUT>
-__device__ __forceinline__ void dequant_chunk(uint2 w, uint32_t sb, float st, int64_t e0, void *out)
+__device__ __forceinline__ void dequant_quad(uint32_t w16, uint32_t sb, float st, int64_t e0, void *out)
 {
-    const uint64_t st2 = f2pack(st, st);
-    uint64_t g[8], m[8], v[8];
-    e2m1x8_values(w.x, g);
-    e2m1x8_values(w.y, g + 4);
+    uint32_t p01, p23;
+    e2m1x4_to_bf16x2(w16, p01, p23);
+    const uint64_t g[2] = {f2pack(__uint_as_float(p01 << 16), __uint_as_float(p01 & 0xFFFF0000u)),
+                           f2pack(__uint_as_float(p23 << 16), __uint_as_float(p23 & 0xFFFF0000u))};
+    uint64_t v[2], m[2];
+    const double st64 = st;
     if (FMT == QFP4_MXFP4) {
         const float h = sb == 255u ? __uint_as_float(0x7FC00000u) : exp2_b128(sb);   // E8M0 0xFF: NaN
         const uint64_t two = f2pack(2.0f, 2.0f), h2 = f2pack(h, h);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = f2mul(f2mul(g[j], two), h2);
+        for (int j = 0; j < 2; ++j) v[j] = f2mul(f2mul(g[j], two), h2);
     } else {
         const float d = (sb & 0x7Fu) == 0x7Fu ? __uint_as_float(0x7FC00000u) : e4m3_value(sb);   // E4M3 NaN
-        const uint64_t d2 = f2pack(d, d);
+        const uint64_t d2 = f2pack(d, d), st2 = f2pack(st, st);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 2; ++j) {
             m[j] = f2mul(g[j], d2);
             v[j] = f2mul(m[j], st2);
         }
     }
     if (OUT == QFP4_F32) {
-        float4 *o = reinterpret_cast<float4 *>(static_cast<float *>(out) + e0);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            float a, b, c, d;
-            f2unpack(v[2 * q], a, b);
-            f2unpack(v[2 * q + 1], c, d);
-            o[q] = make_float4(a, b, c, d);
-        }
+        float a, b, c, d;
+        f2unpack(v[0], a, b);
+        f2unpack(v[1], c, d);
+        *reinterpret_cast<float4 *>(static_cast<float *>(out) + e0) = make_float4(a, b, c, d);
     } else {
-        uint32_t h[8];
+        uint32_t h[2];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 2; ++j) {
             float p[2], mm[2];
             f2unpack(v[j], p[0], p[1]);
             uint32_t b16[2];
@@ -93,39 +76,49 @@ __device__ __forceinline__ void dequant_chunk(uint2 w, uint32_t sb, float st, in
                 b16[0] = __float_as_uint(p[0]) >> 16;          // exact in bfloat16
                 b16[1] = __float_as_uint(p[1]) >> 16;
             } else {
+                // m * s_t is exact in binary64 (at most 6 + 24 significant
+                // bits); one conversion rounds it to bfloat16
                 f2unpack(m[j], mm[0], mm[1]);
 #pragma unroll
                 for (int t = 0; t < 2; ++t) {
-                    const float a = fabsf(p[t]);
-                    if ((a >= 0x1p-100f && a <= 3.0e38f) || mm[t] == 0.0f)
-                        b16[t] = bf16_from_split(p[t], __fmaf_rn(mm[t], st, -p[t]));
-                    else if (a != a)
-                        b16[t] = 0x7FC0u;
-                    else
-                        b16[t] = f64_to_bf16_rn(static_cast<double>(mm[t]) * static_cast<double>(st));
+                    uint16_t r16;
+                    asm("cvt.rn.bf16.f64 %0, %1;" : "=h"(r16) : "d"(static_cast<double>(mm[t]) * st64));
+                    b16[t] = mm[t] != mm[t] ? 0x7FC0u : r16;
                 }
             }
             h[j] = b16[0] | (b16[1] << 16);
         }
-        uint4 *o = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(out) + e0);
-        o[0] = make_uint4(h[0], h[1], h[2], h[3]);
-        o[1] = make_uint4(h[4], h[5], h[6], h[7]);
+        *reinterpret_cast<uint2 *>(static_cast<uint16_t *>(out) + e0) = make_uint2(h[0], h[1]);
     }
 }
 
-// One thread per 16-element chunk (grid-stride loop).
+// Four consecutive elements a thread (a warp covers 128 elements: 64
+// contiguous code bytes in, 512 (binary32) or 256 (bf16) contiguous bytes
+// out), four such quads a thread per loop iteration with all their loads
+// issued first.  n % 16 == 0 (checked on the host).
 template <int FMT, int OUT>
 __global__ void __launch_bounds__(256) k_dequant(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scales,
-                                                 const float *__restrict__ tscale, int64_t n, void *out)
+                                                  const float *__restrict__ tscale, int64_t n, void *out)
 {
-    const int64_t chunks = n / 16;
+    constexpr int U = 4;
+    const int64_t quads = n / 4;
     const float st = FMT == QFP4_NVFP4 ? *tscale : 1.0f;
-    for (int64_t c = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; c < chunks;
-         c += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t e0 = c * 16;
-        const uint2 w = *reinterpret_cast<const uint2 *>(codes + e0 / 2);
-        const uint32_t sb = scales[FMT == QFP4_MXFP4 ? e0 / 32 : e0 / 16];
-        dequant_chunk<FMT, OUT>(w, sb, st, e0, out);
+    const int64_t nth = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    const int64_t t0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const uint16_t *c16 = reinterpret_cast<const uint16_t *>(codes);
+    for (int64_t base = 0; base < quads; base += U * nth) {
+        uint32_t w[U], sb[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t qd = base + t0 + u * nth;
+            w[u] = qd < quads ? c16[qd] : 0u;
+            sb[u] = qd < quads ? scales[FMT == QFP4_MXFP4 ? qd / 8 : qd / 4] : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t qd = base + t0 + u * nth;
+            if (qd < quads) dequant_quad<FMT, OUT>(w[u], sb[u], st, 4 * qd, out);
+        }
     }
 }
 
@@ -133,8 +126,8 @@ int dequantize(const uint8_t *codes, const uint8_t *scales, const float *tscale,
                qfp4_dtype out_dt, void *out, cudaStream_t stream)
 {
     if (n == 0) return QFP4_OK;
-    const int64_t chunks = n / 16;
-    const int grid = static_cast<int>(imin<int64_t>((chunks + 255) / 256, 8 * num_sms()));
+    const int64_t quads = n / 4;
+    const int grid = static_cast<int>(imin<int64_t>((quads + 1023) / 1024, 8 * num_sms()));
     if (fmt == QFP4_MXFP4) {
         if (out_dt == QFP4_F32) k_dequant<QFP4_MXFP4, QFP4_F32><<<grid, 256, 0, stream>>>(codes, scales, tscale, n, out);
         else k_dequant<QFP4_MXFP4, QFP4_BF16><<<grid, 256, 0, stream>>>(codes, scales, tscale, n, out);
