@@ -800,7 +800,7 @@ def run_rows(only=""):
             del x2
         # NVFP4 forward-linear operands: tensor amax, E4M3 scales, four-over-six
         nv = 2 + 0.5 + 1 / 16
-        if want("nvfp4 four-over-six", "nvfp4", "dequantize"):
+        if want("nvfp4 four-over-six", "nvfp4", "dequantize", "scale rules"):
             x3, w3 = bf16(synth.cfg3_X()), bf16(synth.cfg3_W())
             if want("nvfp4 four-over-six"):
                 fp4_row("nvfp4 four-over-six", "X bf16 8192x4096 Student-t(3)*0.5: NVFP4 four-over-six RNE", x3, q.NVFP4,
@@ -823,7 +823,7 @@ def run_rows(only=""):
                 dequant_row("dequantize", "NVFP4 codes of X 8192x4096 -> fp32", x3, q.NVFP4, F32)
             del x3, w3
         # Quartet-style backward: 2D blocks, MXFP8, column-wise 1D, backward GEMMs
-        if want("2d blocks", "column-wise", "mxfp8", "gemm"):
+        if want("2d blocks", "column-wise", "mxfp8", "gemm", "scale rules"):
             g4 = bf16(synth.cfg4_G())
             if want("scale rules"):
                 fp4_row("scale rules", "G bf16 8192x4096: MXFP4 RNE, OCP floor E8M0 exponent", g4, q.MXFP4, q.RNE,

@@ -417,6 +417,30 @@ __device__ __forceinline__ uint32_t e4m3_sr(float v, uint32_t w)
     return e4m3_rne(rr) | sign;
 }
 
+// e4m3_sr on two values at once (a in the low byte), without a branch: in
+// the normal binades (|v| >= 2^-6) the grid keeps 3 of the 23 mantissa bits
+// and up iff (w >> 8) < 16 * (the 20 dropped bits), i.e. (w >> 12) < them,
+// so adding 0xFFFFF - (w >> 12) to the bits and clearing the low 20 rounds
+// (a carry moves into the exponent); below 2^-6 the spacing is 2^-9 and the
+// fraction is compared as in e4m3_sr.  Saturates at 448.
+__device__ __forceinline__ uint32_t e4m3_sr2(float a, float b, uint32_t wa, uint32_t wb)
+{
+    const float v[2] = {a, b};
+    const uint32_t w[2] = {wa, wb};
+    float r[2];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        const uint32_t bits = __float_as_uint(v[t]) & 0x7FFFFFFFu;
+        const uint32_t rn = (bits + (0xFFFFFu - (w[t] >> 12))) & 0xFFF00000u;
+        const float t9 = __fmul_rn(__uint_as_float(bits), 512.0f), f9 = truncf(t9);
+        const float frac24 = __fmul_rn(__fsub_rn(t9, f9), 16777216.0f);
+        const float rs = __fmul_rn(static_cast<float>(w[t] >> 8) < frac24 ? __fadd_rn(f9, 1.0f) : f9, 0.001953125f);
+        const float rr = fminf(bits >= 0x3C800000u ? __uint_as_float(rn) : rs, 448.0f);
+        r[t] = __uint_as_float(__float_as_uint(rr) | (__float_as_uint(v[t]) & 0x80000000u));
+    }
+    return e4m3x2_rne(r[0], r[1]);
+}
+
 // E4M3 byte -> binary32 (exact), from the bit fields.
 __device__ __forceinline__ float e4m3_value(uint32_t b)
 {

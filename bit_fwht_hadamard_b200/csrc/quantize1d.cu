@@ -655,7 +655,7 @@ __device__ __forceinline__ void mxfp8_unit_packed(uint64_t (&p)[UP], uint64_t e0
             f2unpack(pg[2 * t + 1], c, d);
             if (SR) {
                 const uint4 rw = sr_words4(seed, ((e0 + 32 * g) >> 2) + t);
-                w[t] = e4m3_sr(a, rw.x) | (e4m3_sr(b, rw.y) << 8) | (e4m3_sr(c, rw.z) << 16) | (e4m3_sr(d, rw.w) << 24);
+                w[t] = e4m3_sr2(a, b, rw.x, rw.y) | (e4m3_sr2(c, d, rw.z, rw.w) << 16);
             } else {
                 w[t] = e4m3x2_rne(a, b) | (e4m3x2_rne(c, d) << 16);
             }

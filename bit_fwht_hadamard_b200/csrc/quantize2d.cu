@@ -264,7 +264,8 @@ __global__ void __launch_bounds__(256) k_quant2d(const T *__restrict__ x, Q2DPar
 // Transpose a 32 x 32 nibble matrix held as one 128-bit row per lane (4
 // words, nibble j of lane r = element (r, j) in word j / 8); afterwards
 // nibble j of lane r is element (j, r).  Block swaps of 16 and 8 nibbles move
-// whole words, those of 4, 2 and 1 nibbles masked parts of each word.
+// whole words; those of 4, 2 and 1 nibbles are the 16 x 16 transpose's
+// stages on each pair of words.
 __device__ __forceinline__ void transpose32x32_nibbles(uint32_t (&w)[4], int r)
 {
     {   // 16: words {0,1} of the upper lane <-> words {2,3} of the lower lane
@@ -279,14 +280,29 @@ __device__ __forceinline__ void transpose32x32_nibbles(uint32_t (&w)[4], int r)
         const uint32_t b = __shfl_xor_sync(0xFFFFFFFFu, up ? w[2] : w[3], 8);
         if (up) { w[0] = a; w[2] = b; } else { w[1] = a; w[3] = b; }
     }
+    // 4, 2, 1: the byte-permute stages of the 16 x 16 transpose on the word
+    // pairs (0, 1) and (2, 3): one shuffle a pair and stage
 #pragma unroll
-    for (int s = 4; s >= 1; s >>= 1) {
-        const uint32_t m = s == 4 ? 0xFFFF0000u : s == 2 ? 0xFF00FF00u : 0xF0F0F0F0u;   // nibbles with (j & s) != 0
-        const bool up = (r & s) != 0;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const uint32_t o = __shfl_xor_sync(0xFFFFFFFFu, w[k], s);
-            w[k] = up ? ((w[k] & m) | ((o & m) >> (4 * s))) : ((w[k] & ~m) | ((o & ~m) << (4 * s)));
+    for (int k = 0; k < 4; k += 2) {
+        {
+            const bool up = (r & 4) != 0;
+            const uint32_t got = __shfl_xor_sync(0xFFFFFFFFu, __byte_perm(w[k], w[k + 1], up ? 0x5410u : 0x7632u), 4);
+            w[k] = __byte_perm(w[k], got, up ? 0x3254u : 0x5410u);
+            w[k + 1] = __byte_perm(w[k + 1], got, up ? 0x3276u : 0x7610u);
+        }
+        {
+            const bool up = (r & 2) != 0;
+            const uint32_t got = __shfl_xor_sync(0xFFFFFFFFu, __byte_perm(w[k], w[k + 1], up ? 0x6420u : 0x7531u), 2);
+            w[k] = __byte_perm(w[k], got, up ? 0x3514u : 0x5240u);
+            w[k + 1] = __byte_perm(w[k + 1], got, up ? 0x3716u : 0x7260u);
+        }
+        {
+            const bool up = (r & 1) != 0;
+            const uint32_t M = 0x0F0F0F0Fu, km = up ? ~M : M;
+            const uint32_t send = ((w[k] >> (up ? 0 : 4)) & M) | ((w[k + 1] << (up ? 4 : 0)) & ~M);
+            const uint32_t got = __shfl_xor_sync(0xFFFFFFFFu, send, 1);
+            w[k] = (w[k] & km) | ((got << (up ? 0 : 4)) & ~km);
+            w[k + 1] = (w[k + 1] & km) | ((got >> (up ? 4 : 0)) & ~km);
         }
     }
 }
@@ -840,8 +856,9 @@ __global__ void __launch_bounds__(256) k_cols_sr(const uint16_t *__restrict__ x,
             if (MX8) {
                 float q0, q1;
                 f2unpack(qv, q0, q1);
-                code[0][r >> 2] |= e4m3_sr(q0, w0) << (8 * (r & 3));
-                code[1][r >> 2] |= e4m3_sr(q1, w1) << (8 * (r & 3));
+                const uint32_t b2 = e4m3_sr2(q0, q1, w0, w1);   // column 0 in the low byte
+                code[0][r >> 2] |= (b2 & 0xFFu) << (8 * (r & 3));
+                code[1][r >> 2] |= (b2 >> 8) << (8 * (r & 3));
             } else {
                 float g0, g1;
                 f2unpack(e2m1_sr_grid2(qv, w0, w1), g0, g1);
