@@ -58,7 +58,8 @@ def parse():
     ap.add_argument("--no-gemm", action="store_true", help="skip the GEMM sub-measurement")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-cfg5", action="store_true", help="skip the largest-configuration sub-measurements")
-    ap.add_argument("--profile-case", choices=["quant", "gemm", "quant-nvfp4", "backward"], default=None,
+    ap.add_argument("--profile-case", choices=["quant", "gemm", "quant-nvfp4", "backward", "backward-sr", "dequant"],
+                    default=None,
                     help="run a few untimed calls of one kernel family (for ncu captures) and exit")
     ap.add_argument("--rows", nargs="?", const="", default=None, metavar="FILTER",
                     help="time every entry point of the path on its own full-size workload (one JSON line each); "
@@ -639,6 +640,20 @@ def run_profile_case(case):
             q.quantize(g, q.NVFP4, q.RNE, block2d=True, transposed=True)
             q.quantize_mxfp8(g, q.RNE, transposed=True)
             q.quantize(g, q.MXFP4, q.RNE, transposed=True)
+    elif case == "backward-sr":
+        # gradient G 8192 x 4096 with stochastic rounding: 2D NVFP4 with G^T,
+        # 1D NVFP4 rows + independent columns, MXFP8 rows + columns
+        g = torch.from_numpy(synth.cfg4_G().view(np.int16)).view(torch.bfloat16).to(dev)
+        for _ in range(2):
+            q.quantize(g, q.NVFP4, q.SR, block2d=True, transposed=True, seed=11)
+            q.quantize(g, q.NVFP4, q.SR, transposed=True, seed=11)
+            q.quantize_mxfp8(g, q.SR, seed=11, transposed=True)
+    elif case == "dequant":
+        x = torch.from_numpy(synth.cfg3_X().view(np.int16)).view(torch.bfloat16).to(dev)
+        X = q.quantize(x, q.NVFP4, q.RNE)
+        for _ in range(2):
+            q.dequantize(X, 8192, 4096, q.NVFP4, out_dtype=torch.bfloat16)
+            q.dequantize(X, 8192, 4096, q.NVFP4, out_dtype=torch.float32)
     elif case == "quant-nvfp4":
         x = torch.from_numpy(synth.cfg3_X().view(np.int16)).view(torch.bfloat16).to(dev)
         for _ in range(2):
