@@ -671,11 +671,22 @@ __global__ void __launch_bounds__(256) k_cols4(const uint16_t *__restrict__ x, Q
                 dst[1] = make_uint4(w[c][4], w[c][5], w[c][6], w[c][7]);
                 p.scalesT[j * (p.M / 32) + i0 / 32] = static_cast<uint8_t>(sb[0][c]);
             } else {
-                uint2 *dst = reinterpret_cast<uint2 *>(p.codesT + (j * p.M + i0) / 2);
-                dst[0] = make_uint2(w[c][0], w[c][1]);
-                if (rows == 32) dst[1] = make_uint2(w[c][2], w[c][3]);
+                // M % 32 == 0 (always for groups of 32): 16-byte code stores and
+                // the two NVFP4 scale bytes in one 2-byte store, both aligned
+                const bool whole = rows == 32 && (p.M % 32) == 0;
+                if (whole) {
+                    *reinterpret_cast<uint4 *>(p.codesT + (j * p.M + i0) / 2) =
+                        make_uint4(w[c][0], w[c][1], w[c][2], w[c][3]);
+                } else {
+                    uint2 *dst = reinterpret_cast<uint2 *>(p.codesT + (j * p.M + i0) / 2);
+                    dst[0] = make_uint2(w[c][0], w[c][1]);
+                    if (rows == 32) dst[1] = make_uint2(w[c][2], w[c][3]);
+                }
                 if (G == 32) {
                     p.scalesT[j * (p.M / 32) + i0 / 32] = static_cast<uint8_t>(sb[0][c]);
+                } else if (whole) {
+                    *reinterpret_cast<uint16_t *>(p.scalesT + j * (p.M / 16) + i0 / 16) =
+                        static_cast<uint16_t>(sb[0][c] | (sb[NG - 1][c] << 8));
                 } else {
                     p.scalesT[j * (p.M / 16) + i0 / 16] = static_cast<uint8_t>(sb[0][c]);
                     if (rows == 32) p.scalesT[j * (p.M / 16) + i0 / 16 + 1] = static_cast<uint8_t>(sb[NG - 1][c]);
@@ -898,11 +909,22 @@ __global__ void __launch_bounds__(256) k_cols_sr(const uint16_t *__restrict__ x,
                     dst[1] = make_uint4(code[c][4], code[c][5], code[c][6], code[c][7]);
                     p.scalesT[jr * (p.M / 32) + i0 / 32] = static_cast<uint8_t>(sb[0][c]);
                 } else {
-                    uint2 *dst = reinterpret_cast<uint2 *>(p.codesT + (jr * p.M + i0) / 2);
-                    dst[0] = make_uint2(code[c][0], code[c][1]);
-                    if (rows == 32) dst[1] = make_uint2(code[c][2], code[c][3]);
+                    // M % 32 == 0 (always for groups of 32): 16-byte code stores and
+                    // the two NVFP4 scale bytes in one 2-byte store, both aligned
+                    const bool whole = rows == 32 && (p.M % 32) == 0;
+                    if (whole) {
+                        *reinterpret_cast<uint4 *>(p.codesT + (jr * p.M + i0) / 2) =
+                            make_uint4(code[c][0], code[c][1], code[c][2], code[c][3]);
+                    } else {
+                        uint2 *dst = reinterpret_cast<uint2 *>(p.codesT + (jr * p.M + i0) / 2);
+                        dst[0] = make_uint2(code[c][0], code[c][1]);
+                        if (rows == 32) dst[1] = make_uint2(code[c][2], code[c][3]);
+                    }
                     if (G == 32) {
                         p.scalesT[jr * (p.M / 32) + i0 / 32] = static_cast<uint8_t>(sb[0][c]);
+                    } else if (whole) {
+                        *reinterpret_cast<uint16_t *>(p.scalesT + jr * (p.M / 16) + i0 / 16) =
+                            static_cast<uint16_t>(sb[0][c] | (sb[NG - 1][c] << 8));
                     } else {
                         p.scalesT[jr * (p.M / 16) + i0 / 16] = static_cast<uint8_t>(sb[0][c]);
                         if (rows == 32) p.scalesT[jr * (p.M / 16) + i0 / 16 + 1] = static_cast<uint8_t>(sb[NG - 1][c]);
