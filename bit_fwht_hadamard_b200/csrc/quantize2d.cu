@@ -343,7 +343,10 @@ __global__ void __launch_bounds__(256) k_quant2d_mx(const T *__restrict__ x, Q2D
 #pragma unroll
             for (int t = 0; t < 32; ++t) q[t] = __fmul_rn(v[t], mul);
             if (SR) {
-                sr_group<32>(q, static_cast<uint64_t>(i * p.K + bj), p.seed, w);
+                uint64_t qp[16];
+#pragma unroll
+                for (int t = 0; t < 16; ++t) qp[t] = f2pack(q[2 * t], q[2 * t + 1]);
+                sr_group_pairs<32>(qp, static_cast<uint64_t>(i * p.K + bj), p.seed, w);
             } else {
 #pragma unroll
                 for (int t = 0; t < 4; ++t) w[t] = e2m1x8_rne(q + 8 * t);
