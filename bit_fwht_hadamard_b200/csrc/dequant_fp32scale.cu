@@ -11,6 +11,21 @@ __device__ __forceinline__ float exp2_b128(uint32_t b)
     return __uint_as_float(b >= 2u ? (b - 1u) << 23 : 0x00200000u << b);
 }
 
+// E2M1 codes of four elements (16 bits, element t in bits 4t .. 4t + 3) as
+// two bfloat16 pairs (exact: bfloat16 holds every E2M1 value).  The high and
+// low bytes of the eight magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6 (bf16 0x0000,
+// 0x3F00, 0x3F80, 0x3FC0, 0x4000, 0x4040, 0x4080, 0x40C0) are two byte-permute
+// tables indexed by the 3-bit magnitudes, two more permutes interleave them,
+// and the sign bits go to bits 15 and 31.
+__device__ __forceinline__ void e2m1x4_to_bf16x2(uint32_t w16, uint32_t &p01, uint32_t &p23)
+{
+    const uint32_t sel = w16 & 0x7777u;
+    const uint32_t hi = __byte_perm(0x3F3F3F00u, 0x40404040u, sel);
+    const uint32_t lo = __byte_perm(0xC0800000u, 0xC0804000u, sel);
+    p01 = __byte_perm(lo, hi, 0x5140u) | ((w16 << 12) & 0x8000u) | ((w16 << 24) & 0x80000000u);
+    p23 = __byte_perm(lo, hi, 0x7362u) | ((w16 << 4) & 0x8000u) | ((w16 << 16) & 0x80000000u);
+}
+
 // Four consecutive elements e0 .. e0 + 3 from their two code bytes w16 and
 // their scale byte sb.  Every output is the exact value g * scale (* s_t)
 // rounded once:

@@ -287,33 +287,24 @@ __device__ __forceinline__ uint32_t e2m1x8_rne_pairs(uint64_t p0, uint64_t p1, u
     return e2m1x8_rne(v);
 }
 
-// E2M1 codes of four elements (16 bits, element t in bits 4t .. 4t + 3) as
-// two bfloat16 pairs (exact: bfloat16 holds every E2M1 value).  The high and
-// low bytes of the eight magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6 (bf16 0x0000,
-// 0x3F00, 0x3F80, 0x3FC0, 0x4000, 0x4040, 0x4080, 0x40C0) are two byte-permute
-// tables indexed by the 3-bit magnitudes, two more permutes interleave them,
-// and the sign bits go to bits 15 and 31.
-__device__ __forceinline__ void e2m1x4_to_bf16x2(uint32_t w16, uint32_t &p01, uint32_t &p23)
-{
-    const uint32_t sel = w16 & 0x7777u;
-    const uint32_t hi = __byte_perm(0x3F3F3F00u, 0x40404040u, sel);
-    const uint32_t lo = __byte_perm(0xC0800000u, 0xC0804000u, sel);
-    p01 = __byte_perm(lo, hi, 0x5140u) | ((w16 << 12) & 0x8000u) | ((w16 << 24) & 0x80000000u);
-    p23 = __byte_perm(lo, hi, 0x7362u) | ((w16 << 4) & 0x8000u) | ((w16 << 16) & 0x80000000u);
-}
-
-// The eight E2M1 values of a word of nibbles as four packed binary32 pairs
-// (exact), from the byte-permute tables above.  The packed hardware decode
-// (cvt.rn.f16x2.e2m1x2) returned zeros on B200 for bytes 2-3 of words just
-// produced by the E2M1 conversion and for bytes of a 16-bit load, so no
-// path decodes with it.
+// The eight E2M1 values of a word of nibbles as binary32 (exact: binary16
+// holds every E2M1 value, and the widening is exact).
 __device__ __forceinline__ void e2m1x8_values(uint32_t w, uint64_t *g4)
 {
-    uint32_t p[4];
-    e2m1x4_to_bf16x2(w & 0xFFFFu, p[0], p[1]);
-    e2m1x4_to_bf16x2(w >> 16, p[2], p[3]);
+    uint32_t h[4];
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+        : "r"(w));
 #pragma unroll
-    for (int q = 0; q < 4; ++q) g4[q] = f2pack(__uint_as_float(p[q] << 16), __uint_as_float(p[q] & 0xFFFF0000u));
+    for (int q = 0; q < 4; ++q) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h[q]));
+        g4[q] = f2pack(f.x, f.y);
+    }
 }
 
 // E2M1 stochastic rounding of one value (|v| <= 6 or saturating):

@@ -130,10 +130,10 @@ __device__ __forceinline__ void nv_block_rne_pairs(const uint64_t *pp, float S, 
     else nv_codes16_pairs(pp, S, amax, w2);
     if (sse) {
         // Scalar IEEE operations: the multiply feeding the subtraction must
-        // stay two roundings.  The packed f32x2 multiply and subtract gave
-        // different sums on B200 (153 of 16.8 M codes of the full-size
-        // four-over-six test changed, with the E2M1 values from the table
-        // decode), and the sums decide the selection.
+        // stay two roundings.  The packed f32x2 multiply, subtract and tree
+        // gave different sums on B200 (153 of 16.8 M codes of the full-size
+        // four-over-six test changed, with either E2M1 decode), and the sums
+        // decide the selection.
         uint64_t g[8];
         e2m1x8_values(w2[0], g);
         e2m1x8_values(w2[1], g + 4);
