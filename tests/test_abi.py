@@ -123,3 +123,35 @@ def test_kl_calibrate_argument_errors():
     assert C(f, q.BF16, 64, 64, 8, 0, None, None, None, None, f, 1 << 20, None) == q.ERR_ARG    # no clip output
     assert C(f, q.BF16, 64, 64, 8, 0, f, None, None, None, f, 16, None) == q.ERR_ARG            # short workspace
     assert q.qfp4_kl_calibrate_workspace_bytes(2048, 8, 0) > 2048 * 8
+
+
+def test_linear_argument_errors_return_before_any_launch():
+    """Every case below is refused by the host checks before a CUDA call (the
+    pointers are never dereferenced); empty shapes, which may issue memsets,
+    are left out."""
+    f = 1 << 20
+    big = 1 << 40
+    Fw = q.qfp4_linear_forward
+    ok_ws = q.qfp4_linear_forward_workspace_bytes(256, 512, 1024, q.NVFP4)
+    assert ok_ws > 0 and q.qfp4_linear_forward_workspace_bytes(256, 512, 1024, 7) == 0
+    assert Fw(f, f, 256, 512, 1024, 7, 0, q.BF16, f, f, big, None) == q.ERR_ARG                 # format
+    assert Fw(f, f, 256, 512, 1024, q.NVFP4, 0, 9, f, f, big, None) == q.ERR_ARG                # output type
+    assert Fw(f, f, 256, 512, 1024, q.MXFP4, 1, q.BF16, f, f, big, None) == q.ERR_UNSUPPORTED   # four6 on MXFP4
+    assert Fw(f, f, -1, 512, 1024, q.NVFP4, 0, q.BF16, f, f, big, None) == q.ERR_SHAPE
+    assert Fw(f, f, 256, 512, 1000, q.NVFP4, 0, q.BF16, f, f, big, None) == q.ERR_SHAPE         # K % 128
+    assert Fw(f, f, 256, 12, 1024, q.NVFP4, 0, q.BF16, f, f, big, None) == q.ERR_SHAPE          # N % 8, bf16 out
+    assert Fw(f, f, 256, 512, 1024, q.NVFP4, 0, q.BF16, None, f, big, None) == q.ERR_ARG        # no output
+    assert Fw(f + 4, f, 256, 512, 1024, q.NVFP4, 0, q.BF16, f, f, big, None) == q.ERR_ALIGN
+    assert Fw(f, f, 256, 512, 1024, q.NVFP4, 0, q.BF16, f, f, ok_ws - 1, None) == q.ERR_ARG     # short workspace
+    Bw = q.qfp4_linear_backward
+    bws = q.qfp4_linear_backward_workspace_bytes(256, 384, 512, q.NVFP4)
+    assert bws > 0 and q.qfp4_linear_backward_workspace_bytes(256, 384, 512, q.MXFP4) == 0
+    assert Bw(f, f, f, 256, 384, 512, q.MXFP4, 1, q.F32, f, f, f, big, None) == q.ERR_ARG       # format
+    assert Bw(f, f, f, 250, 384, 512, q.NVFP4, 1, q.F32, f, f, f, big, None) == q.ERR_SHAPE     # M % 32
+    assert Bw(f, f, f, 256, 384, 520, q.NVFP4, 1, q.F32, f, f, f, big, None) == q.ERR_SHAPE     # K % 16
+    assert Bw(f, f, f, 256, 384, 528, q.MXFP8, 1, q.F32, f, f, f, big, None) == q.ERR_SHAPE     # K % 32
+    assert Bw(f, f, f, 256, 384, 512, q.NVFP4, 1, q.F32, None, None, f, big, None) == q.ERR_ARG  # no output
+    assert Bw(f, f, None, 256, 384, 512, q.NVFP4, 1, q.F32, f, None, f, big, None) == q.ERR_ARG  # dX without W
+    assert Bw(f, None, f, 256, 384, 512, q.NVFP4, 1, q.F32, None, f, f, big, None) == q.ERR_ARG  # dW without X
+    assert Bw(f, f, f, 256, 384, 512, q.NVFP4, 1, q.F32, f, f + 8, f, big, None) == q.ERR_ALIGN
+    assert Bw(f, f, f, 256, 384, 512, q.NVFP4, 1, q.F32, f, f, f, bws - 1, None) == q.ERR_ARG    # short workspace
