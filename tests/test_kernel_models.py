@@ -342,3 +342,46 @@ def test_kl_warp_kernel_algorithm_matches_the_oracle():
             assert np.array_equal(np.isinf(ref), np.isinf(new))
             f = np.isfinite(ref)
             assert np.allclose(new[f], ref[f], rtol=1e-13, atol=1e-300)
+
+
+# ------------------------------------------------------------------ packed E2M1 stochastic grid
+def _rz_f32(x):
+    """An exact positive rational rounded toward zero to binary32 (normal range)."""
+    from fractions import Fraction
+    e = x.numerator.bit_length() - x.denominator.bit_length()
+    if Fraction(2) ** e > x:
+        e -= 1
+    ulp = Fraction(2) ** (e - 23)
+    return np.float32(float((x // ulp) * ulp))
+
+
+def _e2m1_sr_grid2_model(v, w):
+    """e2m1_sr_grid2 on one element of the pair, step by step in binary32 as
+    the kernel computes it: the spacing exponent clamped below at 127, the
+    round-toward-zero add of 1.5 * 2^47 that leaves floor(q24 / 2^24) * 2^24,
+    the integer compare of the random word's top 24 bits against the
+    fraction, the sign copied; then the saturating E2M1 conversion."""
+    from fractions import Fraction
+    b = _f2u(v) & 0x7FFFFFFF
+    m = max(b >> 23, 127)
+    inv, sp = _u2f((279 - m) << 23), _u2f((m - 25) << 23)
+    C = np.float32(1.5 * 2.0 ** 47)
+    q24 = np.float32(_u2f(b) * inv)
+    assert Fraction(float(q24)) == Fraction(float(_u2f(b))) * Fraction(float(inv))   # a power-of-two scaling
+    fl24 = np.float32(_rz_f32(Fraction(float(q24)) + Fraction(float(C))) - C)
+    frac = np.float32(q24 - fl24)
+    up = np.float32(w >> 8) < frac
+    r = np.float32(np.float32(fl24 + (np.float32(16777216.0) if up else np.float32(0))) * sp)
+    r_signed = _u2f(_f2u(r) | (_f2u(v) & 0x80000000))
+    return oracle.e2m1_rne(float(r_signed))          # cvt.rn.satfinite.e2m1x2: r is a grid value or >= 6
+
+
+def test_packed_e2m1_stochastic_grid_equals_the_definition():
+    rng = np.random.default_rng(11)
+    vals = np.concatenate([rng.standard_normal(500) * s for s in (1e-3, 0.1, 0.4, 1, 2.5, 5)] +
+                          [rng.uniform(-7.9, 7.9, 500),
+                           np.array([0.0, -0.0, 0.25, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0, 6.5, 8.0, 100.0, 1e30,
+                                     2.0 ** -149, -(2.0 ** -126), 0.5 - 2.0 ** -26, 6.0 - 2.0 ** -21])])
+    for v in vals.astype(np.float32):
+        for w in (int(rng.integers(0, 2 ** 32)), int(rng.integers(0, 2 ** 32)), 0, U32, 0x80000000, 0xFF):
+            assert _e2m1_sr_grid2_model(v, w) == oracle.e2m1_sr(float(v), w), (float(v), w)
