@@ -33,6 +33,12 @@ using namespace qfp4;
 
 static bool ok_align(const void *p) { return p == nullptr || aligned16(p); }
 
+// At most 2^38 elements in an M x K operand (a 512 GB bf16 tensor, above one
+// GPU's memory): every byte count fits int64, and the 1D pass's tensor map
+// (rows of 64 elements) stays within its 2^32-row limit.
+constexpr int64_t kMaxElems = int64_t(1) << 38;
+static bool size_ok(int64_t M, int64_t K) { return M <= kMaxElems && K <= kMaxElems && (M == 0 || K <= kMaxElems / M); }
+
 extern "C" size_t qfp4_quantize_workspace_bytes(int64_t M, int64_t K, qfp4_fmt fmt, int rotate, int block2d)
 {
     (void)M; (void)K; (void)rotate; (void)block2d;
@@ -46,7 +52,7 @@ extern "C" int qfp4_quantize_ex(const void *x, qfp4_dtype xdt, int64_t M, int64_
                                 size_t workspace_bytes, qfp4_stream_t stream_)
 {
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-    if (M < 0 || K < 0) return QFP4_ERR_SHAPE;
+    if (M < 0 || K < 0 || !size_ok(M, K)) return QFP4_ERR_SHAPE;
     if (fmt != QFP4_MXFP4 && fmt != QFP4_NVFP4) return QFP4_ERR_ARG;
     if (rounding != QFP4_RNE && rounding != QFP4_SR) return QFP4_ERR_ARG;
     if (xdt != QFP4_BF16 && xdt != QFP4_F32) return QFP4_ERR_ARG;
@@ -115,7 +121,7 @@ extern "C" int qfp4_quantize_mxfp8(const void *x, qfp4_dtype xdt, int64_t M, int
                                    uint64_t seed, uint8_t *codes, uint8_t *scales, uint8_t *codesT, uint8_t *scalesT,
                                    qfp4_stream_t stream)
 {
-    if (M < 0 || K < 0) return QFP4_ERR_SHAPE;
+    if (M < 0 || K < 0 || !size_ok(M, K)) return QFP4_ERR_SHAPE;
     if (rounding != QFP4_RNE && rounding != QFP4_SR) return QFP4_ERR_ARG;
     if (xdt != QFP4_BF16 && xdt != QFP4_F32) return QFP4_ERR_ARG;
     if (M * K > 0 && (!x || !codes || !scales)) return QFP4_ERR_ARG;
@@ -133,7 +139,7 @@ extern "C" int qfp4_quantize_fp32scale(const void *x, qfp4_dtype xdt, int64_t M,
                                        uint8_t *codes, float *scales, void *workspace, size_t workspace_bytes,
                                        qfp4_stream_t stream)
 {
-    if (M < 0 || K < 0) return QFP4_ERR_SHAPE;
+    if (M < 0 || K < 0 || !size_ok(M, K)) return QFP4_ERR_SHAPE;
     if (xdt != QFP4_BF16 && xdt != QFP4_F32) return QFP4_ERR_ARG;
     if (gran < QFP4_GRAN_TENSOR || gran > QFP4_GRAN_GROUP32) return QFP4_ERR_ARG;
     if (M * K > 0 && (!x || !codes || !scales)) return QFP4_ERR_ARG;
@@ -149,7 +155,7 @@ extern "C" int qfp4_quantize_fp32scale(const void *x, qfp4_dtype xdt, int64_t M,
 extern "C" int qfp4_dequantize(const uint8_t *codes, const uint8_t *scales, const float *tscale, int64_t M, int64_t K,
                                qfp4_fmt fmt, qfp4_dtype out_dt, void *out, qfp4_stream_t stream)
 {
-    if (M < 0 || K < 0) return QFP4_ERR_SHAPE;
+    if (M < 0 || K < 0 || !size_ok(M, K)) return QFP4_ERR_SHAPE;
     if (fmt != QFP4_MXFP4 && fmt != QFP4_NVFP4) return QFP4_ERR_ARG;
     if (out_dt != QFP4_BF16 && out_dt != QFP4_F32) return QFP4_ERR_ARG;
     if (M * K > 0 && (!codes || !scales || !out)) return QFP4_ERR_ARG;

@@ -324,7 +324,7 @@ extern "C" int qfp4_kl_calibrate(const void *x, qfp4_dtype xdt, int64_t n, int b
     int st = kl_args_ok(bins, levels, grid);
     if (st != QFP4_OK) return st;
     if (xdt != QFP4_BF16 && xdt != QFP4_F32) return QFP4_ERR_ARG;
-    if (n < 0) return QFP4_ERR_SHAPE;
+    if (n < 0 || n > (int64_t(1) << 38)) return QFP4_ERR_SHAPE;   // the library's element limit
     if (!clip_out || (n > 0 && !x)) return QFP4_ERR_ARG;
     if (!aligned16(x) || !aligned16(workspace) || !aligned16(kl_out) || !aligned16(hist_out)) return QFP4_ERR_ALIGN;
     const KlLayout L = kl_layout(bins, levels, grid);

@@ -975,7 +975,8 @@ static int run_pass(const void *x, qfp4_dtype xdt, int64_t n, QuantParams p, cud
     return QFP4_OK;
 }
 
-// Partial maxima of |x| over a flat range (the NVFP4 tensor-amax pass, no rotation).
+// MXFP8 row-wise codes and E8M0 scales of x[0, n) (bf16, n % 64 == 0) through
+// the TMA kernel.
 int mxfp8_rows(const void *x, int64_t n, bool sr, uint64_t seed, uint8_t *codes, uint8_t *scales, cudaStream_t stream)
 {
     if (n <= 0) return QFP4_OK;
@@ -998,6 +999,7 @@ int mxfp8_rows(const void *x, int64_t n, bool sr, uint64_t seed, uint8_t *codes,
               : launch_tma<MODE_QUANT, FMT_MXFP8, false, false, false>(tm, q, grid, stream);
 }
 
+// Partial maxima of |x| over a flat range (the NVFP4 tensor-amax pass, no rotation).
 int amax_partials(const void *x, qfp4_dtype xdt, int64_t n, float *partials, int *n_parts, cudaStream_t stream)
 {
     QuantParams p{};

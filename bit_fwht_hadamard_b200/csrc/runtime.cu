@@ -59,7 +59,7 @@ extern "C" const char *qfp4_status_string(int status)
     switch (status) {
     case QFP4_OK: return "ok";
     case QFP4_ERR_ARG: return "invalid argument (NULL buffer, bad enum value or short workspace)";
-    case QFP4_ERR_SHAPE: return "shape violates the call's divisibility rules";
+    case QFP4_ERR_SHAPE: return "shape violates the call's divisibility or size rules";
     case QFP4_ERR_UNSUPPORTED: return "unsupported option combination";
     case QFP4_ERR_ALIGN: return "pointer not 16-byte aligned";
     case QFP4_ERR_CUDA: return "CUDA launch or driver call failed";

@@ -35,6 +35,10 @@
  *     E8M0 byte, the scale is 2^(byte-127).  NVFP4 (g = 16): an OCP E4M3
  *     byte, the scale is e4m3(byte) * s_t with s_t the per-tensor scale.
  *   - All buffers need 16-byte aligned base pointers.
+ *   - Size limits (QFP4_ERR_SHAPE beyond them): the quantize, dequantize
+ *     and calibration calls take at most 2^38 elements (M*K, or n), a
+ *     512 GB bf16 tensor; the GEMM and linear calls take M, N, K below
+ *     2^30.  Within them every byte count fits int64.
  */
 #ifndef QFP4_H
 #define QFP4_H
@@ -69,7 +73,7 @@ typedef enum {
 enum {
     QFP4_OK = 0,
     QFP4_ERR_ARG = -1,          /* NULL where a buffer is required, bad enum, short workspace */
-    QFP4_ERR_SHAPE = -2,        /* dimensions violate the call's divisibility rules           */
+    QFP4_ERR_SHAPE = -2,        /* dimensions violate the call's divisibility or size rules   */
     QFP4_ERR_UNSUPPORTED = -3,  /* option combination not defined by the method              */
     QFP4_ERR_ALIGN = -4,        /* a pointer is not 16-byte aligned                           */
     QFP4_ERR_CUDA = -5,         /* a CUDA launch or driver call failed                        */

@@ -155,3 +155,22 @@ def test_linear_argument_errors_return_before_any_launch():
     assert Bw(f, None, f, 256, 384, 512, q.NVFP4, 1, q.F32, None, f, f, big, None) == q.ERR_ARG  # dW without X
     assert Bw(f, f, f, 256, 384, 512, q.NVFP4, 1, q.F32, f, f + 8, f, big, None) == q.ERR_ALIGN
     assert Bw(f, f, f, 256, 384, 512, q.NVFP4, 1, q.F32, f, f, f, bws - 1, None) == q.ERR_ARG    # short workspace
+
+
+def test_size_limits_are_shape_errors():
+    """Operands above 2^38 elements (or with M * K past int64) are refused as
+    shape errors before any launch, as are GEMM dimensions of 2^30 or more."""
+    f = 1 << 20
+    for M, K in ((1 << 20, 1 << 19), (1 << 40, 1 << 40), (1 << 62, 1 << 6)):
+        assert q.qfp4_quantize(f, q.BF16, M, K, q.MXFP4, q.RNE, 0, 0, 0, 0, f, f, None, None, None, None, 0,
+                               None) == q.ERR_SHAPE
+        assert q.qfp4_quantize_mxfp8(f, q.BF16, M, K, q.RNE, 0, f, f, None, None, None) == q.ERR_SHAPE
+        assert q.qfp4_quantize_fp32scale(f, q.BF16, M, K, q.GRAN_ROW, f, f, None, 0, None) == q.ERR_SHAPE
+        assert q.qfp4_dequantize(f, f, f, M, K, q.MXFP4, q.F32, f, None) == q.ERR_SHAPE
+    ws = q.qfp4_kl_calibrate_workspace_bytes(2048, 8, 0)
+    assert ws > 0
+    assert q.qfp4_kl_calibrate(f, q.BF16, (1 << 38) + 32, 2048, 8, 0, f, None, None, None, f, ws, None) == q.ERR_SHAPE
+    big = 1 << 30
+    assert q.qfp4_gemm_blockscaled(f, f, None, f, f, None, big, 256, 256, q.MXFP4, q.F32, f, f, 1 << 40,
+                                   None) == q.ERR_SHAPE
+    assert q.qfp4_status_string(q.ERR_SHAPE) == "shape violates the call's divisibility or size rules"
