@@ -385,3 +385,81 @@ def test_packed_e2m1_stochastic_grid_equals_the_definition():
     for v in vals.astype(np.float32):
         for w in (int(rng.integers(0, 2 ** 32)), int(rng.integers(0, 2 ** 32)), 0, U32, 0x80000000, 0xFF):
             assert _e2m1_sr_grid2_model(v, w) == oracle.e2m1_sr(float(v), w), (float(v), w)
+
+
+# ------------------------------------------------------------------ scale exponents and E4M3 scale bytes
+def _scale_exp_model(amax, top_frac, top_e):
+    """scale_exp: amax = (1 + f 2^-23) 2^e from its bits (subnormals
+    normalised by their leading one), k = e - top_e, plus one when the
+    fraction exceeds top's, clamped to [-127, 127]."""
+    u = _f2u(amax) & 0x7FFFFFFF
+    if u == 0:
+        return -127
+    E = u >> 23
+    if E == 0:
+        lead = u.bit_length() - 1
+        e, f = lead - 149, (u << (23 - lead)) & 0x7FFFFF
+    else:
+        e, f = E - 127, u & 0x7FFFFF
+    k = e - top_e if f <= top_frac else e - top_e + 1
+    return max(-127, min(127, k))
+
+
+def _scale_exp_floor_model(amax, emax):
+    u = _f2u(amax) & 0x7FFFFFFF
+    if u == 0:
+        return -127
+    E = u >> 23
+    e = (u.bit_length() - 1) - 149 if E == 0 else E - 127
+    return max(-127, min(127, e - emax))
+
+
+def _amax_cases(rng):
+    v = [0.0, 2.0 ** -149, 3 * 2.0 ** -149, 2.0 ** -127, 2.0 ** -126, 3.4028234663852886e38, 1.0, 6.0, 4.0, 448.0]
+    for top in (4.0, 6.0, 448.0, 1.0, 8.0):
+        for k in (-149, -140, -130, -127, -126, -120, -3, 0, 1, 7, 100, 119, 120, 125, 126):
+            b = top * 2.0 ** k
+            if b < 3.4e38:
+                f = np.float32(b)
+                v += [float(f), float(np.nextafter(f, np.float32(np.inf))), float(np.nextafter(f, np.float32(0)))]
+    v += list(np.abs(rng.standard_normal(400)) * 10.0 ** rng.integers(-40, 38, 400))
+    return [np.float32(x) for x in v if np.isfinite(np.float32(x))]
+
+
+def test_scale_exponents_from_bits_equal_the_definitions():
+    rng = np.random.default_rng(17)
+    for a in _amax_cases(rng):
+        for top_frac, top_e, top in ((0x400000, 2, 6.0), (0, 2, 4.0), (0x600000, 8, 448.0)):
+            assert _scale_exp_model(a, top_frac, top_e) == oracle.scale_exp(float(a), top), (float(a), top)
+        assert _scale_exp_floor_model(a, 2) == oracle.scale_exp_floor(float(a), 2), float(a)
+
+
+def _e4m3_value_model(b):
+    E, m = (b >> 3) & 15, b & 7
+    mag = np.float32(m) * _u2f(118 << 23) if E == 0 else _u2f(((E + 120) << 23) | (m << 20))
+    return -mag if b & 0x80 else mag
+
+
+def _nv_scale_round_model(r, up):
+    """The last stage of nv_scale_byte: a quotient of 448 or more (or NaN)
+    takes 0x7E; else the nearest E4M3 byte, stepped up once when its value
+    lies below r (rule E4M3_UP)."""
+    if not r < 448.0:
+        return 0x7E
+    enc = oracle.e4m3_rne(float(r))         # the hardware E4M3 conversion, pinned on the GPU
+    if up and enc < 0x7E and _e4m3_value_model(enc) < r:
+        enc += 1
+    return enc
+
+
+def test_e4m3_bit_field_decode_and_round_up_equal_the_definitions():
+    for b in range(256):
+        if b & 0x7F != 0x7F:                 # 0x7F / 0xFF are NaN
+            assert float(_e4m3_value_model(b)) == oracle.e4m3_value(b), b
+    rng = np.random.default_rng(19)
+    ts = [np.float32(x) for x in np.abs(rng.standard_normal(3000)) * 10.0 ** rng.integers(-4, 3, 3000)]
+    ts += [np.float32(oracle.e4m3_value(b)) for b in range(0x7F)]
+    ts += [np.nextafter(t, np.float32(np.inf)) for t in ts[-0x7F:]]
+    ts += [np.float32(x) for x in (2.0 ** -10, 1e-30, 0.0, 448.0, 449.0, 1e30)]
+    for t in ts:
+        assert _nv_scale_round_model(t, True) == oracle.e4m3_up(float(t)), float(t)
