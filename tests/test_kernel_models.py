@@ -463,3 +463,35 @@ def test_e4m3_bit_field_decode_and_round_up_equal_the_definitions():
     ts += [np.float32(x) for x in (2.0 ** -10, 1e-30, 0.0, 448.0, 449.0, 1e30)]
     for t in ts:
         assert _nv_scale_round_model(t, True) == oracle.e4m3_up(float(t)), float(t)
+
+
+def _e4m3_sr_scalar_model(v, w):
+    """e4m3_sr (one value): in the normal binades lo keeps three mantissa
+    bits, the spacing and its inverse come from the exponent field; below
+    2^-6 both come from the 2^-9 grid; up iff fl((w >> 8) 2^-24) < fl((a -
+    lo) / spacing); the result saturates at 448 and takes v's sign bit."""
+    sign = (_f2u(v) >> 24) & 0x80
+    a = np.float32(abs(v))
+    bits = _f2u(a)
+    if a >= np.float32(0.015625):
+        spb = (bits & 0x7F800000) - (3 << 23)
+        lo, sp, inv = _u2f(bits & 0x7FF00000), _u2f(spb), _u2f((254 << 23) - spb)
+    else:
+        lo = np.float32(np.float32(np.trunc(np.float32(a * np.float32(512)))) * np.float32(0.001953125))
+        sp, inv = np.float32(0.001953125), np.float32(512)
+    p = np.float32(np.float32(a - lo) * inv)
+    u = np.float32(np.float32(w >> 8) * np.float32(5.9604644775390625e-08))
+    rr = np.float32(lo + sp) if u < p else lo
+    rr = min(rr, np.float32(448))
+    return oracle.e4m3_rne(float(rr)) | sign
+
+
+def test_scalar_e4m3_stochastic_rule_equals_the_oracle():
+    rng = np.random.default_rng(23)
+    vals = np.concatenate([rng.standard_normal(300) * s for s in (1e-4, 3e-3, 0.02, 1, 30, 200)] +
+                          [np.array([2.0 ** -6, -(2.0 ** -6) * (1 - 2.0 ** -24), 448, -449, 479, 2.0 ** -149,
+                                     2.0 ** -9, 0.0, -0.0])])
+    with np.errstate(over="ignore", invalid="ignore"):
+        for v in vals.astype(np.float32):
+            for w in (int(rng.integers(0, 2 ** 32)), 0, U32, 0x80000000, 0x7FFFF000):
+                assert _e4m3_sr_scalar_model(v, w) == oracle.e4m3_sr(float(v), w), (float(v), w)
