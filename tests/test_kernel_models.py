@@ -495,3 +495,31 @@ def test_scalar_e4m3_stochastic_rule_equals_the_oracle():
         for v in vals.astype(np.float32):
             for w in (int(rng.integers(0, 2 ** 32)), 0, U32, 0x80000000, 0x7FFFF000):
                 assert _e4m3_sr_scalar_model(v, w) == oracle.e4m3_sr(float(v), w), (float(v), w)
+
+
+def _e2m1_sr_grid_scalar_model(v, w):
+    """e2m1_sr_grid (one value): the spacing exponent clamped to [127, 129],
+    so values from 8 on stay in the 4..6 spacing and the result is clamped
+    to 6 in binary32 before the conversion."""
+    from fractions import Fraction
+    a = np.float32(abs(v))
+    m = min(max(_f2u(a) >> 23, 127), 129)
+    inv, sp = _u2f((279 - m) << 23), _u2f((m - 25) << 23)
+    C = np.float32(211106232532992.0)
+    q24 = np.float32(a * inv)
+    fl24 = np.float32(_rz_f32(Fraction(float(q24)) + Fraction(float(C))) - C)
+    frac = np.float32(q24 - fl24)
+    r24 = np.float32(fl24 + np.float32(16777216.0)) if np.float32(w >> 8) < frac else fl24
+    r = min(np.float32(r24 * sp), np.float32(6.0))
+    return oracle.e2m1_rne(float(_u2f(_f2u(r) | (_f2u(v) & 0x80000000))))
+
+
+def test_scalar_e2m1_stochastic_grid_equals_the_definition():
+    rng = np.random.default_rng(29)
+    vals = np.concatenate([rng.standard_normal(400) * s for s in (1e-3, 0.3, 1, 2.5, 5)] +
+                          [rng.uniform(-7.9, 7.9, 400),
+                           np.array([0.0, -0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0, 6.5, 8.0, 100.0, 1e6,
+                                     2.0 ** -149, 0.5 - 2.0 ** -26, 6.0 - 2.0 ** -21])])
+    for v in vals.astype(np.float32):
+        for w in (int(rng.integers(0, 2 ** 32)), 0, U32, 0x80000000):
+            assert _e2m1_sr_grid_scalar_model(v, w) == oracle.e2m1_sr(float(v), w), (float(v), w)
