@@ -523,3 +523,29 @@ def test_scalar_e2m1_stochastic_grid_equals_the_definition():
     for v in vals.astype(np.float32):
         for w in (int(rng.integers(0, 2 ** 32)), 0, U32, 0x80000000):
             assert _e2m1_sr_grid_scalar_model(v, w) == oracle.e2m1_sr(float(v), w), (float(v), w)
+
+
+# ------------------------------------------------------------------ folded rotation normalisation (MXFP4 RNE)
+def test_folded_normalisation_gives_the_same_codes():
+    """The plain MXFP4 round-to-nearest path multiplies the unnormalised
+    butterfly sums once by fl(c 2^-k), c = fl(2^-3.5), instead of by c and
+    then by 2^-k.  For k <= 120 the folded multiplier is exact and both give
+    the same E2M1 code: equal values when the product is normal, and a zero
+    of x's sign both ways when it is subnormal.  The group maximum is
+    fl(amax_raw c) either way (rounding is monotone)."""
+    c = _u2f(0x3DB504F3)
+    rng = np.random.default_rng(31)
+    xs = (rng.standard_normal(4000) * 10.0 ** rng.integers(-38, 38, 4000)).astype(np.float32)
+    xs = np.concatenate([xs, np.array([0.0, -0.0, 2.0 ** -149, -(2.0 ** -126), 3.0e38], np.float32)])
+    for k in (-127, -126, -60, -3, 0, 2, 5, 40, 100, 119, 120):
+        folded = np.float32(c * np.float32(2.0 ** -k))
+        assert float(folded) == float(c) * 2.0 ** -k            # exact for k <= 120
+        with np.errstate(over="ignore"):
+            for x in xs:
+                a = np.float32(x * folded)
+                b = np.float32(np.float32(x * c) * np.float32(2.0 ** -k))
+                if not (np.isfinite(a) and np.isfinite(b)):
+                    continue                                    # beyond any group's range
+                assert oracle.e2m1_rne(float(a)) == oracle.e2m1_rne(float(b)), (float(x), k)
+    raw = np.abs(xs[:64])
+    assert np.float32(raw.max() * c) == np.max(np.abs((raw * c).astype(np.float32)))
