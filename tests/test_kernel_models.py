@@ -119,6 +119,49 @@ def test_stochastic_column_mapping_covers_every_element_once(fmt, M, K):
     _sim_cols_sr(M, K, fmt)
 
 
+def _sim_cols_sr_words(M, K):
+    """The Philox words each element of k_cols_sr gets: in step k the lower
+    lane of a pair draws row k and the upper lane row 16 + k (counter
+    ((i0 + row) K + jb) / 4), each keeps the two words of its own columns
+    and passes the other two to its partner.  Returns {(i, j): (counter,
+    word index)}."""
+    col_blocks, row_blocks = (K + 63) // 64, (M + 31) // 32
+    got_words = {}
+    for task in range(row_blocks * col_blocks):
+        i0 = (task // col_blocks) * 32
+        rows = min(32, M - i0)
+        for pair in range(16):
+            jb = (task % col_blocks) * 64 + 4 * pair
+            if jb >= K:
+                continue
+            for k in range(16):
+                wd = [[(((i0 + k + 16 * q) * K + jb) >> 2, t) for t in range(4)] for q in (0, 1)]
+                own = [(wd[q][2], wd[q][3]) if q else (wd[q][0], wd[q][1]) for q in (0, 1)]
+                sent = [(wd[q][0], wd[q][1]) if q else (wd[q][2], wd[q][3]) for q in (0, 1)]
+                got = [sent[1], sent[0]]
+                for q in (0, 1):
+                    j = jb + 2 * q
+                    use_k = got[q] if q else own[q]
+                    for c in (0, 1):
+                        got_words[(i0 + k, j + c)] = use_k[c]
+                    if 16 + k < rows:
+                        use_16k = own[q] if q else got[q]
+                        for c in (0, 1):
+                            got_words[(i0 + 16 + k, j + c)] = use_16k[c]
+    return got_words
+
+
+@pytest.mark.parametrize("M,K", [(16, 16), (48, 64), (80, 36), (128, 260)])
+def test_stochastic_column_words_are_each_elements_own(M, K):
+    """Every element (i, j) rounds with word (i K + j) mod 4 of Philox call
+    (i K + j) / 4, the word the row-wise pass and the oracle use for it."""
+    words = _sim_cols_sr_words(M, K)
+    assert len(words) == M * K
+    for (i, j), w in words.items():
+        e = i * K + j
+        assert w == (e >> 2, e & 3), (i, j)
+
+
 # ------------------------------------------------------------------ nibble transposes
 M4, NM4 = 0x0F0F0F0F, 0xF0F0F0F0
 PERM = {4: (0x5410, 0x7632, 0x3254, 0x5410, 0x3276, 0x7610),     # send up / lo, merge word 0 up / lo, word 1 up / lo
