@@ -1,14 +1,17 @@
-// gemm.cu -- block-scaled FP4 GEMM on 5th-generation tensor cores:
-// Y[m][n] = sum_k deqA[m][k] deqB[n][k]  (A: M x K, B: N x K, both K-major
-// packed E2M1 codes with row-major scales as qfp4_quantize writes them).
+// gemm.cu -- block-scaled FP4 (and MXFP8) GEMM on 5th-generation tensor
+// cores: Y[m][n] = sum_k deqA[m][k] deqB[n][k]  (A: M x K, B: N x K, both
+// K-major: packed E2M1 codes, or E4M3 bytes for MXFP8, with row-major
+// scales as qfp4_quantize / qfp4_quantize_mxfp8 write them).
 //
-// Method: [QN] §QuTLASS (MXFP4 / NVFP4 operands, FP32 accumulation);
-// [LB] §FP4 (Blackwell FP4 tensor cores).  Two persistent, warp-specialised
-// kernels on sm_100a, both with fp32 accumulators in tensor memory (TMEM),
-// operands staged by TMA with 128-byte swizzle and no multicast:
+// Method: [QN] §QuTLASS (MXFP4 / NVFP4 operands, FP32 accumulation; FP8
+// for the backward); [LB] §FP4 (Blackwell FP4 tensor cores).  Two
+// persistent, warp-specialised kernels on sm_100a, both with fp32
+// accumulators in tensor memory (TMEM), operands staged by TMA with 128-byte
+// swizzle and no multicast:
 //   * k_gemm_bs2 (M > 128): a cluster of two CTAs computes a 256 x 256 tile
 //     with tcgen05.mma.cta_group::2 (kind::mxf4 block32 for MXFP4,
-//     kind::mxf4nvf4 block16 for NVFP4).  The leader's one MMA lane issues;
+//     kind::mxf4nvf4 block16 for NVFP4, kind::mxf8f6f4 block32 with E4M3
+//     operands for MXFP8).  The leader's one MMA lane issues;
 //     a scale producer and four scale warps per CTA move each k-tile's scale
 //     words into a ring of TMEM buffers with tcgen05.st; eight epilogue warps
 //     per CTA read the accumulator (tcgen05.ld), hand it back, then store.
