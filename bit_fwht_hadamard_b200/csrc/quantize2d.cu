@@ -6,21 +6,26 @@
 // rounding; MXFP8 for the sensitive projections), [46] (four-over-six on the
 // column groups of the 1D baseline), [LB] §2-§3 (group scales, E8M0).
 //
-// 2D kernel: a warp covers two horizontally adjacent 16x16 tiles of one
-// 16-row band; lane (h, r) loads row r of tile h (16 bf16 = 32 B, so every
-// 32-byte sector a warp touches is fully used).  The tile amax is a 16-lane
-// shuffle reduction; each lane quantizes its row (RNE or Philox SR keyed on
-// X's element index), stores its 8 code bytes, then a 4-level nibble
-// transpose across the 16 lanes (block swaps of 8, 4, 2, 1 nibbles) gives
-// each lane one column of the tile -- the codes of X^T, bit-identical by
-// construction because every element was rounded once.
+// 2D kernel (`k_quant2d`): a warp task is 64 rows x 32 columns, four 16-row
+// bands of two adjacent 16x16 tiles; lane (h, r) loads row r of tile h in
+// each band (16 bf16 = 32 B, so every 32-byte sector a warp touches is fully
+// used).  The tile amax is a 16-lane shuffle reduction; each lane quantizes
+// its row (RNE or Philox SR keyed on X's element index) and stores its 8
+// code bytes; then a 4-stage nibble transpose across the 16 lanes (byte
+// permutes, one shuffle a stage) gives each lane one column of the tile --
+// the codes of X^T, bit-identical by construction because every element was
+// rounded once -- and the four bands make 32 contiguous bytes of an X^T row.
+// `k_quant2d_mx` is the MXFP4 form on 32x32 tiles (a scale-rule variant).
 //
-// Column-wise outputs (1D X^T baseline, MXFP8 columns): for bf16 input a warp
-// covers 32 rows x 128 columns with 4 adjacent columns a lane (`k_cols4`,
-// 256-byte row loads per warp instruction); binary32 inputs use a 32 x 32
-// tile with one column a lane.  Either way a column group of 32 (or two of
-// 16) sits in one lane's registers.  The row-wise MXFP8 output of a bf16
-// input comes from the TMA kernel of the 1D quantize.
+// Column-wise outputs (1D X^T baseline, MXFP8 columns) from bf16 input:
+// round to nearest in `k_cols4` (32 rows x 128 columns a warp, 4 adjacent
+// columns a lane, 256-byte row loads per warp instruction), stochastic
+// rounding in `k_cols_sr` (32 rows x 64 columns a warp, a lane pair sharing
+// 4 columns and each Philox call); binary32 inputs use `k_quant_cols` /
+// `k_mxfp8` on 32 x 32 tiles with one column a lane.  Either way a column
+// group of 32 (or two of 16) sits in one lane's registers.  The row-wise
+// MXFP8 output of a bf16 input comes from the TMA kernel of the 1D quantize
+// (`k_mxfp8` takes both outputs when M * K is not a multiple of 64).
 #include "qfp4_common.cuh"
 #include "quantize1d.cuh"
 
