@@ -174,3 +174,46 @@ def test_size_limits_are_shape_errors():
     assert q.qfp4_gemm_blockscaled(f, f, None, f, f, None, big, 256, 256, q.MXFP4, q.F32, f, f, 1 << 40,
                                    None) == q.ERR_SHAPE
     assert q.qfp4_status_string(q.ERR_SHAPE) == "shape violates the call's divisibility or size rules"
+
+
+def test_header_is_plain_c_and_a_c_program_links_and_runs(tmp_path):
+    """include/qfp4.h compiles as strict C99 (warnings are errors), a C
+    program links against libqfp4.so taking the address of every declared
+    entry point, and its host-only calls and a validation error run."""
+    import subprocess
+    from bit_fwht_hadamard_b200 import build
+    build.build()
+    names = _declared()
+    refs = ",\n    ".join(f"(void (*)(void)){n}" for n in names)
+    src = f"""#include <stdio.h>
+#include <string.h>
+#include "qfp4.h"
+static void (*const entry_points[])(void) = {{
+    {refs}
+}};
+int main(void)
+{{
+    size_t i;
+    for (i = 0; i < sizeof entry_points / sizeof entry_points[0]; ++i)
+        if (!entry_points[i]) return 10;
+    if (qfp4_version() < 100) return 11;
+    if (strcmp(qfp4_status_string(QFP4_OK), "ok") != 0) return 12;
+    if (qfp4_quantize((const void *)0, QFP4_BF16, 4, 64, (qfp4_fmt)7, QFP4_RNE, 0, 0, 0, 0,
+                      (unsigned char *)0, (unsigned char *)0, (unsigned char *)0, (unsigned char *)0,
+                      (float *)0, (void *)0, 0, (qfp4_stream_t)0) != QFP4_ERR_ARG) return 13;
+    printf("%u entry points\\n", (unsigned)(sizeof entry_points / sizeof entry_points[0]));
+    return 0;
+}}
+"""
+    c = tmp_path / "abi_check.c"
+    c.write_text(src)
+    exe = tmp_path / "abi_check"
+    libdir = os.path.join(ROOT, "bit_fwht_hadamard_b200")
+    cc = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                         "-I", os.path.join(ROOT, "include"), str(c), "-o", str(exe),
+                         "-L", libdir, "-l:libqfp4.so", f"-Wl,-rpath,{libdir}"],
+                        capture_output=True, text=True)
+    assert cc.returncode == 0, cc.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0, (run.returncode, run.stderr)
+    assert run.stdout.strip() == f"{len(names)} entry points"
