@@ -268,6 +268,17 @@ def _check(st, where):
         raise QFP4Error(st, where)
 
 
+def _input(t, name, dims=2):
+    """An input tensor the C ABI can read as a plain pointer: on a CUDA
+    device, contiguous (row-major), with `dims` dimensions (None: any)."""
+    if not getattr(t, "is_cuda", False):
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (row-major)")
+    if dims is not None and t.dim() != dims:
+        raise ValueError(f"{name} must have {dims} dimensions, not {t.dim()}")
+
+
 def quantize(x, fmt=MXFP4, rounding=RNE, rotate=False, block2d=False, four6=False, seed=0, transposed=False,
              stream=None, out=None, workspace=None, rule=SCALE_DEFAULT, amax_in=None, amax_out=None):
     """Quantize a contiguous (M, K) bf16/fp32 CUDA tensor; returns a dict of
@@ -276,7 +287,7 @@ def quantize(x, fmt=MXFP4, rounding=RNE, rotate=False, block2d=False, four6=Fals
     ``rule``, ``amax_in`` / ``amax_out`` (one-element float32 CUDA tensors)
     are qfp4_quantize_ex's scale rule and tensor-amax options."""
     torch = _torch()
-    assert x.is_cuda and x.is_contiguous() and x.dim() == 2
+    _input(x, "x")
     M, K = x.shape
     g = 32 if fmt == MXFP4 else 16
     dev = x.device
@@ -301,6 +312,7 @@ def quantize(x, fmt=MXFP4, rounding=RNE, rotate=False, block2d=False, four6=Fals
 
 def quantize_mxfp8(x, rounding=RNE, seed=0, transposed=False, stream=None, out=None):
     torch = _torch()
+    _input(x, "x")
     M, K = x.shape
     dev = x.device
     o = dict(out) if out is not None else {}
@@ -318,6 +330,7 @@ def quantize_mxfp8(x, rounding=RNE, seed=0, transposed=False, stream=None, out=N
 
 def quantize_fp32scale(x, gran, stream=None, out=None):
     torch = _torch()
+    _input(x, "x")
     M, K = x.shape
     dev = x.device
     n_scales = {GRAN_TENSOR: 1, GRAN_ROW: M, GRAN_GROUP16: M * K // 16, GRAN_GROUP32: M * K // 32}[gran]
@@ -367,6 +380,7 @@ def gemm_fused_rq(A_bf16, B, N, fmt=NVFP4, rotate=True, four6=False, out_dtype=N
     A_amax_in / A_amax_out: NVFP4 tensor amax of A supplied / reported
     (one-element float32 CUDA tensors)."""
     torch = _torch()
+    _input(A_bf16, "A_bf16")
     M, K = A_bf16.shape
     out_dtype = torch.float32 if out_dtype is None else out_dtype
     if out is None:
@@ -385,6 +399,8 @@ def linear_forward(X, W, fmt=NVFP4, four6=False, out_dtype=None, out=None, works
     """Y = X W^T through rotated FP4 operands (qfp4_linear_forward); X (M, K)
     and W (N, K) bf16 CUDA tensors."""
     torch = _torch()
+    _input(X, "X")
+    _input(W, "W")
     M, K = X.shape
     N = W.shape[0]
     if out is None:
@@ -403,6 +419,10 @@ def linear_backward(G, X, W, fmt=NVFP4, seed=0, out_dtype=None, want_dx=True, wa
     """(dX, dW) = (G W, G^T X) through quantized operands
     (qfp4_linear_backward); G (M, N), X (M, K), W (N, K) bf16 CUDA tensors."""
     torch = _torch()
+    _input(G, "G")
+    for t, name in ((X, "X"), (W, "W")):
+        if t is not None:
+            _input(t, name)
     M, N = G.shape
     K = X.shape[1] if X is not None else W.shape[1]
     dt = torch.float32 if out_dtype is None else out_dtype
@@ -425,6 +445,7 @@ def kl_calibrate(x, bins=2048, levels=8, grid=0, stream=None, out=None):
     dict(clip (1,) float32, best (1,) int32, kl (bins - first + 1,) float64,
     hist (bins,) int64 holding the uint64 counts)."""
     torch = _torch()
+    _input(x, "x", dims=None)
     dev = x.device
     first = 8 if grid else levels
     o = dict(out) if out is not None else {

@@ -217,3 +217,45 @@ int main(void)
     run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert run.returncode == 0, (run.returncode, run.stderr)
     assert run.stdout.strip() == f"{len(names)} entry points"
+
+
+def test_python_wrappers_refuse_inputs_the_c_abi_cannot_read():
+    """The torch-level wrappers pass plain pointers, so they refuse a host
+    tensor, a non-contiguous view or a wrong rank before any call."""
+    import pytest
+    import torch
+    x = torch.zeros((64, 64), dtype=torch.bfloat16)
+    cases = [
+        (lambda: q.quantize(x, q.MXFP4), "CUDA"),
+        (lambda: q.quantize_mxfp8(x), "CUDA"),
+        (lambda: q.quantize_fp32scale(x, q.GRAN_ROW), "CUDA"),
+        (lambda: q.gemm_fused_rq(x, {}, 64), "CUDA"),
+        (lambda: q.linear_forward(x, x), "CUDA"),
+        (lambda: q.linear_backward(x, None, x), "CUDA"),
+        (lambda: q.kl_calibrate(x), "CUDA"),
+    ]
+    for call, what in cases:
+        with pytest.raises(ValueError, match=what):
+            call()
+    with pytest.raises(ValueError, match="contiguous"):
+        q._input(_FakeCuda(False, 2), "x")
+    with pytest.raises(ValueError, match="dimensions"):
+        q._input(_FakeCuda(True, 3), "x")
+    q._input(_FakeCuda(True, 2), "x")
+    q._input(_FakeCuda(True, 1), "x", dims=None)
+
+
+class _FakeCuda:
+    """Stands in for a CUDA tensor's attributes (no GPU here)."""
+    is_cuda = True
+
+    def __new__(cls, contiguous=True, dims=2):
+        o = object.__new__(cls)
+        o._c, o._d = contiguous, dims
+        return o
+
+    def is_contiguous(self):
+        return self._c
+
+    def dim(self):
+        return self._d
