@@ -210,8 +210,8 @@ int qfp4_quantize_mxfp8(const void *x, qfp4_dtype xdt, int64_t M, int64_t K,
  * scale modes of [LB] §1-§2: S = amax / 6 in binary32 over the tensor, each
  * row, or each group of 16 or 32 along K; v = x / S rounded to the nearest
  * E2M1 value (ties to even, saturating); S == 0 gives +0 codes.
- * scales: 1, M, M*K/16 or M*K/32 binary32 values.  Needs K % 2 == 0 and
- * K % g == 0 for the group modes.  workspace: qfp4_quantize_workspace_bytes
+ * scales: 1, M, M*K/16 or M*K/32 binary32 values.  Needs K % 16 == 0
+ * (K % 32 == 0 for QFP4_GRAN_GROUP32).  workspace: qfp4_quantize_workspace_bytes
  * (M, K, QFP4_NVFP4, 0, 0) bytes for QFP4_GRAN_TENSOR, else may be NULL.
  * ---------------------------------------------------------------------- */
 int qfp4_quantize_fp32scale(const void *x, qfp4_dtype xdt, int64_t M, int64_t K,
@@ -389,7 +389,8 @@ int qfp4_linear_backward(const void *G, const void *X, const void *W, int64_t M,
  *   hist_out       device uint64[bins] (or NULL): the histogram.
  *   workspace      qfp4_kl_calibrate_workspace_bytes(bins, levels, grid).
  * Errors: QFP4_ERR_ARG for bins, levels or grid out of range, a NULL x
- * (n > 0) or clip_out, a short workspace.
+ * (n > 0) or clip_out, a short workspace; QFP4_ERR_SHAPE for n < 0 or
+ * n > 2^38; QFP4_ERR_ALIGN for a pointer off 16 bytes.
  * ---------------------------------------------------------------------- */
 size_t qfp4_kl_calibrate_workspace_bytes(int bins, int levels, int grid);
 
