@@ -91,14 +91,6 @@ __device__ __forceinline__ int e2m1_level_of_bin(int64_t b, int64_t i)
     return level;
 }
 
-__device__ __forceinline__ int kl_level(int b, int i, int levels, int grid)
-{
-    if (grid) return e2m1_level_of_bin(b, i);
-    const int per = i / levels;
-    const int l = b / per;
-    return l < levels ? l : levels - 1;
-}
-
 // Prefix sums of the histogram and of its count of nonzero bins, so that a
 // level's kept mass and nonzero count are two lookups: ph[b] = sum of
 // hist[0 .. b), pnz[b] = number of nonzero bins in [0, b), b = 0 .. bins.
