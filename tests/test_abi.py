@@ -259,3 +259,14 @@ class _FakeCuda:
 
     def dim(self):
         return self._d
+
+
+def test_a_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """No CPU fallback: without the built library every call path raises."""
+    import pytest
+    monkeypatch.setattr(q, "_lib", None)
+    monkeypatch.setattr(q, "LIB_PATH", str(tmp_path / "libqfp4.so"))
+    with pytest.raises(ImportError, match="not built"):
+        q.lib()
+    with pytest.raises(ImportError):
+        q.qfp4_version()
