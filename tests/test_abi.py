@@ -270,3 +270,25 @@ def test_a_missing_library_fails_loudly(monkeypatch, tmp_path):
         q.lib()
     with pytest.raises(ImportError):
         q.qfp4_version()
+
+
+def test_product_path_never_touches_the_oracle():
+    """The package and its native sources neither import, load nor name the
+    oracle library; importing the package and loading libqfp4 leaves the
+    oracle unloaded; the library does not link it."""
+    import subprocess
+    import sys
+    pkg = os.path.join(ROOT, "bit_fwht_hadamard_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", text, re.M), f
+                assert "liboracle" not in text and "qfp4_oracle" not in text, f
+    code = ("import sys; import bit_fwht_hadamard_b200 as q; q.lib(); "
+            "print('oracle' in sys.modules, any('liboracle' in l for l in open('/proc/self/maps')))")
+    out = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0, out.stderr
+    assert out.stdout.split() == ["False", "False"]
+    ldd = subprocess.run(["ldd", os.path.join(pkg, "libqfp4.so")], capture_output=True, text=True)
+    assert "oracle" not in ldd.stdout
