@@ -292,3 +292,14 @@ def test_product_path_never_touches_the_oracle():
     assert out.stdout.split() == ["False", "False"]
     ldd = subprocess.run(["ldd", os.path.join(pkg, "libqfp4.so")], capture_output=True, text=True)
     assert "oracle" not in ldd.stdout
+
+
+def test_oracle_shares_no_code_with_the_product():
+    """The oracle and the input generators include no product header and
+    import nothing from the product package."""
+    for d in ("oracle", "synth"):
+        for f in os.listdir(os.path.join(ROOT, d)):
+            if f.endswith((".py", ".c", ".h")):
+                text = open(os.path.join(ROOT, d, f), encoding="utf-8").read()
+                assert '#include "qfp4.h"' not in text and "csrc/" not in text, f
+                assert not re.search(r"^\s*(import|from)\s+bit_fwht_hadamard_b200\b", text, re.M), f
