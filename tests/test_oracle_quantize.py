@@ -385,6 +385,20 @@ def test_four6_prefers_amax_over_4_when_values_sit_in_the_4_to_6_gap():
     assert pick == 0
 
 
+def test_four6_tie_keeps_amax_over_6():
+    """Equal errors keep the amax/6 candidate (reading c7): when both
+    candidate quotients saturate at 448 they encode the same scale, the
+    codes and errors are identical, and the block must keep amax/6."""
+    rng = np.random.default_rng(37)
+    for _ in range(50):
+        x = (rng.standard_normal(16) * rng.uniform(0.1, 3)).astype(np.float32)
+        s_t = np.float32(np.abs(x).max() / np.float32(2 * 2688))        # both quotients >= 448
+        pick, enc, _ = oracle.four6_pick(x, float(s_t))
+        assert pick == 0 and enc == 0x7E
+    pick, enc, codes = oracle.four6_pick(np.zeros(16, np.float32), 1.0)  # amax 0: both scales 0
+    assert pick == 0 and enc == 0 and not codes.any()
+
+
 def test_four6_in_quantize_matches_pick():
     M, K = 8, 64
     x = synth.cfg3_X(M, K, seed=33)
