@@ -101,6 +101,19 @@ def test_all_zero_groups_and_tensor():
     assert (oracle.quantize(x, oracle.MXFP4)["codes"] == 0).all()
 
 
+def test_nvfp4_block_whose_scale_underflows_gets_plus_zero_codes():
+    """Reading c6: a block whose E4M3 scale rounds to 0 under the tensor scale
+    (values far below amax_t / 2688 * 2^-9) has S = 0 and +0 codes, also for
+    its negative values, with RNE and SR alike."""
+    x = np.zeros((1, 32), np.float32)
+    x[0, :16] = np.array([1e-6, -2e-6, 3e-7, -1e-6] * 4, np.float32)
+    x[0, 16], x[0, 17:] = 1000.0, -3.0
+    for rounding in (oracle.RNE, oracle.SR):
+        q = oracle.quantize(synth.f32_to_bf16_bits(x), oracle.NVFP4, rounding, seed=5)
+        assert q["scales"][0, 0] == 0 and q["scales"][0, 1] == 0x7E      # 1000 / 6 / s_t = 448
+        assert not q["codes"][0, :8].any()
+
+
 def test_effective_bits_match_the_page():
     tb = _tables()["effective_bits"]
     M, K = 64, 256
